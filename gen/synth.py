@@ -1,0 +1,202 @@
+"""Seeded input generation for the sparse-attention workloads.
+
+One ``numpy.random.Generator(PCG64(seed))`` stream per workload, drawn in a
+fixed order: q, k / kv, v, dO, sinks, index sets, topk lengths.  Normal values
+are drawn in float32 and rounded to bfloat16 (round to nearest, ties to even);
+bfloat16 tensors are carried as their raw uint16 bit patterns.
+
+Nothing here computes attention: the only arithmetic is drawing numbers,
+rounding them to bfloat16 and the mean-pooling that stands in for the upstream
+KV compressor (whose algorithm the pages do not give).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .configs import Workload
+
+_CHUNK = 1 << 24
+
+
+def bf16_bits_from_f32(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bfloat16 (RNE); return the uint16 bit patterns."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    bias = np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
+    return ((u + bias) >> np.uint32(16)).astype(np.uint16)
+
+
+def f32_from_bf16_bits(u: np.ndarray) -> np.ndarray:
+    """Widen bfloat16 bit patterns to float32 (exact)."""
+    return (np.ascontiguousarray(u, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def _normal_bf16(rng: np.random.Generator, shape, mul: float = 1.0) -> np.ndarray:
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint16)
+    for lo in range(0, n, _CHUNK):
+        hi = min(n, lo + _CHUNK)
+        x = rng.standard_normal(hi - lo, dtype=np.float32)
+        if mul != 1.0:
+            x *= np.float32(mul)
+        out[lo:hi] = bf16_bits_from_f32(x)
+    return out.reshape(shape)
+
+
+def _block_indices(rng, w: Workload, S: int, allow_future: bool) -> np.ndarray:
+    """[S, Hkv, topk] int32 block indices for one sequence."""
+    bs, topk, Hkv = w.block_size, w.topk, w.Hkv
+    nblk = (S + bs - 1) // bs
+    idx = np.full((S, Hkv, topk), -1, dtype=np.int32)
+    for J in range(nblk):
+        t0, t1 = J * bs, min(S, (J + 1) * bs)
+        rows = (t1 - t0) * Hkv
+        if w.select == "diag_uniform":
+            # slot 0 = own (diagonal) block, then distinct uniform earlier blocks
+            ncand = nblk if allow_future else J
+            cand = np.array([c for c in range(ncand) if c != J], dtype=np.int64)
+            k = min(topk - 1, len(cand))
+            sel = np.full((rows, topk), -1, dtype=np.int64)
+            sel[:, 0] = J
+            if k > 0:
+                keys = rng.random((rows, len(cand)))
+                order = np.argsort(keys, axis=1, kind="stable")[:, :k]
+                sel[:, 1:1 + k] = cand[order]
+        elif w.select == "zipf":
+            # distinct blocks from [0, diag] (or all blocks), weight (b+1)^-s,
+            # sequential weighted sampling without replacement via exponential keys
+            ncand = nblk if allow_future else J + 1
+            wts = (np.arange(ncand, dtype=np.float64) + 1.0) ** (-w.zipf_s)
+            k = min(topk, ncand)
+            u = rng.random((rows, ncand))
+            keys = -np.log1p(-u) / wts
+            order = np.argsort(keys, axis=1, kind="stable")[:, :k]
+            sel = np.full((rows, topk), -1, dtype=np.int64)
+            sel[:, :k] = order
+        else:
+            raise ValueError(f"block selection {w.select!r}")
+        idx[t0:t1] = sel.reshape(t1 - t0, Hkv, topk).astype(np.int32)
+    if w.p_drop > 0:
+        drop = rng.random(idx.shape) < w.p_drop
+        idx[drop] = -1
+    return idx
+
+
+def _token_indices(rng, w: Workload, S: int) -> np.ndarray:
+    """[S, Hkv, topk] int32 distinct token indices in [0, t] (uniform), -1 padded."""
+    topk, Hkv = w.topk, w.Hkv
+    idx = np.full((S, Hkv, topk), -1, dtype=np.int32)
+    for t in range(S):
+        n = t + 1
+        for g in range(Hkv):
+            keys = rng.random(n)
+            if n <= topk:
+                sel = np.argsort(keys, kind="stable")
+            else:
+                sel = np.argpartition(keys, topk - 1)[:topk]
+            idx[t, g, :len(sel)] = sel
+    return idx
+
+
+def _cmp_indices(rng, w: Workload, S: int, any_pos: bool) -> np.ndarray:
+    """[S, Hkv, cmp_topk] distinct compressed-row indices, -1 padded.
+
+    By default each token draws from the compressed rows whose whole source
+    group lies at or before it ((c+1)*ratio - 1 <= t); ``any_pos`` draws from
+    every compressed row of the sequence instead (used by tests to exercise the
+    compressed causal mask).
+    """
+    r, k, Hkv = w.cmp_ratio, w.cmp_topk, w.Hkv
+    Tc = S // r
+    idx = np.full((S, Hkv, k), -1, dtype=np.int32)
+    for t in range(S):
+        n = Tc if any_pos else (t + 1) // r
+        if n == 0:
+            continue
+        for g in range(Hkv):
+            keys = rng.random(n)
+            if n <= k:
+                sel = np.argsort(keys, kind="stable")
+            else:
+                sel = np.argpartition(keys, k - 1)[:k]
+            idx[t, g, :len(sel)] = sel
+    return idx
+
+
+def make_inputs(w: Workload, *, allow_future: bool = False, cmp_any: bool = False,
+                ori_len_range: tuple | None = None) -> dict:
+    """Draw every input of workload ``w``.
+
+    Returns a dict of numpy arrays.  bf16 tensors are uint16 bit patterns with
+    shape [B, S, H, d] (BSND) or [T, H, d] (TND); index tensors are int32 with
+    shape [..., Hkv, slots]; topk lengths are int32 [..., Hkv].
+
+    Test-only knobs: ``allow_future`` lets block selections name blocks after
+    the diagonal (the causal mask must then hide them); ``cmp_any`` draws cmp
+    indices from all compressed rows; ``ori_len_range`` adds a per-row ori topk
+    length drawn uniformly from the inclusive range.
+    """
+    rng = np.random.Generator(np.random.PCG64(w.seed))
+    lens = w.seq_lengths
+    T = sum(lens)
+    lead = (w.B, w.S) if w.layout == "BSND" else (T,)
+    out: dict = {}
+
+    out["q"] = _normal_bf16(rng, lead + (w.Hq, w.d_qk))
+    if w.kv_shared:
+        out["kv"] = _normal_bf16(rng, lead + (w.Hkv, w.d_qk))
+    else:
+        out["k"] = _normal_bf16(rng, lead + (w.Hkv, w.d_qk))
+        out["v"] = _normal_bf16(rng, lead + (w.Hkv, w.d_v))
+    out["do"] = _normal_bf16(rng, lead + (w.Hq, w.d_v), mul=w.do_scale)
+    if w.sinks:
+        out["sinks"] = rng.standard_normal(w.Hq, dtype=np.float32)
+
+    starts = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+
+    if w.topk > 0:
+        parts = []
+        for b, L in enumerate(lens):
+            if w.mode == "block":
+                parts.append(_block_indices(rng, w, L, allow_future))
+            elif w.mode == "token":
+                parts.append(_token_indices(rng, w, L))
+            else:
+                raise ValueError(f"ori indices in mode {w.mode!r}")
+        idx = np.concatenate(parts, axis=0)
+        out["ori_idx"] = idx.reshape(lead + (w.Hkv, w.topk))
+
+    if w.cmp_topk > 0:
+        kvkey = "kv" if w.kv_shared else "k"
+        src = out[kvkey].reshape((T, w.Hkv, w.d_qk))
+        cmp_parts, cmp_lens = [], []
+        for b, L in enumerate(lens):
+            Tc = L // w.cmp_ratio
+            seg = f32_from_bf16_bits(src[starts[b]:starts[b] + Tc * w.cmp_ratio]).astype(np.float64)
+            pooled = seg.reshape(Tc, w.cmp_ratio, w.Hkv, w.d_qk).mean(axis=1)
+            cmp_parts.append(bf16_bits_from_f32(pooled.astype(np.float32)))
+            cmp_lens.append(Tc)
+        out["cmp_kv"] = np.concatenate(cmp_parts, axis=0)
+        out["cu_seqlens_cmp"] = np.concatenate([[0], np.cumsum(cmp_lens)]).astype(np.int32)
+        out["cmp_residual"] = np.array([L % w.cmp_ratio for L in lens], dtype=np.int32)
+        cidx = np.concatenate([_cmp_indices(rng, w, L, cmp_any) for L in lens], axis=0)
+        out["cmp_idx"] = cidx.reshape(lead + (w.Hkv, w.cmp_topk))
+
+    if ori_len_range is not None and w.topk > 0:
+        lo, hi = ori_len_range
+        out["ori_topk_len"] = rng.integers(lo, hi + 1, size=lead + (w.Hkv,)).astype(np.int32)
+
+    if w.cmp_topk > 0:
+        lo, hi = w.cmp_len_range
+        raw = rng.integers(lo, hi + 1, size=(T, w.Hkv))
+        cap = np.empty((T, w.Hkv), dtype=np.int64)
+        for b, L in enumerate(lens):
+            t = np.arange(L)
+            n = (np.full(L, L // w.cmp_ratio) if cmp_any else (t + 1) // w.cmp_ratio)
+            cap[starts[b]:starts[b] + L] = n[:, None]
+        out["cmp_topk_len"] = np.minimum(raw, cap).astype(np.int32).reshape(lead + (w.Hkv,))
+
+    if w.layout == "TND":
+        out["cu_seqlens_q"] = starts.astype(np.int32)
+        out["cu_seqlens_kv"] = starts.astype(np.int32)
+    return out

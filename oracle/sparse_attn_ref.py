@@ -1,0 +1,397 @@
+"""Float64 CPU oracle for top-k index-selected sparse attention: forward and backward.
+
+TEST INFRASTRUCTURE ONLY.  The parity tests, the smoke check and the CPU-baseline
+leg of the benchmark may import this module; the CUDA product path never does,
+and this module imports nothing from it.
+
+What it computes is the plain definition, one query token at a time, in float64
+(NumPy matmul as the only library step):
+
+* Selection.  aclnnSparseFlashAttentionGrad, "Formula": selectedKey/selectedValue
+  = Gather(key/value, topkIndices[i]) for 0 <= i < selectBlockCount, each index
+  naming a block of contiguous rows.  SparseFlashMlaGrad, "Computation formula",
+  Stage 1: cmp_ratio = 1 (SWA) selects the original KV, cmp_ratio = 4 (SCFA)
+  concatenates the original KV with Gather(cmpKv, topkIndices[i]); the
+  "Parameter Description" table adds oriSparseIndices (token rows of the
+  original KV), oriTopkLength / cmpTopkLength (usable slots per query row),
+  oriMaskMode / cmpMaskMode and oriWinLeft / oriWinRight.
+* Forward.  aclnnNsaSelectedAttentionInfer, "Formula":
+  Softmax(query . key_topk^T / sqrt(d)) . value_topk, with the scale attribute
+  (scaleValue) in place of 1/sqrt(d), an optional per-head sink logit in the
+  softmax denominator, and lse = log of that denominator (natural log).
+* Backward.  SparseFlashMlaGrad, "Computation formula", Stages 2-3, and
+  aclnnSparseFlashAttentionGrad, "Formula", Phases 1-3:
+      P  = SimpleSoftmax(Mask(Q selKv^T scale), lse) = exp(S - lse)
+      dP = dO V^T
+      dS = P o (dP - rowsum(dO o O))          (o = elementwise product)
+      dQ = dS K scale,  dK = dS^T Q scale,  dV = P^T dO  (dKV = dK + dV if K = V)
+      dSinks = sum over rows of -P_sink * sum_j P_j dP_j,  P_sink = exp(sink - lse)
+
+Readings taken where the pages are silent or garbled (each is listed with its
+reason in the design notes of this repository):
+  - the "@" inside the dS formula of aclnnSparseFlashAttentionGrad is the
+    elementwise product (SparseFlashMlaGrad prints "x");
+  - block x covers rows [x*bs, (x+1)*bs) of the same sequence, rows past the
+    sequence end are dropped;
+  - an index < 0, or a slot at or past the row's topk length, selects nothing;
+  - causal masks align the last query with the last key (bottom-right); the
+    band mask keeps rows in [t - winLeft, t + winRight]; a compressed row c is
+    visible when its last source token, (c + 1) * cmp_ratio - 1, is <= t;
+  - duplicates in a row's index list are gathered with multiplicity;
+  - a row with no visible key and no sink has lse = +inf and O = 0, and gives
+    zero gradients;
+  - with K = V, V is the first d_v columns of the shared KV row;
+  - TND indices are positions local to their own sequence, like BSND.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "widen_bf16",
+    "round_to_bf16_bits",
+    "Problem",
+    "visible_rows",
+    "unit_forward",
+    "unit_backward",
+    "forward",
+    "backward",
+    "unit_flops",
+]
+
+
+# ----------------------------------------------------------------------------
+# bfloat16 <-> float64 (the oracle's own conversions)
+# ----------------------------------------------------------------------------
+
+def widen_bf16(u16: np.ndarray) -> np.ndarray:
+    """bfloat16 bit patterns -> float64, exactly (a bf16 is the top half of a binary32)."""
+    u = np.asarray(u16, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return u.view(np.float32).astype(np.float64)
+
+
+def round_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float64 -> bfloat16 bit patterns, round to nearest, ties to even, in one step.
+
+    A bfloat16 keeps 8 significant bits, so for |x| in [2^(e-1), 2^e) its spacing
+    is 2^(e-8) (never below 2^-133, the subnormal spacing).  Dividing by that
+    power of two is exact, np.rint rounds half to even, and the result is exactly
+    representable in binary32, whose top 16 bits are the bfloat16.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)
+    spacing = np.ldexp(1.0, np.maximum(e - 8, -133))
+    q = np.rint(x / spacing) * spacing
+    q = np.where(np.isfinite(x), q, x)
+    bits = q.astype(np.float32).view(np.uint32) >> np.uint32(16)
+    return bits.astype(np.uint16)
+
+
+# ----------------------------------------------------------------------------
+# Problem description
+# ----------------------------------------------------------------------------
+
+class Problem:
+    """All inputs of one sparse-attention call, token-major, in float64.
+
+    Arrays (T = total query tokens, Tk = total original KV rows, Tc = total
+    compressed KV rows):
+      q      [T, Hq, d_qk]
+      k_ori  [Tk, Hkv, d_qk],  v_ori [Tk, Hkv, d_v]   (K = V: v_ori is k_ori[..., :d_v])
+      k_cmp  [Tc, Hkv, d_qk],  v_cmp [Tc, Hkv, d_v]   (compressed KV, always K = V)
+      ori_idx [T, Hkv, topk] int, cmp_idx [T, Hkv, cmp_topk] int (or None)
+      ori_topk_len / cmp_topk_len [T, Hkv] int (or None)
+      sinks [Hq] (or None)
+    Sequences: q_start/q_len, kv_start/kv_len, cmp_start/cmp_len per batch.
+    """
+
+    def __init__(self, *, q, k_ori, v_ori, kv_shared, q_lens, kv_lens, Hq, Hkv,
+                 d_qk, d_v, scale, block_size=1, ori_idx=None, ori_topk_len=None,
+                 k_cmp=None, v_cmp=None, cmp_lens=None, cmp_idx=None,
+                 cmp_topk_len=None, cmp_ratio=1, ori_mask="causal",
+                 cmp_mask="causal", win_left=0, win_right=0, sinks=None):
+        self.q = np.asarray(q, dtype=np.float64)
+        self.k_ori = np.asarray(k_ori, dtype=np.float64)
+        self.v_ori = np.asarray(v_ori, dtype=np.float64)
+        self.kv_shared = bool(kv_shared)
+        self.Hq, self.Hkv, self.d_qk, self.d_v = Hq, Hkv, d_qk, d_v
+        assert Hq % Hkv == 0
+        self.G = Hq // Hkv
+        self.scale = float(scale)
+        self.block_size = int(block_size)
+        self.ori_idx = None if ori_idx is None else np.asarray(ori_idx, dtype=np.int64)
+        self.ori_topk_len = None if ori_topk_len is None else np.asarray(ori_topk_len, dtype=np.int64)
+        self.k_cmp = None if k_cmp is None else np.asarray(k_cmp, dtype=np.float64)
+        self.v_cmp = None if v_cmp is None else np.asarray(v_cmp, dtype=np.float64)
+        self.cmp_idx = None if cmp_idx is None else np.asarray(cmp_idx, dtype=np.int64)
+        self.cmp_topk_len = None if cmp_topk_len is None else np.asarray(cmp_topk_len, dtype=np.int64)
+        self.cmp_ratio = int(cmp_ratio)
+        self.ori_mask, self.cmp_mask = ori_mask, cmp_mask
+        self.win_left, self.win_right = int(win_left), int(win_right)
+        self.sinks = None if sinks is None else np.asarray(sinks, dtype=np.float64)
+        self.q_len = np.asarray(q_lens, dtype=np.int64)
+        self.kv_len = np.asarray(kv_lens, dtype=np.int64)
+        self.q_start = np.concatenate([[0], np.cumsum(self.q_len)])[:-1]
+        self.kv_start = np.concatenate([[0], np.cumsum(self.kv_len)])[:-1]
+        if cmp_lens is None:
+            cmp_lens = np.zeros_like(self.q_len)
+        self.cmp_len = np.asarray(cmp_lens, dtype=np.int64)
+        self.cmp_start = np.concatenate([[0], np.cumsum(self.cmp_len)])[:-1]
+        self.T = int(self.q_len.sum())
+        self._batch_of = np.repeat(np.arange(len(self.q_len)), self.q_len)
+        assert self.q.shape == (self.T, Hq, d_qk)
+
+    @property
+    def has_cmp(self) -> bool:
+        return self.k_cmp is not None
+
+    def batch_of(self, tq: int) -> int:
+        return int(self._batch_of[tq])
+
+    @classmethod
+    def from_inputs(cls, w, inp: dict) -> "Problem":
+        """Build from a workload description and the generator's arrays (bf16 as uint16)."""
+        T = w.T
+        q = widen_bf16(inp["q"]).reshape(T, w.Hq, w.d_qk)
+        if w.kv_shared:
+            kv = widen_bf16(inp["kv"]).reshape(T, w.Hkv, w.d_qk)
+            k_ori, v_ori = kv, kv[..., :w.d_v]
+        else:
+            k_ori = widen_bf16(inp["k"]).reshape(T, w.Hkv, w.d_qk)
+            v_ori = widen_bf16(inp["v"]).reshape(T, w.Hkv, w.d_v)
+        lens = list(w.seq_lengths)
+        kw = {}
+        if "ori_idx" in inp:
+            kw["ori_idx"] = inp["ori_idx"].reshape(T, w.Hkv, -1)
+        if "ori_topk_len" in inp:
+            kw["ori_topk_len"] = inp["ori_topk_len"].reshape(T, w.Hkv)
+        if "cmp_kv" in inp:
+            ck = widen_bf16(inp["cmp_kv"]).reshape(-1, w.Hkv, w.d_qk)
+            kw.update(k_cmp=ck, v_cmp=ck[..., :w.d_v],
+                      cmp_lens=np.diff(inp["cu_seqlens_cmp"]),
+                      cmp_idx=inp["cmp_idx"].reshape(T, w.Hkv, -1))
+            if "cmp_topk_len" in inp:
+                kw["cmp_topk_len"] = inp["cmp_topk_len"].reshape(T, w.Hkv)
+        if "sinks" in inp:
+            kw["sinks"] = inp["sinks"].astype(np.float64)
+        return cls(q=q, k_ori=k_ori, v_ori=v_ori, kv_shared=w.kv_shared, q_lens=lens,
+                   kv_lens=lens, Hq=w.Hq, Hkv=w.Hkv, d_qk=w.d_qk, d_v=w.d_v,
+                   scale=w.scale, block_size=w.block_size, cmp_ratio=w.cmp_ratio,
+                   ori_mask=w.ori_mask, cmp_mask=w.cmp_mask, win_left=w.win_left,
+                   win_right=w.win_right, **kw)
+
+
+# ----------------------------------------------------------------------------
+# Selection (Stage 1 / the Gather formula) and masks
+# ----------------------------------------------------------------------------
+
+def visible_rows(p: Problem, tq: int, g: int):
+    """Visible KV rows of query token ``tq`` (global) under kv-head ``g``.
+
+    Returns (ori_rows, cmp_rows): int64 arrays of row numbers local to the
+    token's sequence, in slot order (duplicates kept).
+    """
+    b = p.batch_of(tq)
+    t = tq - int(p.q_start[b])
+    Lk = int(p.kv_len[b])
+    ta = t + (Lk - int(p.q_len[b]))           # query position on the key axis
+
+    # original KV: gathered through the ori indices, else all of it (SWA / SCFA / CFA)
+    if p.ori_idx is not None:
+        n = p.ori_idx.shape[2]
+        if p.ori_topk_len is not None:
+            n = max(0, min(n, int(p.ori_topk_len[tq, g])))
+        idx = p.ori_idx[tq, g, :n]
+        idx = idx[idx >= 0]
+        bs = p.block_size
+        if np.any(idx * bs >= Lk):
+            raise IndexError(f"ori index out of range at token {tq}, kv-head {g}")
+        ori = (idx[:, None] * bs + np.arange(bs)[None, :]).reshape(-1)
+        ori = ori[ori < Lk]
+    else:
+        ori = np.arange(Lk, dtype=np.int64)
+    if p.ori_mask == "causal":
+        ori = ori[ori <= ta]
+    elif p.ori_mask == "band":
+        ori = ori[(ori >= ta - p.win_left) & (ori <= ta + p.win_right)]
+    elif p.ori_mask != "none":
+        raise ValueError(p.ori_mask)
+
+    # compressed KV: gathered through the cmp indices (SCFA)
+    cmp = np.zeros(0, dtype=np.int64)
+    if p.has_cmp and p.cmp_idx is not None:
+        n = p.cmp_idx.shape[2]
+        if p.cmp_topk_len is not None:
+            n = max(0, min(n, int(p.cmp_topk_len[tq, g])))
+        c = p.cmp_idx[tq, g, :n]
+        c = c[c >= 0]
+        if np.any(c >= int(p.cmp_len[b])):
+            raise IndexError(f"cmp index out of range at token {tq}, kv-head {g}")
+        if p.cmp_mask == "causal":
+            c = c[(c + 1) * p.cmp_ratio - 1 <= ta]
+        elif p.cmp_mask != "none":
+            raise ValueError(p.cmp_mask)
+        cmp = c
+    elif p.has_cmp:
+        raise NotImplementedError("compressed KV without cmp indices (CFA)")
+    return ori, cmp
+
+
+def _gather(p: Problem, tq: int, g: int):
+    b = p.batch_of(tq)
+    ori, cmp = visible_rows(p, tq, g)
+    K = p.k_ori[p.kv_start[b] + ori, g]
+    V = p.v_ori[p.kv_start[b] + ori, g]
+    if len(cmp):
+        K = np.concatenate([K, p.k_cmp[p.cmp_start[b] + cmp, g]])
+        V = np.concatenate([V, p.v_cmp[p.cmp_start[b] + cmp, g]])
+    return ori, cmp, K, V
+
+
+# ----------------------------------------------------------------------------
+# Forward (selected attention with optional sinks)
+# ----------------------------------------------------------------------------
+
+def unit_forward(p: Problem, tq: int, g: int):
+    """O [G, d_v] and lse [G] (float64) for the G query heads of kv-head g at token tq."""
+    hs = slice(g * p.G, (g + 1) * p.G)
+    Q = p.q[tq, hs]
+    _, _, K, V = _gather(p, tq, g)
+    S = p.scale * (Q @ K.T)                               # [G, n] scaled scores
+    sink = None if p.sinks is None else p.sinks[hs]
+    if K.shape[0] == 0 and sink is None:
+        return np.zeros((p.G, p.d_v)), np.full(p.G, np.inf)
+    m = np.full(p.G, -np.inf)
+    if K.shape[0]:
+        m = S.max(axis=1)
+    if sink is not None:
+        m = np.maximum(m, sink)
+    Z = np.exp(S - m[:, None]).sum(axis=1)
+    if sink is not None:
+        Z = Z + np.exp(sink - m)
+    lse = m + np.log(Z)
+    P = np.exp(S - lse[:, None])
+    return P @ V, lse
+
+
+def forward(p: Problem, units=None, rounded: bool = True):
+    """Forward over all units (token, kv-head), or only over ``units``.
+
+    Returns (O, lse): O [T, Hq, d_v], lse [T, Hq].  Rounded: O as bf16 bits and
+    lse as float32; otherwise float64.  Units not computed hold zeros.
+    """
+    O = np.zeros((p.T, p.Hq, p.d_v))
+    lse = np.zeros((p.T, p.Hq))
+    if units is None:
+        units = [(tq, g) for tq in range(p.T) for g in range(p.Hkv)]
+    for tq, g in units:
+        o, l = unit_forward(p, tq, g)
+        O[tq, g * p.G:(g + 1) * p.G] = o
+        lse[tq, g * p.G:(g + 1) * p.G] = l
+    if rounded:
+        return round_to_bf16_bits(O), lse.astype(np.float32)
+    return O, lse
+
+
+# ----------------------------------------------------------------------------
+# Backward (Stages 2-3 / Phases 1-3)
+# ----------------------------------------------------------------------------
+
+def unit_backward(p: Problem, tq: int, g: int, O, lse, dO):
+    """Everything the backward derives for one unit.
+
+    ``O`` [G, d_v], ``lse`` [G], ``dO`` [G, d_v] are the float64 inputs of this
+    unit.  Returns a dict with ori/cmp rows, S, P, dP, Delta, dS, dQ [G, d_qk],
+    dK_rows [n, d_qk], dV_rows [n, d_v], P_sink [G] and dSinks [G].
+    """
+    hs = slice(g * p.G, (g + 1) * p.G)
+    Q = p.q[tq, hs]
+    ori, cmp, K, V = _gather(p, tq, g)
+    S = p.scale * (Q @ K.T)
+    P = np.exp(S - lse[:, None])                          # SimpleSoftmax(S, lse)
+    dP = dO @ V.T
+    Delta = (dO * O).sum(axis=1)                          # rowsum(dO o O)
+    dS = P * (dP - Delta[:, None])
+    out = dict(ori=ori, cmp=cmp, S=S, P=P, dP=dP, Delta=Delta, dS=dS,
+               dQ=p.scale * (dS @ K),
+               dK_rows=p.scale * (dS.T @ Q),
+               dV_rows=P.T @ dO)
+    if p.sinks is not None:
+        psink = np.exp(p.sinks[hs] - lse)
+        out["P_sink"] = psink
+        out["dSinks"] = -psink * (P * dP).sum(axis=1)
+    return out
+
+
+def _scatter_add(dst, rows, vals):
+    """dst[rows] += vals, adding repeated rows once per occurrence."""
+    if len(np.unique(rows)) == len(rows):
+        dst[rows] += vals
+    else:
+        np.add.at(dst, rows, vals)
+
+
+def backward(p: Problem, O, lse, dO, units=None, rounded: bool = True):
+    """Backward over all units, or over ``units`` only (partial sums for dK/dV).
+
+    ``O``, ``dO`` [T, Hq, d_v] and ``lse`` [T, Hq] as float64 (widen bf16 / fp32
+    first).  Returns a dict: dq [T, Hq, d_qk]; dk [Tk, Hkv, d_qk] and dv
+    [Tk, Hkv, d_v], or dkv [Tk, Hkv, d_qk] when K = V; dcmp [Tc, Hkv, d_qk] when
+    there is a compressed KV; dsinks [Hq] when there are sinks.  Rounded: bf16
+    bits for every tensor but dsinks (float32); otherwise float64.
+    """
+    O = np.asarray(O, dtype=np.float64)
+    dO = np.asarray(dO, dtype=np.float64)
+    lse = np.asarray(lse, dtype=np.float64)
+    Tk = p.k_ori.shape[0]
+    dq = np.zeros_like(p.q)
+    dk = np.zeros((Tk, p.Hkv, p.d_qk))
+    dv = np.zeros((Tk, p.Hkv, p.d_v))
+    Tc = 0 if p.k_cmp is None else p.k_cmp.shape[0]
+    dkc = np.zeros((Tc, p.Hkv, p.d_qk))
+    dvc = np.zeros((Tc, p.Hkv, p.d_v))
+    dsinks = np.zeros(p.Hq)
+    if units is None:
+        units = [(tq, g) for tq in range(p.T) for g in range(p.Hkv)]
+    for tq, g in units:
+        hs = slice(g * p.G, (g + 1) * p.G)
+        r = unit_backward(p, tq, g, O[tq, hs], lse[tq, hs], dO[tq, hs])
+        dq[tq, hs] = r["dQ"]
+        b = p.batch_of(tq)
+        no = len(r["ori"])
+        _scatter_add(dk[:, g], p.kv_start[b] + r["ori"], r["dK_rows"][:no])
+        _scatter_add(dv[:, g], p.kv_start[b] + r["ori"], r["dV_rows"][:no])
+        if len(r["cmp"]):
+            _scatter_add(dkc[:, g], p.cmp_start[b] + r["cmp"], r["dK_rows"][no:])
+            _scatter_add(dvc[:, g], p.cmp_start[b] + r["cmp"], r["dV_rows"][no:])
+        if p.sinks is not None:
+            dsinks[hs] += r["dSinks"]
+    res = {"dq": dq}
+    if p.kv_shared:
+        dkv = dk.copy()
+        dkv[..., :p.d_v] += dv
+        res["dkv"] = dkv
+    else:
+        res["dk"], res["dv"] = dk, dv
+    if p.k_cmp is not None:
+        dc = dkc.copy()
+        dc[..., :p.d_v] += dvc
+        res["dcmp"] = dc
+    if p.sinks is not None:
+        res["dsinks"] = dsinks
+    if rounded:
+        for key in list(res):
+            if key == "dsinks":
+                res[key] = res[key].astype(np.float32)
+            else:
+                res[key] = round_to_bf16_bits(res[key])
+    return res
+
+
+def unit_flops(p: Problem, tq: int, g: int) -> tuple:
+    """(forward, backward) FLOPs of one unit counted over visible (row, head, key) triples."""
+    ori, cmp = visible_rows(p, tq, g)
+    n = (len(ori) + len(cmp)) * p.G
+    return 2 * (p.d_qk + p.d_v) * n, 2 * (3 * p.d_qk + 2 * p.d_v) * n
+
