@@ -1,0 +1,477 @@
+#!/usr/bin/env python
+"""Benchmark of top-k index-selected sparse attention on B200.
+
+One step = the whole hot path on one batch: forward (O, lse) then backward
+(rowsum(dO o O), the fused backward, finalize) through the C ABI.  Prints ONE
+JSON line (rank 0): the backward TFLOP/s counted over selected, visible
+(row, head, key) triples, the roofline fraction of the dominant kernel, the
+forward TFLOP/s, an end-to-end figure with host buffers, and the float64
+oracle timed on the host cores as a CPU baseline.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+       [--workload cfg2] [--no-cpu-baseline] [--no-e2e]
+For N > 1 launch under torchrun; every rank runs an independent replica of the
+workload (the path has no exchange step), timing is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gen import get_workload, make_inputs  # noqa: E402
+
+METRIC = "sparse-attn bwd TFLOP/s (selected-KV FLOPs) and % of roofline; fwd TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------
+# workload accounting (host side, from the index tensors)
+# ----------------------------------------------------------------------------
+
+def count_work(w, inputs) -> dict:
+    """Visible (row, key) pairs per unit and the bytes the selection names.
+
+    visible  -- keys that survive selection, topk lengths and masks (FLOP count)
+    gathered -- rows the selection names before masking (block rows clipped to
+                the sequence, one row per token / compressed index, the window)
+    """
+    lens = list(w.seq_lengths)
+    T = w.T
+    vis = np.zeros((T, w.Hkv), dtype=np.int64)
+    gat = np.zeros((T, w.Hkv), dtype=np.int64)
+    start = 0
+    for L in lens:
+        t = np.arange(L)[:, None, None]
+        ta = t  # equal query / key lengths
+        if w.topk:
+            idx = inputs["ori_idx"].reshape(T, w.Hkv, -1)[start:start + L].astype(np.int64)
+            slot = np.arange(idx.shape[2])[None, None, :]
+            ok = idx >= 0
+            if "ori_topk_len" in inputs:
+                ok &= slot < inputs["ori_topk_len"].reshape(T, w.Hkv)[start:start + L, :, None]
+            if w.block_size > 1:
+                first = idx * w.block_size
+                ok &= first < L
+                last = np.minimum(first + w.block_size, L) - 1
+                lo, hi = first, last
+                if w.ori_mask == "causal":
+                    hi = np.minimum(hi, ta)
+                elif w.ori_mask == "band":
+                    lo = np.maximum(lo, ta - w.win_left)
+                    hi = np.minimum(hi, ta + w.win_right)
+                v = np.where(ok, np.maximum(hi - lo + 1, 0), 0)
+                g = np.where(ok, last - first + 1, 0)
+            else:
+                ok &= idx < L
+                m = ok.copy()
+                if w.ori_mask == "causal":
+                    m &= idx <= ta
+                elif w.ori_mask == "band":
+                    m &= (idx >= ta - w.win_left) & (idx <= ta + w.win_right)
+                v, g = m, ok
+            vis[start:start + L] += v.sum(-1)
+            gat[start:start + L] += g.sum(-1)
+        else:
+            tt = np.arange(L)
+            lo, hi = np.zeros(L, dtype=np.int64), np.full(L, L - 1)
+            if w.ori_mask == "causal":
+                hi = np.minimum(hi, tt)
+            elif w.ori_mask == "band":
+                lo = np.maximum(lo, tt - w.win_left)
+                hi = np.minimum(hi, tt + w.win_right)
+            n = np.maximum(hi - lo + 1, 0)[:, None]
+            vis[start:start + L] += n
+            gat[start:start + L] += n
+        if w.cmp_topk:
+            cidx = inputs["cmp_idx"].reshape(T, w.Hkv, -1)[start:start + L].astype(np.int64)
+            slot = np.arange(cidx.shape[2])[None, None, :]
+            ok = (cidx >= 0) & (cidx < L // w.cmp_ratio)
+            if "cmp_topk_len" in inputs:
+                ok &= slot < inputs["cmp_topk_len"].reshape(T, w.Hkv)[start:start + L, :, None]
+            m = ok & ((cidx + 1) * w.cmp_ratio - 1 <= ta)
+            vis[start:start + L] += m.sum(-1)
+            gat[start:start + L] += ok.sum(-1)
+        start += L
+    G = w.G
+    triples = int(vis.sum()) * G
+    row_bytes = (w.d_qk + (0 if w.kv_shared else w.d_v)) * 2
+    gathered = int(gat.sum()) * row_bytes
+    Tk = T
+    n_q, n_v = T * w.Hq * w.d_qk * 2, T * w.Hq * w.d_v * 2
+    lse_b = T * w.Hq * 4
+    kv_out = Tk * w.Hkv * (w.d_qk + (0 if w.kv_shared else w.d_v)) * 2
+    if w.cmp_topk:
+        kv_out += sum(L // w.cmp_ratio for L in lens) * w.Hkv * w.d_qk * 2
+    return {
+        "triples": triples,
+        "fwd_flops": 2 * (w.d_qk + w.d_v) * triples,
+        "bwd_flops": 2 * (3 * w.d_qk + 2 * w.d_v) * triples,
+        "gathered_bytes": gathered,
+        # forward kernel: gathered rows + read Q + write O, lse
+        "fwd_bytes": gathered + n_q + n_v + lse_b,
+        # fused backward kernel: gathered rows + read Q, dO, lse, Delta + write dQ + dK/dV once
+        "bwd_main_bytes": gathered + n_q + n_v + 2 * lse_b + n_q + kv_out,
+        "units": T * w.Hkv,
+    }
+
+
+def load_peaks() -> tuple:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches this build."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        data = json.load(f)
+    ent = data.get(f"{kernel}@{workload}")
+    if not ent:
+        return None
+    if ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "top_sparse_attention_attn_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# the CPU baseline: the float64 oracle on a bounded sample of units
+# ----------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_baseline(w, inputs, budget_s: float = 12.0, seed: int = 0) -> dict:
+    """Time the oracle's backward on random units of the workload (forward for the
+    same units computed first, untimed)."""
+    import oracle  # the CPU baseline leg is the one place the benchmark runs the oracle
+    p = oracle.Problem.from_inputs(w, inputs)
+    rng = np.random.default_rng(seed)
+    do = inputs["do"].reshape(w.T, w.Hq, w.d_v)
+    flops = 0
+    elapsed = 0.0
+    n_units = 0
+    G = w.G
+    while elapsed < budget_s:
+        batch = [(int(rng.integers(w.T)), int(rng.integers(w.Hkv))) for _ in range(32)]
+        fw = oracle.forward(p, units=batch)
+
+        class Rows:
+            def __init__(self, k):
+                self.k = k
+
+            def __getitem__(self, key):
+                tq, hs = key
+                g = hs.start // G
+                return fw[(tq, g)][self.k]
+
+        t0 = time.perf_counter()
+        oracle.backward(p, Rows(0), Rows(1), do, units=batch)
+        elapsed += time.perf_counter() - t0
+        for tq, g in batch:
+            flops += oracle.unit_flops(p, tq, g)[1]
+        n_units += len(batch)
+    return {"value": flops / elapsed / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{n_units} random (token, kv-head) units of {w.name}, float64 NumPy backward "
+                      f"({elapsed:.1f} s of CPU time)"}
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+def workload_of(args):
+    """The named workload, optionally with overrides ("S=2048,B=1") for profiling runs."""
+    w = get_workload(args.workload)
+    ov = getattr(args, "override", None)
+    if ov:
+        from gen import scaled
+        kw = {}
+        for item in ov.split(","):
+            k, v = item.split("=")
+            kw[k.strip()] = type(getattr(w, k.strip()))(v)
+        w = scaled(w, "override", **kw)
+    return w
+
+
+def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
+    import torch
+    from gen.torch_io import to_torch
+    from top_sparse_attention_attn_b200 import SparseAttention
+    from top_sparse_attention_attn_b200 import _lib as L
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workload_of(args)
+    inputs = make_inputs(w)
+    work = count_work(w, inputs)
+    t = to_torch(inputs, dev)
+    sa = SparseAttention.from_workload(w, t)
+    stream = torch.cuda.current_stream(dev)
+    o, lse = sa.alloc_fwd()
+    grads = sa.alloc_bwd()
+    ws_f = sa.fwd_workspace()
+    ws_b = sa.bwd_workspace()
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        sa.forward(o, lse, ws_f)
+        sa.backward(o, lse, t["do"], grads, ws_b)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for e in ev:  # materialise the raw cudaEvent_t handles
+        for x in e:
+            x.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    launches0 = L.sa_kernel_launch_count()
+    with ClockSampler(local_rank) as clk:
+        for k in range(K):
+            flush.zero_()                          # L2 flushed between timed steps
+            e0, e1, e2, mb, me = ev[k]
+            e0.record(stream)
+            sa.forward(o, lse, ws_f)
+            e1.record(stream)
+            L.sa_set_timing_events(mb.cuda_event, me.cuda_event)
+            sa.backward(o, lse, t["do"], grads, ws_b)
+            L.sa_set_timing_events(None, None)
+            e2.record(stream)
+        torch.cuda.synchronize()
+    launches = L.sa_kernel_launch_count() - launches0
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    main_ms = sum(e[3].elapsed_time(e[4]) for e in ev) / K
+    step_ms = fwd_ms + bwd_ms
+    times = torch.tensor([fwd_ms, bwd_ms, main_ms, step_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    fwd_ms, bwd_ms, main_ms, step_ms = times.tolist()
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host_in = {k: v.cpu().pin_memory() for k, v in t.items()}
+        host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in grads.items()}
+        h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+        d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+
+        def e2e_step():
+            for k_, v in host_in.items():
+                t[k_].copy_(v, non_blocking=True)
+            sa.forward(o, lse, ws_f)
+            sa.backward(o, lse, t["do"], grads, ws_b)
+            for k_, v in host_out.items():
+                v.copy_(grads[k_], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for k in range(K):
+            flush.zero_()
+            es[k][0].record(stream)
+            e2e_step()
+            es[k][1].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in es) / K], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
+        e2e = {"value": world * work["bwd_flops"] / (e2e_ms.item() * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms.item(),
+               "note": "bwd FLOPs over the whole step: H2D of inputs, forward, backward, D2H of gradients"}
+
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    bwd_tflops = world * work["bwd_flops"] / (bwd_ms * 1e-3) / 1e12
+    fwd_tflops = world * work["fwd_flops"] / (fwd_ms * 1e-3) / 1e12
+    # roofline of the dominant kernel (fused backward)
+    t_bytes = work["bwd_main_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_flops = work["bwd_flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
+    bound = "hbm" if t_bytes >= t_flops else "tensor"
+    if bound == "hbm":
+        achieved = work["bwd_main_bytes"] / (main_ms * 1e-3) / 1e9
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved = work["bwd_flops"] / (main_ms * 1e-3) / 1e12
+        peak, unit = peaks["bf16_tflops_sustained"], "TFLOP/s"
+    roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": load_traffic("bwd_kernel", w.name),
+            "kernel": "bwd_kernel (fused backward)", "kernel_ms": main_ms,
+            "algorithmic_bytes": work["bwd_main_bytes"], "algorithmic_flops": work["bwd_flops"],
+            "peak_source": f"{peak_src} MEASURED_PEAKS.json" if peak_src == "measured" else "fallback",
+            "t_roof_ms": max(t_bytes, t_flops) * 1e3}
+    line = {
+        "metric": METRIC, "value": bwd_tflops, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv,
+                   "d_qk": w.d_qk, "d_v": w.d_v, "block_size": w.block_size, "topk": w.topk,
+                   "parallelism": f"replicas{world}", "l2": "flushed between timed steps",
+                   "visible_triples": work["triples"], "gathered_bytes": work["gathered_bytes"]},
+        "fwd_tflops": fwd_tflops, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+        "bwd_roofline_frac": max(t_bytes, t_flops) * 1e3 / bwd_ms,
+        "roofline": roof, "clocks": clk.summary(), "gpu_launches": launches,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_baseline(w, inputs)
+    return line
+
+
+# ----------------------------------------------------------------------------
+# reference arm: the oracle on the host cores
+# ----------------------------------------------------------------------------
+
+def run_reference(args, rank: int) -> dict | None:
+    if rank != 0:
+        return None
+    w = workload_of(args)
+    inputs = make_inputs(w)
+    per_step = getattr(args, "step_budget", None) or max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_baseline(w, inputs, budget_s=1.0, seed=1)
+    vals = [oracle_baseline(w, inputs, budget_s=per_step, seed=100 + k) for k in range(args.steps)]
+    v = statistics.mean(x["value"] for x in vals)
+    return {"metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "impl": "reference",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": vals[0]["cores"],
+                             "kind": "oracle", "sample": vals[0]["sample"]},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="cfg2")
+    ap.add_argument("--override", default=None, help="workload overrides for profiling, e.g. S=2048")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        line = run_reference(args, rank)
+    else:
+        if world > 1:
+            import datetime
+            import torch
+            torch.cuda.set_device(local_rank)
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        line = run_ours(args, rank, world, local_rank)
+        if world > 1:
+            import torch
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

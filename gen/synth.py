@@ -43,6 +43,14 @@ def _normal_bf16(rng: np.random.Generator, shape, mul: float = 1.0) -> np.ndarra
     return out.reshape(shape)
 
 
+def _smallest_k(keys: np.ndarray, k: int) -> np.ndarray:
+    """Column positions of the k smallest keys of each row, in increasing key order."""
+    n = keys.shape[1]
+    part = np.argpartition(keys, k - 1, axis=1)[:, :k] if k < n else np.tile(np.arange(n), (keys.shape[0], 1))
+    order = np.argsort(np.take_along_axis(keys, part, axis=1), axis=1, kind="stable")
+    return np.take_along_axis(part, order, axis=1)
+
+
 def _block_indices(rng, w: Workload, S: int, allow_future: bool) -> np.ndarray:
     """[S, Hkv, topk] int32 block indices for one sequence."""
     bs, topk, Hkv = w.block_size, w.topk, w.Hkv
@@ -60,8 +68,7 @@ def _block_indices(rng, w: Workload, S: int, allow_future: bool) -> np.ndarray:
             sel[:, 0] = J
             if k > 0:
                 keys = rng.random((rows, len(cand)))
-                order = np.argsort(keys, axis=1, kind="stable")[:, :k]
-                sel[:, 1:1 + k] = cand[order]
+                sel[:, 1:1 + k] = cand[_smallest_k(keys, k)]
         elif w.select == "zipf":
             # distinct blocks from [0, diag] (or all blocks), weight (b+1)^-s,
             # sequential weighted sampling without replacement via exponential keys
@@ -70,9 +77,8 @@ def _block_indices(rng, w: Workload, S: int, allow_future: bool) -> np.ndarray:
             k = min(topk, ncand)
             u = rng.random((rows, ncand))
             keys = -np.log1p(-u) / wts
-            order = np.argsort(keys, axis=1, kind="stable")[:, :k]
             sel = np.full((rows, topk), -1, dtype=np.int64)
-            sel[:, :k] = order
+            sel[:, :k] = _smallest_k(keys, k)
         else:
             raise ValueError(f"block selection {w.select!r}")
         idx[t0:t1] = sel.reshape(t1 - t0, Hkv, topk).astype(np.int32)

@@ -1,0 +1,222 @@
+/*
+ * sparse_attn.h -- C ABI of libsparse_attn.so: top-k index-selected sparse
+ * attention (forward and backward) on one NVIDIA B200 (sm_100a).
+ *
+ * The operation.  For every query token t and kv-head g, a set of KV rows is
+ * selected and attended to by the G = Hq / Hkv query heads that share g:
+ *
+ *   - block-level selection: aclnnSparseFlashAttentionGrad, "Formula" --
+ *     selectedKey = Gather(key, topkIndices[i]), 0 <= i < selectBlockCount,
+ *     each index naming block_size contiguous rows;
+ *   - token-level selection of a shared latent KV (K = V) and the sliding
+ *     window / compressed-KV concatenation: SparseFlashMlaGrad, "Computation
+ *     formula", Stage 1, with the oriSparseIndices / cmpSparseIndices,
+ *     oriTopkLength / cmpTopkLength, oriMaskMode / cmpMaskMode, oriWinLeft /
+ *     oriWinRight and sinks rows of its "Parameter Description" table;
+ *   - forward: aclnnNsaSelectedAttentionInfer, "Formula" --
+ *     O = Softmax(Q K_sel^T * scale) V_sel, lse = ln(sum exp(scores) [+ exp(sink)]);
+ *   - backward: SparseFlashMlaGrad, "Computation formula", Stages 2-3, and
+ *     aclnnSparseFlashAttentionGrad, "Formula", Phases 1-3 --
+ *     P = exp(S - lse), dP = dO V^T, dS = P o (dP - rowsum(dO o O)),
+ *     dQ = dS K scale, dK = dS^T Q scale, dV = P^T dO (dKV = dK + dV when K = V),
+ *     dSinks = sum over rows of -P_sink * sum_j P_j dP_j.
+ *
+ * Call shape.  Like the pages' two-phase API: *_get_workspace_size validates
+ * the arguments on the host and returns the workspace the call needs; the
+ * second call re-validates, enqueues its kernels on the caller's stream and
+ * returns without synchronising.  The library never allocates device memory:
+ * the caller owns every buffer, including the workspace.
+ *
+ * Pointers.  Every tensor pointer is a DEVICE pointer (bf16 = 2-byte bfloat16,
+ * row-major, innermost dimension contiguous, 16-byte aligned).  The sa_args /
+ * sa_fwd_out / sa_bwd_io structs themselves are host memory read during the
+ * call only.  `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *
+ * Layouts (layout = SA_LAYOUT_BSND or SA_LAYOUT_TND, shared by Q and KV):
+ *   BSND: q [B, s_q, Hq, d_qk]   k [B, s_kv, Hkv, d_qk]   v [B, s_kv, Hkv, d_v]
+ *         kv [B, s_kv, Hkv, d_qk] (K = V)  cmp_kv [B, s_kv / cmp_ratio, Hkv, d_qk]
+ *         ori_idx [B, s_q, Hkv, topk]  cmp_idx [B, s_q, Hkv, cmp_topk]
+ *         ori_topk_len / cmp_topk_len [B, s_q, Hkv]
+ *         o / d_o [B, s_q, Hq, d_v]   lse [B, s_q, Hq] (fp32)
+ *   TND:  the same with the leading [B, s] replaced by a packed token axis:
+ *         q [t_q, ...], k / v / kv [t_kv, ...], cmp_kv [t_cmp, ...]; sequence b
+ *         spans [cu_seqlens_x[b], cu_seqlens_x[b+1]) (B + 1 int32 offsets).
+ * Index values are positions local to their own sequence: a block index x
+ * covers rows [x * block_size, (x + 1) * block_size) clipped to the sequence;
+ * a token / compressed index is one row.  A negative index, or a slot at or
+ * past the row's topk length, selects nothing.  Indices past the end of the
+ * sequence are never read: they select nothing, and with SA_FLAG_CHECK the
+ * call reports SA_ERR_INDEX.
+ *
+ * Masks (applied per query row t, aligned bottom-right: ta = t + len_kv - len_q):
+ *   ori: NONE; CAUSAL row r <= ta; BAND ta - ori_win_left <= r <= ta + ori_win_right.
+ *   cmp: NONE; CAUSAL compressed row c visible iff (c + 1) * cmp_ratio - 1 <= ta.
+ * Without ori indices the whole original KV enters the selection under the ori
+ * mask (sliding window when BAND); cmp indices add compressed rows (SCFA).
+ *
+ * Empty rows.  A query row with no visible key and no sink gets lse = +inf and
+ * O = 0 and contributes no gradient.  A call with no query tokens returns
+ * SA_OK without launching anything.
+ *
+ * Determinism.  The backward accumulates dK / dV / dKV / dSinks with fp32
+ * atomics, so results may differ in the last bits from run to run.
+ *
+ * Errors.  Every entry point returns an sa_status.  Argument errors are found
+ * on the host before anything is enqueued.  CUDA launch errors come back as
+ * SA_ERR_CUDA (the library calls cudaGetLastError after its launches).
+ */
+#ifndef SPARSE_ATTN_H_
+#define SPARSE_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SA_ABI_VERSION 1
+
+typedef enum sa_status {
+  SA_OK = 0,
+  SA_ERR_NULLPTR = 1,      /* a required pointer is NULL */
+  SA_ERR_PARAM = 2,        /* a size, mode or attribute is out of range */
+  SA_ERR_UNSUPPORTED = 3,  /* valid per the pages but not built (e.g. fp16, CFA) */
+  SA_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than *_get_workspace_size */
+  SA_ERR_INDEX = 5,        /* SA_FLAG_CHECK found an index past its sequence */
+  SA_ERR_TIMEOUT = 6,      /* a bounded device wait gave up */
+  SA_ERR_CUDA = 7          /* a CUDA runtime error */
+} sa_status;
+
+typedef enum sa_layout { SA_LAYOUT_BSND = 0, SA_LAYOUT_TND = 1 } sa_layout;
+typedef enum sa_mask { SA_MASK_NONE = 0, SA_MASK_CAUSAL = 1, SA_MASK_BAND = 2 } sa_mask;
+typedef enum sa_dtype { SA_DTYPE_BF16 = 0, SA_DTYPE_FP16 = 1 } sa_dtype;
+
+/* flags */
+#define SA_FLAG_CHECK 1u   /* validate every index on the device first; the call then
+                              synchronises `stream` and returns SA_ERR_INDEX if one is
+                              past its sequence (nothing else is computed) */
+
+/* The problem description shared by every entry point (host struct). */
+typedef struct sa_args {
+  int32_t layout;          /* sa_layout */
+  int32_t dtype;           /* sa_dtype; only SA_DTYPE_BF16 is built */
+  int32_t batch;           /* B >= 0 */
+  int32_t s_q, s_kv;       /* BSND sequence lengths (ignored for TND) */
+  int32_t t_q, t_kv, t_cmp;/* TND packed token counts (ignored for BSND) */
+  int32_t n_heads_q;       /* Hq, a multiple of n_heads_kv */
+  int32_t n_heads_kv;      /* Hkv */
+  int32_t d_qk;            /* score head dim; multiple of 16, <= 576 */
+  int32_t d_v;             /* value head dim; multiple of 16, <= 512; <= d_qk if kv_shared */
+  int32_t kv_shared;       /* 1: K = V = kv, V is the first d_v columns of each kv row */
+  int32_t block_size;      /* rows per ori index (1 = token-level); <= 64 or a multiple of 64 */
+  int32_t topk;            /* ori index slots per (token, kv-head); 0 = no ori indices */
+  int32_t cmp_topk;        /* cmp index slots per (token, kv-head); 0 = no compressed KV */
+  int32_t cmp_ratio;       /* >= 1; cmp_kv has len_kv / cmp_ratio rows per sequence */
+  int32_t ori_mask_mode;   /* sa_mask */
+  int32_t cmp_mask_mode;   /* SA_MASK_NONE or SA_MASK_CAUSAL */
+  int64_t ori_win_left;    /* BAND: past rows kept (>= 0) */
+  int64_t ori_win_right;   /* BAND: future rows kept (>= 0) */
+  float scale;             /* scaleValue: multiplies Q K^T */
+  uint32_t flags;          /* SA_FLAG_* */
+  const void* q;           /* bf16, required */
+  const void* k;           /* bf16, required when !kv_shared */
+  const void* v;           /* bf16, required when !kv_shared */
+  const void* kv;          /* bf16, required when kv_shared */
+  const void* cmp_kv;      /* bf16, required when cmp_topk > 0 */
+  const int32_t* ori_idx;  /* required when topk > 0 */
+  const int32_t* cmp_idx;  /* required when cmp_topk > 0 */
+  const int32_t* cu_seqlens_q;   /* TND: B + 1 offsets, required */
+  const int32_t* cu_seqlens_kv;  /* TND: B + 1 offsets, required */
+  const int32_t* cu_seqlens_cmp; /* TND with cmp_topk > 0: B + 1 offsets, required */
+  const int32_t* ori_topk_len;   /* optional (NULL = all topk slots usable) */
+  const int32_t* cmp_topk_len;   /* optional (NULL = all cmp_topk slots usable) */
+  const int32_t* cmp_residual;   /* optional, [B]: len_kv mod cmp_ratio; accepted, not used */
+  const float* sinks;            /* optional, [Hq] fp32 sink logits */
+} sa_args;
+
+/* Forward outputs (device): O bf16 [.., Hq, d_v]; lse fp32 [.., Hq]. */
+typedef struct sa_fwd_out {
+  void* o;
+  float* lse;
+} sa_fwd_out;
+
+/* Backward inputs and outputs (device).  o / lse are the forward's outputs.
+ * dq is required.  dk and dv (separate K, V) or dkv (K = V) are required.
+ * dcmp_kv is required when cmp_topk > 0, dsinks when sinks != NULL. */
+typedef struct sa_bwd_io {
+  const void* o;           /* bf16 [.., Hq, d_v] */
+  const void* d_o;         /* bf16 [.., Hq, d_v] */
+  const float* lse;        /* fp32 [.., Hq] */
+  void* dq;                /* bf16, shape of q */
+  void* dk;                /* bf16, shape of k */
+  void* dv;                /* bf16, shape of v */
+  void* dkv;               /* bf16, shape of kv */
+  void* dcmp_kv;           /* bf16, shape of cmp_kv */
+  float* dsinks;           /* fp32 [Hq] */
+} sa_bwd_io;
+
+/* ---- forward ---------------------------------------------------------- */
+
+/* Phase 1: validate `args` (host only) and return the forward workspace size. */
+sa_status sa_fwd_get_workspace_size(const sa_args* args, size_t* ws_bytes);
+
+/* Phase 2: compute O and lse.  `ws` must hold at least the phase-1 size
+ * (may be NULL when that size is 0).  Enqueued on `stream`, asynchronous. */
+sa_status sa_fwd(const sa_args* args, const sa_fwd_out* out, void* ws, size_t ws_bytes,
+                 void* stream);
+
+/* ---- backward --------------------------------------------------------- */
+
+/* Phase 1: validate `args` (host only) and return the backward workspace size
+ * (fp32 accumulators for dK/dV, dKV and dCmpKv, the rowsum(dO o O) vector and
+ * the inverse index used by the key-stationary kernels). */
+sa_status sa_bwd_get_workspace_size(const sa_args* args, size_t* ws_bytes);
+
+/* Phase 2: compute dQ, dK/dV (or dKV), dCmpKv and dSinks from dO, O and lse.
+ * Every output is fully overwritten.  Enqueued on `stream`, asynchronous. */
+sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_bytes,
+                 void* stream);
+
+/* rowsum(dO o O) alone -- the "FlashSoftmaxGrad(dO, O)" / "SoftmaxGrad(dO, O)"
+ * term of aclnnSparseFlashAttentionGrad Phase 2 and SparseFlashMlaGrad Stage 2:
+ * delta[token, h] = sum_c d_o[token, h, c] * o[token, h, c] in fp32.
+ * o, d_o bf16 [.., Hq, d_v]; delta fp32 [.., Hq] (device).  Asynchronous. */
+sa_status sa_softmax_grad_preprocess(const sa_args* args, const void* o, const void* d_o,
+                                     float* delta, void* stream);
+
+/* ---- inspection ------------------------------------------------------- */
+
+/* The visible KV set of every (query token, kv-head) unit exactly as the
+ * kernels resolve it (Stage 1 selection plus masks).  rows: int32
+ * [units, max_rows] with unit = token * Hkv + g; original-KV row r is written
+ * as r, compressed row c as (0x40000000 | c), in slot order; entries past the
+ * count are left untouched.  counts: int32 [units], the full count (may exceed
+ * max_rows, in which case only max_rows entries are written).  Asynchronous. */
+sa_status sa_debug_resolve(const sa_args* args, int32_t* rows, int32_t* counts,
+                           int32_t max_rows, void* stream);
+
+/* ---- benchmarking hooks ------------------------------------------------ */
+
+/* Timing hook (process-wide, not thread-safe): when both are non-NULL, the
+ * next sa_fwd / sa_bwd calls record ev_begin right before and ev_end right
+ * after their main kernel (the forward kernel; the fused backward kernel), on
+ * the call's stream.  Both are cudaEvent_t created by the caller; pass NULL,
+ * NULL to disable. */
+void sa_set_timing_events(void* ev_begin, void* ev_end);
+
+/* Number of kernels this library has launched since it was loaded
+ * (memsets excluded). */
+int64_t sa_kernel_launch_count(void);
+
+/* Human-readable name of a status code (static string). */
+const char* sa_status_string(int32_t status);
+
+/* SA_ABI_VERSION of the built library. */
+int32_t sa_abi_version(void);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* SPARSE_ATTN_H_ */

@@ -88,12 +88,23 @@ def round_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     return bits.astype(np.uint16)
 
 
+def as_f64(x) -> np.ndarray:
+    """float64 view of an array slice: bf16 bit patterns (uint16) are widened exactly."""
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return widen_bf16(x)
+    return x.astype(np.float64, copy=False)
+
+
 # ----------------------------------------------------------------------------
 # Problem description
 # ----------------------------------------------------------------------------
 
 class Problem:
-    """All inputs of one sparse-attention call, token-major, in float64.
+    """All inputs of one sparse-attention call, token-major.
+
+    Tensors may be float64 or bf16 bit patterns (uint16); the latter are
+    widened exactly to float64 row by row when a unit reads them.
 
     Arrays (T = total query tokens, Tk = total original KV rows, Tc = total
     compressed KV rows):
@@ -111,9 +122,9 @@ class Problem:
                  k_cmp=None, v_cmp=None, cmp_lens=None, cmp_idx=None,
                  cmp_topk_len=None, cmp_ratio=1, ori_mask="causal",
                  cmp_mask="causal", win_left=0, win_right=0, sinks=None):
-        self.q = np.asarray(q, dtype=np.float64)
-        self.k_ori = np.asarray(k_ori, dtype=np.float64)
-        self.v_ori = np.asarray(v_ori, dtype=np.float64)
+        self.q = np.asarray(q)
+        self.k_ori = np.asarray(k_ori)
+        self.v_ori = np.asarray(v_ori)
         self.kv_shared = bool(kv_shared)
         self.Hq, self.Hkv, self.d_qk, self.d_v = Hq, Hkv, d_qk, d_v
         assert Hq % Hkv == 0
@@ -122,8 +133,8 @@ class Problem:
         self.block_size = int(block_size)
         self.ori_idx = None if ori_idx is None else np.asarray(ori_idx, dtype=np.int64)
         self.ori_topk_len = None if ori_topk_len is None else np.asarray(ori_topk_len, dtype=np.int64)
-        self.k_cmp = None if k_cmp is None else np.asarray(k_cmp, dtype=np.float64)
-        self.v_cmp = None if v_cmp is None else np.asarray(v_cmp, dtype=np.float64)
+        self.k_cmp = None if k_cmp is None else np.asarray(k_cmp)
+        self.v_cmp = None if v_cmp is None else np.asarray(v_cmp)
         self.cmp_idx = None if cmp_idx is None else np.asarray(cmp_idx, dtype=np.int64)
         self.cmp_topk_len = None if cmp_topk_len is None else np.asarray(cmp_topk_len, dtype=np.int64)
         self.cmp_ratio = int(cmp_ratio)
@@ -143,6 +154,17 @@ class Problem:
         assert self.q.shape == (self.T, Hq, d_qk)
 
     @property
+    def Tk(self) -> int:
+        return int(self.k_ori.shape[0])
+
+    @property
+    def Tc(self) -> int:
+        return 0 if self.k_cmp is None else int(self.k_cmp.shape[0])
+
+    def all_units(self):
+        return [(tq, g) for tq in range(self.T) for g in range(self.Hkv)]
+
+    @property
     def has_cmp(self) -> bool:
         return self.k_cmp is not None
 
@@ -151,15 +173,16 @@ class Problem:
 
     @classmethod
     def from_inputs(cls, w, inp: dict) -> "Problem":
-        """Build from a workload description and the generator's arrays (bf16 as uint16)."""
+        """Build from a workload description and the generator's arrays (bf16 as uint16,
+        kept as bit patterns and widened when read)."""
         T = w.T
-        q = widen_bf16(inp["q"]).reshape(T, w.Hq, w.d_qk)
+        q = inp["q"].reshape(T, w.Hq, w.d_qk)
         if w.kv_shared:
-            kv = widen_bf16(inp["kv"]).reshape(T, w.Hkv, w.d_qk)
+            kv = inp["kv"].reshape(T, w.Hkv, w.d_qk)
             k_ori, v_ori = kv, kv[..., :w.d_v]
         else:
-            k_ori = widen_bf16(inp["k"]).reshape(T, w.Hkv, w.d_qk)
-            v_ori = widen_bf16(inp["v"]).reshape(T, w.Hkv, w.d_v)
+            k_ori = inp["k"].reshape(T, w.Hkv, w.d_qk)
+            v_ori = inp["v"].reshape(T, w.Hkv, w.d_v)
         lens = list(w.seq_lengths)
         kw = {}
         if "ori_idx" in inp:
@@ -167,7 +190,7 @@ class Problem:
         if "ori_topk_len" in inp:
             kw["ori_topk_len"] = inp["ori_topk_len"].reshape(T, w.Hkv)
         if "cmp_kv" in inp:
-            ck = widen_bf16(inp["cmp_kv"]).reshape(-1, w.Hkv, w.d_qk)
+            ck = inp["cmp_kv"].reshape(-1, w.Hkv, w.d_qk)
             kw.update(k_cmp=ck, v_cmp=ck[..., :w.d_v],
                       cmp_lens=np.diff(inp["cu_seqlens_cmp"]),
                       cmp_idx=inp["cmp_idx"].reshape(T, w.Hkv, -1))
@@ -241,11 +264,11 @@ def visible_rows(p: Problem, tq: int, g: int):
 def _gather(p: Problem, tq: int, g: int):
     b = p.batch_of(tq)
     ori, cmp = visible_rows(p, tq, g)
-    K = p.k_ori[p.kv_start[b] + ori, g]
-    V = p.v_ori[p.kv_start[b] + ori, g]
+    K = as_f64(p.k_ori[p.kv_start[b] + ori, g])
+    V = as_f64(p.v_ori[p.kv_start[b] + ori, g])
     if len(cmp):
-        K = np.concatenate([K, p.k_cmp[p.cmp_start[b] + cmp, g]])
-        V = np.concatenate([V, p.v_cmp[p.cmp_start[b] + cmp, g]])
+        K = np.concatenate([K, as_f64(p.k_cmp[p.cmp_start[b] + cmp, g])])
+        V = np.concatenate([V, as_f64(p.v_cmp[p.cmp_start[b] + cmp, g])])
     return ori, cmp, K, V
 
 
@@ -256,7 +279,7 @@ def _gather(p: Problem, tq: int, g: int):
 def unit_forward(p: Problem, tq: int, g: int):
     """O [G, d_v] and lse [G] (float64) for the G query heads of kv-head g at token tq."""
     hs = slice(g * p.G, (g + 1) * p.G)
-    Q = p.q[tq, hs]
+    Q = as_f64(p.q[tq, hs])
     _, _, K, V = _gather(p, tq, g)
     S = p.scale * (Q @ K.T)                               # [G, n] scaled scores
     sink = None if p.sinks is None else p.sinks[hs]
@@ -276,22 +299,24 @@ def unit_forward(p: Problem, tq: int, g: int):
 
 
 def forward(p: Problem, units=None, rounded: bool = True):
-    """Forward over all units (token, kv-head), or only over ``units``.
+    """Forward over every unit (token, kv-head), or over ``units`` only.
 
-    Returns (O, lse): O [T, Hq, d_v], lse [T, Hq].  Rounded: O as bf16 bits and
-    lse as float32; otherwise float64.  Units not computed hold zeros.
+    With ``units=None`` returns (O, lse): O [T, Hq, d_v], lse [T, Hq].  With a
+    list of units returns a dict {(tq, g): (O [G, d_v], lse [G])}.  Rounded: O
+    as bf16 bits and lse as float32; otherwise float64.
     """
+    def fin(o, l):
+        return (round_to_bf16_bits(o), l.astype(np.float32)) if rounded else (o, l)
+
+    if units is not None:
+        return {(tq, g): fin(*unit_forward(p, tq, g)) for tq, g in units}
     O = np.zeros((p.T, p.Hq, p.d_v))
     lse = np.zeros((p.T, p.Hq))
-    if units is None:
-        units = [(tq, g) for tq in range(p.T) for g in range(p.Hkv)]
-    for tq, g in units:
+    for tq, g in p.all_units():
         o, l = unit_forward(p, tq, g)
         O[tq, g * p.G:(g + 1) * p.G] = o
         lse[tq, g * p.G:(g + 1) * p.G] = l
-    if rounded:
-        return round_to_bf16_bits(O), lse.astype(np.float32)
-    return O, lse
+    return fin(O, lse)
 
 
 # ----------------------------------------------------------------------------
@@ -306,7 +331,7 @@ def unit_backward(p: Problem, tq: int, g: int, O, lse, dO):
     dK_rows [n, d_qk], dV_rows [n, d_v], P_sink [G] and dSinks [G].
     """
     hs = slice(g * p.G, (g + 1) * p.G)
-    Q = p.q[tq, hs]
+    Q = as_f64(p.q[tq, hs])
     ori, cmp, K, V = _gather(p, tq, g)
     S = p.scale * (Q @ K.T)
     P = np.exp(S - lse[:, None])                          # SimpleSoftmax(S, lse)
@@ -333,31 +358,34 @@ def _scatter_add(dst, rows, vals):
 
 
 def backward(p: Problem, O, lse, dO, units=None, rounded: bool = True):
-    """Backward over all units, or over ``units`` only (partial sums for dK/dV).
+    """Backward over every unit, or over ``units`` only (then dK/dV are partial sums).
 
-    ``O``, ``dO`` [T, Hq, d_v] and ``lse`` [T, Hq] as float64 (widen bf16 / fp32
-    first).  Returns a dict: dq [T, Hq, d_qk]; dk [Tk, Hkv, d_qk] and dv
-    [Tk, Hkv, d_v], or dkv [Tk, Hkv, d_qk] when K = V; dcmp [Tc, Hkv, d_qk] when
-    there is a compressed KV; dsinks [Hq] when there are sinks.  Rounded: bf16
-    bits for every tensor but dsinks (float32); otherwise float64.
+    ``O``, ``dO`` [T, Hq, d_v] and ``lse`` [T, Hq]: float64 arrays, or bf16 bit
+    patterns / float32 (widened exactly when read).  Returns a dict: dq
+    [T, Hq, d_qk] (a dict {(tq, g): [G, d_qk]} when ``units`` is given); dk
+    [Tk, Hkv, d_qk] and dv [Tk, Hkv, d_v], or dkv [Tk, Hkv, d_qk] when K = V;
+    dcmp [Tc, Hkv, d_qk] when there is a compressed KV; dsinks [Hq] when there
+    are sinks.  Rounded: bf16 bits for every tensor but dsinks (float32);
+    otherwise float64.
     """
-    O = np.asarray(O, dtype=np.float64)
-    dO = np.asarray(dO, dtype=np.float64)
-    lse = np.asarray(lse, dtype=np.float64)
-    Tk = p.k_ori.shape[0]
-    dq = np.zeros_like(p.q)
-    dk = np.zeros((Tk, p.Hkv, p.d_qk))
-    dv = np.zeros((Tk, p.Hkv, p.d_v))
-    Tc = 0 if p.k_cmp is None else p.k_cmp.shape[0]
-    dkc = np.zeros((Tc, p.Hkv, p.d_qk))
-    dvc = np.zeros((Tc, p.Hkv, p.d_v))
+    dk = np.zeros((p.Tk, p.Hkv, p.d_qk))
+    dv = np.zeros((p.Tk, p.Hkv, p.d_v))
+    dkc = np.zeros((p.Tc, p.Hkv, p.d_qk))
+    dvc = np.zeros((p.Tc, p.Hkv, p.d_v))
     dsinks = np.zeros(p.Hq)
     if units is None:
-        units = [(tq, g) for tq in range(p.T) for g in range(p.Hkv)]
-    for tq, g in units:
+        dq = np.zeros((p.T, p.Hq, p.d_qk))
+        todo = p.all_units()
+    else:
+        dq = {}
+        todo = units
+    for tq, g in todo:
         hs = slice(g * p.G, (g + 1) * p.G)
-        r = unit_backward(p, tq, g, O[tq, hs], lse[tq, hs], dO[tq, hs])
-        dq[tq, hs] = r["dQ"]
+        r = unit_backward(p, tq, g, as_f64(O[tq, hs]), as_f64(lse[tq, hs]), as_f64(dO[tq, hs]))
+        if units is None:
+            dq[tq, hs] = r["dQ"]
+        else:
+            dq[(tq, g)] = r["dQ"]
         b = p.batch_of(tq)
         no = len(r["ori"])
         _scatter_add(dk[:, g], p.kv_start[b] + r["ori"], r["dK_rows"][:no])
@@ -384,6 +412,8 @@ def backward(p: Problem, O, lse, dO, units=None, rounded: bool = True):
         for key in list(res):
             if key == "dsinks":
                 res[key] = res[key].astype(np.float32)
+            elif key == "dq" and units is not None:
+                res[key] = {u: round_to_bf16_bits(v) for u, v in res[key].items()}
             else:
                 res[key] = round_to_bf16_bits(res[key])
     return res

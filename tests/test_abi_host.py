@@ -1,0 +1,189 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+symbol, its structs match the ctypes mirror, and argument validation returns
+the documented status codes without touching a GPU."""
+
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+from top_sparse_attention_attn_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sparse_attn.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(sa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared_functions()
+    assert len(names) >= 8
+    lib = L.lib()
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in sparse_attn.h but not exported"
+    assert sorted(L.EXPORTS) == names
+
+
+def test_abi_version_and_status_strings():
+    m = re.search(r"#define SA_ABI_VERSION (\d+)", open(HEADER).read())
+    assert L.sa_abi_version() == int(m.group(1))
+    for s in range(8):
+        assert L.status_string(s).startswith("SA_")
+    assert "unknown" in L.status_string(99)
+
+
+C_PROBE = r"""
+#include <stdio.h>
+#include <stddef.h>
+#include "sparse_attn.h"
+#define F(S, m) printf("%s.%s %zu\n", #S, #m, offsetof(S, m));
+int main(void) {
+  printf("sa_args %zu\nsa_fwd_out %zu\nsa_bwd_io %zu\n", sizeof(sa_args), sizeof(sa_fwd_out), sizeof(sa_bwd_io));
+  F(sa_args, ori_win_left) F(sa_args, scale) F(sa_args, flags) F(sa_args, q) F(sa_args, sinks)
+  F(sa_args, cmp_idx) F(sa_args, cu_seqlens_cmp) F(sa_bwd_io, dsinks) F(sa_bwd_io, dcmp_kv)
+  return 0;
+}
+"""
+
+
+def test_struct_layout_matches_header():
+    with tempfile.TemporaryDirectory() as d:
+        src = os.path.join(d, "probe.c")
+        exe = os.path.join(d, "probe")
+        open(src, "w").write(C_PROBE)
+        subprocess.run(["gcc", "-std=c11", "-I", os.path.dirname(HEADER), src, "-o", exe], check=True)
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = dict(line.split() for line in out if line.strip())
+    assert int(got["sa_args"]) == ctypes.sizeof(L.SaArgs)
+    assert int(got["sa_fwd_out"]) == ctypes.sizeof(L.SaFwdOut)
+    assert int(got["sa_bwd_io"]) == ctypes.sizeof(L.SaBwdIo)
+    for key, val in got.items():
+        if "." in key:
+            s, m = key.split(".")
+            cls = {"sa_args": L.SaArgs, "sa_bwd_io": L.SaBwdIo}[s]
+            assert getattr(cls, m).offset == int(val), key
+
+
+# ----------------------------------------------------------------------------
+# validation (host only: every call below fails before any CUDA call)
+# ----------------------------------------------------------------------------
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: these calls fail validation first
+
+
+def _args(**kw):
+    a = L.SaArgs()
+    a.layout = L.SA_LAYOUT_BSND
+    a.dtype = L.SA_DTYPE_BF16
+    a.batch, a.s_q, a.s_kv = 2, 128, 128
+    a.n_heads_q, a.n_heads_kv = 16, 4
+    a.d_qk, a.d_v = 192, 128
+    a.block_size, a.topk = 64, 4
+    a.cmp_ratio = 1
+    a.ori_mask_mode = L.SA_MASK_CAUSAL
+    a.scale = 0.1
+    a.q = a.k = a.v = a.ori_idx = FAKE
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def _ws(a):
+    n = ctypes.c_size_t(0)
+    st = L.lib().sa_bwd_get_workspace_size(ctypes.byref(a), ctypes.byref(n))
+    return st, n.value
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(), L.SA_OK),
+    (dict(n_heads_q=15), L.SA_ERR_PARAM),
+    (dict(n_heads_kv=0), L.SA_ERR_PARAM),
+    (dict(dtype=L.SA_DTYPE_FP16), L.SA_ERR_UNSUPPORTED),
+    (dict(dtype=7), L.SA_ERR_PARAM),
+    (dict(d_qk=96, d_v=96), L.SA_ERR_UNSUPPORTED),
+    (dict(d_qk=100), L.SA_ERR_PARAM),
+    (dict(d_qk=640), L.SA_ERR_PARAM),
+    (dict(block_size=100), L.SA_ERR_PARAM),
+    (dict(block_size=0), L.SA_ERR_PARAM),
+    (dict(topk=-1), L.SA_ERR_PARAM),
+    (dict(q=None), L.SA_ERR_NULLPTR),
+    (dict(ori_idx=None), L.SA_ERR_NULLPTR),
+    (dict(v=None), L.SA_ERR_NULLPTR),
+    (dict(layout=5), L.SA_ERR_PARAM),
+    (dict(ori_mask_mode=L.SA_MASK_BAND, ori_win_left=-1), L.SA_ERR_PARAM),
+    (dict(cmp_mask_mode=L.SA_MASK_BAND), L.SA_ERR_PARAM),
+    (dict(cmp_ratio=0), L.SA_ERR_PARAM),
+    (dict(scale=float("nan")), L.SA_ERR_PARAM),
+    (dict(cmp_topk=8, cmp_kv=FAKE, cmp_idx=FAKE), L.SA_ERR_UNSUPPORTED),   # compressed KV needs K = V
+    (dict(layout=L.SA_LAYOUT_TND, t_q=256, t_kv=256), L.SA_ERR_NULLPTR),    # no cu_seqlens
+    (dict(kv_shared=1, d_qk=128, d_v=128, k=None, v=None), L.SA_ERR_NULLPTR),
+    (dict(kv_shared=1, d_qk=128, d_v=128, k=None, v=None, kv=FAKE), L.SA_OK),
+    (dict(kv_shared=1, d_qk=128, d_v=256, kv=FAKE), L.SA_ERR_PARAM),
+])
+def test_validation_codes(kw, status):
+    st, _ = _ws(_args(**kw))
+    assert st == status, L.status_string(st)
+    n = ctypes.c_size_t(0)
+    assert L.lib().sa_fwd_get_workspace_size(ctypes.byref(_args(**kw)), ctypes.byref(n)) == status
+
+
+def test_null_args_and_null_size():
+    n = ctypes.c_size_t(0)
+    assert L.lib().sa_fwd_get_workspace_size(None, ctypes.byref(n)) == L.SA_ERR_NULLPTR
+    assert L.lib().sa_bwd_get_workspace_size(ctypes.byref(_args()), None) == L.SA_ERR_NULLPTR
+
+
+def _align(x):
+    return (x + 255) // 256 * 256
+
+
+def test_bwd_workspace_size_contract():
+    a = _args()
+    st, n = _ws(a)
+    Tq, Tk = 2 * 128, 2 * 128
+    expect = 256 + _align(Tq * 16 * 4) + _align(Tk * 4 * 192 * 4) + _align(Tk * 4 * 128 * 4)
+    assert st == L.SA_OK and n == expect
+    a = _args(kv_shared=1, d_qk=576, d_v=512, kv=FAKE, n_heads_q=64, n_heads_kv=1, block_size=1,
+              layout=L.SA_LAYOUT_TND, t_q=1000, t_kv=1000, t_cmp=250, cmp_topk=16, cmp_ratio=4,
+              cmp_kv=FAKE, cmp_idx=FAKE, cu_seqlens_q=FAKE, cu_seqlens_kv=FAKE, cu_seqlens_cmp=FAKE)
+    st, n = _ws(a)
+    expect = 256 + _align(1000 * 64 * 4) + _align(1000 * 576 * 4) + _align(250 * 576 * 4)
+    assert st == L.SA_OK and n == expect
+
+
+def test_calls_fail_before_launch():
+    a = _args()
+    n = _ws(a)[1]
+    io = L.SaBwdIo(o=FAKE, d_o=FAKE, lse=FAKE, dq=FAKE, dk=FAKE, dv=FAKE)
+    # workspace too small / missing
+    assert L.lib().sa_bwd(ctypes.byref(a), ctypes.byref(io), FAKE, n - 1, None) == L.SA_ERR_WORKSPACE
+    assert L.lib().sa_bwd(ctypes.byref(a), ctypes.byref(io), None, n, None) == L.SA_ERR_WORKSPACE
+    # missing outputs
+    io2 = L.SaBwdIo(o=FAKE, d_o=FAKE, lse=FAKE, dq=FAKE, dk=FAKE)
+    assert L.lib().sa_bwd(ctypes.byref(a), ctypes.byref(io2), FAKE, n, None) == L.SA_ERR_NULLPTR
+    assert L.lib().sa_bwd(ctypes.byref(a), None, FAKE, n, None) == L.SA_ERR_NULLPTR
+    out = L.SaFwdOut(o=FAKE, lse=None)
+    assert L.lib().sa_fwd(ctypes.byref(a), ctypes.byref(out), FAKE, 256, None) == L.SA_ERR_NULLPTR
+    # misaligned tensor
+    out = L.SaFwdOut(o=FAKE, lse=FAKE)
+    a.q = FAKE + 2
+    assert L.lib().sa_fwd(ctypes.byref(a), ctypes.byref(out), FAKE, 256, None) == L.SA_ERR_PARAM
+
+
+def test_empty_query_is_a_no_op():
+    """An empty query returns directly (the pages: 'If the query is an empty Tensor: return directly')."""
+    a = _args(s_q=0)
+    out = L.SaFwdOut(o=None, lse=None)
+    assert L.lib().sa_fwd(ctypes.byref(a), ctypes.byref(out), None, 0, None) == L.SA_OK
+    io = L.SaBwdIo()
+    assert L.lib().sa_bwd(ctypes.byref(a), ctypes.byref(io), None, 0, None) == L.SA_OK
+    a = _args(batch=0)
+    assert L.lib().sa_fwd(ctypes.byref(a), ctypes.byref(out), None, 0, None) == L.SA_OK
+    assert L.lib().sa_softmax_grad_preprocess(ctypes.byref(a), None, None, None, None) == L.SA_OK

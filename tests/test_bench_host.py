@@ -1,0 +1,59 @@
+"""Host-side checks of the benchmark's accounting: the FLOP and byte counters
+read from the index tensors agree with the oracle's own visible-set count."""
+
+import numpy as np
+import pytest
+
+import bench
+import oracle
+from gen import get_workload, make_inputs, scaled
+
+CASES = [
+    ("cfg1", {}, {}),
+    ("cfg2", dict(S=700, Hq=32, Hkv=2), dict(allow_future=True, ori_len_range=(0, 16))),
+    ("cfg3", dict(S=300, Hq=16, topk=64), {}),
+    ("cfg4", dict(seqlens=(100, 300, 37), Hq=16, cmp_topk=64, cmp_len_range=(16, 64)), dict(cmp_any=True)),
+    ("cfg5", dict(S=1024, Hq=16, Hkv=4), {}),
+    ("cfg4", dict(seqlens=(50, 90), Hq=8, cmp_topk=16, cmp_len_range=(2, 16), win_left=10, win_right=3), {}),
+]
+
+
+@pytest.mark.parametrize("name,ov,kw", CASES)
+def test_flop_count_matches_oracle(name, ov, kw):
+    w = scaled(name, **ov) if ov else get_workload(name)
+    inp = make_inputs(w, **kw)
+    c = bench.count_work(w, inp)
+    p = oracle.Problem.from_inputs(w, inp)
+    fwd = bwd = 0
+    for tq, g in p.all_units():
+        f, b = oracle.unit_flops(p, tq, g)
+        fwd += f
+        bwd += b
+    assert c["fwd_flops"] == fwd and c["bwd_flops"] == bwd
+
+
+def test_cfg1_matches_published_plan():
+    """Config 1 totals: 0.526 GFLOP backward, 60.8 MB of gathered rows."""
+    w = get_workload("cfg1")
+    c = bench.count_work(w, make_inputs(w))
+    assert abs(c["bwd_flops"] / 1e9 - 0.526) < 0.001
+    assert abs(c["gathered_bytes"] / 1e6 - 60.8) < 0.1
+
+
+def test_oracle_baseline_runs_briefly():
+    w = scaled("cfg2", S=256, Hq=16, Hkv=1)
+    r = bench.oracle_baseline(w, make_inputs(w), budget_s=0.5)
+    assert r["value"] > 0 and r["cores"] >= 1 and r["kind"] == "oracle"
+
+
+def test_reference_arm_line():
+    class A:
+        workload = "cfg1"
+        override = None
+        steps = 1
+        warmup = 0
+        step_budget = 1.0
+    line = bench.run_reference(A(), rank=0)
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert bench.run_reference(A(), rank=1) is None

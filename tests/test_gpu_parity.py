@@ -1,0 +1,59 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
+seeded inputs.  Small workloads compare every output element; the five
+full-size workloads compare sampled units and tail KV rows in the launch
+configuration the benchmark times."""
+
+import numpy as np
+import pytest
+import torch
+
+from gen import get_workload, make_inputs, scaled
+from gpu_harness import run_full_comparison, run_sampled
+
+pytestmark = pytest.mark.gpu
+
+
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA GPU is required for -m gpu tests")
+
+
+SMALL = {
+    "cfg1_full": (get_workload("cfg1"), {}),
+    "cfg2_small": (scaled("cfg2", S=700, Hq=32, Hkv=2, seed=21), {}),
+    "cfg2_future_len": (scaled("cfg2", "future", S=448, Hq=16, Hkv=1, seed=22),
+                        dict(allow_future=True, ori_len_range=(0, 16))),
+    "cfg3_small": (scaled("cfg3", S=700, Hq=32, topk=256, seed=23), {}),
+    "cfg4_small": (scaled("cfg4", seqlens=(100, 300, 37), Hq=16, cmp_topk=64,
+                          cmp_len_range=(16, 64), seed=24), {}),
+    "cfg4_cmp_any_band": (scaled("cfg4", "any", seqlens=(130, 71), Hq=16, cmp_topk=32,
+                                 cmp_len_range=(8, 32), win_left=40, win_right=5, seed=25),
+                          dict(cmp_any=True)),
+    "cfg5_small": (scaled("cfg5", S=2048, Hq=16, Hkv=4, seed=26), {}),
+    "cfg5_empty_rows": (scaled("cfg5", "empty", S=512, Hq=8, Hkv=2, p_drop=0.6, seed=27), {}),
+    "block_g24_128": (scaled("cfg2", "g24", S=320, Hq=48, Hkv=2, d_qk=128, d_v=128, topk=6,
+                             seed=28), {}),
+    "block_bs16_d64": (scaled("cfg1", "bs16", S=300, Hq=8, Hkv=2, block_size=16, topk=6,
+                              seed=29), {}),
+    "block_bs128_d64": (scaled("cfg1", "bs128", S=600, Hq=4, Hkv=1, block_size=128, topk=3,
+                               seed=30), {}),
+    "block_tnd": (scaled("cfg1", "tnd", layout="TND", seqlens=(200, 64, 333), Hq=8, Hkv=1,
+                         seed=31), {}),
+    "token_shared_128_nomask": (scaled("cfg3", "nomask", S=333, Hq=16, d_qk=128, d_v=128,
+                                       topk=100, ori_mask="none", seed=32), {}),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_workload_all_elements(name):
+    _need_gpu()
+    w, kw = SMALL[name]
+    run_full_comparison(w, kw)
+
+
+@pytest.mark.parametrize("cfg", ["cfg2", "cfg1", "cfg5", "cfg4", "cfg3"])
+def test_full_size_sampled(cfg):
+    _need_gpu()
+    w = get_workload(cfg)
+    tail = 16 if cfg == "cfg3" else 64
+    run_sampled(w, n_units=16 if cfg == "cfg3" else 24, tail_rows=tail)

@@ -1,0 +1,161 @@
+"""ctypes binding of libsparse_attn.so (include/sparse_attn.h).
+
+Argument marshalling only: every entry point here converts Python values into
+the C structs and calls the library; all computation happens in the CUDA
+kernels behind the C ABI.  Loading fails loudly when the library is missing.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libsparse_attn.so")
+
+SA_OK = 0
+SA_ERR_NULLPTR = 1
+SA_ERR_PARAM = 2
+SA_ERR_UNSUPPORTED = 3
+SA_ERR_WORKSPACE = 4
+SA_ERR_INDEX = 5
+SA_ERR_TIMEOUT = 6
+SA_ERR_CUDA = 7
+
+SA_LAYOUT_BSND = 0
+SA_LAYOUT_TND = 1
+SA_MASK_NONE = 0
+SA_MASK_CAUSAL = 1
+SA_MASK_BAND = 2
+SA_DTYPE_BF16 = 0
+SA_DTYPE_FP16 = 1
+SA_FLAG_CHECK = 1
+
+MASKS = {"none": SA_MASK_NONE, "causal": SA_MASK_CAUSAL, "band": SA_MASK_BAND}
+LAYOUTS = {"BSND": SA_LAYOUT_BSND, "TND": SA_LAYOUT_TND}
+
+_vp = ctypes.c_void_p
+_ip = ctypes.POINTER(ctypes.c_int32)
+_fp = ctypes.POINTER(ctypes.c_float)
+
+
+class SaArgs(ctypes.Structure):
+    _fields_ = [
+        ("layout", ctypes.c_int32), ("dtype", ctypes.c_int32), ("batch", ctypes.c_int32),
+        ("s_q", ctypes.c_int32), ("s_kv", ctypes.c_int32),
+        ("t_q", ctypes.c_int32), ("t_kv", ctypes.c_int32), ("t_cmp", ctypes.c_int32),
+        ("n_heads_q", ctypes.c_int32), ("n_heads_kv", ctypes.c_int32),
+        ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32), ("kv_shared", ctypes.c_int32),
+        ("block_size", ctypes.c_int32), ("topk", ctypes.c_int32), ("cmp_topk", ctypes.c_int32),
+        ("cmp_ratio", ctypes.c_int32), ("ori_mask_mode", ctypes.c_int32),
+        ("cmp_mask_mode", ctypes.c_int32), ("ori_win_left", ctypes.c_int64),
+        ("ori_win_right", ctypes.c_int64), ("scale", ctypes.c_float), ("flags", ctypes.c_uint32),
+        ("q", _vp), ("k", _vp), ("v", _vp), ("kv", _vp), ("cmp_kv", _vp),
+        ("ori_idx", _vp), ("cmp_idx", _vp),
+        ("cu_seqlens_q", _vp), ("cu_seqlens_kv", _vp), ("cu_seqlens_cmp", _vp),
+        ("ori_topk_len", _vp), ("cmp_topk_len", _vp), ("cmp_residual", _vp), ("sinks", _vp),
+    ]
+
+
+class SaFwdOut(ctypes.Structure):
+    _fields_ = [("o", _vp), ("lse", _vp)]
+
+
+class SaBwdIo(ctypes.Structure):
+    _fields_ = [("o", _vp), ("d_o", _vp), ("lse", _vp), ("dq", _vp), ("dk", _vp), ("dv", _vp),
+                ("dkv", _vp), ("dcmp_kv", _vp), ("dsinks", _vp)]
+
+
+class SaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+_lib = None
+
+# every symbol include/sparse_attn.h declares
+EXPORTS = ["sa_fwd_get_workspace_size", "sa_fwd", "sa_bwd_get_workspace_size", "sa_bwd",
+           "sa_softmax_grad_preprocess", "sa_debug_resolve", "sa_status_string", "sa_abi_version",
+           "sa_set_timing_events", "sa_kernel_launch_count"]
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsparse_attn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m top_sparse_attention_attn_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER
+        L.sa_fwd_get_workspace_size.argtypes = [P(SaArgs), P(ctypes.c_size_t)]
+        L.sa_fwd.argtypes = [P(SaArgs), P(SaFwdOut), _vp, ctypes.c_size_t, _vp]
+        L.sa_bwd_get_workspace_size.argtypes = [P(SaArgs), P(ctypes.c_size_t)]
+        L.sa_bwd.argtypes = [P(SaArgs), P(SaBwdIo), _vp, ctypes.c_size_t, _vp]
+        L.sa_softmax_grad_preprocess.argtypes = [P(SaArgs), _vp, _vp, _vp, _vp]
+        L.sa_debug_resolve.argtypes = [P(SaArgs), _vp, _vp, ctypes.c_int32, _vp]
+        L.sa_status_string.argtypes = [ctypes.c_int32]
+        L.sa_status_string.restype = ctypes.c_char_p
+        L.sa_abi_version.argtypes = []
+        L.sa_set_timing_events.argtypes = [_vp, _vp]
+        L.sa_set_timing_events.restype = None
+        L.sa_kernel_launch_count.argtypes = []
+        L.sa_kernel_launch_count.restype = ctypes.c_int64
+        for name in EXPORTS:
+            if name not in ("sa_status_string", "sa_set_timing_events", "sa_kernel_launch_count"):
+                getattr(L, name).restype = ctypes.c_int32
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().sa_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != SA_OK:
+        raise SaError(status, where)
+
+
+# ---- the entry points, same names as the C ABI -------------------------------
+
+def sa_fwd_get_workspace_size(args: SaArgs) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().sa_fwd_get_workspace_size(ctypes.byref(args), ctypes.byref(n)), "sa_fwd_get_workspace_size")
+    return n.value
+
+
+def sa_fwd(args: SaArgs, out: SaFwdOut, ws: int, ws_bytes: int, stream: int = 0) -> None:
+    _check(lib().sa_fwd(ctypes.byref(args), ctypes.byref(out), ws, ws_bytes, stream), "sa_fwd")
+
+
+def sa_bwd_get_workspace_size(args: SaArgs) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().sa_bwd_get_workspace_size(ctypes.byref(args), ctypes.byref(n)), "sa_bwd_get_workspace_size")
+    return n.value
+
+
+def sa_bwd(args: SaArgs, io: SaBwdIo, ws: int, ws_bytes: int, stream: int = 0) -> None:
+    _check(lib().sa_bwd(ctypes.byref(args), ctypes.byref(io), ws, ws_bytes, stream), "sa_bwd")
+
+
+def sa_softmax_grad_preprocess(args: SaArgs, o: int, d_o: int, delta: int, stream: int = 0) -> None:
+    _check(lib().sa_softmax_grad_preprocess(ctypes.byref(args), o, d_o, delta, stream),
+           "sa_softmax_grad_preprocess")
+
+
+def sa_debug_resolve(args: SaArgs, rows: int, counts: int, max_rows: int, stream: int = 0) -> None:
+    _check(lib().sa_debug_resolve(ctypes.byref(args), rows, counts, max_rows, stream), "sa_debug_resolve")
+
+
+def sa_abi_version() -> int:
+    return int(lib().sa_abi_version())
+
+
+def sa_set_timing_events(ev_begin: int | None, ev_end: int | None) -> None:
+    lib().sa_set_timing_events(ev_begin, ev_end)
+
+
+def sa_kernel_launch_count() -> int:
+    return int(lib().sa_kernel_launch_count())

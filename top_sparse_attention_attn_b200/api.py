@@ -1,0 +1,198 @@
+"""Thin PyTorch-facing wrapper over the C ABI.
+
+`SparseAttention` holds the device tensors and attributes of one problem,
+marshals them into an `SaArgs`, allocates outputs and workspace with torch
+(device memory is PyTorch's job here) and calls `sa_fwd` / `sa_bwd`.  No
+arithmetic of the method happens in Python.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+from . import _lib as L
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else int(t.data_ptr())
+
+
+@dataclass
+class SparseAttention:
+    layout: str                  # "BSND" | "TND"
+    Hq: int
+    Hkv: int
+    d_qk: int
+    d_v: int
+    scale: float
+    q: torch.Tensor
+    k: torch.Tensor | None = None
+    v: torch.Tensor | None = None
+    kv: torch.Tensor | None = None
+    kv_shared: bool = False
+    batch: int = 1
+    s_q: int = 0
+    s_kv: int = 0
+    t_q: int = 0
+    t_kv: int = 0
+    t_cmp: int = 0
+    block_size: int = 1
+    ori_idx: torch.Tensor | None = None
+    ori_topk_len: torch.Tensor | None = None
+    cmp_kv: torch.Tensor | None = None
+    cmp_idx: torch.Tensor | None = None
+    cmp_topk_len: torch.Tensor | None = None
+    cmp_ratio: int = 1
+    cu_seqlens_q: torch.Tensor | None = None
+    cu_seqlens_kv: torch.Tensor | None = None
+    cu_seqlens_cmp: torch.Tensor | None = None
+    cmp_residual: torch.Tensor | None = None
+    sinks: torch.Tensor | None = None
+    ori_mask: str = "causal"
+    cmp_mask: str = "causal"
+    win_left: int = 0
+    win_right: int = 0
+    flags: int = 0
+    _keep: list = field(default_factory=list, repr=False)
+
+    # ---- marshalling -------------------------------------------------------
+    @property
+    def topk(self) -> int:
+        return 0 if self.ori_idx is None else int(self.ori_idx.shape[-1])
+
+    @property
+    def cmp_topk(self) -> int:
+        return 0 if self.cmp_idx is None else int(self.cmp_idx.shape[-1])
+
+    @property
+    def n_tokens(self) -> int:
+        return self.batch * self.s_q if self.layout == "BSND" else self.t_q
+
+    def args(self) -> L.SaArgs:
+        a = L.SaArgs()
+        a.layout = L.LAYOUTS[self.layout]
+        a.dtype = L.SA_DTYPE_BF16
+        a.batch = self.batch
+        a.s_q, a.s_kv = self.s_q, self.s_kv
+        a.t_q, a.t_kv, a.t_cmp = self.t_q, self.t_kv, self.t_cmp
+        a.n_heads_q, a.n_heads_kv = self.Hq, self.Hkv
+        a.d_qk, a.d_v = self.d_qk, self.d_v
+        a.kv_shared = 1 if self.kv_shared else 0
+        a.block_size = self.block_size
+        a.topk, a.cmp_topk = self.topk, self.cmp_topk
+        a.cmp_ratio = self.cmp_ratio
+        a.ori_mask_mode = L.MASKS[self.ori_mask]
+        a.cmp_mask_mode = L.MASKS[self.cmp_mask]
+        a.ori_win_left, a.ori_win_right = self.win_left, self.win_right
+        a.scale = self.scale
+        a.flags = self.flags
+        a.q, a.k, a.v, a.kv = _ptr(self.q), _ptr(self.k), _ptr(self.v), _ptr(self.kv)
+        a.cmp_kv = _ptr(self.cmp_kv)
+        a.ori_idx, a.cmp_idx = _ptr(self.ori_idx), _ptr(self.cmp_idx)
+        a.cu_seqlens_q, a.cu_seqlens_kv = _ptr(self.cu_seqlens_q), _ptr(self.cu_seqlens_kv)
+        a.cu_seqlens_cmp = _ptr(self.cu_seqlens_cmp)
+        a.ori_topk_len, a.cmp_topk_len = _ptr(self.ori_topk_len), _ptr(self.cmp_topk_len)
+        a.cmp_residual = _ptr(self.cmp_residual)
+        a.sinks = _ptr(self.sinks)
+        return a
+
+    # ---- allocation helpers ------------------------------------------------
+    def _lead(self) -> tuple:
+        return (self.batch, self.s_q) if self.layout == "BSND" else (self.t_q,)
+
+    def alloc_fwd(self):
+        dev = self.q.device
+        o = torch.empty(self._lead() + (self.Hq, self.d_v), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(self._lead() + (self.Hq,), dtype=torch.float32, device=dev)
+        return o, lse
+
+    def alloc_bwd(self) -> dict:
+        dev = self.q.device
+        g = {"dq": torch.empty_like(self.q)}
+        if self.kv_shared:
+            g["dkv"] = torch.empty_like(self.kv)
+        else:
+            g["dk"], g["dv"] = torch.empty_like(self.k), torch.empty_like(self.v)
+        if self.cmp_kv is not None:
+            g["dcmp"] = torch.empty_like(self.cmp_kv)
+        if self.sinks is not None:
+            g["dsinks"] = torch.empty(self.Hq, dtype=torch.float32, device=dev)
+        return g
+
+    def fwd_workspace(self) -> torch.Tensor:
+        n = L.sa_fwd_get_workspace_size(self.args())
+        return torch.empty(max(n, 1), dtype=torch.uint8, device=self.q.device)
+
+    def bwd_workspace(self) -> torch.Tensor:
+        n = L.sa_bwd_get_workspace_size(self.args())
+        return torch.empty(max(n, 1), dtype=torch.uint8, device=self.q.device)
+
+    # ---- calls -------------------------------------------------------------
+    def forward(self, o=None, lse=None, ws=None, stream=None):
+        if o is None:
+            o, lse = self.alloc_fwd()
+        if ws is None:
+            ws = self.fwd_workspace()
+        out = L.SaFwdOut(o=_ptr(o), lse=_ptr(lse))
+        st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+        L.sa_fwd(self.args(), out, _ptr(ws), ws.numel(), st)
+        return o, lse
+
+    def backward(self, o, lse, d_o, grads=None, ws=None, stream=None) -> dict:
+        if grads is None:
+            grads = self.alloc_bwd()
+        if ws is None:
+            ws = self.bwd_workspace()
+        io = L.SaBwdIo(o=_ptr(o), d_o=_ptr(d_o), lse=_ptr(lse), dq=_ptr(grads["dq"]),
+                       dk=_ptr(grads.get("dk")), dv=_ptr(grads.get("dv")),
+                       dkv=_ptr(grads.get("dkv")), dcmp_kv=_ptr(grads.get("dcmp")),
+                       dsinks=_ptr(grads.get("dsinks")))
+        st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+        L.sa_bwd(self.args(), io, _ptr(ws), ws.numel(), st)
+        return grads
+
+    def delta(self, o, d_o, stream=None) -> torch.Tensor:
+        out = torch.empty(self._lead() + (self.Hq,), dtype=torch.float32, device=self.q.device)
+        st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+        L.sa_softmax_grad_preprocess(self.args(), _ptr(o), _ptr(d_o), _ptr(out), st)
+        return out
+
+    def debug_resolve(self, max_rows: int, stream=None):
+        n_units = self.n_tokens * self.Hkv
+        rows = torch.full((n_units, max(max_rows, 1)), -1, dtype=torch.int32, device=self.q.device)
+        counts = torch.zeros(n_units, dtype=torch.int32, device=self.q.device)
+        st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+        L.sa_debug_resolve(self.args(), _ptr(rows), _ptr(counts), max_rows, st)
+        return rows, counts
+
+    # ---- construction from a workload description ---------------------------
+    @classmethod
+    def from_workload(cls, w, t: dict, flags: int = 0) -> "SparseAttention":
+        """``w``: an object with the workload attributes (see gen.configs.Workload);
+        ``t``: device tensors keyed like the generator's arrays (bf16 as torch.bfloat16)."""
+        kw = dict(layout=w.layout, Hq=w.Hq, Hkv=w.Hkv, d_qk=w.d_qk, d_v=w.d_v, scale=w.scale,
+                  q=t["q"], kv_shared=w.kv_shared, block_size=w.block_size,
+                  cmp_ratio=w.cmp_ratio, ori_mask=w.ori_mask, cmp_mask=w.cmp_mask,
+                  win_left=w.win_left, win_right=w.win_right, flags=flags)
+        if w.kv_shared:
+            kw["kv"] = t["kv"]
+        else:
+            kw["k"], kw["v"] = t["k"], t["v"]
+        for key in ("ori_idx", "ori_topk_len", "cmp_kv", "cmp_idx", "cmp_topk_len",
+                    "cu_seqlens_q", "cu_seqlens_kv", "cu_seqlens_cmp", "cmp_residual", "sinks"):
+            if key in t:
+                kw[key] = t[key]
+        if w.layout == "BSND":
+            kw.update(batch=w.B, s_q=w.S, s_kv=w.S)
+        else:
+            T = sum(w.seqlens)
+            kw.update(batch=len(w.seqlens), t_q=T, t_kv=T,
+                      t_cmp=int(t["cmp_kv"].shape[0]) if "cmp_kv" in t else 0)
+        return cls(**kw)
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,316 @@
+// sa_api.cu -- the extern "C" entry points declared in include/sparse_attn.h:
+// host-side argument validation, workspace sizing and kernel dispatch.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/sparse_attn.h"
+#include "sa_device.cuh"
+#include "sa_launch.h"
+
+namespace {
+
+using sa::bf16;
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Sizes {
+  long long Tq, Tkv, Tcmp;
+};
+
+Sizes sizes_of(const sa_args* a) {
+  Sizes s;
+  if (a->layout == SA_LAYOUT_BSND) {
+    s.Tq = (long long)a->batch * a->s_q;
+    s.Tkv = (long long)a->batch * a->s_kv;
+    s.Tcmp = a->cmp_topk > 0 ? (long long)a->batch * (a->s_kv / (a->cmp_ratio > 0 ? a->cmp_ratio : 1)) : 0;
+  } else {
+    s.Tq = a->t_q;
+    s.Tkv = a->t_kv;
+    s.Tcmp = a->cmp_topk > 0 ? a->t_cmp : 0;
+  }
+  return s;
+}
+
+sa_status validate(const sa_args* a) {
+  if (!a) return SA_ERR_NULLPTR;
+  if (a->dtype == SA_DTYPE_FP16) return SA_ERR_UNSUPPORTED;
+  if (a->dtype != SA_DTYPE_BF16) return SA_ERR_PARAM;
+  if (a->layout != SA_LAYOUT_BSND && a->layout != SA_LAYOUT_TND) return SA_ERR_PARAM;
+  if (a->batch < 0) return SA_ERR_PARAM;
+  if (a->layout == SA_LAYOUT_BSND) {
+    if (a->s_q < 0 || a->s_kv < 0) return SA_ERR_PARAM;
+  } else {
+    if (a->t_q < 0 || a->t_kv < 0 || a->t_cmp < 0) return SA_ERR_PARAM;
+  }
+  if (a->n_heads_q < 1 || a->n_heads_kv < 1 || a->n_heads_q % a->n_heads_kv) return SA_ERR_PARAM;
+  if (a->d_qk < 16 || a->d_v < 16 || a->d_qk % 16 || a->d_v % 16) return SA_ERR_PARAM;
+  if (a->d_qk > 576 || a->d_v > 512) return SA_ERR_PARAM;
+  if (a->kv_shared && a->d_v > a->d_qk) return SA_ERR_PARAM;
+  if (a->block_size < 1 || (a->block_size > sa::kTileRows && a->block_size % sa::kTileRows)) return SA_ERR_PARAM;
+  if (a->topk < 0 || a->cmp_topk < 0) return SA_ERR_PARAM;
+  if (a->cmp_ratio < 1) return SA_ERR_PARAM;
+  if (a->ori_mask_mode < SA_MASK_NONE || a->ori_mask_mode > SA_MASK_BAND) return SA_ERR_PARAM;
+  if (a->cmp_mask_mode != SA_MASK_NONE && a->cmp_mask_mode != SA_MASK_CAUSAL) return SA_ERR_PARAM;
+  if (a->ori_mask_mode == SA_MASK_BAND && (a->ori_win_left < 0 || a->ori_win_right < 0)) return SA_ERR_PARAM;
+  if (!isfinite(a->scale)) return SA_ERR_PARAM;
+  Sizes s = sizes_of(a);
+  if (s.Tq >= (1ll << 30) || s.Tkv >= (1ll << 30) || s.Tcmp >= (1ll << 30)) return SA_ERR_PARAM;
+  const int G = a->n_heads_q / a->n_heads_kv;
+  if (s.Tq * a->n_heads_kv * ((G + 15) / 16) >= (1ll << 31)) return SA_ERR_PARAM;
+  // pointers
+  if (s.Tq > 0) {
+    if (!a->q) return SA_ERR_NULLPTR;
+    if (a->kv_shared ? !a->kv : (!a->k || !a->v)) return SA_ERR_NULLPTR;
+    if (a->topk > 0 && !a->ori_idx) return SA_ERR_NULLPTR;
+    if (a->cmp_topk > 0 && (!a->cmp_kv || !a->cmp_idx)) return SA_ERR_NULLPTR;
+    if (a->layout == SA_LAYOUT_TND) {
+      if (!a->cu_seqlens_q || !a->cu_seqlens_kv) return SA_ERR_NULLPTR;
+      if (a->cmp_topk > 0 && !a->cu_seqlens_cmp) return SA_ERR_NULLPTR;
+      if (a->batch < 1) return SA_ERR_PARAM;
+    }
+  }
+  // combinations that are valid on the pages but not built here
+  if (a->cmp_topk > 0 && !a->kv_shared) return SA_ERR_UNSUPPORTED;
+  if (!sa::kernels_built(a->d_qk, a->d_v, a->kv_shared != 0)) return SA_ERR_UNSUPPORTED;
+  return SA_OK;
+}
+
+sa::Prob make_prob(const sa_args* a, int* status) {
+  sa::Prob p;
+  memset(&p, 0, sizeof(p));
+  Sizes s = sizes_of(a);
+  p.layout = a->layout;
+  p.B = a->batch;
+  p.s_q = a->s_q;
+  p.s_kv = a->s_kv;
+  p.Tq = (int)s.Tq;
+  p.Tkv = (int)s.Tkv;
+  p.Tcmp = (int)s.Tcmp;
+  p.Hq = a->n_heads_q;
+  p.Hkv = a->n_heads_kv;
+  p.G = a->n_heads_q / a->n_heads_kv;
+  p.dqk = a->d_qk;
+  p.dv = a->d_v;
+  p.shared = a->kv_shared ? 1 : 0;
+  p.bs = a->block_size;
+  p.topk = a->topk;
+  p.cmp_topk = a->cmp_topk;
+  p.ratio = a->cmp_ratio;
+  p.ori_mask = a->ori_mask_mode;
+  p.cmp_mask = a->cmp_mask_mode;
+  p.wl = a->ori_win_left;
+  p.wr = a->ori_win_right;
+  p.scale = a->scale;
+  p.scale_log2 = a->scale * 1.4426950408889634f;
+  p.q = static_cast<const bf16*>(a->q);
+  if (a->kv_shared) {
+    p.k = static_cast<const bf16*>(a->kv);
+    p.v = static_cast<const bf16*>(a->kv);
+  } else {
+    p.k = static_cast<const bf16*>(a->k);
+    p.v = static_cast<const bf16*>(a->v);
+  }
+  p.cmpk = a->cmp_topk > 0 ? static_cast<const bf16*>(a->cmp_kv) : nullptr;
+  p.ori_idx = a->topk > 0 ? a->ori_idx : nullptr;
+  p.cmp_idx = a->cmp_topk > 0 ? a->cmp_idx : nullptr;
+  p.cu_q = a->cu_seqlens_q;
+  p.cu_kv = a->cu_seqlens_kv;
+  p.cu_cmp = a->cu_seqlens_cmp;
+  p.ori_len = a->topk > 0 ? a->ori_topk_len : nullptr;
+  p.cmp_len = a->cmp_topk > 0 ? a->cmp_topk_len : nullptr;
+  p.sinks = a->sinks;
+  p.status = status;
+  return p;
+}
+
+bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15u) == 0; }
+
+sa_status check_tensor_alignment(const sa_args* a) {
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->kv) ||
+      !aligned16(a->cmp_kv))
+    return SA_ERR_PARAM;
+  return SA_OK;
+}
+
+// Workspace: [status word][delta][dK or dKV acc][dV acc][dCmp acc]
+struct BwdWs {
+  size_t status, delta, dk, dv, dcmp, total;
+};
+
+BwdWs bwd_ws_layout(const sa_args* a) {
+  Sizes s = sizes_of(a);
+  BwdWs w;
+  size_t off = 0;
+  w.status = off;
+  off += kAlign;
+  w.delta = off;
+  off += align_up((size_t)s.Tq * a->n_heads_q * sizeof(float));
+  w.dk = off;
+  off += align_up((size_t)s.Tkv * a->n_heads_kv * a->d_qk * sizeof(float));
+  w.dv = off;
+  if (!a->kv_shared) off += align_up((size_t)s.Tkv * a->n_heads_kv * a->d_v * sizeof(float));
+  w.dcmp = off;
+  off += align_up((size_t)s.Tcmp * a->n_heads_kv * a->d_qk * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+sa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
+
+// SA_FLAG_CHECK: validate every usable index on the device, synchronously.
+sa_status run_check(const sa_args* a, int* status, cudaStream_t st) {
+  sa::Prob p = make_prob(a, status);
+  if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return SA_ERR_CUDA;
+  if (sa::launch_check(p, st) != cudaSuccess) return SA_ERR_CUDA;
+  int host = 0;
+  if (cudaMemcpyAsync(&host, status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SA_ERR_CUDA;
+  return (host & sa::kStatusIndexRange) ? SA_ERR_INDEX : SA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t sa_abi_version(void) { return SA_ABI_VERSION; }
+
+void sa_set_timing_events(void* ev_begin, void* ev_end) {
+  sa::g_ev_begin = static_cast<cudaEvent_t>(ev_begin);
+  sa::g_ev_end = static_cast<cudaEvent_t>(ev_end);
+}
+
+int64_t sa_kernel_launch_count(void) { return __atomic_load_n(&sa::g_launches, __ATOMIC_RELAXED); }
+
+const char* sa_status_string(int32_t s) {
+  switch (s) {
+    case SA_OK: return "SA_OK";
+    case SA_ERR_NULLPTR: return "SA_ERR_NULLPTR: a required pointer is NULL";
+    case SA_ERR_PARAM: return "SA_ERR_PARAM: a size, mode or attribute is out of range";
+    case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED: combination not built";
+    case SA_ERR_WORKSPACE: return "SA_ERR_WORKSPACE: workspace missing or too small";
+    case SA_ERR_INDEX: return "SA_ERR_INDEX: an index lies past its sequence";
+    case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT: a bounded device wait gave up";
+    case SA_ERR_CUDA: return "SA_ERR_CUDA: CUDA runtime error";
+    default: return "unknown sa_status";
+  }
+}
+
+sa_status sa_fwd_get_workspace_size(const sa_args* args, size_t* ws_bytes) {
+  if (!ws_bytes) return SA_ERR_NULLPTR;
+  sa_status st = validate(args);
+  if (st != SA_OK) return st;
+  *ws_bytes = kAlign;  // status word
+  return SA_OK;
+}
+
+sa_status sa_fwd(const sa_args* args, const sa_fwd_out* out, void* ws, size_t ws_bytes, void* stream) {
+  sa_status st = validate(args);
+  if (st != SA_OK) return st;
+  if (!out) return SA_ERR_NULLPTR;
+  Sizes s = sizes_of(args);
+  if (s.Tq == 0) return SA_OK;
+  if (!out->o || !out->lse) return SA_ERR_NULLPTR;
+  if (!ws || ws_bytes < kAlign) return SA_ERR_WORKSPACE;
+  if (check_tensor_alignment(args) != SA_OK || !aligned16(out->o)) return SA_ERR_PARAM;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  if (args->flags & SA_FLAG_CHECK) {
+    st = run_check(args, status, cs);
+    if (st != SA_OK) return st;
+  }
+  sa::Prob p = make_prob(args, status);
+  if (cudaMemsetAsync(status, 0, sizeof(int), cs) != cudaSuccess) return SA_ERR_CUDA;
+  return cuda_status(sa::launch_fwd(p, static_cast<bf16*>(out->o), out->lse, cs));
+}
+
+sa_status sa_bwd_get_workspace_size(const sa_args* args, size_t* ws_bytes) {
+  if (!ws_bytes) return SA_ERR_NULLPTR;
+  sa_status st = validate(args);
+  if (st != SA_OK) return st;
+  *ws_bytes = bwd_ws_layout(args).total;
+  return SA_OK;
+}
+
+sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_bytes, void* stream) {
+  sa_status st = validate(args);
+  if (st != SA_OK) return st;
+  if (!io) return SA_ERR_NULLPTR;
+  Sizes s = sizes_of(args);
+  const bool sinks = args->sinks != nullptr;
+  if (s.Tq == 0) return SA_OK;
+  if (!io->o || !io->d_o || !io->lse || !io->dq) return SA_ERR_NULLPTR;
+  if (args->kv_shared ? !io->dkv : (!io->dk || !io->dv)) return SA_ERR_NULLPTR;
+  if (args->cmp_topk > 0 && !io->dcmp_kv) return SA_ERR_NULLPTR;
+  if (sinks && !io->dsinks) return SA_ERR_NULLPTR;
+  BwdWs w = bwd_ws_layout(args);
+  if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
+  if (check_tensor_alignment(args) != SA_OK || !aligned16(io->o) || !aligned16(io->d_o) ||
+      !aligned16(io->dq) || !aligned16(io->dk) || !aligned16(io->dv) || !aligned16(io->dkv) ||
+      !aligned16(io->dcmp_kv))
+    return SA_ERR_PARAM;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(ws);
+  int* status = reinterpret_cast<int*>(base + w.status);
+  if (args->flags & SA_FLAG_CHECK) {
+    st = run_check(args, status, cs);
+    if (st != SA_OK) return st;
+  }
+  sa::Prob p = make_prob(args, status);
+  float* delta = reinterpret_cast<float*>(base + w.delta);
+  sa::BwdOut out;
+  out.dq = static_cast<bf16*>(io->dq);
+  out.dk_acc = reinterpret_cast<float*>(base + w.dk);
+  out.dv_acc = args->kv_shared ? nullptr : reinterpret_cast<float*>(base + w.dv);
+  out.dcmp_acc = args->cmp_topk > 0 ? reinterpret_cast<float*>(base + w.dcmp) : nullptr;
+  out.dsinks = sinks ? io->dsinks : nullptr;
+  const long long nk = s.Tkv * args->n_heads_kv * args->d_qk;
+  const long long nv = s.Tkv * args->n_heads_kv * args->d_v;
+  const long long nc = s.Tcmp * args->n_heads_kv * args->d_qk;
+  // zero the accumulators (one contiguous range) and dSinks
+  if (cudaMemsetAsync(base, 0, w.total, cs) != cudaSuccess) return SA_ERR_CUDA;
+  if (sinks && cudaMemsetAsync(io->dsinks, 0, sizeof(float) * args->n_heads_q, cs) != cudaSuccess)
+    return SA_ERR_CUDA;
+  cudaError_t e = sa::launch_delta(static_cast<const bf16*>(io->o), static_cast<const bf16*>(io->d_o), delta,
+                                   s.Tq * args->n_heads_q, args->d_v, cs);
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+  e = sa::launch_bwd(p, static_cast<const bf16*>(io->o), static_cast<const bf16*>(io->d_o), io->lse, delta,
+                     out, cs);
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+  if (args->kv_shared) {
+    e = sa::launch_to_bf16(out.dk_acc, static_cast<bf16*>(io->dkv), nk, cs);
+  } else {
+    e = sa::launch_to_bf16(out.dk_acc, static_cast<bf16*>(io->dk), nk, cs);
+    if (e == cudaSuccess) e = sa::launch_to_bf16(out.dv_acc, static_cast<bf16*>(io->dv), nv, cs);
+  }
+  if (e == cudaSuccess && args->cmp_topk > 0)
+    e = sa::launch_to_bf16(out.dcmp_acc, static_cast<bf16*>(io->dcmp_kv), nc, cs);
+  return cuda_status(e);
+}
+
+sa_status sa_softmax_grad_preprocess(const sa_args* args, const void* o, const void* d_o, float* delta,
+                                     void* stream) {
+  sa_status st = validate(args);
+  if (st != SA_OK) return st;
+  Sizes s = sizes_of(args);
+  if (s.Tq == 0) return SA_OK;
+  if (!o || !d_o || !delta) return SA_ERR_NULLPTR;
+  if (!aligned16(o) || !aligned16(d_o)) return SA_ERR_PARAM;
+  return cuda_status(sa::launch_delta(static_cast<const bf16*>(o), static_cast<const bf16*>(d_o), delta,
+                                      s.Tq * args->n_heads_q, args->d_v, static_cast<cudaStream_t>(stream)));
+}
+
+sa_status sa_debug_resolve(const sa_args* args, int32_t* rows, int32_t* counts, int32_t max_rows, void* stream) {
+  sa_status st = validate(args);
+  if (st != SA_OK) return st;
+  if (max_rows < 0) return SA_ERR_PARAM;
+  Sizes s = sizes_of(args);
+  if (s.Tq == 0) return SA_OK;
+  if (!counts || (max_rows > 0 && !rows)) return SA_ERR_NULLPTR;
+  sa::Prob p = make_prob(args, nullptr);
+  return cuda_status(sa::launch_debug_resolve(p, rows, counts, max_rows, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,295 @@
+// sa_device.cuh -- device-side problem description, selection (Stage 1) and
+// warp-level MMA helpers shared by the sparse-attention kernels.
+//
+// Selection follows aclnnSparseFlashAttentionGrad "Formula" (block Gather
+// through topkIndices) and SparseFlashMlaGrad "Computation formula" Stage 1
+// (original KV, optionally through token indices, concatenated with gathered
+// compressed KV), with the masks and topk lengths of the SparseFlashMlaGrad
+// "Parameter Description" table.  Every (query token, kv-head) "unit" sees a
+// list of tiles; a tile is 64 KV rows, each resolved to a global row code or
+// to -1 (invisible).  Row codes: original-KV row -> its global row number;
+// compressed row -> kCmpFlag | global compressed row.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sa {
+
+typedef __nv_bfloat16 bf16;
+
+constexpr int kTileRows = 64;
+constexpr int kCmpFlag = 0x40000000;
+
+enum { kLayoutBSND = 0, kLayoutTND = 1 };
+enum { kMaskNone = 0, kMaskCausal = 1, kMaskBand = 2 };
+enum { kOriNone = 0, kOriBlock = 1, kOriToken = 2, kOriRange = 3 };
+
+// Status bits written by kernels into the workspace status word.
+enum { kStatusIndexRange = 1, kStatusTimeout = 2 };
+
+struct Prob {
+  int layout, B, s_q, s_kv;
+  int Tq, Tkv, Tcmp;
+  int Hq, Hkv, G, dqk, dv, shared, bs, topk, cmp_topk, ratio, ori_mask, cmp_mask;
+  long long wl, wr;
+  float scale;        // scaleValue
+  float scale_log2;   // scale * log2(e)
+  const bf16* q;
+  const bf16* k;      // K (or the shared KV)
+  const bf16* v;      // V (or the shared KV)
+  const bf16* cmpk;   // compressed KV (K = V)
+  const int* ori_idx;
+  const int* cmp_idx;
+  const int* cu_q;
+  const int* cu_kv;
+  const int* cu_cmp;
+  const int* ori_len;
+  const int* cmp_len;
+  const float* sinks;
+  int* status;        // device status word (may be null)
+};
+
+struct Unit {
+  int tq, g, b, t, ta, Lk, Lc, kv0, cmp0;
+  int ori_mode, n_ori_slots, n_cmp_slots, lo, hi, tps;
+  int n_ori_tiles, n_tiles;
+};
+
+__device__ __forceinline__ int find_batch(const int* cu, int B, int tq) {
+  int lo = 0, hi = B - 1;  // largest b with cu[b] <= tq
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu + mid) <= tq) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ Unit make_unit(const Prob& p, int tq, int g) {
+  Unit u;
+  u.tq = tq;
+  u.g = g;
+  int Lq;
+  if (p.layout == kLayoutBSND) {
+    u.b = tq / p.s_q;
+    u.t = tq - u.b * p.s_q;
+    Lq = p.s_q;
+    u.Lk = p.s_kv;
+    u.kv0 = u.b * p.s_kv;
+    u.Lc = p.cmp_topk > 0 ? p.s_kv / p.ratio : 0;
+    u.cmp0 = u.b * u.Lc;
+  } else {
+    // offsets are clamped to the packed extents, so inconsistent cu_seqlens can
+    // shrink a sequence but never make a kernel read outside its tensors
+    u.b = find_batch(p.cu_q, p.B, tq);
+    int q0 = __ldg(p.cu_q + u.b);
+    Lq = max(__ldg(p.cu_q + u.b + 1) - q0, 0);
+    u.t = tq - q0;
+    u.kv0 = min(max(__ldg(p.cu_kv + u.b), 0), p.Tkv);
+    u.Lk = min(max(__ldg(p.cu_kv + u.b + 1), u.kv0), p.Tkv) - u.kv0;
+    if (p.cmp_topk > 0) {
+      u.cmp0 = min(max(__ldg(p.cu_cmp + u.b), 0), p.Tcmp);
+      u.Lc = min(max(__ldg(p.cu_cmp + u.b + 1), u.cmp0), p.Tcmp) - u.cmp0;
+    } else {
+      u.cmp0 = 0;
+      u.Lc = 0;
+    }
+  }
+  u.ta = u.t + u.Lk - Lq;
+  const long long ug = (long long)tq * p.Hkv + g;
+  u.tps = 1;
+  u.lo = 0;
+  u.hi = -1;
+  if (p.topk > 0) {
+    int n = p.topk;
+    if (p.ori_len) n = min(n, max(0, __ldg(p.ori_len + ug)));
+    u.n_ori_slots = n;
+    if (p.bs > 1) {
+      u.ori_mode = kOriBlock;
+      u.tps = (p.bs + kTileRows - 1) / kTileRows;
+      u.n_ori_tiles = n * u.tps;
+    } else {
+      u.ori_mode = kOriToken;
+      u.n_ori_tiles = (n + kTileRows - 1) / kTileRows;
+    }
+  } else {
+    u.ori_mode = kOriRange;
+    u.n_ori_slots = 0;
+    long long lo = 0, hi = (long long)u.Lk - 1;
+    if (p.ori_mask == kMaskCausal) {
+      hi = min(hi, (long long)u.ta);
+    } else if (p.ori_mask == kMaskBand) {
+      lo = max(lo, (long long)u.ta - p.wl);
+      hi = min(hi, (long long)u.ta + p.wr);
+    }
+    if (hi < lo) { lo = 0; hi = -1; }
+    u.lo = (int)lo;
+    u.hi = (int)hi;
+    u.n_ori_tiles = (int)((hi - lo + 1 + kTileRows - 1) / kTileRows);
+  }
+  if (p.cmp_topk > 0) {
+    int n = p.cmp_topk;
+    if (p.cmp_len) n = min(n, max(0, __ldg(p.cmp_len + ug)));
+    u.n_cmp_slots = n;
+  } else {
+    u.n_cmp_slots = 0;
+  }
+  u.n_tiles = u.n_ori_tiles + (u.n_cmp_slots + kTileRows - 1) / kTileRows;
+  return u;
+}
+
+__device__ __forceinline__ bool ori_mask_ok(const Prob& p, const Unit& u, int r) {
+  if (p.ori_mask == kMaskCausal) return r <= u.ta;
+  if (p.ori_mask == kMaskBand) return (long long)r >= (long long)u.ta - p.wl && (long long)r <= (long long)u.ta + p.wr;
+  return true;
+}
+
+// True when a tile (ori block slot) is empty before looking at its rows; lets
+// callers skip whole slots cheaply.  Only used as a hint.
+__device__ __forceinline__ bool tile_is_empty_slot(const Prob& p, const Unit& u, int tile) {
+  if (tile < u.n_ori_tiles && u.ori_mode == kOriBlock) {
+    int s = tile / u.tps;
+    int x = __ldg(p.ori_idx + ((long long)u.tq * p.Hkv + u.g) * p.topk + s);
+    return x < 0;
+  }
+  return false;
+}
+
+// Resolve row r (0..63) of tile `tile` of unit u to a global row code, or -1.
+__device__ __forceinline__ int resolve_row(const Prob& p, const Unit& u, int tile, int r) {
+  if (tile < u.n_ori_tiles) {
+    const long long ug = (long long)u.tq * p.Hkv + u.g;
+    if (u.ori_mode == kOriBlock) {
+      int s = tile / u.tps, sub = tile - s * u.tps;
+      int x = __ldg(p.ori_idx + ug * p.topk + s);
+      if (x < 0) return -1;
+      int within = sub * kTileRows + r;
+      if (within >= p.bs) return -1;
+      long long first = (long long)x * p.bs;
+      if (first >= u.Lk) {
+        if (p.status && r == 0 && sub == 0) atomicOr(p.status, kStatusIndexRange);
+        return -1;
+      }
+      long long row = first + within;
+      if (row >= u.Lk || !ori_mask_ok(p, u, (int)row)) return -1;
+      return u.kv0 + (int)row;
+    } else if (u.ori_mode == kOriToken) {
+      int s = tile * kTileRows + r;
+      if (s >= u.n_ori_slots) return -1;
+      int x = __ldg(p.ori_idx + ug * p.topk + s);
+      if (x < 0) return -1;
+      if (x >= u.Lk) {
+        if (p.status) atomicOr(p.status, kStatusIndexRange);
+        return -1;
+      }
+      if (!ori_mask_ok(p, u, x)) return -1;
+      return u.kv0 + x;
+    } else {
+      int row = u.lo + tile * kTileRows + r;
+      if (row > u.hi) return -1;
+      return u.kv0 + row;
+    }
+  }
+  int s = (tile - u.n_ori_tiles) * kTileRows + r;
+  if (s >= u.n_cmp_slots) return -1;
+  const long long ug = (long long)u.tq * p.Hkv + u.g;
+  int c = __ldg(p.cmp_idx + ug * p.cmp_topk + s);
+  if (c < 0) return -1;
+  if (c >= u.Lc) {
+    if (p.status) atomicOr(p.status, kStatusIndexRange);
+    return -1;
+  }
+  if (p.cmp_mask == kMaskCausal && (long long)(c + 1) * p.ratio - 1 > u.ta) return -1;
+  return kCmpFlag | (u.cmp0 + c);
+}
+
+// Element offsets of a row's K and V vectors (kv-head g) for a row code >= 0.
+__device__ __forceinline__ const bf16* row_k_ptr(const Prob& p, int code, int g) {
+  if (code & kCmpFlag) return p.cmpk + ((long long)(code & ~kCmpFlag) * p.Hkv + g) * p.dqk;
+  return p.k + ((long long)code * p.Hkv + g) * p.dqk;
+}
+__device__ __forceinline__ const bf16* row_v_ptr(const Prob& p, int code, int g) {
+  if (code & kCmpFlag) return p.cmpk + ((long long)(code & ~kCmpFlag) * p.Hkv + g) * p.dqk;
+  if (p.shared) return p.k + ((long long)code * p.Hkv + g) * p.dqk;
+  return p.v + ((long long)code * p.Hkv + g) * p.dv;
+}
+
+// ---------------------------------------------------------------------------
+// shared-memory tiles: rows of D bf16 (D % 64 == 0), 16-byte chunks XOR-swizzled
+// by (row & 7) so ldmatrix phases hit distinct banks.
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ uint32_t swz(uint32_t base, int row, int chunk) {
+  return base + (uint32_t)(row * D * 2) + (uint32_t)(((chunk ^ (row & 7))) << 4);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  int n = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// A fragment (16 x 16) at rows r0.., k-chunk kc (k0 = 8*kc) of a row-major swizzled tile.
+template <int D>
+__device__ __forceinline__ void load_a(uint32_t (&a)[4], uint32_t base, int r0, int kc, int lane) {
+  ldsm_x4(a, swz<D>(base, r0 + (lane & 15), kc + (lane >> 4)));
+}
+// B fragments for two n-tiles (rows n0..n0+15 of a row-major [N][D] tile, B[k][n] = T[n][k]),
+// k-chunk kc: b[0],b[1] -> n-tile n0; b[2],b[3] -> n-tile n0+8.
+template <int D>
+__device__ __forceinline__ void load_b_nk(uint32_t (&b)[4], uint32_t base, int n0, int kc, int lane) {
+  ldsm_x4(b, swz<D>(base, n0 + (lane & 7) + ((lane >> 4) << 3), kc + ((lane >> 3) & 1)));
+}
+// B fragments for two n-tiles from a row-major [K][D] tile with B[k][n] = T[k][n]
+// (k rows k0..k0+15, columns n-chunk nc and nc+1).
+template <int D>
+__device__ __forceinline__ void load_b_kn(uint32_t (&b)[4], uint32_t base, int k0, int nc, int lane) {
+  ldsm_x4_t(b, swz<D>(base, k0 + (lane & 7) + (((lane >> 3) & 1) << 3), nc + (lane >> 4)));
+}
+// A fragment of the transpose: A[m][k] = T[k][m] from a row-major [K][D] tile,
+// m rows from column-chunk mc (m0 = 8*mc), k rows k0..k0+15.
+template <int D>
+__device__ __forceinline__ void load_a_t(uint32_t (&a)[4], uint32_t base, int k0, int mc, int lane) {
+  ldsm_x4_t(a, swz<D>(base, k0 + (lane & 7) + ((lane >> 4) << 3), mc + ((lane >> 3) & 1)));
+}
+
+__device__ __forceinline__ float warp_max4(float v) {
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+  return v;
+}
+__device__ __forceinline__ float warp_sum4(float v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  return v;
+}
+
+}  // namespace sa
