@@ -178,6 +178,29 @@ sa_status sa_bwd_get_workspace_size(const sa_args* args, size_t* ws_bytes);
 sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_bytes,
                  void* stream);
 
+/* The backward pass for callers that cannot allocate device memory.  The
+ * pages have no counterpart to this entry point.  Some callers cannot call
+ * cudaMalloc where they run the backward: a plugin whose host framework owns
+ * all device memory through its own pre-reserved pool and forbids allocation
+ * during execution, or a latency-critical loop that cannot absorb the device
+ * synchronisation an allocation implies.  This entry point needs no
+ * workspace: it runs sa_bwd on a fixed scratch array compiled into the
+ * library (sa_bwd_no_alloc_max_workspace() bytes, held on every GPU that loads
+ * the library until the process exits) and allocates nothing.
+ *   - Problems whose sa_bwd_get_workspace_size exceeds that size are rejected
+ *     with SA_ERR_WORKSPACE before anything is enqueued.
+ *   - The first call on a device (with that device current) resolves the
+ *     array's device address once; make that first call before any stream
+ *     capture.
+ *   - All calls share the one array: calls whose work overlaps on the GPU
+ *     (other streams, other host threads on the same device) race.  Each call
+ *     re-zeroes the parts it uses, so nothing carries over between calls.
+ * Inputs, outputs and errors are as for sa_bwd.  Asynchronous. */
+sa_status sa_bwd_no_alloc(const sa_args* args, const sa_bwd_io* io, void* stream);
+
+/* Size in bytes of the scratch array behind sa_bwd_no_alloc. */
+size_t sa_bwd_no_alloc_max_workspace(void);
+
 /* rowsum(dO o O) alone -- the "FlashSoftmaxGrad(dO, O)" / "SoftmaxGrad(dO, O)"
  * term of aclnnSparseFlashAttentionGrad Phase 2 and SparseFlashMlaGrad Stage 2:
  * delta[token, h] = sum_c d_o[token, h, c] * o[token, h, c] in fp32.

@@ -178,7 +178,7 @@ def test_calls_fail_before_launch():
 
 
 def test_empty_query_is_a_no_op():
-    """An empty query returns directly (the pages: 'If the query is an empty Tensor: return directly')."""
+    """An empty query is a successful no-op (aclnnSparseFlashAttentionGrad, Constraints, empty inputs)."""
     a = _args(s_q=0)
     out = L.SaFwdOut(o=None, lse=None)
     assert L.lib().sa_fwd(ctypes.byref(a), ctypes.byref(out), None, 0, None) == L.SA_OK
@@ -187,3 +187,14 @@ def test_empty_query_is_a_no_op():
     a = _args(batch=0)
     assert L.lib().sa_fwd(ctypes.byref(a), ctypes.byref(out), None, 0, None) == L.SA_OK
     assert L.lib().sa_softmax_grad_preprocess(ctypes.byref(a), None, None, None, None) == L.SA_OK
+
+
+def test_no_alloc_rejects_oversized_problem_on_the_host():
+    """sa_bwd_no_alloc refuses problems whose workspace exceeds its fixed scratch."""
+    cap = L.sa_bwd_no_alloc_max_workspace()
+    assert cap >= 1 << 20
+    a = _args(batch=8, s_q=8192, s_kv=8192)                 # ~ hundreds of MB of accumulators
+    assert _ws(a)[1] > cap
+    io = L.SaBwdIo(o=FAKE, d_o=FAKE, lse=FAKE, dq=FAKE, dk=FAKE, dv=FAKE)
+    assert L.lib().sa_bwd_no_alloc(ctypes.byref(a), ctypes.byref(io), None) == L.SA_ERR_WORKSPACE
+    assert L.lib().sa_bwd_no_alloc(ctypes.byref(_args(n_heads_q=15)), ctypes.byref(io), None) == L.SA_ERR_PARAM

@@ -77,7 +77,8 @@ _lib = None
 # every symbol include/sparse_attn.h declares
 EXPORTS = ["sa_fwd_get_workspace_size", "sa_fwd", "sa_bwd_get_workspace_size", "sa_bwd",
            "sa_softmax_grad_preprocess", "sa_debug_resolve", "sa_status_string", "sa_abi_version",
-           "sa_set_timing_events", "sa_kernel_launch_count"]
+           "sa_set_timing_events", "sa_kernel_launch_count", "sa_bwd_no_alloc",
+           "sa_bwd_no_alloc_max_workspace"]
 
 
 def lib() -> ctypes.CDLL:
@@ -102,8 +103,12 @@ def lib() -> ctypes.CDLL:
         L.sa_set_timing_events.restype = None
         L.sa_kernel_launch_count.argtypes = []
         L.sa_kernel_launch_count.restype = ctypes.c_int64
+        L.sa_bwd_no_alloc.argtypes = [P(SaArgs), P(SaBwdIo), _vp]
+        L.sa_bwd_no_alloc_max_workspace.argtypes = []
+        L.sa_bwd_no_alloc_max_workspace.restype = ctypes.c_size_t
         for name in EXPORTS:
-            if name not in ("sa_status_string", "sa_set_timing_events", "sa_kernel_launch_count"):
+            if name not in ("sa_status_string", "sa_set_timing_events", "sa_kernel_launch_count",
+                            "sa_bwd_no_alloc_max_workspace"):
                 getattr(L, name).restype = ctypes.c_int32
         _lib = L
     return _lib
@@ -138,6 +143,15 @@ def sa_bwd_get_workspace_size(args: SaArgs) -> int:
 
 def sa_bwd(args: SaArgs, io: SaBwdIo, ws: int, ws_bytes: int, stream: int = 0) -> None:
     _check(lib().sa_bwd(ctypes.byref(args), ctypes.byref(io), ws, ws_bytes, stream), "sa_bwd")
+
+
+def sa_bwd_no_alloc(args: SaArgs, io: SaBwdIo, stream: int = 0) -> None:
+    """Backward on the library's fixed scratch array (no workspace, no allocation)."""
+    _check(lib().sa_bwd_no_alloc(ctypes.byref(args), ctypes.byref(io), stream), "sa_bwd_no_alloc")
+
+
+def sa_bwd_no_alloc_max_workspace() -> int:
+    return int(lib().sa_bwd_no_alloc_max_workspace())
 
 
 def sa_softmax_grad_preprocess(args: SaArgs, o: int, d_o: int, delta: int, stream: int = 0) -> None:
