@@ -51,6 +51,7 @@ def count_work(w, inputs) -> dict:
     T = w.T
     vis = np.zeros((T, w.Hkv), dtype=np.int64)
     gat = np.zeros((T, w.Hkv), dtype=np.int64)
+    npair = np.zeros((T, w.Hkv), dtype=np.int64)   # (token, kv-head, usable block slot) with a visible row
     start = 0
     for L in lens:
         t = np.arange(L)[:, None, None]
@@ -73,6 +74,7 @@ def count_work(w, inputs) -> dict:
                     hi = np.minimum(hi, ta + w.win_right)
                 v = np.where(ok, np.maximum(hi - lo + 1, 0), 0)
                 g = np.where(ok, last - first + 1, 0)
+                npair[start:start + L] += (v > 0).sum(-1)
             else:
                 ok &= idx < L
                 m = ok.copy()
@@ -106,6 +108,7 @@ def count_work(w, inputs) -> dict:
         start += L
     G = w.G
     triples = int(vis.sum()) * G
+    n_pairs = int(npair.sum())
     row_bytes = (w.d_qk + (0 if w.kv_shared else w.d_v)) * 2
     gathered = int(gat.sum()) * row_bytes
     Tk = T
@@ -123,6 +126,13 @@ def count_work(w, inputs) -> dict:
         "fwd_bytes": gathered + n_q + n_v + lse_b,
         # fused backward kernel: gathered rows + read Q, dO, lse, Delta + write dQ + dK/dV once
         "bwd_main_bytes": gathered + n_q + n_v + 2 * lse_b + n_q + kv_out,
+        # key-stationary dK/dV kernel: S, dP, dV, dK contractions; streams each selecting
+        # token's G query and dO rows once per (token, slot) plus the KV blocks once
+        "kv_flops": 4 * (w.d_qk + w.d_v) * triples,
+        "kv_bytes": n_pairs * w.G * (w.d_qk + w.d_v) * 2 + 2 * n_pairs * w.G * 4 + kv_out + kv_out,
+        # query-stationary dQ pass: S, dP, dQ contractions over the gathered rows
+        "dq_flops": 2 * (2 * w.d_qk + w.d_v) * triples,
+        "dq_bytes": gathered + n_q + n_v + 2 * lse_b + n_q,
         "units": T * w.Hkv,
     }
 
@@ -327,9 +337,9 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
             e0.record(stream)
             sa.forward(o, lse, ws_f)
             e1.record(stream)
-            L.sa_set_timing_events(mb.cuda_event, me.cuda_event)
+            L.sa_set_timing_events(mb.cuda_event, me.cuda_event, L.TIME_BWD_KV)
             sa.backward(o, lse, t["do"], grads, ws_b)
-            L.sa_set_timing_events(None, None)
+            L.sa_set_timing_events(None, None, -1)
             e2.record(stream)
         torch.cuda.synchronize()
     launches = L.sa_kernel_launch_count() - launches0
@@ -337,10 +347,26 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
     main_ms = sum(e[3].elapsed_time(e[4]) for e in ev) / K
     step_ms = fwd_ms + bwd_ms
-    times = torch.tensor([fwd_ms, bwd_ms, main_ms, step_ms], dtype=torch.float64, device=dev)
+    # attribution pass (not part of the timed steps): the separate dQ kernel, if any
+    dq_ms = 0.0
+    evq = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a_, b_ in evq:
+        a_.record(stream)
+        b_.record(stream)
+    torch.cuda.synchronize()
+    for k in range(K):
+        flush.zero_()
+        L.sa_set_timing_events(evq[k][0].cuda_event, evq[k][1].cuda_event, L.TIME_BWD_DQ)
+        sa.backward(o, lse, t["do"], grads, ws_b)
+        L.sa_set_timing_events(None, None, -1)
+    torch.cuda.synchronize()
+    dq_ms = sum(a_.elapsed_time(b_) for a_, b_ in evq) / K
+    if dq_ms < 1e-3:
+        dq_ms = 0.0
+    times = torch.tensor([fwd_ms, bwd_ms, main_ms, step_ms, dq_ms], dtype=torch.float64, device=dev)
     if world > 1:
         torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    fwd_ms, bwd_ms, main_ms, step_ms = times.tolist()
+    fwd_ms, bwd_ms, main_ms, step_ms, dq_ms = times.tolist()
 
     # end to end through the public API with host buffers
     e2e = None
@@ -383,22 +409,32 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     peaks, peak_src = load_peaks()
     bwd_tflops = world * work["bwd_flops"] / (bwd_ms * 1e-3) / 1e12
     fwd_tflops = world * work["fwd_flops"] / (fwd_ms * 1e-3) / 1e12
-    # roofline of the dominant kernel (fused backward)
-    t_bytes = work["bwd_main_bytes"] / (peaks["hbm_gbs"] * 1e9)
-    t_flops = work["bwd_flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
+    # roofline of the dominant backward kernel
+    keystat = dq_ms > 0.0
+    kern = []
+    if keystat:
+        kern.append(("kv_bwd_kernel (key-stationary dK/dV)", main_ms, work["kv_flops"], work["kv_bytes"]))
+        kern.append(("bwd_kernel<SCATTER=false> (query-stationary dQ)", dq_ms, work["dq_flops"], work["dq_bytes"]))
+    else:
+        kern.append(("bwd_kernel (fused query-stationary backward)", main_ms, work["bwd_flops"],
+                     work["bwd_main_bytes"]))
+    name, kms, kflops, kbytes = max(kern, key=lambda x: x[1])
+    t_bytes = kbytes / (peaks["hbm_gbs"] * 1e9)
+    t_flops = kflops / (peaks["bf16_tflops_sustained"] * 1e12)
     bound = "hbm" if t_bytes >= t_flops else "tensor"
     if bound == "hbm":
-        achieved = work["bwd_main_bytes"] / (main_ms * 1e-3) / 1e9
+        achieved = kbytes / (kms * 1e-3) / 1e9
         peak, unit = peaks["hbm_gbs"], "GB/s"
     else:
-        achieved = work["bwd_flops"] / (main_ms * 1e-3) / 1e12
+        achieved = kflops / (kms * 1e-3) / 1e12
         peak, unit = peaks["bf16_tflops_sustained"], "TFLOP/s"
     roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-            "frac": achieved / peak, "traffic": load_traffic("bwd_kernel", w.name),
-            "kernel": "bwd_kernel (fused backward)", "kernel_ms": main_ms,
-            "algorithmic_bytes": work["bwd_main_bytes"], "algorithmic_flops": work["bwd_flops"],
+            "frac": achieved / peak, "traffic": load_traffic(name.split(" ")[0], w.name),
+            "kernel": name, "kernel_ms": kms,
+            "algorithmic_bytes": kbytes, "algorithmic_flops": kflops,
             "peak_source": f"{peak_src} MEASURED_PEAKS.json" if peak_src == "measured" else "fallback",
-            "t_roof_ms": max(t_bytes, t_flops) * 1e3}
+            "t_roof_ms": max(t_bytes, t_flops) * 1e3,
+            "kernels_ms": {k_[0]: k_[1] for k_ in kern}}
     line = {
         "metric": METRIC, "value": bwd_tflops, "unit": "TFLOP/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
@@ -408,6 +444,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
                    "parallelism": f"replicas{world}", "l2": "flushed between timed steps",
                    "visible_triples": work["triples"], "gathered_bytes": work["gathered_bytes"]},
         "fwd_tflops": fwd_tflops, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+        "bwd_path": "key-stationary dK/dV + query-stationary dQ" if keystat else "query-stationary fused",
         "bwd_roofline_frac": max(t_bytes, t_flops) * 1e3 / bwd_ms,
         "roofline": roof, "clocks": clk.summary(), "gpu_launches": launches,
         "e2e": e2e,

@@ -96,6 +96,17 @@ typedef enum sa_dtype { SA_DTYPE_BF16 = 0, SA_DTYPE_FP16 = 1 } sa_dtype;
 #define SA_FLAG_CHECK 1u   /* validate every index on the device first; the call then
                               synchronises `stream` and returns SA_ERR_INDEX if one is
                               past its sequence (nothing else is computed) */
+/* Backward kernel choice (results agree within rounding; the default is the
+ * fastest measured).  Block-level selection with block_size 64, BSND, equal
+ * query / key lengths, separate K and V and no sinks runs key-stationary by
+ * default: one CTA per (kv block, chunk of the tokens that select it)
+ * accumulates dK / dV on the tensor cores, and dQ comes from a query-stationary
+ * pass.  Every other problem runs query-stationary. */
+#define SA_FLAG_QUERY_STATIONARY_BWD 2u  /* force the query-stationary backward
+                                            (dK / dV by fp32 scatter-add) */
+#define SA_FLAG_DQ_ATOMIC 4u   /* key-stationary backward: form dQ in the same kernel and
+                                  add it with fp32 atomics (needs Tq*Hq*d_qk*4 more
+                                  workspace bytes) instead of a separate pass */
 
 /* The problem description shared by every entry point (host struct). */
 typedef struct sa_args {
@@ -221,16 +232,30 @@ sa_status sa_debug_resolve(const sa_args* args, int32_t* rows, int32_t* counts,
 
 /* ---- benchmarking hooks ------------------------------------------------ */
 
-/* Timing hook (process-wide, not thread-safe): when both are non-NULL, the
- * next sa_fwd / sa_bwd calls record ev_begin right before and ev_end right
- * after their main kernel (the forward kernel; the fused backward kernel), on
- * the call's stream.  Both are cudaEvent_t created by the caller; pass NULL,
- * NULL to disable. */
-void sa_set_timing_events(void* ev_begin, void* ev_end);
+/* Timing hook (process-wide, not thread-safe): when both events are
+ * non-NULL, later sa_fwd / sa_bwd calls record ev_begin right before and
+ * ev_end right after one of their kernels, on the call's stream:
+ *   which = 0: the forward kernel;
+ *   which = 1: the backward kernel that forms dK / dV (key-stationary kernel,
+ *              or the fused query-stationary kernel);
+ *   which = 2: the query-stationary dQ pass of the key-stationary backward.
+ * Both are cudaEvent_t created by the caller; pass NULL, NULL to disable. */
+void sa_set_timing_events(void* ev_begin, void* ev_end, int32_t which);
 
 /* Number of kernels this library has launched since it was loaded
  * (memsets excluded). */
 int64_t sa_kernel_launch_count(void);
+
+/* Self-check of the tensor-core building blocks used by the key-stationary
+ * backward: one CTA computes D = A B with TMA loads (boxes of box_rows x 64),
+ * 128-byte swizzled shared-memory operands, tcgen05.mma and TMEM loads.
+ * A is K-major [M][K] (a_mn = 0) or MN-major [K][M] (a_mn = 1); B is K-major
+ * [N][K] (b_mn = 0) or MN-major [K][N] (b_mn = 1); all bf16 row-major, device.
+ * D fp32 [M][N] (device).  M in {64, 128}; N, K multiples of 64, N <= 256,
+ * K <= 256; box_rows in {8, 16, 32, 64}.  *status (device int) gets the
+ * timeout bit if a bounded wait gives up.  Asynchronous. */
+sa_status sa_selftest_mma(int32_t M, int32_t N, int32_t K, int32_t a_mn, int32_t b_mn, int32_t box_rows,
+                          const void* A, const void* B, float* D, int32_t* status, void* stream);
 
 /* Human-readable name of a status code (static string). */
 const char* sa_status_string(int32_t status);

@@ -145,11 +145,20 @@ def _align(x):
 
 
 def test_bwd_workspace_size_contract():
-    a = _args()
+    # query-stationary backward: status word, Delta, fp32 dK and dV accumulators
+    a = _args(flags=L.SA_FLAG_QUERY_STATIONARY_BWD)
     st, n = _ws(a)
     Tq, Tk = 2 * 128, 2 * 128
-    expect = 256 + _align(Tq * 16 * 4) + _align(Tk * 4 * 192 * 4) + _align(Tk * 4 * 128 * 4)
-    assert st == L.SA_OK and n == expect
+    base = 256 + _align(Tq * 16 * 4) + _align(Tk * 4 * 192 * 4) + _align(Tk * 4 * 128 * 4)
+    assert st == L.SA_OK and n == base
+    # key-stationary backward (block-level, BSND, 64-row blocks): + the inverse index
+    n_lists, n_slots = 2 * 4 * 2, 2 * 128 * 4 * 4
+    index = 2 * _align(4 * n_lists) + 2 * _align(4 * (n_lists + 1)) + 256 + _align(4 * n_slots)
+    st, n = _ws(_args())
+    assert st == L.SA_OK and n == base + index
+    # ... + an fp32 dQ accumulator when dQ is formed in the same kernel
+    st, n = _ws(_args(flags=L.SA_FLAG_DQ_ATOMIC))
+    assert st == L.SA_OK and n == base + index + _align(Tq * 16 * 192 * 4)
     a = _args(kv_shared=1, d_qk=576, d_v=512, kv=FAKE, n_heads_q=64, n_heads_kv=1, block_size=1,
               layout=L.SA_LAYOUT_TND, t_q=1000, t_kv=1000, t_cmp=250, cmp_topk=16, cmp_ratio=4,
               cmp_kv=FAKE, cmp_idx=FAKE, cu_seqlens_q=FAKE, cu_seqlens_kv=FAKE, cu_seqlens_cmp=FAKE)

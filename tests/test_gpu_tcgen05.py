@@ -1,0 +1,39 @@
+"""The tensor-core building blocks (TMA tile loads into 128-byte swizzled
+shared memory, matrix descriptors for K-major and MN-major operands,
+tcgen05.mma, TMEM accumulators of height 64 and 128) against a plain fp32
+matmul of the same bf16 operands."""
+
+import pytest
+import torch
+
+from top_sparse_attention_attn_b200 import _lib as L
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # M, N, K, a_mn, b_mn, box_rows
+    (128, 64, 64, 0, 0, 64), (128, 64, 192, 0, 0, 16), (128, 256, 128, 0, 0, 8),
+    (128, 64, 128, 1, 1, 64), (128, 64, 128, 1, 1, 16), (64, 64, 128, 1, 1, 32),
+    (128, 192, 64, 0, 1, 64), (128, 128, 256, 1, 0, 16), (64, 128, 64, 0, 0, 8),
+    (64, 192, 128, 1, 1, 64), (128, 192, 128, 1, 0, 8),
+]
+
+
+@pytest.mark.parametrize("M,N,K,a_mn,b_mn,box", CASES)
+def test_tcgen05_mma_matches_matmul(M, N, K, a_mn, b_mn, box):
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA GPU is required for -m gpu tests")
+    g = torch.Generator(device="cuda").manual_seed(M * 1000 + N * 10 + K + a_mn + 2 * b_mn)
+    A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+    B = torch.randn(K, N, device="cuda", generator=g).to(torch.bfloat16)
+    a_store = A.t().contiguous() if a_mn else A.contiguous()          # [K][M] or [M][K]
+    b_store = B.contiguous() if b_mn else B.t().contiguous()          # [K][N] or [N][K]
+    D = torch.full((M, N), float("nan"), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.sa_selftest_mma(M, N, K, a_mn, b_mn, box, a_store.data_ptr(), b_store.data_ptr(), D.data_ptr(),
+                      status.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ref = A.float() @ B.float()
+    err = (D - ref).abs().max().item()
+    assert err <= 1e-3 * ref.abs().max().item(), f"max err {err}"

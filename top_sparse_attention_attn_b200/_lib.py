@@ -30,6 +30,8 @@ SA_MASK_BAND = 2
 SA_DTYPE_BF16 = 0
 SA_DTYPE_FP16 = 1
 SA_FLAG_CHECK = 1
+SA_FLAG_QUERY_STATIONARY_BWD = 2
+SA_FLAG_DQ_ATOMIC = 4
 
 MASKS = {"none": SA_MASK_NONE, "causal": SA_MASK_CAUSAL, "band": SA_MASK_BAND}
 LAYOUTS = {"BSND": SA_LAYOUT_BSND, "TND": SA_LAYOUT_TND}
@@ -78,7 +80,7 @@ _lib = None
 EXPORTS = ["sa_fwd_get_workspace_size", "sa_fwd", "sa_bwd_get_workspace_size", "sa_bwd",
            "sa_softmax_grad_preprocess", "sa_debug_resolve", "sa_status_string", "sa_abi_version",
            "sa_set_timing_events", "sa_kernel_launch_count", "sa_bwd_no_alloc",
-           "sa_bwd_no_alloc_max_workspace"]
+           "sa_bwd_no_alloc_max_workspace", "sa_selftest_mma"]
 
 
 def lib() -> ctypes.CDLL:
@@ -99,13 +101,14 @@ def lib() -> ctypes.CDLL:
         L.sa_status_string.argtypes = [ctypes.c_int32]
         L.sa_status_string.restype = ctypes.c_char_p
         L.sa_abi_version.argtypes = []
-        L.sa_set_timing_events.argtypes = [_vp, _vp]
+        L.sa_set_timing_events.argtypes = [_vp, _vp, ctypes.c_int32]
         L.sa_set_timing_events.restype = None
         L.sa_kernel_launch_count.argtypes = []
         L.sa_kernel_launch_count.restype = ctypes.c_int64
         L.sa_bwd_no_alloc.argtypes = [P(SaArgs), P(SaBwdIo), _vp]
         L.sa_bwd_no_alloc_max_workspace.argtypes = []
         L.sa_bwd_no_alloc_max_workspace.restype = ctypes.c_size_t
+        L.sa_selftest_mma.argtypes = [ctypes.c_int32] * 6 + [_vp, _vp, _vp, _vp, _vp]
         for name in EXPORTS:
             if name not in ("sa_status_string", "sa_set_timing_events", "sa_kernel_launch_count",
                             "sa_bwd_no_alloc_max_workspace"):
@@ -154,6 +157,11 @@ def sa_bwd_no_alloc_max_workspace() -> int:
     return int(lib().sa_bwd_no_alloc_max_workspace())
 
 
+def sa_selftest_mma(M: int, N: int, K: int, a_mn: int, b_mn: int, box_rows: int, A: int, B: int,
+                    D: int, status: int, stream: int = 0) -> None:
+    _check(lib().sa_selftest_mma(M, N, K, a_mn, b_mn, box_rows, A, B, D, status, stream), "sa_selftest_mma")
+
+
 def sa_softmax_grad_preprocess(args: SaArgs, o: int, d_o: int, delta: int, stream: int = 0) -> None:
     _check(lib().sa_softmax_grad_preprocess(ctypes.byref(args), o, d_o, delta, stream),
            "sa_softmax_grad_preprocess")
@@ -167,8 +175,11 @@ def sa_abi_version() -> int:
     return int(lib().sa_abi_version())
 
 
-def sa_set_timing_events(ev_begin: int | None, ev_end: int | None) -> None:
-    lib().sa_set_timing_events(ev_begin, ev_end)
+TIME_FWD, TIME_BWD_KV, TIME_BWD_DQ = 0, 1, 2
+
+
+def sa_set_timing_events(ev_begin: int | None, ev_end: int | None, which: int = TIME_BWD_KV) -> None:
+    lib().sa_set_timing_events(ev_begin, ev_end, which)
 
 
 def sa_kernel_launch_count() -> int:

@@ -7,6 +7,7 @@
 
 #include "../../include/sparse_attn.h"
 #include "sa_device.cuh"
+#include "sa_kv_bwd.h"
 #include "sa_launch.h"
 
 namespace {
@@ -135,14 +136,52 @@ sa_status check_tensor_alignment(const sa_args* a) {
   return SA_OK;
 }
 
+// The key-stationary backward applies to block-level BSND selection with
+// 64-row blocks, equal query / key lengths, separate K / V and no sinks.
+bool use_kv_path(const sa_args* a) {
+  if (a->flags & SA_FLAG_QUERY_STATIONARY_BWD) return false;
+  const int G = a->n_heads_q / a->n_heads_kv;
+  return a->layout == SA_LAYOUT_BSND && a->topk > 0 && a->block_size == 64 && a->s_q == a->s_kv &&
+         !a->kv_shared && a->cmp_topk == 0 && a->sinks == nullptr && G <= 128 &&
+         sa::kv_path_built(a->d_qk, a->d_v);
+}
+
+struct KvGeom {
+  int RPT, TPT, nblk, n_lists, chunk;
+  long long n_slots, max_work;
+};
+
+KvGeom kv_geometry(const sa_args* a) {
+  KvGeom k;
+  const int G = a->n_heads_q / a->n_heads_kv;
+  k.RPT = (G + 7) / 8 * 8;
+  k.TPT = 128 / k.RPT;
+  k.nblk = (a->s_kv + 63) / 64;
+  k.n_lists = a->batch * a->n_heads_kv * k.nblk;
+  k.n_slots = (long long)a->batch * a->s_q * a->n_heads_kv * a->topk;
+  // chunk of tokens per CTA: ~4 work items per SM, between 4 tiles and 512 tokens
+  long long want = (k.n_slots + 148 * 4 - 1) / (148 * 4);
+  long long lo = 4ll * k.TPT, hi = (512 / k.TPT) * k.TPT;
+  if (want < lo) want = lo;
+  if (want > hi) want = hi;
+  want = (want + k.TPT - 1) / k.TPT * k.TPT;
+  k.chunk = (int)want;
+  k.max_work = (k.n_slots + k.chunk - 1) / k.chunk + k.n_lists;
+  return k;
+}
+
 // Workspace: [status word][delta][dK or dKV acc][dV acc][dCmp acc]
+//            + key-stationary path: [counts][cursor][list_off][chunk_off][work][entries][dQ acc]
 struct BwdWs {
-  size_t status, delta, dk, dv, dcmp, total;
+  size_t status, delta, dk, dv, dcmp;
+  size_t counts, cursor, list_off, chunk_off, work, entries, dq;
+  size_t total;
 };
 
 BwdWs bwd_ws_layout(const sa_args* a) {
   Sizes s = sizes_of(a);
   BwdWs w;
+  memset(&w, 0, sizeof(w));
   size_t off = 0;
   w.status = off;
   off += kAlign;
@@ -154,6 +193,25 @@ BwdWs bwd_ws_layout(const sa_args* a) {
   if (!a->kv_shared) off += align_up((size_t)s.Tkv * a->n_heads_kv * a->d_v * sizeof(float));
   w.dcmp = off;
   off += align_up((size_t)s.Tcmp * a->n_heads_kv * a->d_qk * sizeof(float));
+  if (use_kv_path(a)) {
+    KvGeom k = kv_geometry(a);
+    w.counts = off;
+    off += align_up(sizeof(int) * k.n_lists);
+    w.cursor = off;
+    off += align_up(sizeof(int) * k.n_lists);
+    w.list_off = off;
+    off += align_up(sizeof(int) * (k.n_lists + 1));
+    w.chunk_off = off;
+    off += align_up(sizeof(int) * (k.n_lists + 1));
+    w.work = off;
+    off += kAlign;
+    w.entries = off;
+    off += align_up(sizeof(int) * (size_t)k.n_slots);
+    if (a->flags & SA_FLAG_DQ_ATOMIC) {
+      w.dq = off;
+      off += align_up((size_t)s.Tq * a->n_heads_q * a->d_qk * sizeof(float));
+    }
+  }
   w.total = off;
   return w;
 }
@@ -177,9 +235,10 @@ extern "C" {
 
 int32_t sa_abi_version(void) { return SA_ABI_VERSION; }
 
-void sa_set_timing_events(void* ev_begin, void* ev_end) {
+void sa_set_timing_events(void* ev_begin, void* ev_end, int32_t which) {
   sa::g_ev_begin = static_cast<cudaEvent_t>(ev_begin);
   sa::g_ev_end = static_cast<cudaEvent_t>(ev_end);
+  sa::g_ev_which = which;
 }
 
 int64_t sa_kernel_launch_count(void) { return __atomic_load_n(&sa::g_launches, __ATOMIC_RELAXED); }
@@ -269,15 +328,85 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
   const long long nk = s.Tkv * args->n_heads_kv * args->d_qk;
   const long long nv = s.Tkv * args->n_heads_kv * args->d_v;
   const long long nc = s.Tcmp * args->n_heads_kv * args->d_qk;
-  // zero the accumulators (one contiguous range) and dSinks
-  if (cudaMemsetAsync(base, 0, w.total, cs) != cudaSuccess) return SA_ERR_CUDA;
+  // zero the accumulators and dSinks (the index region is cleared by its own kernels)
+  const size_t zero_end = w.counts ? w.counts : w.total;
+  if (cudaMemsetAsync(base, 0, zero_end, cs) != cudaSuccess) return SA_ERR_CUDA;
+  if (w.dq && cudaMemsetAsync(base + w.dq, 0, w.total - w.dq, cs) != cudaSuccess) return SA_ERR_CUDA;
   if (sinks && cudaMemsetAsync(io->dsinks, 0, sizeof(float) * args->n_heads_q, cs) != cudaSuccess)
     return SA_ERR_CUDA;
   cudaError_t e = sa::launch_delta(static_cast<const bf16*>(io->o), static_cast<const bf16*>(io->d_o), delta,
                                    s.Tq * args->n_heads_q, args->d_v, cs);
   if (e != cudaSuccess) return SA_ERR_CUDA;
-  e = sa::launch_bwd(p, static_cast<const bf16*>(io->o), static_cast<const bf16*>(io->d_o), io->lse, delta,
-                     out, cs);
+  if (w.counts) {
+    // key-stationary: inverse index, then dK / dV per KV block (+ dQ)
+    KvGeom k = kv_geometry(args);
+    sa::KvIndexArgs ia;
+    memset(&ia, 0, sizeof(ia));
+    ia.ori_idx = args->ori_idx;
+    ia.ori_len = args->ori_topk_len;
+    ia.n_slots = k.n_slots;
+    ia.topk = args->topk;
+    ia.Hkv = args->n_heads_kv;
+    ia.S = args->s_q;
+    ia.nblk = k.nblk;
+    ia.n_lists = k.n_lists;
+    ia.chunk_tokens = k.chunk;
+    ia.ori_mask = args->ori_mask_mode;
+    ia.wl = args->ori_win_left;
+    ia.wr = args->ori_win_right;
+    ia.counts = reinterpret_cast<int*>(base + w.counts);
+    ia.cursor = reinterpret_cast<int*>(base + w.cursor);
+    ia.list_off = reinterpret_cast<int*>(base + w.list_off);
+    ia.chunk_off = reinterpret_cast<int*>(base + w.chunk_off);
+    ia.entries = reinterpret_cast<int*>(base + w.entries);
+    ia.work_count = reinterpret_cast<int*>(base + w.work);
+    if (sa::launch_kv_index(ia, cs) != cudaSuccess) return SA_ERR_CUDA;
+    sa::KvLaunch kl;
+    memset(&kl, 0, sizeof(kl));
+    sa::KvArgs& ka = kl.args;
+    ka.S = args->s_q;
+    ka.Hq = args->n_heads_q;
+    ka.Hkv = args->n_heads_kv;
+    ka.G = args->n_heads_q / args->n_heads_kv;
+    ka.RPT = k.RPT;
+    ka.TPT = k.TPT;
+    ka.nblk = k.nblk;
+    ka.n_lists = k.n_lists;
+    ka.chunk_tokens = k.chunk;
+    ka.ori_mask = args->ori_mask_mode;
+    ka.wl = args->ori_win_left;
+    ka.wr = args->ori_win_right;
+    ka.scale = args->scale;
+    ka.scale_log2 = args->scale * 1.4426950408889634f;
+    ka.list_off = ia.list_off;
+    ka.chunk_off = ia.chunk_off;
+    ka.entries = ia.entries;
+    ka.work_count = ia.work_count;
+    ka.lse = io->lse;
+    ka.delta = delta;
+    ka.dk_acc = out.dk_acc;
+    ka.dv_acc = out.dv_acc;
+    ka.dq_acc = w.dq ? reinterpret_cast<float*>(base + w.dq) : nullptr;
+    ka.status = status;
+    kl.q = args->q;
+    kl.d_o = io->d_o;
+    kl.k = args->k;
+    kl.v = args->v;
+    kl.Tq = s.Tq;
+    kl.Tkv = s.Tkv;
+    kl.dqk = args->d_qk;
+    kl.dv = args->d_v;
+    kl.max_work = k.max_work;
+    if (sa::launch_kv_bwd(kl, w.dq != 0, cs) != cudaSuccess) return SA_ERR_CUDA;
+    if (w.dq) {
+      e = sa::launch_to_bf16(ka.dq_acc, static_cast<bf16*>(io->dq), s.Tq * args->n_heads_q * args->d_qk, cs);
+    } else {
+      e = sa::launch_bwd_dq(p, static_cast<const bf16*>(io->d_o), io->lse, delta, out, cs);
+    }
+  } else {
+    e = sa::launch_bwd(p, static_cast<const bf16*>(io->o), static_cast<const bf16*>(io->d_o), io->lse, delta,
+                       out, cs);
+  }
   if (e != cudaSuccess) return SA_ERR_CUDA;
   if (args->kv_shared) {
     e = sa::launch_to_bf16(out.dk_acc, static_cast<bf16*>(io->dkv), nk, cs);

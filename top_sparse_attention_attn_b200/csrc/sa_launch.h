@@ -1,6 +1,7 @@
 // sa_launch.h -- host-side launchers behind the C ABI (internal).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 
@@ -18,16 +19,29 @@ struct BwdOut {
 };
 
 // Process-wide benchmarking hooks (see sa_set_timing_events).
+enum { kTimeFwd = 0, kTimeBwdKV = 1, kTimeBwdDQ = 2 };
 extern cudaEvent_t g_ev_begin, g_ev_end;
+extern int g_ev_which;
 extern long long g_launches;
 inline void count_launch() { __atomic_fetch_add(&g_launches, 1, __ATOMIC_RELAXED); }
-inline void mark_begin(cudaStream_t st) { if (g_ev_begin && g_ev_end) cudaEventRecord(g_ev_begin, st); }
-inline void mark_end(cudaStream_t st) { if (g_ev_begin && g_ev_end) cudaEventRecord(g_ev_end, st); }
+inline void mark_begin(cudaStream_t st, int which) {
+  if (g_ev_begin && g_ev_end && which == g_ev_which) cudaEventRecord(g_ev_begin, st);
+}
+inline void mark_end(cudaStream_t st, int which) {
+  if (g_ev_begin && g_ev_end && which == g_ev_which) cudaEventRecord(g_ev_end, st);
+}
+
+// TMA tensor map over a [rows][cols] bf16 matrix (row stride in bytes), boxes
+// of box_rows x 64 columns, 128-byte swizzle, zero fill out of range.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
+                    uint32_t box_rows);
 
 // Returns false when no kernel is built for (dqk, dv, shared).
 bool kernels_built(int dqk, int dv, bool shared);
 
 cudaError_t launch_fwd(const Prob& p, bf16* o, float* lse, cudaStream_t st);
+cudaError_t launch_bwd_dq(const Prob& p, const bf16* d_o, const float* lse, const float* delta,
+                          const BwdOut& out, cudaStream_t st);
 cudaError_t launch_delta(const bf16* o, const bf16* d_o, float* delta, long long rows, int dv,
                          cudaStream_t st);
 cudaError_t launch_bwd(const Prob& p, const bf16* o, const bf16* d_o, const float* lse,

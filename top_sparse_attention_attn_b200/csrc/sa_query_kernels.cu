@@ -25,6 +25,7 @@
 namespace sa {
 
 cudaEvent_t g_ev_begin = nullptr, g_ev_end = nullptr;
+int g_ev_which = -1;
 long long g_launches = 0;
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -258,7 +259,7 @@ __device__ __forceinline__ void red_add2(float* addr, float a, float b) {
   atomicAdd(reinterpret_cast<float2*>(addr), make_float2(a, b));
 }
 
-template <int DQK, int DV, bool SHARED>
+template <int DQK, int DV, bool SHARED, bool SCATTER>
 __global__ void __launch_bounds__(128) bwd_kernel(const Prob p, const bf16* __restrict__ dO,
                                                   const float* __restrict__ LSE,
                                                   const float* __restrict__ Delta, BwdOut out) {
@@ -373,7 +374,7 @@ __global__ void __launch_bounds__(128) bwd_kernel(const Prob p, const bf16* __re
     if (code1 >= 0)
       kdst1 = (code1 & kCmpFlag) ? out.dcmp_acc + ((long long)(code1 & ~kCmpFlag) * p.Hkv + g) * DQK
                                  : out.dk_acc + ((long long)code1 * p.Hkv + g) * DQK;
-    if (__any_sync(0xffffffffu, code0 >= 0 || code1 >= 0)) {
+    if (SCATTER && __any_sync(0xffffffffu, code0 >= 0 || code1 >= 0)) {
       uint32_t adsT[4], apT[4];
       load_a_t<64>(adsT, sDS, 0, warp * 2, lane);
       load_a_t<64>(apT, sP, 0, warp * 2, lane);
@@ -588,25 +589,26 @@ static cudaError_t fwd_t(const Prob& p, bf16* o, float* lse, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kBytes);
   if (e != cudaSuccess) return e;
   long long grid = (long long)p.Tq * p.Hkv * ((p.G + 15) / 16);
-  mark_begin(st);
+  mark_begin(st, kTimeFwd);
   k<<<(unsigned)grid, 128, PL::kBytes, st>>>(p, o, lse);
   count_launch();
-  mark_end(st);
+  mark_end(st, kTimeFwd);
   return cudaGetLastError();
 }
 
-template <int DQK, int DV, bool SHARED>
+template <int DQK, int DV, bool SHARED, bool SCATTER = true>
 static cudaError_t bwd_t(const Prob& p, const bf16* d_o, const float* lse, const float* delta,
                          const BwdOut& out, cudaStream_t st) {
   using PL = Plan<DQK, DV, SHARED>;
-  auto k = bwd_kernel<DQK, DV, SHARED>;
+  auto k = bwd_kernel<DQK, DV, SHARED, SCATTER>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kBytes);
   if (e != cudaSuccess) return e;
   long long grid = (long long)p.Tq * p.Hkv * ((p.G + 15) / 16);
-  mark_begin(st);
+  const int which = SCATTER ? kTimeBwdKV : kTimeBwdDQ;
+  mark_begin(st, which);
   k<<<(unsigned)grid, 128, PL::kBytes, st>>>(p, d_o, lse, delta, out);
   count_launch();
-  mark_end(st);
+  mark_end(st, which);
   return cudaGetLastError();
 }
 
@@ -625,6 +627,15 @@ cudaError_t launch_bwd(const Prob& p, const bf16* o, const bf16* d_o, const floa
   if (p.dqk == A && p.dv == B && (bool)p.shared == C) return bwd_t<A, B, C>(p, d_o, lse, delta, out, st);
   SA_FOR_EACH_SHAPE(X)
 #undef X
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd_dq(const Prob& p, const bf16* d_o, const float* lse, const float* delta,
+                          const BwdOut& out, cudaStream_t st) {
+  // dQ only (dK / dV come from the key-stationary kernel); dSinks needs no sinks here
+  if (p.dqk == 64 && p.dv == 64 && !p.shared) return bwd_t<64, 64, false, false>(p, d_o, lse, delta, out, st);
+  if (p.dqk == 128 && p.dv == 128 && !p.shared) return bwd_t<128, 128, false, false>(p, d_o, lse, delta, out, st);
+  if (p.dqk == 192 && p.dv == 128 && !p.shared) return bwd_t<192, 128, false, false>(p, d_o, lse, delta, out, st);
   return cudaErrorInvalidValue;
 }
 

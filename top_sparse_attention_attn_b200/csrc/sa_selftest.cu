@@ -1,0 +1,127 @@
+// sa_selftest.cu -- sa_selftest_mma: one CTA computes D = A * B through the
+// same TMA loads, shared-memory matrix descriptors, tcgen05.mma and TMEM loads
+// that the key-stationary backward kernel is built from, so that each operand
+// orientation (K-major, MN-major) and each accumulator height (M = 64, 128)
+// can be checked against a plain matmul.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sparse_attn.h"
+#include "sa_launch.h"
+#include "sa_tc.cuh"
+
+namespace sa {
+
+struct SelftestArgs {
+  int M, N, K, a_mn, b_mn, box_rows;
+};
+
+__global__ void __launch_bounds__(128) selftest_mma_kernel(const __grid_constant__ CUtensorMap mapA,
+                                                           const __grid_constant__ CUtensorMap mapB,
+                                                           const SelftestArgs a, float* __restrict__ D,
+                                                           int* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte aligned operand area
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t bar_load, bar_mma;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sA = smem_u32(smem);
+  const uint32_t sB = sA + a.M * a.K * 2;
+  const uint32_t ncols = a.N <= 64 ? 64 : (a.N <= 128 ? 128 : 256);
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar_load, 1);
+    mbar_init(&bar_mma, 1);
+    mbar_fence_init();
+  }
+  if (warp == 0) tmem_alloc(&tmem_base, ncols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  if (threadIdx.x == 0) {
+    // operand tiles: K-major -> slabs over K of [rows][64]; MN-major -> slabs over M/N of [K][64]
+    mbar_arrive_tx(&bar_load, (uint32_t)((a.M + a.N) * a.K * 2));
+    const int br = a.box_rows;
+    if (!a.a_mn) {
+      for (int s = 0; s < a.K / 64; ++s)
+        for (int r = 0; r < a.M; r += br) tma_load_2d(sA + s * a.M * 128 + r * 128, &mapA, 64 * s, r, &bar_load);
+    } else {
+      for (int s = 0; s < a.M / 64; ++s)
+        for (int r = 0; r < a.K; r += br) tma_load_2d(sA + s * a.K * 128 + r * 128, &mapA, 64 * s, r, &bar_load);
+    }
+    if (!a.b_mn) {
+      for (int s = 0; s < a.K / 64; ++s)
+        for (int r = 0; r < a.N; r += br) tma_load_2d(sB + s * a.N * 128 + r * 128, &mapB, 64 * s, r, &bar_load);
+    } else {
+      for (int s = 0; s < a.N / 64; ++s)
+        for (int r = 0; r < a.K; r += br) tma_load_2d(sB + s * a.K * 128 + r * 128, &mapB, 64 * s, r, &bar_load);
+    }
+    if (mbar_wait(&bar_load, 0, &abort_flag, status)) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16(a.M, a.N, a.a_mn != 0, a.b_mn != 0);
+      for (int kk = 0; kk < a.K / 16; ++kk) {
+        uint64_t da = a.a_mn ? sdesc(sA + kk * 2048, a.K * 128, 1024)
+                             : sdesc(sA + (kk >> 2) * a.M * 128 + (kk & 3) * 32, 16, 1024);
+        uint64_t db = a.b_mn ? sdesc(sB + kk * 2048, a.K * 128, 1024)
+                             : sdesc(sB + (kk >> 2) * a.N * 128 + (kk & 3) * 32, 16, 1024);
+        mma_bf16(tmem_base, da, db, idesc, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(&bar_mma);
+    }
+  }
+  __syncwarp();
+  bool ok = mbar_wait(&bar_mma, 0, &abort_flag, status);
+  tc_fence_after();
+  if (ok) {
+    const int sub = warp & 3;
+    int m = -1;
+    if (a.M == 128) m = 32 * sub + lane;
+    else if (lane < 16) m = 16 * sub + lane;
+    for (int c = 0; c < a.N; c += 16) {
+      uint32_t r[16];
+      tmem_ld16(tmem_base + ((uint32_t)(32 * sub) << 16) + c, r);
+      tmem_wait_ld();
+      reg_dep16(r);
+      if (m >= 0)
+        for (int i = 0; i < 16; ++i) D[(long long)m * a.N + c + i] = __uint_as_float(r[i]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, ncols);
+    tmem_relinquish();
+  }
+}
+
+}  // namespace sa
+
+extern "C" sa_status sa_selftest_mma(int32_t M, int32_t N, int32_t K, int32_t a_mn, int32_t b_mn,
+                                     int32_t box_rows, const void* A, const void* B, float* D, int32_t* status,
+                                     void* stream) {
+  if (!A || !B || !D || !status) return SA_ERR_NULLPTR;
+  if ((M != 64 && M != 128) || N < 64 || N > 256 || N % 64 || K < 64 || K > 256 || K % 64) return SA_ERR_PARAM;
+  if (box_rows != 8 && box_rows != 16 && box_rows != 32 && box_rows != 64) return SA_ERR_PARAM;
+  CUtensorMap ma, mb;
+  // A: K-major [M][K] or MN-major [K][M]; B: K-major [N][K] or MN-major [K][N]
+  bool okA = a_mn ? sa::make_tmap_bf16(&ma, A, K, M, (uint64_t)M * 2, box_rows)
+                  : sa::make_tmap_bf16(&ma, A, M, K, (uint64_t)K * 2, box_rows);
+  bool okB = b_mn ? sa::make_tmap_bf16(&mb, B, K, N, (uint64_t)N * 2, box_rows)
+                  : sa::make_tmap_bf16(&mb, B, N, K, (uint64_t)K * 2, box_rows);
+  if (!okA || !okB) return SA_ERR_PARAM;
+  sa::SelftestArgs args{M, N, K, a_mn, b_mn, box_rows};
+  const int smem = (M + N) * K * 2 + 1024;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaFuncSetAttribute(sa::selftest_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return SA_ERR_CUDA;
+  sa::selftest_mma_kernel<<<1, 128, smem, st>>>(ma, mb, args, D, status);
+  sa::count_launch();
+  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
