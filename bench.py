@@ -187,7 +187,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", str(self.dev)],
+                 "-lms", "100", "-i", str(self.dev)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -304,7 +304,10 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     inputs = make_inputs(w)
     work = count_work(w, inputs)
     t = to_torch(inputs, dev)
-    sa = SparseAttention.from_workload(w, t)
+    flags = 0
+    for f in filter(None, args.flags.split(",")):
+        flags |= {"dq_atomic": L.SA_FLAG_DQ_ATOMIC, "query_stationary": L.SA_FLAG_QUERY_STATIONARY_BWD}[f]
+    sa = SparseAttention.from_workload(w, t, flags=flags)
     stream = torch.cuda.current_stream(dev)
     o, lse = sa.alloc_fwd()
     grads = sa.alloc_bwd()
@@ -442,6 +445,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         "config": {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv,
                    "d_qk": w.d_qk, "d_v": w.d_v, "block_size": w.block_size, "topk": w.topk,
                    "parallelism": f"replicas{world}", "l2": "flushed between timed steps",
+                   "flags": args.flags or "default",
                    "visible_triples": work["triples"], "gathered_bytes": work["gathered_bytes"]},
         "fwd_tflops": fwd_tflops, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
         "bwd_path": "key-stationary dK/dV + query-stationary dQ" if keystat else "query-stationary fused",
@@ -480,13 +484,14 @@ def run_reference(args, rank: int) -> dict | None:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="cfg2")
     ap.add_argument("--override", default=None, help="workload overrides for profiling, e.g. S=2048")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--flags", default="", help="backward variant for measurements: dq_atomic | query_stationary")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

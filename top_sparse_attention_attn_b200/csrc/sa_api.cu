@@ -9,6 +9,7 @@
 #include "sa_device.cuh"
 #include "sa_kv_bwd.h"
 #include "sa_launch.h"
+#include "sa_qblock.h"
 
 namespace {
 
@@ -144,6 +145,43 @@ bool use_kv_path(const sa_args* a) {
   return a->layout == SA_LAYOUT_BSND && a->topk > 0 && a->block_size == 64 && a->s_q == a->s_kv &&
          !a->kv_shared && a->cmp_topk == 0 && a->sinks == nullptr && G <= 128 &&
          sa::kv_path_built(a->d_qk, a->d_v);
+}
+
+// Query-stationary block kernels (TMA-fed): 64-row blocks, separate K / V, no compressed KV.
+bool use_qb_path(const sa_args* a) {
+  return a->topk > 0 && a->topk <= 256 && a->block_size == 64 && !a->kv_shared && a->cmp_topk == 0 &&
+         sa::qb_path_built(a->d_qk, a->d_v);
+}
+
+sa::QbArgs make_qb_args(const sa_args* a, int* status) {
+  sa::QbArgs q;
+  memset(&q, 0, sizeof(q));
+  Sizes s = sizes_of(a);
+  q.layout = a->layout;
+  q.B = a->batch;
+  q.s_q = a->s_q;
+  q.s_kv = a->s_kv;
+  q.Tq = (int)s.Tq;
+  q.Tkv = (int)s.Tkv;
+  q.Hq = a->n_heads_q;
+  q.Hkv = a->n_heads_kv;
+  q.G = a->n_heads_q / a->n_heads_kv;
+  q.dqk = a->d_qk;
+  q.dv = a->d_v;
+  q.topk = a->topk;
+  q.ori_mask = a->ori_mask_mode;
+  q.wl = a->ori_win_left;
+  q.wr = a->ori_win_right;
+  q.scale = a->scale;
+  q.scale_log2 = a->scale * 1.4426950408889634f;
+  q.q = static_cast<const bf16*>(a->q);
+  q.ori_idx = a->ori_idx;
+  q.ori_len = a->ori_topk_len;
+  q.cu_q = a->cu_seqlens_q;
+  q.cu_kv = a->cu_seqlens_kv;
+  q.sinks = a->sinks;
+  q.status = status;
+  return q;
 }
 
 struct KvGeom {
@@ -282,6 +320,12 @@ sa_status sa_fwd(const sa_args* args, const sa_fwd_out* out, void* ws, size_t ws
   }
   sa::Prob p = make_prob(args, status);
   if (cudaMemsetAsync(status, 0, sizeof(int), cs) != cudaSuccess) return SA_ERR_CUDA;
+  if (use_qb_path(args)) {
+    sa::QbArgs q = make_qb_args(args, status);
+    q.o = static_cast<bf16*>(out->o);
+    q.lse = out->lse;
+    return cuda_status(sa::launch_qb(q, args->k, args->v, false, cs));
+  }
   return cuda_status(sa::launch_fwd(p, static_cast<bf16*>(out->o), out->lse, cs));
 }
 
@@ -401,7 +445,12 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
     if (w.dq) {
       e = sa::launch_to_bf16(ka.dq_acc, static_cast<bf16*>(io->dq), s.Tq * args->n_heads_q * args->d_qk, cs);
     } else {
-      e = sa::launch_bwd_dq(p, static_cast<const bf16*>(io->d_o), io->lse, delta, out, cs);
+      sa::QbArgs q = make_qb_args(args, status);
+      q.d_o = static_cast<const bf16*>(io->d_o);
+      q.lse = const_cast<float*>(io->lse);
+      q.delta = delta;
+      q.dq = static_cast<bf16*>(io->dq);
+      e = sa::launch_qb(q, args->k, args->v, true, cs);
     }
   } else {
     e = sa::launch_bwd(p, static_cast<const bf16*>(io->o), static_cast<const bf16*>(io->d_o), io->lse, delta,

@@ -1,0 +1,32 @@
+// sa_qblock.h -- arguments of the query-stationary block kernels (forward, dQ pass).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sa_device.cuh"
+
+namespace sa {
+
+struct QbArgs {
+  int layout, B, s_q, s_kv, Tq, Tkv, Hq, Hkv, G, dqk, dv, topk, ori_mask;
+  long long wl, wr;
+  float scale, scale_log2;
+  const bf16* q;
+  const bf16* d_o;      // dQ pass
+  const int* ori_idx;
+  const int* ori_len;
+  const int* cu_q;
+  const int* cu_kv;
+  const float* sinks;   // forward
+  bf16* o;              // forward output
+  float* lse;           // forward output / dQ-pass input
+  const float* delta;   // dQ pass
+  bf16* dq;             // dQ-pass output
+  int* status;
+};
+
+bool qb_path_built(int dqk, int dv);
+cudaError_t launch_qb(const QbArgs& a, const void* k, const void* v, bool dq, cudaStream_t st);
+
+}  // namespace sa
