@@ -130,6 +130,11 @@ def count_work(w, inputs) -> dict:
         # token's G query and dO rows once per (token, slot) plus the KV blocks once
         "kv_flops": 4 * (w.d_qk + w.d_v) * triples,
         "kv_bytes": n_pairs * w.G * (w.d_qk + w.d_v) * 2 + 2 * n_pairs * w.G * 4 + kv_out + kv_out,
+        # ... with dQ formed in the same kernel: + the dQ contraction and the dQ partials
+        # (fp32, added once per (token, slot)) read-modify-written through L2
+        "kvq_flops": 2 * (3 * w.d_qk + 2 * w.d_v) * triples,
+        "kvq_bytes": n_pairs * w.G * (w.d_qk + w.d_v) * 2 + 2 * n_pairs * w.G * 4 + kv_out + kv_out
+                     + T * w.Hq * w.d_qk * 4 * 2,
         # query-stationary dQ pass: S, dP, dQ contractions over the gathered rows
         "dq_flops": 2 * (2 * w.d_qk + w.d_v) * triples,
         "dq_bytes": gathered + n_q + n_v + 2 * lse_b + n_q,
@@ -306,7 +311,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     t = to_torch(inputs, dev)
     flags = 0
     for f in filter(None, args.flags.split(",")):
-        flags |= {"dq_atomic": L.SA_FLAG_DQ_ATOMIC, "query_stationary": L.SA_FLAG_QUERY_STATIONARY_BWD}[f]
+        flags |= {"dq_separate": L.SA_FLAG_DQ_SEPARATE, "query_stationary": L.SA_FLAG_QUERY_STATIONARY_BWD}[f]
     sa = SparseAttention.from_workload(w, t, flags=flags)
     stream = torch.cuda.current_stream(dev)
     o, lse = sa.alloc_fwd()
@@ -413,12 +418,17 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     bwd_tflops = world * work["bwd_flops"] / (bwd_ms * 1e-3) / 1e12
     fwd_tflops = world * work["fwd_flops"] / (fwd_ms * 1e-3) / 1e12
     # roofline of the dominant backward kernel
-    keystat = dq_ms > 0.0
     kern = []
-    if keystat:
+    keystat = w.mode == "block" and w.block_size == 64 and "query_stationary" not in args.flags
+    if keystat and dq_ms > 0.0:
+        bwd_path = "key-stationary dK/dV + query-stationary dQ pass"
         kern.append(("kv_bwd_kernel (key-stationary dK/dV)", main_ms, work["kv_flops"], work["kv_bytes"]))
-        kern.append(("bwd_kernel<SCATTER=false> (query-stationary dQ)", dq_ms, work["dq_flops"], work["dq_bytes"]))
+        kern.append(("qb_kernel<dQ> (query-stationary dQ pass)", dq_ms, work["dq_flops"], work["dq_bytes"]))
+    elif keystat:
+        bwd_path = "key-stationary dK/dV/dQ (dQ by fp32 atomics)"
+        kern.append(("kv_bwd_kernel (key-stationary dK/dV/dQ)", main_ms, work["kvq_flops"], work["kvq_bytes"]))
     else:
+        bwd_path = "query-stationary fused (dK/dV scatter-add)"
         kern.append(("bwd_kernel (fused query-stationary backward)", main_ms, work["bwd_flops"],
                      work["bwd_main_bytes"]))
     name, kms, kflops, kbytes = max(kern, key=lambda x: x[1])
@@ -448,7 +458,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
                    "flags": args.flags or "default",
                    "visible_triples": work["triples"], "gathered_bytes": work["gathered_bytes"]},
         "fwd_tflops": fwd_tflops, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
-        "bwd_path": "key-stationary dK/dV + query-stationary dQ" if keystat else "query-stationary fused",
+        "bwd_path": bwd_path,
         "bwd_roofline_frac": max(t_bytes, t_flops) * 1e3 / bwd_ms,
         "roofline": roof, "clocks": clk.summary(), "gpu_launches": launches,
         "e2e": e2e,
@@ -491,7 +501,7 @@ def main():
     ap.add_argument("--override", default=None, help="workload overrides for profiling, e.g. S=2048")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--flags", default="", help="backward variant for measurements: dq_atomic | query_stationary")
+    ap.add_argument("--flags", default="", help="backward variant for measurements: dq_separate | query_stationary")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -100,13 +100,13 @@ typedef enum sa_dtype { SA_DTYPE_BF16 = 0, SA_DTYPE_FP16 = 1 } sa_dtype;
  * fastest measured).  Block-level selection with block_size 64, BSND, equal
  * query / key lengths, separate K and V and no sinks runs key-stationary by
  * default: one CTA per (kv block, chunk of the tokens that select it)
- * accumulates dK / dV on the tensor cores, and dQ comes from a query-stationary
- * pass.  Every other problem runs query-stationary. */
+ * accumulates dK / dV on the tensor cores and adds its dQ contributions to an
+ * fp32 accumulator with vector atomics (Tq*Hq*d_qk*4 workspace bytes).
+ * Every other problem runs query-stationary. */
 #define SA_FLAG_QUERY_STATIONARY_BWD 2u  /* force the query-stationary backward
                                             (dK / dV by fp32 scatter-add) */
-#define SA_FLAG_DQ_ATOMIC 4u   /* key-stationary backward: form dQ in the same kernel and
-                                  add it with fp32 atomics (needs Tq*Hq*d_qk*4 more
-                                  workspace bytes) instead of a separate pass */
+#define SA_FLAG_DQ_SEPARATE 4u  /* key-stationary backward: take dQ from a separate
+                                   query-stationary pass instead of atomics */
 
 /* The problem description shared by every entry point (host struct). */
 typedef struct sa_args {

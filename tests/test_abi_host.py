@@ -154,10 +154,10 @@ def test_bwd_workspace_size_contract():
     # key-stationary backward (block-level, BSND, 64-row blocks): + the inverse index
     n_lists, n_slots = 2 * 4 * 2, 2 * 128 * 4 * 4
     index = 2 * _align(4 * n_lists) + 2 * _align(4 * (n_lists + 1)) + 256 + _align(4 * n_slots)
-    st, n = _ws(_args())
+    st, n = _ws(_args(flags=L.SA_FLAG_DQ_SEPARATE))
     assert st == L.SA_OK and n == base + index
-    # ... + an fp32 dQ accumulator when dQ is formed in the same kernel
-    st, n = _ws(_args(flags=L.SA_FLAG_DQ_ATOMIC))
+    # ... + an fp32 dQ accumulator when dQ is formed in the same kernel (the default)
+    st, n = _ws(_args())
     assert st == L.SA_OK and n == base + index + _align(Tq * 16 * 192 * 4)
     a = _args(kv_shared=1, d_qk=576, d_v=512, kv=FAKE, n_heads_q=64, n_heads_kv=1, block_size=1,
               layout=L.SA_LAYOUT_TND, t_q=1000, t_kv=1000, t_cmp=250, cmp_topk=16, cmp_ratio=4,

@@ -54,15 +54,15 @@ def test_small_workload_all_elements(name):
 BLOCK_CASES = ["cfg1_full", "cfg2_small", "cfg2_future_len", "cfg5_small", "cfg5_empty_rows", "block_g24_128"]
 
 
-@pytest.mark.parametrize("flag", ["dq_atomic", "query_stationary"])
+@pytest.mark.parametrize("flag", ["dq_separate", "query_stationary"])
 @pytest.mark.parametrize("name", BLOCK_CASES)
 def test_block_level_backward_variants(name, flag):
-    """The block-level workloads through the other backward kernels: dQ formed in the
-    key-stationary kernel (fp32 atomics), and the fused query-stationary kernel."""
+    """The block-level workloads through the other backward kernels: dQ from a separate
+    query-stationary pass, and the fused query-stationary kernel."""
     _need_gpu()
     from top_sparse_attention_attn_b200 import _lib as L
     w, kw = SMALL[name]
-    flags = {"dq_atomic": L.SA_FLAG_DQ_ATOMIC, "query_stationary": L.SA_FLAG_QUERY_STATIONARY_BWD}[flag]
+    flags = {"dq_separate": L.SA_FLAG_DQ_SEPARATE, "query_stationary": L.SA_FLAG_QUERY_STATIONARY_BWD}[flag]
     run_full_comparison(w, kw, flags=flags)
 
 

@@ -31,7 +31,7 @@ SA_DTYPE_BF16 = 0
 SA_DTYPE_FP16 = 1
 SA_FLAG_CHECK = 1
 SA_FLAG_QUERY_STATIONARY_BWD = 2
-SA_FLAG_DQ_ATOMIC = 4
+SA_FLAG_DQ_SEPARATE = 4
 
 MASKS = {"none": SA_MASK_NONE, "causal": SA_MASK_CAUSAL, "band": SA_MASK_BAND}
 LAYOUTS = {"BSND": SA_LAYOUT_BSND, "TND": SA_LAYOUT_TND}

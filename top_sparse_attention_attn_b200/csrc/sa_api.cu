@@ -245,7 +245,7 @@ BwdWs bwd_ws_layout(const sa_args* a) {
     off += kAlign;
     w.entries = off;
     off += align_up(sizeof(int) * (size_t)k.n_slots);
-    if (a->flags & SA_FLAG_DQ_ATOMIC) {
+    if (!(a->flags & SA_FLAG_DQ_SEPARATE)) {
       w.dq = off;
       off += align_up((size_t)s.Tq * a->n_heads_q * a->d_qk * sizeof(float));
     }

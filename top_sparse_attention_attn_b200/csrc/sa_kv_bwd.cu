@@ -140,33 +140,47 @@ __global__ void __launch_bounds__(192, 1) kv_bwd_kernel(const __grid_constant__ 
   const uint32_t tmem = bars.tmem_base;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producer (whole warp)
+    // lane u issues the TMA loads of token u of the tile; the next tile's token
+    // ids are fetched while the current stage is being waited for.
+    const int row0 = b * a.S + 64 * j;
     if (lane == 0) {
       tma_prefetch_desc(&mapQ);
       tma_prefetch_desc(&mapDO);
-      const int row0 = b * a.S + 64 * j;
       mbar_arrive_tx(&bars.kv_full, (uint32_t)(64 * (DQK + DV) * 2));
       for (int s = 0; s < DQK / 64; ++s) tma_load_2d(sK + s * 64 * 128, &mapK, g * DQK + 64 * s, row0, &bars.kv_full);
       for (int s = 0; s < DV / 64; ++s) tma_load_2d(sV + s * 64 * 128, &mapV, g * DV + 64 * s, row0, &bars.kv_full);
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
-        const int st = i & 1;
-        if (i >= 2 && !mbar_wait(&bars.q_empty[st], ((i >> 1) - 1) & 1, abort_flag, a.status)) break;
-        const int n = min(TPT, ntok - i * TPT);
-        issued = i + 1;
-        mbar_arrive_tx(&bars.q_full[st], (uint32_t)(n * a.G * (DQK + DV) * 2));
-        for (int u = 0; u < n; ++u) {
-          const int tq = __ldg(toks + i * TPT + u);
-          const int row = tq * a.Hq + g * a.G;
-          const uint32_t off = (uint32_t)(u * RPT * 128);
-          for (int s = 0; s < DQK / 64; ++s)
-            tma_load_2d(sQ + st * PL::kQStage + s * 128 * 128 + off, &mapQ, 64 * s, row, &bars.q_full[st]);
-          for (int s = 0; s < DV / 64; ++s)
-            tma_load_2d(sDO + st * PL::kDOStage + s * 128 * 128 + off, &mapDO, 64 * s, row, &bars.q_full[st]);
-        }
+    }
+    int issued = 0;
+    int tq_next = (lane < TPT && lane < ntok) ? __ldg(toks + lane) : 0;
+    for (int i = 0; i < ntiles; ++i) {
+      const int st = i & 1;
+      const int n = min(TPT, ntok - i * TPT);
+      const int tq = tq_next;
+      if (i + 1 < ntiles) {
+        const int u2 = (i + 1) * TPT + lane;
+        tq_next = (lane < TPT && u2 < ntok) ? __ldg(toks + u2) : 0;
       }
-      // drain: before the CTA can exit, every TMA load it issued must have landed
-      // (on an abort some stages are never consumed)
+      bool ok = true;
+      if (lane == 0 && i >= 2) ok = mbar_wait(&bars.q_empty[st], ((i >> 1) - 1) & 1, abort_flag, a.status);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      issued = i + 1;
+      if (lane == 0) mbar_arrive_tx(&bars.q_full[st], (uint32_t)(n * a.G * (DQK + DV) * 2));
+      __syncwarp();
+      if (lane < n) {
+        const int row = tq * a.Hq + g * a.G;
+        const uint32_t off = (uint32_t)(lane * RPT * 128);
+        for (int s = 0; s < DQK / 64; ++s)
+          tma_load_2d(sQ + st * PL::kQStage + s * 128 * 128 + off, &mapQ, 64 * s, row, &bars.q_full[st]);
+        for (int s = 0; s < DV / 64; ++s)
+          tma_load_2d(sDO + st * PL::kDOStage + s * 128 * 128 + off, &mapDO, 64 * s, row, &bars.q_full[st]);
+      }
+      __syncwarp();
+    }
+    // drain: before the CTA can exit, every TMA load it issued must have landed
+    // (on an abort some stages are never consumed)
+    if (lane == 0) {
       mbar_wait_drain(&bars.kv_full, 0);
       for (int st = 0; st < 2; ++st) {
         int last = -1;
@@ -236,18 +250,30 @@ __global__ void __launch_bounds__(192, 1) kv_bwd_kernel(const __grid_constant__ 
     const int u = r / RPT, hh = r - u * RPT;
     const int blk_row0 = 64 * j;
     bool ok = true;
+    // row metadata of tile i (token, lse, Delta), fetched one tile ahead
+    int tq_n = 0;
+    float lse_n = INFINITY, dlt_n = 0.f;
+    auto fetch = [&](int i2) {
+      const int n2 = min(TPT, ntok - i2 * TPT);
+      tq_n = 0;
+      lse_n = INFINITY;
+      dlt_n = 0.f;
+      if (i2 < ntiles && u < n2 && hh < a.G) {
+        tq_n = __ldg(toks + i2 * TPT + u);
+        const long long ih = (long long)tq_n * a.Hq + g * a.G + hh;
+        lse_n = __ldg(a.lse + ih);
+        dlt_n = __ldg(a.delta + ih);
+      }
+    };
+    fetch(0);
     for (int i = 0; i < ntiles && ok; ++i) {
       const int n = min(TPT, ntok - i * TPT);
       const bool vrow = (u < n) && (hh < a.G);
-      int tq = 0, ta = 0;
-      float lse2 = INFINITY, dlt = 0.f;
-      if (vrow) {
-        tq = __ldg(toks + i * TPT + u);
-        ta = tq - b * a.S;  // equal query / key lengths (BSND)
-        const long long ih = (long long)tq * a.Hq + g * a.G + hh;
-        lse2 = __ldg(a.lse + ih) * kLog2eKv;
-        dlt = __ldg(a.delta + ih);
-      }
+      const int tq = tq_n;
+      const int ta = tq - b * a.S;  // equal query / key lengths (BSND)
+      const float lse2 = vrow ? lse_n * kLog2eKv : INFINITY;
+      const float dlt = vrow ? dlt_n : 0.f;
+      fetch(i + 1);
       // visible key rows of this block for this query row
       int vlo = 0, vhi = -1;
       if (vrow) {

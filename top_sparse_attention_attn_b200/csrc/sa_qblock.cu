@@ -33,7 +33,7 @@ template <int DQK, int DV, bool DQ>
 struct QbPlan {
   static constexpr int kStage = 64 * (DQK + DV) * 2;  // K block + V block
   static constexpr int kComb = 4 * 16 * (DQ ? DQK : DV) * 4 + 4 * 16 * 2 * 4;  // partials + (m, l)
-  static constexpr int kBudget = 227 * 1024 - 1024 - kComb - 5 * 1024;  // 5 KB static shared memory
+  static constexpr int kBudget = 227 * 1024 - 1024 - kComb - 6 * 1024;  // 6 KB static shared memory
   static constexpr int kStages = (kBudget / kStage) > 6 ? 6 : (kBudget / kStage);
   static constexpr int oRing = 0;
   static constexpr int oComb = kStages * kStage;
@@ -51,24 +51,32 @@ struct QbBars {
   int abort_flag;
 };
 
-// Per work item: the usable slots (valid, in range, not fully masked), in slot order.
-__device__ __forceinline__ int qb_slots(const QbArgs& a, const Unit& u, int* xs) {
+// Warp-collective: the usable slots of a work item (valid, in range, not fully
+// masked), in slot order, written to xs (shared); returns their number.
+__device__ __forceinline__ int qb_slots(const QbArgs& a, const Unit& u, int* xs, int lane) {
   const long long ug = (long long)u.tq * a.Hkv + u.g;
   int n = a.topk;
   if (a.ori_len) n = min(n, max(0, __ldg(a.ori_len + ug)));
   int cnt = 0;
-  for (int s = 0; s < n; ++s) {
-    const int x = __ldg(a.ori_idx + ug * a.topk + s);
-    if (x < 0) continue;
-    const long long first = (long long)x * 64;
-    if (first >= u.Lk) continue;
-    if (a.ori_mask == kMaskCausal && first > u.ta) continue;
-    if (a.ori_mask == kMaskBand) {
-      const long long last = min(first + 63, (long long)u.Lk - 1);
-      if (first > (long long)u.ta + a.wr || last < (long long)u.ta - a.wl) continue;
+  for (int s0 = 0; s0 < n; s0 += 32) {
+    const int s = s0 + lane;
+    bool ok = false;
+    int x = -1;
+    if (s < n) {
+      x = __ldg(a.ori_idx + ug * a.topk + s);
+      const long long first = (long long)x * 64;
+      ok = x >= 0 && first < u.Lk;
+      if (a.ori_mask == kMaskCausal) ok = ok && first <= u.ta;
+      if (a.ori_mask == kMaskBand) {
+        const long long last = min(first + 63, (long long)u.Lk - 1);
+        ok = ok && first <= (long long)u.ta + a.wr && last >= (long long)u.ta - a.wl;
+      }
     }
-    xs[cnt++] = x;
+    const unsigned m = __ballot_sync(0xffffffffu, ok);
+    if (ok) xs[cnt + __popc(m & ((1u << lane) - 1u))] = x;
+    cnt += __popc(m);
   }
+  __syncwarp();
   return cnt;
 }
 
@@ -103,7 +111,7 @@ __global__ void __launch_bounds__(160, 1) qb_kernel(const __grid_constant__ CUte
   constexpr int NV = DV / 16;    // k steps over d_v
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ QbBars bars;
-  __shared__ int slot_x[4][256];  // per consumer warp: the current item's usable block indices
+  __shared__ int slot_x[5][256];  // per warp: the current item's usable block indices
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t ring = smem_u32(smem + PL::oRing);
@@ -124,31 +132,41 @@ __global__ void __launch_bounds__(160, 1) qb_kernel(const __grid_constant__ CUte
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
+    int* xs = slot_x[4];
+    long long t = 0;  // blocks streamed so far
+    bool ok = true;
     if (lane == 0) {
-      int xs[256];
-      long long t = 0;  // blocks streamed so far
-      bool ok = true;
-      for (long long it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
-        const int unit = (int)(it / n_hsl);
-        const int tq = unit / a.Hkv, g = unit - tq * a.Hkv;
-        const Unit u = qb_unit(a, tq, g);
-        const int n = qb_slots(a, u, xs);
-        for (int i = 0; i < n; ++i, ++t) {
-          const int st = (int)(t % S);
+      tma_prefetch_desc(&mapK);
+      tma_prefetch_desc(&mapV);
+    }
+    for (long long it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+      const int unit = (int)(it / n_hsl);
+      const int tq = unit / a.Hkv, g = unit - tq * a.Hkv;
+      const Unit u = qb_unit(a, tq, g);
+      const int n = qb_slots(a, u, xs, lane);
+      for (int i = 0; i < n; ++i, ++t) {
+        const int st = (int)(t % S);
+        if (lane == 0) {
           if (t >= S && !mbar_wait(&bars.empty[st], (uint32_t)(((t / S) - 1) & 1), abort_flag, a.status)) {
             ok = false;
-            break;
+          } else {
+            const uint32_t sk = ring + st * PL::kStage, sv = sk + 64 * DQK * 2;
+            const int row = u.kv0 + 64 * xs[i];
+            mbar_arrive_tx(&bars.full[st], (uint32_t)PL::kStage);
+            for (int s2 = 0; s2 < DQK / 64; ++s2)
+              tma_load_2d(sk + s2 * 8192, &mapK, g * DQK + 64 * s2, row, &bars.full[st]);
+            for (int s2 = 0; s2 < DV / 64; ++s2)
+              tma_load_2d(sv + s2 * 8192, &mapV, g * DV + 64 * s2, row, &bars.full[st]);
           }
-          const uint32_t sk = ring + st * PL::kStage, sv = sk + 64 * DQK * 2;
-          const int row = u.kv0 + 64 * xs[i];
-          mbar_arrive_tx(&bars.full[st], (uint32_t)PL::kStage);
-          for (int s = 0; s < DQK / 64; ++s) tma_load_2d(sk + s * 8192, &mapK, g * DQK + 64 * s, row, &bars.full[st]);
-          for (int s = 0; s < DV / 64; ++s) tma_load_2d(sv + s * 8192, &mapV, g * DV + 64 * s, row, &bars.full[st]);
         }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
       }
-      // drain: the last S stages must have landed before the CTA exits
-      for (long long k = (t > S ? t - S : 0); k < t; ++k) mbar_wait_drain(&bars.full[k % S], (uint32_t)((k / S) & 1));
+      __syncwarp();
     }
+    // drain: the last S stages must have landed before the CTA exits
+    if (lane == 0)
+      for (long long k = (t > S ? t - S : 0); k < t; ++k) mbar_wait_drain(&bars.full[k % S], (uint32_t)((k / S) & 1));
     return;
   }
 
@@ -164,10 +182,7 @@ __global__ void __launch_bounds__(160, 1) qb_kernel(const __grid_constant__ CUte
     const int h0 = g * a.G + hsl * 16;
     const int nh = min(16, a.G - hsl * 16);
     int* xs = slot_x[warp];
-    int n = 0;
-    if (lane == 0) n = qb_slots(a, u, xs);
-    n = __shfl_sync(0xffffffffu, n, 0);
-    __syncwarp();
+    const int n = qb_slots(a, u, xs, lane);
 
     // query rows as A fragments (rows >= nh are zero)
     uint32_t qf[NQK][4];
