@@ -185,7 +185,7 @@ sa::QbArgs make_qb_args(const sa_args* a, int* status) {
 }
 
 struct KvGeom {
-  int RPT, TPT, nblk, n_lists, chunk;
+  int RPT, TPT, nblk, n_lists, chunk, nwin, win_tokens;
   long long n_slots, max_work;
 };
 
@@ -195,7 +195,21 @@ KvGeom kv_geometry(const sa_args* a) {
   k.RPT = (G + 7) / 8 * 8;
   k.TPT = 128 / k.RPT;
   k.nblk = (a->s_kv + 63) / 64;
-  k.n_lists = a->batch * a->n_heads_kv * k.nblk;
+  // token windows: with dQ added by atomics, a window's fp32 dQ rows (~24 MB) stay
+  // in L2 while the CTAs of that window run
+  // Windows pay off only when a window's dQ rows fit in L2 (<= 48 MB) while each
+  // (window, block) cell still holds enough tokens (>= 128 on average) that the
+  // extra dK / dV flushes stay cheap; otherwise one window spans the sequence.
+  k.win_tokens = a->s_q > 0 ? a->s_q : 1;
+  if (!(a->flags & SA_FLAG_DQ_SEPARATE) && a->topk > 0) {
+    long long fit = (48ll << 20) / ((long long)a->n_heads_q * a->d_qk * 4);
+    fit = fit / 64 * 64;
+    const long long need = 128ll * k.nblk / a->topk;
+    if (fit >= 64 && fit >= need && fit < k.win_tokens) k.win_tokens = (int)fit;
+  }
+  k.nwin = (a->s_q + k.win_tokens - 1) / k.win_tokens;
+  if (k.nwin < 1) k.nwin = 1;
+  k.n_lists = a->batch * k.nwin * a->n_heads_kv * k.nblk;
   k.n_slots = (long long)a->batch * a->s_q * a->n_heads_kv * a->topk;
   // chunk of tokens per CTA: ~4 work items per SM, between 4 tiles and 512 tokens
   long long want = (k.n_slots + 148 * 4 - 1) / (148 * 4);
@@ -209,11 +223,12 @@ KvGeom kv_geometry(const sa_args* a) {
 }
 
 // Workspace: [status word][delta][dK or dKV acc][dV acc][dCmp acc]
-//            + key-stationary path: [counts][cursor][list_off][chunk_off][work][entries][dQ acc]
+//            + key-stationary path: [dQ acc][counts][cursor] | [list_off][chunk_off][work][entries]
+// Everything before `zero_end` is cleared at the start of each call with one memset.
 struct BwdWs {
   size_t status, delta, dk, dv, dcmp;
-  size_t counts, cursor, list_off, chunk_off, work, entries, dq;
-  size_t total;
+  size_t dq, counts, cursor, list_off, chunk_off, work, entries;
+  size_t zero_end, total;
 };
 
 BwdWs bwd_ws_layout(const sa_args* a) {
@@ -233,10 +248,15 @@ BwdWs bwd_ws_layout(const sa_args* a) {
   off += align_up((size_t)s.Tcmp * a->n_heads_kv * a->d_qk * sizeof(float));
   if (use_kv_path(a)) {
     KvGeom k = kv_geometry(a);
+    if (!(a->flags & SA_FLAG_DQ_SEPARATE)) {
+      w.dq = off;
+      off += align_up((size_t)s.Tq * a->n_heads_q * a->d_qk * sizeof(float));
+    }
     w.counts = off;
     off += align_up(sizeof(int) * k.n_lists);
     w.cursor = off;
     off += align_up(sizeof(int) * k.n_lists);
+    w.zero_end = off;
     w.list_off = off;
     off += align_up(sizeof(int) * (k.n_lists + 1));
     w.chunk_off = off;
@@ -245,10 +265,8 @@ BwdWs bwd_ws_layout(const sa_args* a) {
     off += kAlign;
     w.entries = off;
     off += align_up(sizeof(int) * (size_t)k.n_slots);
-    if (!(a->flags & SA_FLAG_DQ_SEPARATE)) {
-      w.dq = off;
-      off += align_up((size_t)s.Tq * a->n_heads_q * a->d_qk * sizeof(float));
-    }
+  } else {
+    w.zero_end = off;
   }
   w.total = off;
   return w;
@@ -372,10 +390,8 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
   const long long nk = s.Tkv * args->n_heads_kv * args->d_qk;
   const long long nv = s.Tkv * args->n_heads_kv * args->d_v;
   const long long nc = s.Tcmp * args->n_heads_kv * args->d_qk;
-  // zero the accumulators and dSinks (the index region is cleared by its own kernels)
-  const size_t zero_end = w.counts ? w.counts : w.total;
-  if (cudaMemsetAsync(base, 0, zero_end, cs) != cudaSuccess) return SA_ERR_CUDA;
-  if (w.dq && cudaMemsetAsync(base + w.dq, 0, w.total - w.dq, cs) != cudaSuccess) return SA_ERR_CUDA;
+  // zero the accumulators and the index counters (one memset), and dSinks
+  if (cudaMemsetAsync(base, 0, w.zero_end, cs) != cudaSuccess) return SA_ERR_CUDA;
   if (sinks && cudaMemsetAsync(io->dsinks, 0, sizeof(float) * args->n_heads_q, cs) != cudaSuccess)
     return SA_ERR_CUDA;
   cudaError_t e = sa::launch_delta(static_cast<const bf16*>(io->o), static_cast<const bf16*>(io->d_o), delta,
@@ -394,6 +410,8 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
     ia.S = args->s_q;
     ia.nblk = k.nblk;
     ia.n_lists = k.n_lists;
+    ia.nwin = k.nwin;
+    ia.win_tokens = k.win_tokens;
     ia.chunk_tokens = k.chunk;
     ia.ori_mask = args->ori_mask_mode;
     ia.wl = args->ori_win_left;
@@ -416,6 +434,7 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
     ka.TPT = k.TPT;
     ka.nblk = k.nblk;
     ka.n_lists = k.n_lists;
+    ka.nwin = k.nwin;
     ka.chunk_tokens = k.chunk;
     ka.ori_mask = args->ori_mask_mode;
     ka.wl = args->ori_win_left;
@@ -442,9 +461,7 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
     kl.dv = args->d_v;
     kl.max_work = k.max_work;
     if (sa::launch_kv_bwd(kl, w.dq != 0, cs) != cudaSuccess) return SA_ERR_CUDA;
-    if (w.dq) {
-      e = sa::launch_to_bf16(ka.dq_acc, static_cast<bf16*>(io->dq), s.Tq * args->n_heads_q * args->d_qk, cs);
-    } else {
+    if (!w.dq) {
       sa::QbArgs q = make_qb_args(args, status);
       q.d_o = static_cast<const bf16*>(io->d_o);
       q.lse = const_cast<float*>(io->lse);
@@ -457,14 +474,20 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
                        out, cs);
   }
   if (e != cudaSuccess) return SA_ERR_CUDA;
-  if (args->kv_shared) {
-    e = sa::launch_to_bf16(out.dk_acc, static_cast<bf16*>(io->dkv), nk, cs);
-  } else {
-    e = sa::launch_to_bf16(out.dk_acc, static_cast<bf16*>(io->dk), nk, cs);
-    if (e == cudaSuccess) e = sa::launch_to_bf16(out.dv_acc, static_cast<bf16*>(io->dv), nv, cs);
+  {
+    sa::Cvt jobs[4];
+    int nj = 0;
+    if (args->kv_shared) {
+      jobs[nj++] = sa::Cvt{out.dk_acc, static_cast<bf16*>(io->dkv), nk};
+    } else {
+      jobs[nj++] = sa::Cvt{out.dk_acc, static_cast<bf16*>(io->dk), nk};
+      jobs[nj++] = sa::Cvt{out.dv_acc, static_cast<bf16*>(io->dv), nv};
+    }
+    if (args->cmp_topk > 0) jobs[nj++] = sa::Cvt{out.dcmp_acc, static_cast<bf16*>(io->dcmp_kv), nc};
+    if (w.dq) jobs[nj++] = sa::Cvt{reinterpret_cast<float*>(base + w.dq), static_cast<bf16*>(io->dq),
+                                   s.Tq * args->n_heads_q * args->d_qk};
+    e = sa::launch_to_bf16_multi(jobs, nj, cs);
   }
-  if (e == cudaSuccess && args->cmp_topk > 0)
-    e = sa::launch_to_bf16(out.dcmp_acc, static_cast<bf16*>(io->dcmp_kv), nc, cs);
   return cuda_status(e);
 }
 

@@ -20,8 +20,8 @@
 // At the end dK^T / dV^T (scaled) are added to the fp32 dK / dV accumulators;
 // blocks split into several chunks meet there.
 //
-// Warp roles (6 warps): 0 = TMA producer, 1 = MMA issuer + TMEM owner,
-// 2..5 = softmax / epilogue (thread = query row = TMEM lane).
+// Warp roles: 0 = TMA producer, 1 = MMA issuer + TMEM owner, 2..5 = softmax /
+// dK-dV epilogue (thread = query row = TMEM lane), 6..9 (with dQ) = dQ epilogue.
 // Every wait is bounded (sa_tc.cuh): on timeout the CTA raises the status
 // word, skips the rest of its work, drains and frees TMEM.
 #include <cuda.h>
@@ -71,7 +71,7 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 }
 
 template <int DQK, int DV, bool WITH_DQ>
-__global__ void __launch_bounds__(192, 1) kv_bwd_kernel(const __grid_constant__ CUtensorMap mapQ,
+__global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __grid_constant__ CUtensorMap mapQ,
                                                         const __grid_constant__ CUtensorMap mapDO,
                                                         const __grid_constant__ CUtensorMap mapK,
                                                         const __grid_constant__ CUtensorMap mapV,
@@ -93,9 +93,10 @@ __global__ void __launch_bounds__(192, 1) kv_bwd_kernel(const __grid_constant__ 
   }
   const int L = lo;
   const int chunk = w - __ldg(a.chunk_off + L);
+  // list id = ((batch * nwin + window) * Hkv + kv-head) * nblk + block
   const int j = L % a.nblk;
-  const int bg = L / a.nblk;
-  const int g = bg % a.Hkv, b = bg / a.Hkv;
+  const int rest = L / a.nblk;
+  const int g = rest % a.Hkv, b = (rest / a.Hkv) / a.nwin;
   const int list_begin = __ldg(a.list_off + L), list_end = __ldg(a.list_off + L + 1);
   const int tok0 = list_begin + chunk * a.chunk_tokens;
   const int ntok = min(a.chunk_tokens, list_end - tok0);
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(192, 1) kv_bwd_kernel(const __grid_constant__ 
       }
       mma_commit(&bars.acc_done);
     }
-  } else {
+  } else if (warp < 6) {
     // ------------------------------------------------------------ softmax / epilogue
     const int sub = warp & 3;
     const int r = 32 * sub + lane;  // query row of the tile = TMEM lane
@@ -288,35 +289,39 @@ __global__ void __launch_bounds__(192, 1) kv_bwd_kernel(const __grid_constant__ 
       }
       if (!mbar_wait(&bars.s_full, i & 1, abort_flag, a.status)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[4][16], dr[4][16];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld16(lane_base + PL::cS + 16 * c, sr[c]);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld16(lane_base + PL::cDP + 16 * c, dr[c]);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        reg_dep16(sr[c]);
-        reg_dep16(dr[c]);
-      }
-      // P and dS for the 64 key rows, packed to bf16 pairs
+      // P and dS for the 64 key rows, packed to bf16 pairs; two halves of 32
+      // columns keep the register footprint small
       uint32_t pk[32], dk[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sr[2][16], dr[2][16];
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          float pv[2], dsv[2];
+        for (int c = 0; c < 2; ++c) tmem_ld16(lane_base + PL::cS + 32 * half + 16 * c, sr[c]);
 #pragma unroll
-          for (int q2 = 0; q2 < 2; ++q2) {
-            const int col = 16 * c + e + q2;
-            const bool vis = col >= vlo && col <= vhi;
-            const float p = vis ? exp2f(__uint_as_float(sr[c][e + q2]) * a.scale_log2 - lse2) : 0.f;
-            pv[q2] = p;
-            dsv[q2] = p * (__uint_as_float(dr[c][e + q2]) - dlt);
-          }
-          pk[(16 * c + e) >> 1] = pack_bf16(pv[0], pv[1]);
-          dk[(16 * c + e) >> 1] = pack_bf16(dsv[0], dsv[1]);
+        for (int c = 0; c < 2; ++c) tmem_ld16(lane_base + PL::cDP + 32 * half + 16 * c, dr[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          reg_dep16(sr[c]);
+          reg_dep16(dr[c]);
         }
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            float pv[2], dsv[2];
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+              const int col = 32 * half + 16 * c + e + q2;
+              const bool vis = col >= vlo && col <= vhi;
+              const float p = vis ? exp2f(__uint_as_float(sr[c][e + q2]) * a.scale_log2 - lse2) : 0.f;
+              pv[q2] = p;
+              dsv[q2] = p * (__uint_as_float(dr[c][e + q2]) - dlt);
+            }
+            pk[(32 * half + 16 * c + e) >> 1] = pack_bf16(pv[0], pv[1]);
+            dk[(32 * half + 16 * c + e) >> 1] = pack_bf16(dsv[0], dsv[1]);
+          }
+      }
       tc_fence_before();
       // the P / dS buffer is free once the previous tile's dK^T (and dQ) MMAs are done
       if (i > 0 && !mbar_wait(&bars.tile_done, (i - 1) & 1, abort_flag, a.status)) { ok = false; break; }
@@ -336,26 +341,6 @@ __global__ void __launch_bounds__(192, 1) kv_bwd_kernel(const __grid_constant__ 
                      : "memory");
       fence_async_smem();
       mbar_arrive(&bars.ds_full);
-      if (WITH_DQ) {
-        if (!mbar_wait(&bars.dq_full, i & 1, abort_flag, a.status)) { ok = false; break; }
-        tc_fence_after();
-        float* dst = a.dq_acc + ((long long)tq * a.Hq + g * a.G + hh) * DQK;
-#pragma unroll 1
-        for (int c = 0; c < DQK; c += 16) {
-          uint32_t v[16];
-          tmem_ld16(lane_base + PL::cDQ + c, v);
-          tmem_wait_ld();
-          reg_dep16(v);
-          if (vrow) {
-#pragma unroll
-            for (int e = 0; e < 16; e += 4)
-              red_add_v4(dst + c + e, __uint_as_float(v[e]) * a.scale, __uint_as_float(v[e + 1]) * a.scale,
-                         __uint_as_float(v[e + 2]) * a.scale, __uint_as_float(v[e + 3]) * a.scale);
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(&bars.dq_free);
-      }
     }
     // ---- epilogue: dV^T and dK^T (scaled) into the fp32 accumulators
     if (ok && mbar_wait(&bars.acc_done, 0, abort_flag, a.status)) {
@@ -390,6 +375,38 @@ __global__ void __launch_bounds__(192, 1) kv_bwd_kernel(const __grid_constant__ 
       }
     }
     tc_fence_before();
+  } else if (WITH_DQ) {
+    // ------------------------------------------------------------ dQ epilogue (warps 6..9)
+    // reads each tile's dQ partial from TMEM and adds it (scaled) to the fp32 dQ
+    // accumulator with vector atomics, overlapping the next tile's softmax
+    const int sub = warp & 3;
+    const int r = 32 * sub + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * sub) << 16);
+    const int u = r / RPT, hh = r - u * RPT;
+    int tq_n = (u < min(TPT, ntok) && hh < a.G) ? __ldg(toks + u) : -1;
+    for (int i = 0; i < ntiles; ++i) {
+      const int tq = tq_n;
+      const int n2 = min(TPT, ntok - (i + 1) * TPT);
+      tq_n = (i + 1 < ntiles && u < n2 && hh < a.G) ? __ldg(toks + (i + 1) * TPT + u) : -1;
+      if (!mbar_wait(&bars.dq_full, i & 1, abort_flag, a.status)) break;
+      tc_fence_after();
+      float* dst = a.dq_acc + ((long long)(tq < 0 ? 0 : tq) * a.Hq + g * a.G + hh) * DQK;
+#pragma unroll 1
+      for (int c = 0; c < DQK; c += 16) {
+        uint32_t v[16];
+        tmem_ld16(lane_base + PL::cDQ + c, v);
+        tmem_wait_ld();
+        reg_dep16(v);
+        if (tq >= 0) {
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            red_add_v4(dst + c + e, __uint_as_float(v[e]) * a.scale, __uint_as_float(v[e + 1]) * a.scale,
+                       __uint_as_float(v[e + 2]) * a.scale, __uint_as_float(v[e + 3]) * a.scale);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars.dq_free);
+    }
   }
   __syncthreads();
   if (warp == 1) {
@@ -400,7 +417,8 @@ __global__ void __launch_bounds__(192, 1) kv_bwd_kernel(const __grid_constant__ 
 }
 
 // ---------------------------------------------------------------------------
-// inverse index: for every (batch, kv-head, block) the tokens that select it
+// inverse index: for every (batch, token window, kv-head, block) the tokens
+// of the window that select the block
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ bool kv_slot_list(const KvIndexArgs& a, long long e, int* list, int* tq_out) {
   const int slot = (int)(e % a.topk);
@@ -419,7 +437,10 @@ __device__ __forceinline__ bool kv_slot_list(const KvIndexArgs& a, long long e, 
     long long last = min(first + 63, (long long)a.S - 1);
     if (first > (long long)ta + a.wr || last < (long long)ta - a.wl) return false;
   }
-  *list = (b * a.Hkv + g) * a.nblk + x;
+  // keyed by the token's window first, so that CTAs launched together add their dQ
+  // contributions to a window of tokens whose fp32 accumulators stay in L2
+  const int win = ta / a.win_tokens;
+  *list = ((b * a.nwin + win) * a.Hkv + g) * a.nblk + x;
   *tq_out = tq;
   return true;
 }
@@ -510,15 +531,14 @@ static cudaError_t kv_launch_t(const KvLaunch& L, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   if (L.max_work == 0) return cudaSuccess;
   mark_begin(st, kTimeBwdKV);
-  k<<<(unsigned)L.max_work, 192, PL::kSmem, st>>>(mq, mdo, mk, mv, a);
+  k<<<(unsigned)L.max_work, WITH_DQ ? 320 : 192, PL::kSmem, st>>>(mq, mdo, mk, mv, a);
   count_launch();
   mark_end(st, kTimeBwdKV);
   return cudaGetLastError();
 }
 
 cudaError_t launch_kv_index(const KvIndexArgs& a, cudaStream_t st) {
-  if (cudaMemsetAsync(a.counts, 0, sizeof(int) * a.n_lists, st) != cudaSuccess) return cudaErrorUnknown;
-  if (cudaMemsetAsync(a.cursor, 0, sizeof(int) * a.n_lists, st) != cudaSuccess) return cudaErrorUnknown;
+  // counts and cursor arrive zeroed (cleared with the rest of the workspace)
   if (a.n_slots > 0) {
     kv_count_kernel<<<(unsigned)((a.n_slots + 255) / 256), 256, 0, st>>>(a);
     count_launch();

@@ -14,6 +14,7 @@ struct KvIndexArgs {
   const int* ori_len;   // [Tq, Hkv] or null
   long long n_slots;    // Tq * Hkv * topk
   int topk, Hkv, S, nblk, n_lists, chunk_tokens, ori_mask;
+  int nwin, win_tokens;  // lists are keyed by (batch, token window, kv-head, block)
   long long wl, wr;
   int* counts;          // [n_lists]
   int* cursor;          // [n_lists]
@@ -25,6 +26,7 @@ struct KvIndexArgs {
 
 struct KvArgs {
   int S, Hq, Hkv, G, RPT, TPT, nblk, n_lists, chunk_tokens, ori_mask;
+  int nwin;
   long long wl, wr;
   float scale, scale_log2;
   const int* list_off;

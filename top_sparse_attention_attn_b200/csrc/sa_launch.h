@@ -47,6 +47,13 @@ cudaError_t launch_delta(const bf16* o, const bf16* d_o, float* delta, long long
 cudaError_t launch_bwd(const Prob& p, const bf16* o, const bf16* d_o, const float* lse,
                        const float* delta, const BwdOut& out, cudaStream_t st);
 cudaError_t launch_to_bf16(const float* src, bf16* dst, long long n, cudaStream_t st);
+// Up to four fp32 -> bf16 conversions in one launch (each n a multiple of 8).
+struct Cvt {
+  const float* src;
+  bf16* dst;
+  long long n;
+};
+cudaError_t launch_to_bf16_multi(const Cvt* jobs, int njobs, cudaStream_t st);
 cudaError_t launch_check(const Prob& p, cudaStream_t st);
 cudaError_t launch_debug_resolve(const Prob& p, int* rows, int* counts, int max_rows,
                                  cudaStream_t st);

@@ -529,6 +529,30 @@ __global__ void __launch_bounds__(256) to_bf16_kernel(const float* __restrict__ 
   }
 }
 
+struct CvtJobs {
+  Cvt job[4];
+  long long end8[4];  // cumulative 8-element group counts
+  int n;
+};
+
+__global__ void __launch_bounds__(256) to_bf16_multi_kernel(const CvtJobs J) {
+  const long long total = J.end8[J.n - 1];
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    int k = 0;
+    while (i >= J.end8[k]) ++k;
+    const long long li = i - (k ? J.end8[k - 1] : 0);
+    const float4* src = reinterpret_cast<const float4*>(J.job[k].src);
+    float4 a = __ldg(src + 2 * li), b = __ldg(src + 2 * li + 1);
+    uint4 r;
+    r.x = pack_bf16(a.x, a.y);
+    r.y = pack_bf16(a.z, a.w);
+    r.z = pack_bf16(b.x, b.y);
+    r.w = pack_bf16(b.z, b.w);
+    reinterpret_cast<uint4*>(J.job[k].dst)[li] = r;
+  }
+}
+
 __global__ void check_kernel(const Prob p) {
   long long ug = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (ug >= (long long)p.Tq * p.Hkv) return;
@@ -653,6 +677,25 @@ cudaError_t launch_to_bf16(const float* src, bf16* dst, long long n, cudaStream_
   long long blocks = (n8 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   to_bf16_kernel<<<(unsigned)blocks, 256, 0, st>>>(src, dst, n8);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_to_bf16_multi(const Cvt* jobs, int njobs, cudaStream_t st) {
+  CvtJobs J;
+  J.n = 0;
+  long long acc = 0;
+  for (int k = 0; k < njobs && k < 4; ++k) {
+    if (jobs[k].n <= 0) continue;
+    J.job[J.n] = jobs[k];
+    acc += jobs[k].n / 8;
+    J.end8[J.n] = acc;
+    ++J.n;
+  }
+  if (J.n == 0) return cudaSuccess;
+  long long blocks = (acc + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  to_bf16_multi_kernel<<<(unsigned)blocks, 256, 0, st>>>(J);
   count_launch();
   return cudaGetLastError();
 }
