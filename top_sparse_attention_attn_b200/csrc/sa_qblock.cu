@@ -230,15 +230,26 @@ __global__ void __launch_bounds__(160, 1) qb_kernel(const __grid_constant__ CUte
         const uint32_t sk = ring + st * PL::kStage, sv = sk + 64 * DQK * 2;
         const int x = xs[i];
         // S_w = Q K_w^T: the warp's 16 block rows
+        // two independent accumulation chains per n tile (even / odd k steps)
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int k = 0; k < NQK; ++k) {
           uint32_t b[4];
           const int rr = 16 * warp + (lane & 7) + ((lane >> 4) << 3);
           ldsm_x4(b, slab_addr(sk, 64, rr, 2 * k + ((lane >> 3) & 1)));
-          mma16816(s[0], qf[k], b[0], b[1]);
-          mma16816(s[1], qf[k], b[2], b[3]);
+          if (k & 1) {
+            mma16816(s2[0], qf[k], b[0], b[1]);
+            mma16816(s2[1], qf[k], b[2], b[3]);
+          } else {
+            mma16816(s[0], qf[k], b[0], b[1]);
+            mma16816(s[1], qf[k], b[2], b[3]);
+          }
         }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) s[nt][j] += s2[nt][j];
         // visibility of the warp's block rows for this query token
         const int rbase = 64 * x + 16 * warp;
         bool vis[2][2];
