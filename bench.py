@@ -329,52 +329,79 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     torch.cuda.synchronize()
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-    for e in ev:  # materialise the raw cudaEvent_t handles
-        for x in e:
-            x.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    launches0 = L.sa_kernel_launch_count()
-    with ClockSampler(local_rank) as clk:
+    # The timed steps replay a CUDA graph of each call (forward, backward) unless
+    # --no-graph: the calls enqueue only kernels and memsets on the stream, so they
+    # capture as they are, and replays drop the host-side launch gaps that would
+    # otherwise dominate small problems.
+    use_graph = not args.no_graph
+    launches_per_step = None
+    if use_graph:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        g_fwd, g_bwd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        n0 = L.sa_kernel_launch_count()
+        with torch.cuda.graph(g_fwd):
+            sa.forward(o, lse, ws_f)
+        with torch.cuda.graph(g_bwd):
+            sa.backward(o, lse, t["do"], grads, ws_b)
+        launches_per_step = L.sa_kernel_launch_count() - n0
+        for _ in range(2):
+            g_fwd.replay()
+            g_bwd.replay()
+        torch.cuda.synchronize()
+
+    def timed_pass(which):
+        """K steps bracketed by events; optionally times one kernel through the hook."""
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+        for e in ev:  # materialise the raw cudaEvent_t handles
+            for x in e:
+                x.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
         for k in range(K):
             flush.zero_()                          # L2 flushed between timed steps
             e0, e1, e2, mb, me = ev[k]
             e0.record(stream)
-            sa.forward(o, lse, ws_f)
-            e1.record(stream)
-            L.sa_set_timing_events(mb.cuda_event, me.cuda_event, L.TIME_BWD_KV)
-            sa.backward(o, lse, t["do"], grads, ws_b)
-            L.sa_set_timing_events(None, None, -1)
+            if which is None and use_graph:
+                g_fwd.replay()
+                e1.record(stream)
+                g_bwd.replay()
+            else:
+                sa.forward(o, lse, ws_f)
+                e1.record(stream)
+                if which is not None:
+                    L.sa_set_timing_events(mb.cuda_event, me.cuda_event, which)
+                sa.backward(o, lse, t["do"], grads, ws_b)
+                L.sa_set_timing_events(None, None, -1)
             e2.record(stream)
         torch.cuda.synchronize()
+        fwd = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+        bwd = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+        kern = sum(e[3].elapsed_time(e[4]) for e in ev) / K
+        return fwd, bwd, kern
+
+    launches0 = L.sa_kernel_launch_count()
+    with ClockSampler(local_rank) as clk:
+        fwd_ms, bwd_ms, _ = timed_pass(None)
     launches = L.sa_kernel_launch_count() - launches0
-    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
-    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
-    main_ms = sum(e[3].elapsed_time(e[4]) for e in ev) / K
+    if use_graph:
+        launches = launches_per_step * K
     step_ms = fwd_ms + bwd_ms
-    # attribution pass (not part of the timed steps): the separate dQ kernel, if any
-    dq_ms = 0.0
-    evq = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    for a_, b_ in evq:
-        a_.record(stream)
-        b_.record(stream)
-    torch.cuda.synchronize()
-    for k in range(K):
-        flush.zero_()
-        L.sa_set_timing_events(evq[k][0].cuda_event, evq[k][1].cuda_event, L.TIME_BWD_DQ)
-        sa.backward(o, lse, t["do"], grads, ws_b)
-        L.sa_set_timing_events(None, None, -1)
-    torch.cuda.synchronize()
-    dq_ms = sum(a_.elapsed_time(b_) for a_, b_ in evq) / K
-    if dq_ms < 1e-3:
-        dq_ms = 0.0
-    times = torch.tensor([fwd_ms, bwd_ms, main_ms, step_ms, dq_ms], dtype=torch.float64, device=dev)
+    # attribution passes (not part of the timed steps): eager calls with the timing
+    # hook around the dK/dV kernel and around the separate dQ pass, if any
+    fwd_eager_ms, bwd_eager_ms, main_ms = timed_pass(L.TIME_BWD_KV)
+    _, _, dq_ms = timed_pass(L.TIME_BWD_DQ) if "dq_separate" in args.flags else (0.0, 0.0, 0.0)
+    times = torch.tensor([fwd_ms, bwd_ms, main_ms, step_ms, dq_ms, fwd_eager_ms, bwd_eager_ms],
+                         dtype=torch.float64, device=dev)
     if world > 1:
         torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    fwd_ms, bwd_ms, main_ms, step_ms, dq_ms = times.tolist()
+    fwd_ms, bwd_ms, main_ms, step_ms, dq_ms, fwd_eager_ms, bwd_eager_ms = times.tolist()
 
     # end to end through the public API with host buffers
     e2e = None
@@ -459,6 +486,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
                    "flags": args.flags or "default",
                    "visible_triples": work["triples"], "gathered_bytes": work["gathered_bytes"]},
         "fwd_tflops": fwd_tflops, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+        "timing": "CUDA-graph replays" if use_graph else "eager calls",
+        "fwd_eager_ms": fwd_eager_ms, "bwd_eager_ms": bwd_eager_ms,
         "bwd_path": bwd_path,
         # the benchmark spec's roofline for the whole backward: the slower of tensor peak and
         # gathered + compulsory bytes at HBM bandwidth
@@ -507,6 +536,7 @@ def main():
     ap.add_argument("--override", default=None, help="workload overrides for profiling, e.g. S=2048")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time eager calls instead of CUDA-graph replays")
     ap.add_argument("--flags", default="", help="backward variant for measurements: dq_separate | query_stationary")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -72,3 +72,45 @@ def test_full_size_sampled(cfg):
     w = get_workload(cfg)
     tail = 16 if cfg == "cfg3" else 64
     run_sampled(w, n_units=16 if cfg == "cfg3" else 24, tail_rows=tail)
+
+
+@pytest.mark.parametrize("name", ["cfg2_small", "cfg4_small"])
+def test_calls_capture_in_a_cuda_graph(name):
+    """sa_fwd / sa_bwd enqueue only kernels and memsets on the caller's stream, so a
+    CUDA graph of them replays to the same results as the eager calls."""
+    _need_gpu()
+    from gpu_harness import check_close, device_problem, grads_to_host, widen
+    from gen.torch_io import bf16_bits
+    w, kw = SMALL[name]
+    sa, t = device_problem(w, make_inputs(w, **kw))
+    o, lse = sa.alloc_fwd()
+    grads = sa.alloc_bwd()
+    ws_f, ws_b = sa.fwd_workspace(), sa.bwd_workspace()
+    sa.forward(o, lse, ws_f)
+    sa.backward(o, lse, t["do"], grads, ws_b)
+    torch.cuda.synchronize()
+    ref_o, ref_lse, ref_g = bf16_bits(o), lse.cpu().numpy(), grads_to_host(grads)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g1, g2 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g1):
+            sa.forward(o, lse, ws_f)
+        with torch.cuda.graph(g2):
+            sa.backward(o, lse, t["do"], grads, ws_b)
+    torch.cuda.current_stream().wait_stream(side)
+    o.fill_(float("nan"))
+    for v in grads.values():
+        v.fill_(float("nan"))
+    for _ in range(2):
+        g1.replay()
+        g2.replay()
+    torch.cuda.synchronize()
+    check_close("graph:O", widen(bf16_bits(o)), widen(ref_o))
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=1e-5)
+    got = grads_to_host(grads)
+    for key in ref_g:
+        if key == "dsinks":
+            check_close(f"graph:{key}", got[key], ref_g[key])
+        else:
+            check_close(f"graph:{key}", widen(got[key]), widen(ref_g[key]))

@@ -211,9 +211,10 @@ KvGeom kv_geometry(const sa_args* a) {
   if (k.nwin < 1) k.nwin = 1;
   k.n_lists = a->batch * k.nwin * a->n_heads_kv * k.nblk;
   k.n_slots = (long long)a->batch * a->s_q * a->n_heads_kv * a->topk;
-  // chunk of tokens per CTA: ~4 work items per SM, between 4 tiles and 512 tokens
+  // chunk of tokens per CTA: ~4 work items per SM, between 1 tile and 512 tokens
+  // (small problems get one tile per CTA: latency, not throughput, bounds them)
   long long want = (k.n_slots + 148 * 4 - 1) / (148 * 4);
-  long long lo = 4ll * k.TPT, hi = (512 / k.TPT) * k.TPT;
+  long long lo = k.TPT, hi = (512 / k.TPT) * k.TPT;
   if (want < lo) want = lo;
   if (want > hi) want = hi;
   want = (want + k.TPT - 1) / k.TPT * k.TPT;

@@ -34,7 +34,10 @@ struct QbPlan {
   static constexpr int kStage = 64 * (DQK + DV) * 2;  // K block + V block
   static constexpr int kComb = 4 * 16 * (DQ ? DQK : DV) * 4 + 4 * 16 * 2 * 4;  // partials + (m, l)
   static constexpr int kBudget = 227 * 1024 - 1024 - kComb - 6 * 1024;  // 6 KB static shared memory
-  static constexpr int kStages = (kBudget / kStage) > 6 ? 6 : (kBudget / kStage);
+  // small stages (d <= 64): a short ring keeps the CTA small enough for two or
+  // more per SM, which small problems need more than pipeline depth
+  static constexpr int kMaxStages = kStage <= 16384 ? 3 : 6;
+  static constexpr int kStages = (kBudget / kStage) > kMaxStages ? kMaxStages : (kBudget / kStage);
   static constexpr int oRing = 0;
   static constexpr int oComb = kStages * kStage;
   static constexpr int kSmem = oComb + kComb + 1024;
@@ -441,11 +444,14 @@ static cudaError_t qb_launch_t(const QbArgs& a, const void* k, const void* v, cu
   auto kern = qb_kernel<DQK, DV, DQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kSmem);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
+  int dev = 0, sms = 148, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 160, PL::kSmem) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
   const long long n_items = (long long)a.Tq * a.Hkv * ((a.G + 15) / 16);
-  const long long grid = n_items < sms ? n_items : sms;
+  const long long slots = (long long)sms * per_sm;
+  const long long grid = n_items < slots ? n_items : slots;
   if (grid == 0) return cudaSuccess;
   mark_begin(st, time_id);
   kern<<<(unsigned)grid, 160, PL::kSmem, st>>>(mk, mv, a);
