@@ -29,14 +29,22 @@ namespace sa {
 constexpr float kLog2eQb = 1.4426950408889634f;
 constexpr float kLn2Qb = 0.6931471805599453f;
 
-template <int DQK, int DV, bool DQ>
+// NCTA = CTAs per SM the plan is sized for.  With two, the ring is two stages
+// and the per-warp partials are merged in two column halves, so two CTAs (eight
+// consumer warps) share an SM: the forward is bound by mma.sync dependency
+// latency, which more resident warps hide.
+template <int DQK, int DV, bool DQ, int NCTA>
 struct QbPlan {
   static constexpr int kStage = 64 * (DQK + DV) * 2;  // K block + V block
-  static constexpr int kComb = 4 * 16 * (DQ ? DQK : DV) * 4 + 4 * 16 * 2 * 4;  // partials + (m, l)
-  static constexpr int kBudget = 227 * 1024 - 1024 - kComb - 6 * 1024;  // 6 KB static shared memory
+  static constexpr int W = DQ ? DQK : DV;              // accumulator width
+  static constexpr int NR = (NCTA > 1 && W > 64) ? 2 : 1;  // merge rounds
+  static constexpr int WC = W / NR;                    // columns merged per round
+  static constexpr int kComb = 4 * 16 * WC * 4 + 4 * 16 * 2 * 4;  // partials + (m, l)
+  static constexpr int kStatic = 6 * 1024;             // static shared memory
+  static constexpr int kBudget = (227 * 1024) / NCTA - 1024 - kComb - kStatic;
   // small stages (d <= 64): a short ring keeps the CTA small enough for two or
   // more per SM, which small problems need more than pipeline depth
-  static constexpr int kMaxStages = kStage <= 16384 ? 3 : 6;
+  static constexpr int kMaxStages = NCTA > 1 ? 2 : (kStage <= 16384 ? 3 : 6);
   static constexpr int kStages = (kBudget / kStage) > kMaxStages ? kMaxStages : (kBudget / kStage);
   static constexpr int oRing = 0;
   static constexpr int oComb = kStages * kStage;
@@ -105,10 +113,10 @@ __device__ __forceinline__ Unit qb_unit(const QbArgs& a, int tq, int g) {
   return make_unit(p, tq, g);
 }
 
-template <int DQK, int DV, bool DQ>
-__global__ void __launch_bounds__(160, 1) qb_kernel(const __grid_constant__ CUtensorMap mapK,
-                                                    const __grid_constant__ CUtensorMap mapV, const QbArgs a) {
-  using PL = QbPlan<DQK, DV, DQ>;
+template <int DQK, int DV, bool DQ, int NCTA>
+__global__ void __launch_bounds__(160, NCTA) qb_kernel(const __grid_constant__ CUtensorMap mapK,
+                                                       const __grid_constant__ CUtensorMap mapV, const QbArgs a) {
+  using PL = QbPlan<DQK, DV, DQ, NCTA>;
   constexpr int S = PL::kStages;
   constexpr int NQK = DQK / 16;  // k steps over d_qk
   constexpr int NV = DV / 16;    // k steps over d_v
@@ -355,77 +363,82 @@ __global__ void __launch_bounds__(160, 1) qb_kernel(const __grid_constant__ CUte
       if (lane == 0) mbar_arrive(&bars.empty[st]);
     }
 
-    // ---- merge the four warps' partials (named barrier over the consumer warps)
-    constexpr int W = DQ ? DQK : DV;
-    float* part = comb;                  // [4][16][W]
-    float* stat = comb + 4 * 16 * W;     // [4][16][2]
-#pragma unroll
-    for (int c = 0; c < NACC; ++c) {
-      const int col = 8 * c + cq;
-      *reinterpret_cast<float2*>(part + (warp * 16 + r0) * W + col) = make_float2(acc[c][0], acc[c][1]);
-      *reinterpret_cast<float2*>(part + (warp * 16 + r0 + 8) * W + col) = make_float2(acc[c][2], acc[c][3]);
-    }
+    // ---- merge the four warps' partials (named barrier over the consumer warps),
+    // PL::NR rounds of PL::WC columns
+    constexpr int W = PL::W, WC = PL::WC;
+    float* part = comb;                   // [4][16][WC]
+    float* stat = comb + 4 * 16 * WC;     // [4][16][2]
     if (!DQ && (lane & 3) == 0) {
       stat[(warp * 16 + r0) * 2] = m[0];
       stat[(warp * 16 + r0) * 2 + 1] = l[0];
       stat[(warp * 16 + r0 + 8) * 2] = m[1];
       stat[(warp * 16 + r0 + 8) * 2 + 1] = l[1];
     }
-    asm volatile("bar.sync 1, 128;\n" ::: "memory");
-    // 128 consumer threads: thread -> (row, column group)
-    const int ct = threadIdx.x;  // 0..127
+    const int ct = threadIdx.x;  // 0..127: thread -> (row, column group of 8)
     const int row = ct >> 3, cg = ct & 7;
-    if (row < nh) {
-      const long long ih = (long long)tq * a.Hq + h0 + row;
-      if (!DQ) {
-        float M = a.sinks ? __ldg(a.sinks + h0 + row) * kLog2eQb : -INFINITY;
-        for (int w2 = 0; w2 < 4; ++w2) M = fmaxf(M, stat[(w2 * 16 + row) * 2]);
-        const float Mu = M == -INFINITY ? 0.f : M;
-        float al[4], Lsum = a.sinks ? exp2f(__ldg(a.sinks + h0 + row) * kLog2eQb - Mu) : 0.f;
-        for (int w2 = 0; w2 < 4; ++w2) {
-          al[w2] = exp2f(stat[(w2 * 16 + row) * 2] - Mu);
-          Lsum += al[w2] * stat[(w2 * 16 + row) * 2 + 1];
-        }
-        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-        bf16* orow = a.o + ih * DV;
-        for (int c = cg * 8; c < DV; c += 64) {
-          float v[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            float s2 = 0.f;
+    for (int hr = 0; hr < PL::NR; ++hr) {
 #pragma unroll
-            for (int w2 = 0; w2 < 4; ++w2) s2 += al[w2] * part[(w2 * 16 + row) * W + c + e];
-            v[e] = s2 * inv;
+      for (int c = 0; c < NACC; ++c) {
+        if (c / (WC / 8) != hr) continue;
+        const int col = 8 * c + cq - hr * WC;
+        *reinterpret_cast<float2*>(part + (warp * 16 + r0) * WC + col) = make_float2(acc[c][0], acc[c][1]);
+        *reinterpret_cast<float2*>(part + (warp * 16 + r0 + 8) * WC + col) = make_float2(acc[c][2], acc[c][3]);
+      }
+      asm volatile("bar.sync 1, 128;\n" ::: "memory");
+      if (row < nh) {
+        const long long ih = (long long)tq * a.Hq + h0 + row;
+        if (!DQ) {
+          float M = a.sinks ? __ldg(a.sinks + h0 + row) * kLog2eQb : -INFINITY;
+          for (int w2 = 0; w2 < 4; ++w2) M = fmaxf(M, stat[(w2 * 16 + row) * 2]);
+          const float Mu = M == -INFINITY ? 0.f : M;
+          float al[4], Lsum = a.sinks ? exp2f(__ldg(a.sinks + h0 + row) * kLog2eQb - Mu) : 0.f;
+          for (int w2 = 0; w2 < 4; ++w2) {
+            al[w2] = exp2f(stat[(w2 * 16 + row) * 2] - Mu);
+            Lsum += al[w2] * stat[(w2 * 16 + row) * 2 + 1];
           }
-          uint4 pk;
-          pk.x = pack_bf16(v[0], v[1]);
-          pk.y = pack_bf16(v[2], v[3]);
-          pk.z = pack_bf16(v[4], v[5]);
-          pk.w = pack_bf16(v[6], v[7]);
-          *reinterpret_cast<uint4*>(orow + c) = pk;
-        }
-        if (cg == 0) a.lse[ih] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2Qb : INFINITY;
-      } else {
-        bf16* qrow = a.dq + ih * DQK;
-        for (int c = cg * 8; c < DQK; c += 64) {
-          float v[8];
+          const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+          bf16* orow = a.o + ih * DV + hr * WC;
+          for (int c = cg * 8; c < WC; c += 64) {
+            float v[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            float s2 = 0.f;
+            for (int e = 0; e < 8; ++e) {
+              float s2 = 0.f;
 #pragma unroll
-            for (int w2 = 0; w2 < 4; ++w2) s2 += part[(w2 * 16 + row) * W + c + e];
-            v[e] = s2 * a.scale;
+              for (int w2 = 0; w2 < 4; ++w2) s2 += al[w2] * part[(w2 * 16 + row) * WC + c + e];
+              v[e] = s2 * inv;
+            }
+            uint4 pk;
+            pk.x = pack_bf16(v[0], v[1]);
+            pk.y = pack_bf16(v[2], v[3]);
+            pk.z = pack_bf16(v[4], v[5]);
+            pk.w = pack_bf16(v[6], v[7]);
+            *reinterpret_cast<uint4*>(orow + c) = pk;
           }
-          uint4 pk;
-          pk.x = pack_bf16(v[0], v[1]);
-          pk.y = pack_bf16(v[2], v[3]);
-          pk.z = pack_bf16(v[4], v[5]);
-          pk.w = pack_bf16(v[6], v[7]);
-          *reinterpret_cast<uint4*>(qrow + c) = pk;
+          if (cg == 0 && hr == 0) a.lse[ih] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2Qb : INFINITY;
+        } else {
+          bf16* qrow = a.dq + ih * DQK + hr * WC;
+          for (int c = cg * 8; c < WC; c += 64) {
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              float s2 = 0.f;
+#pragma unroll
+              for (int w2 = 0; w2 < 4; ++w2) s2 += part[(w2 * 16 + row) * WC + c + e];
+              v[e] = s2 * a.scale;
+            }
+            uint4 pk;
+            pk.x = pack_bf16(v[0], v[1]);
+            pk.y = pack_bf16(v[2], v[3]);
+            pk.z = pack_bf16(v[4], v[5]);
+            pk.w = pack_bf16(v[6], v[7]);
+            *reinterpret_cast<uint4*>(qrow + c) = pk;
+          }
         }
       }
+      asm volatile("bar.sync 1, 128;\n" ::: "memory");
     }
-    asm volatile("bar.sync 1, 128;\n" ::: "memory");
+    (void)W;
   }
 }
 
@@ -436,12 +449,13 @@ bool qb_path_built(int dqk, int dv) {
 
 template <int DQK, int DV, bool DQ>
 static cudaError_t qb_launch_t(const QbArgs& a, const void* k, const void* v, cudaStream_t st, int time_id) {
-  using PL = QbPlan<DQK, DV, DQ>;
+  constexpr int NCTA = DQ ? 1 : 2;  // the dQ pass needs more registers per thread
+  using PL = QbPlan<DQK, DV, DQ, NCTA>;
   CUtensorMap mk, mv;
   if (!make_tmap_bf16(&mk, k, (uint64_t)a.Tkv, (uint64_t)a.Hkv * DQK, (uint64_t)a.Hkv * DQK * 2, 64) ||
       !make_tmap_bf16(&mv, v, (uint64_t)a.Tkv, (uint64_t)a.Hkv * DV, (uint64_t)a.Hkv * DV * 2, 64))
     return cudaErrorInvalidValue;
-  auto kern = qb_kernel<DQK, DV, DQ>;
+  auto kern = qb_kernel<DQK, DV, DQ, NCTA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kSmem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148, per_sm = 1;
