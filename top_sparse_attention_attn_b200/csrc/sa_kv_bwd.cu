@@ -289,9 +289,13 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
       }
       if (!mbar_wait(&bars.s_full, i & 1, abort_flag, a.status)) { ok = false; break; }
       tc_fence_after();
-      // P and dS for the 64 key rows, packed to bf16 pairs; two halves of 32
-      // columns keep the register footprint small
-      uint32_t pk[32], dk[32];
+      // The P / dS buffer is free once the previous tile's dK^T and dQ MMAs are
+      // done; those were committed before this tile's S and dP, so after s_full
+      // this wait returns at once.  P goes to shared memory as it is formed; only
+      // dS (bf16 pairs) stays in registers until p_free.
+      if (i > 0 && !mbar_wait(&bars.tile_done, (i - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+      const uint32_t rowaddr = sPS + r * 128;
+      uint32_t dk[32];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t sr[2][16], dr[2][16];
@@ -305,6 +309,7 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
           reg_dep16(sr[c]);
           reg_dep16(dr[c]);
         }
+        uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
@@ -318,19 +323,18 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
               pv[q2] = p;
               dsv[q2] = p * (__uint_as_float(dr[c][e + q2]) - dlt);
             }
-            pk[(32 * half + 16 * c + e) >> 1] = pack_bf16(pv[0], pv[1]);
+            pk[(16 * c + e) >> 1] = pack_bf16(pv[0], pv[1]);
             dk[(32 * half + 16 * c + e) >> 1] = pack_bf16(dsv[0], dsv[1]);
           }
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int cc = 4 * half + ch;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(rowaddr + ((cc ^ (r & 7)) << 4)),
+                       "r"(pk[4 * ch]), "r"(pk[4 * ch + 1]), "r"(pk[4 * ch + 2]), "r"(pk[4 * ch + 3])
+                       : "memory");
+        }
       }
       tc_fence_before();
-      // the P / dS buffer is free once the previous tile's dK^T (and dQ) MMAs are done
-      if (i > 0 && !mbar_wait(&bars.tile_done, (i - 1) & 1, abort_flag, a.status)) { ok = false; break; }
-      const uint32_t rowaddr = sPS + r * 128;
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(rowaddr + ((ch ^ (r & 7)) << 4)),
-                     "r"(pk[4 * ch]), "r"(pk[4 * ch + 1]), "r"(pk[4 * ch + 2]), "r"(pk[4 * ch + 3])
-                     : "memory");
       fence_async_smem();
       mbar_arrive(&bars.p_full);
       if (!mbar_wait(&bars.p_free, i & 1, abort_flag, a.status)) { ok = false; break; }
