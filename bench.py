@@ -297,6 +297,20 @@ def workload_of(args):
     return w
 
 
+def max_over_ranks(values, world: int, device=None) -> list:
+    """Element-wise max of per-rank timings (every rank gets the result)."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_rate(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return world * units_per_rank / (max_ms * 1e-3)
+
+
 def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     import torch
     from gen.torch_io import to_torch
@@ -397,11 +411,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     # hook around the dK/dV kernel and around the separate dQ pass, if any
     fwd_eager_ms, bwd_eager_ms, main_ms = timed_pass(L.TIME_BWD_KV)
     _, _, dq_ms = timed_pass(L.TIME_BWD_DQ) if "dq_separate" in args.flags else (0.0, 0.0, 0.0)
-    times = torch.tensor([fwd_ms, bwd_ms, main_ms, step_ms, dq_ms, fwd_eager_ms, bwd_eager_ms],
-                         dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    fwd_ms, bwd_ms, main_ms, step_ms, dq_ms, fwd_eager_ms, bwd_eager_ms = times.tolist()
+    fwd_ms, bwd_ms, main_ms, step_ms, dq_ms, fwd_eager_ms, bwd_eager_ms = max_over_ranks(
+        [fwd_ms, bwd_ms, main_ms, step_ms, dq_ms, fwd_eager_ms, bwd_eager_ms], world, dev)
 
     # end to end through the public API with host buffers
     e2e = None
@@ -442,8 +453,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     if rank != 0:
         return None
     peaks, peak_src = load_peaks()
-    bwd_tflops = world * work["bwd_flops"] / (bwd_ms * 1e-3) / 1e12
-    fwd_tflops = world * work["fwd_flops"] / (fwd_ms * 1e-3) / 1e12
+    bwd_tflops = aggregate_rate(work["bwd_flops"], world, bwd_ms) / 1e12
+    fwd_tflops = aggregate_rate(work["fwd_flops"], world, fwd_ms) / 1e12
     # roofline of the dominant backward kernel
     kern = []
     keystat = (w.mode == "block" and w.block_size == 64 and w.layout == "BSND" and not w.sinks
