@@ -252,10 +252,13 @@ int64_t sa_kernel_launch_count(void);
  * A is K-major [M][K] (a_mn = 0) or MN-major [K][M] (a_mn = 1); B is K-major
  * [N][K] (b_mn = 0) or MN-major [K][N] (b_mn = 1); all bf16 row-major, device.
  * D fp32 [M][N] (device).  M in {64, 128}; N, K multiples of 64, N <= 256,
- * K <= 256; box_rows in {8, 16, 32, 64}.  *status (device int) gets the
- * timeout bit if a bounded wait gives up.  Asynchronous. */
+ * K <= 256; box_rows in {8, 16, 32, 64}.  d_lane: TMEM lane offset of the
+ * accumulator, 0, or 16 with M = 64 (an M = 64 accumulator occupies 16 lanes of
+ * each 32-lane sub-partition, so two of them can share columns).  *status
+ * (device int) gets the timeout bit if a bounded wait gives up.  Asynchronous. */
 sa_status sa_selftest_mma(int32_t M, int32_t N, int32_t K, int32_t a_mn, int32_t b_mn, int32_t box_rows,
-                          const void* A, const void* B, float* D, int32_t* status, void* stream);
+                          int32_t d_lane, const void* A, const void* B, float* D, int32_t* status,
+                          void* stream);
 
 /* Human-readable name of a status code (static string). */
 const char* sa_status_string(int32_t status);

@@ -152,8 +152,16 @@ def test_bwd_workspace_size_contract():
     base = 256 + _align(Tq * 16 * 4) + _align(Tk * 4 * 192 * 4) + _align(Tk * 4 * 128 * 4)
     assert st == L.SA_OK and n == base
     # key-stationary backward (block-level, BSND, 64-row blocks): + the inverse index
+    # counts, cursor, list offsets, work items (16 B each; a small problem gets
+    # chunks of ceil(n_slots / 148) tokens rounded up to whole 128-row tiles), the
+    # work count and the entries; a problem this small also takes the bucketed
+    # index: per bucket of 512 slots, each list's count and offset
     n_lists, n_slots = 2 * 4 * 2, 2 * 128 * 4 * 4
-    index = 2 * _align(4 * n_lists) + 2 * _align(4 * (n_lists + 1)) + 256 + _align(4 * n_slots)
+    chunk = -(-(-(-n_slots // 148)) // 16) * 16  # G = 4: 8 rows per token, 16 tokens per tile
+    max_work = -(-n_slots // chunk) + n_lists
+    cells = -(-n_slots // 512) * n_lists
+    index = (2 * _align(4 * n_lists) + _align(4 * (n_lists + 1)) + _align(16 * max_work) + 256
+             + _align(4 * n_slots) + 2 * _align(4 * cells))
     st, n = _ws(_args(flags=L.SA_FLAG_DQ_SEPARATE))
     assert st == L.SA_OK and n == base + index
     # ... + an fp32 dQ accumulator when dQ is formed in the same kernel (the default)

@@ -11,16 +11,19 @@ from top_sparse_attention_attn_b200 import _lib as L
 pytestmark = pytest.mark.gpu
 
 CASES = [
-    # M, N, K, a_mn, b_mn, box_rows
+    # M, N, K, a_mn, b_mn, box_rows[, d_lane]
     (128, 64, 64, 0, 0, 64), (128, 64, 192, 0, 0, 16), (128, 256, 128, 0, 0, 8),
     (128, 64, 128, 1, 1, 64), (128, 64, 128, 1, 1, 16), (64, 64, 128, 1, 1, 32),
     (128, 192, 64, 0, 1, 64), (128, 128, 256, 1, 0, 16), (64, 128, 64, 0, 0, 8),
     (64, 192, 128, 1, 1, 64), (128, 192, 128, 1, 0, 8),
+    (64, 64, 128, 1, 1, 64, 16), (64, 128, 64, 0, 0, 16, 16),
 ]
 
 
-@pytest.mark.parametrize("M,N,K,a_mn,b_mn,box", CASES)
-def test_tcgen05_mma_matches_matmul(M, N, K, a_mn, b_mn, box):
+@pytest.mark.parametrize("case", CASES, ids=[str(c) for c in CASES])
+def test_tcgen05_mma_matches_matmul(case):
+    M, N, K, a_mn, b_mn, box = case[:6]
+    d_lane = case[6] if len(case) > 6 else 0
     if not torch.cuda.is_available():
         pytest.fail("a CUDA GPU is required for -m gpu tests")
     g = torch.Generator(device="cuda").manual_seed(M * 1000 + N * 10 + K + a_mn + 2 * b_mn)
@@ -31,7 +34,7 @@ def test_tcgen05_mma_matches_matmul(M, N, K, a_mn, b_mn, box):
     D = torch.full((M, N), float("nan"), device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     L.sa_selftest_mma(M, N, K, a_mn, b_mn, box, a_store.data_ptr(), b_store.data_ptr(), D.data_ptr(),
-                      status.data_ptr(), torch.cuda.current_stream().cuda_stream)
+                      status.data_ptr(), torch.cuda.current_stream().cuda_stream, d_lane=d_lane)
     torch.cuda.synchronize()
     assert status.item() == 0
     ref = A.float() @ B.float()

@@ -108,7 +108,7 @@ def lib() -> ctypes.CDLL:
         L.sa_bwd_no_alloc.argtypes = [P(SaArgs), P(SaBwdIo), _vp]
         L.sa_bwd_no_alloc_max_workspace.argtypes = []
         L.sa_bwd_no_alloc_max_workspace.restype = ctypes.c_size_t
-        L.sa_selftest_mma.argtypes = [ctypes.c_int32] * 6 + [_vp, _vp, _vp, _vp, _vp]
+        L.sa_selftest_mma.argtypes = [ctypes.c_int32] * 7 + [_vp, _vp, _vp, _vp, _vp]
         for name in EXPORTS:
             if name not in ("sa_status_string", "sa_set_timing_events", "sa_kernel_launch_count",
                             "sa_bwd_no_alloc_max_workspace"):
@@ -158,8 +158,9 @@ def sa_bwd_no_alloc_max_workspace() -> int:
 
 
 def sa_selftest_mma(M: int, N: int, K: int, a_mn: int, b_mn: int, box_rows: int, A: int, B: int,
-                    D: int, status: int, stream: int = 0) -> None:
-    _check(lib().sa_selftest_mma(M, N, K, a_mn, b_mn, box_rows, A, B, D, status, stream), "sa_selftest_mma")
+                    D: int, status: int, stream: int = 0, d_lane: int = 0) -> None:
+    _check(lib().sa_selftest_mma(M, N, K, a_mn, b_mn, box_rows, d_lane, A, B, D, status, stream),
+           "sa_selftest_mma")
 
 
 def sa_softmax_grad_preprocess(args: SaArgs, o: int, d_o: int, delta: int, stream: int = 0) -> None:

@@ -211,10 +211,12 @@ KvGeom kv_geometry(const sa_args* a) {
   if (k.nwin < 1) k.nwin = 1;
   k.n_lists = a->batch * k.nwin * a->n_heads_kv * k.nblk;
   k.n_slots = (long long)a->batch * a->s_q * a->n_heads_kv * a->topk;
-  // chunk of tokens per CTA: ~4 work items per SM, between 1 tile and 512 tokens
-  // (small problems get one tile per CTA: latency, not throughput, bounds them)
+  // chunk of tokens per CTA: ~4 work items per SM, at most 512 tokens.  A problem
+  // too small for that gets one wave of CTAs (about one item per SM) instead:
+  // latency bounds it, and each extra chunk of a block costs one more dK / dV flush.
   long long want = (k.n_slots + 148 * 4 - 1) / (148 * 4);
   long long lo = k.TPT, hi = (512 / k.TPT) * k.TPT;
+  if (want < lo) want = (k.n_slots + 147) / 148;
   if (want < lo) want = lo;
   if (want > hi) want = hi;
   want = (want + k.TPT - 1) / k.TPT * k.TPT;
@@ -224,13 +226,16 @@ KvGeom kv_geometry(const sa_args* a) {
 }
 
 // Workspace: [status word][delta][dK or dKV acc][dV acc][dCmp acc]
-//            + key-stationary path: [dQ acc][counts][cursor] | [list_off][chunk_off][work][entries]
+//            + key-stationary path: [dQ acc][counts][cursor] | [list_off][items][work][entries]
 // Everything before `zero_end` is cleared at the start of each call with one memset.
 struct BwdWs {
   size_t status, delta, dk, dv, dcmp;
-  size_t dq, counts, cursor, list_off, chunk_off, work, entries;
+  size_t dq, counts, cursor, list_off, items, work, entries, bucket_cnt, bucket_off;
   size_t zero_end, total;
 };
+
+// Small key-stationary problems take the bucketed index (one preparation launch).
+bool kv_bucketed(const sa_args* a, const KvGeom& k) { return sa::kv_bucketed_fits(k.n_slots, k.n_lists, k.chunk); }
 
 BwdWs bwd_ws_layout(const sa_args* a) {
   Sizes s = sizes_of(a);
@@ -260,12 +265,19 @@ BwdWs bwd_ws_layout(const sa_args* a) {
     w.zero_end = off;
     w.list_off = off;
     off += align_up(sizeof(int) * (k.n_lists + 1));
-    w.chunk_off = off;
-    off += align_up(sizeof(int) * (k.n_lists + 1));
+    w.items = off;
+    off += align_up(sizeof(int4) * (size_t)k.max_work);
     w.work = off;
     off += kAlign;
     w.entries = off;
     off += align_up(sizeof(int) * (size_t)k.n_slots);
+    if (kv_bucketed(a, k)) {
+      const size_t cells = (size_t)sa::kv_bucket_count(k.n_slots) * k.n_lists;
+      w.bucket_cnt = off;
+      off += align_up(sizeof(int) * cells);
+      w.bucket_off = off;
+      off += align_up(sizeof(int) * cells);
+    }
   } else {
     w.zero_end = off;
   }
@@ -391,16 +403,24 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
   const long long nk = s.Tkv * args->n_heads_kv * args->d_qk;
   const long long nv = s.Tkv * args->n_heads_kv * args->d_v;
   const long long nc = s.Tcmp * args->n_heads_kv * args->d_qk;
-  // zero the accumulators and the index counters (one memset), and dSinks
-  if (cudaMemsetAsync(base, 0, w.zero_end, cs) != cudaSuccess) return SA_ERR_CUDA;
+  KvGeom k;
+  memset(&k, 0, sizeof(k));
+  if (w.counts) k = kv_geometry(args);
+  // small key-stationary problems: one launch clears, forms Delta and builds the index
+  // small problems: one launch builds a bucketed index, clears and forms Delta
+  const bool prep_small = w.counts && kv_bucketed(args, k);
+  cudaError_t e = cudaSuccess;
+  if (!prep_small) {
+    // zero the accumulators and the index counters (one memset), then Delta
+    if (cudaMemsetAsync(base, 0, w.zero_end, cs) != cudaSuccess) return SA_ERR_CUDA;
+    e = sa::launch_delta(static_cast<const bf16*>(io->o), static_cast<const bf16*>(io->d_o), delta,
+                         s.Tq * args->n_heads_q, args->d_v, cs);
+    if (e != cudaSuccess) return SA_ERR_CUDA;
+  }
   if (sinks && cudaMemsetAsync(io->dsinks, 0, sizeof(float) * args->n_heads_q, cs) != cudaSuccess)
     return SA_ERR_CUDA;
-  cudaError_t e = sa::launch_delta(static_cast<const bf16*>(io->o), static_cast<const bf16*>(io->d_o), delta,
-                                   s.Tq * args->n_heads_q, args->d_v, cs);
-  if (e != cudaSuccess) return SA_ERR_CUDA;
   if (w.counts) {
     // key-stationary: inverse index, then dK / dV per KV block (+ dQ)
-    KvGeom k = kv_geometry(args);
     sa::KvIndexArgs ia;
     memset(&ia, 0, sizeof(ia));
     ia.ori_idx = args->ori_idx;
@@ -420,10 +440,29 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
     ia.counts = reinterpret_cast<int*>(base + w.counts);
     ia.cursor = reinterpret_cast<int*>(base + w.cursor);
     ia.list_off = reinterpret_cast<int*>(base + w.list_off);
-    ia.chunk_off = reinterpret_cast<int*>(base + w.chunk_off);
+    ia.items = reinterpret_cast<int4*>(base + w.items);
     ia.entries = reinterpret_cast<int*>(base + w.entries);
     ia.work_count = reinterpret_cast<int*>(base + w.work);
-    if (sa::launch_kv_index(ia, cs) != cudaSuccess) return SA_ERR_CUDA;
+    if (prep_small) {
+      ia.n_buckets = sa::kv_bucket_count(k.n_slots);
+      ia.bucket_cnt = reinterpret_cast<int*>(base + w.bucket_cnt);
+      ia.bucket_off = reinterpret_cast<int*>(base + w.bucket_off);
+    }
+    if (prep_small) {
+      sa::KvPrepArgs pa;
+      // the accumulators and counters after Delta (Delta is formed in the same launch)
+      pa.status = status;
+      pa.zero = reinterpret_cast<float4*>(base + w.dk);
+      pa.zero_n16 = (long long)((w.zero_end - w.dk) / 16);
+      pa.o = static_cast<const bf16*>(io->o);
+      pa.d_o = static_cast<const bf16*>(io->d_o);
+      pa.delta = delta;
+      pa.rows = s.Tq * args->n_heads_q;
+      pa.dv = args->d_v;
+      if (sa::launch_kv_prep_small(ia, pa, cs) != cudaSuccess) return SA_ERR_CUDA;
+    } else if (sa::launch_kv_index(ia, cs) != cudaSuccess) {
+      return SA_ERR_CUDA;
+    }
     sa::KvLaunch kl;
     memset(&kl, 0, sizeof(kl));
     sa::KvArgs& ka = kl.args;
@@ -442,8 +481,7 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
     ka.wr = args->ori_win_right;
     ka.scale = args->scale;
     ka.scale_log2 = args->scale * 1.4426950408889634f;
-    ka.list_off = ia.list_off;
-    ka.chunk_off = ia.chunk_off;
+    ka.items = ia.items;
     ka.entries = ia.entries;
     ka.work_count = ia.work_count;
     ka.lse = io->lse;
@@ -452,6 +490,9 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
     ka.dv_acc = out.dv_acc;
     ka.dq_acc = w.dq ? reinterpret_cast<float*>(base + w.dq) : nullptr;
     ka.status = status;
+    ka.n_buckets = ia.n_buckets;
+    ka.bucket_cnt = ia.bucket_cnt;
+    ka.bucket_off = ia.bucket_off;
     kl.q = args->q;
     kl.d_o = io->d_o;
     kl.k = args->k;

@@ -292,4 +292,36 @@ __device__ __forceinline__ float warp_sum4(float v) {
   return v;
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may begin while the kernel before it on the stream is still
+// running; pdl_wait() returns once that kernel has completed and its memory is
+// visible (at once when there is no such predecessor), so everything before it
+// may touch only this CTA's own shared memory and TMEM.  pdl_trigger() lets the
+// next kernel on the stream start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+// Delta of one row: sum_d a[d] * b[d] over n bf16 (n a multiple of 8, 16-byte
+// aligned rows) in fp32, by one warp; every lane returns the sum.
+__device__ __forceinline__ float warp_row_dot_bf16(const bf16* __restrict__ a, const bf16* __restrict__ b, int n,
+                                                   int lane) {
+  const uint4* a4 = reinterpret_cast<const uint4*>(a);
+  const uint4* b4 = reinterpret_cast<const uint4*>(b);
+  float acc = 0.f;
+  for (int i = lane; i < n / 8; i += 32) {
+    uint4 x = __ldg(a4 + i), y = __ldg(b4 + i);
+    const __nv_bfloat162* px = reinterpret_cast<const __nv_bfloat162*>(&x);
+    const __nv_bfloat162* py = reinterpret_cast<const __nv_bfloat162*>(&y);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 fx = __bfloat1622float2(px[j]), fy = __bfloat1622float2(py[j]);
+      acc = fmaf(fx.x, fy.x, acc);
+      acc = fmaf(fx.y, fy.y, acc);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  return acc;
+}
+
 }  // namespace sa

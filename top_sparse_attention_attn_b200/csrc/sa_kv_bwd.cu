@@ -48,14 +48,28 @@ struct KvPlan {
   static constexpr int oK = oDO + 2 * kDOStage;    // NSQ slabs of 64 rows
   static constexpr int oV = oK + NSQ * 64 * 128;   // NSV slabs of 64 rows
   static constexpr int oPS = oV + NSV * 64 * 128;  // P, then dS: 128 rows x 128 B
-  static constexpr int kBytes = oPS + 128 * 128;
+  static constexpr int oTok = oPS + 128 * 128;     // bucketed mode: the chunk's token ids
+  static constexpr int kBytes = oTok + kBucketMaxChunk * 4;
   static constexpr int kSmem = kBytes + 1024;      // + alignment slack
   static constexpr int NV = (DV + 127) / 128;      // M tiles of dV^T
   static constexpr int NK = (DQK + 127) / 128;     // M tiles of dK^T
-  static constexpr int cS = 0, cDP = 64, cDV = 128, cDK = cDV + 64 * NV, cDQ = cDK + 64 * NK;
+  // d_qk = d_v = 64: dV^T and dK^T are both M = 64 accumulators (16 lanes of each
+  // sub-partition), so they share columns at lane offsets 0 and 16 and the plan
+  // fits 256 columns (two CTAs per SM)
+  static constexpr bool kPack = DQK == 64 && DV == 64;
+  static constexpr int kDkLane = kPack ? 16 : 0;
+  static constexpr int cS = 0, cDP = 64, cDV = 128;
+  static constexpr int cDK = kPack ? cDV : cDV + 64 * NV;
+  static constexpr int cDQ = kPack ? cDV + 64 : cDK + 64 * NK;
   static constexpr int kCols = cDQ + (WITH_DQ ? DQK : 0);
   static constexpr uint32_t kAlloc = kCols <= 256 ? 256 : 512;
   static_assert(kCols <= 512, "TMEM plan too large");
+  // epilogue staging of dV^T / dK^T as fp32 [key][dim] over the (then idle) Q / dO
+  // stages; with packed accumulators the dK rows start 16 banks after the dV rows
+  // so that the two lane halves of a warp store without bank conflicts
+  static constexpr int oStV = oQ;
+  static constexpr int oStK = oStV + 64 * DV * 4 + (kPack ? 64 : 0);
+  static_assert(oStK + 64 * DQK * 4 <= oK, "epilogue staging does not fit the Q / dO stages");
   static_assert(kSmem <= 227 * 1024, "shared memory plan too large");
 };
 
@@ -63,11 +77,95 @@ struct KvBars {
   uint64_t kv_full, q_full[2], q_empty[2], s_full, p_full, p_free, ds_full, tile_done, acc_done, dq_full, dq_free;
   uint32_t tmem_base;
   int abort_flag;
+  int item_L, item_c, item_ntok;  // the work item: list, chunk of the list, tokens
+  int bstart[kBucketMax];         // bucketed mode: first rank of each bucket in the list
+  int boff[kBucketMax];           // bucketed mode: the list's offset within each bucket
 };
+
+// The list that block x of one token's selections joins: (batch b, token window,
+// kv-head g, block x), or -1 when the block is out of range or keeps no visible
+// row for the token (offset ta within its sequence).  A is KvArgs or KvIndexArgs.
+template <class A>
+__device__ __forceinline__ int kv_block_list(const A& a, int x, int b, int ta, int g) {
+  if (x < 0) return -1;
+  const long long first = (long long)x * 64;
+  if (first >= a.S) return -1;
+  if (a.ori_mask == kMaskCausal && first > ta) return -1;
+  if (a.ori_mask == kMaskBand) {
+    const long long last = min(first + 63, (long long)a.S - 1);
+    if (first > (long long)ta + a.wr || last < (long long)ta - a.wl) return -1;
+  }
+  // keyed by the token's window first, so that CTAs launched together add their dQ
+  // contributions to a window of tokens whose fp32 accumulators stay in L2
+  return ((b * a.nwin + ta / a.win_tokens) * a.Hkv + g) * a.nblk + x;
+}
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
+}
+
+// Work item w from the bucketed index (every thread of the CTA).  Warp 0 sums
+// each list's counts over the buckets, turns them into chunk counts, finds the
+// list and chunk of item w, and where each bucket's part of that list starts (in
+// rank order) and sits; then the CTA gathers the chunk's token ids into `toks`.
+// Fills bars.item_* (item_L = -1 past the last item).
+__device__ void kv_bucket_item(const KvArgs& a, int w, int* toks, KvBars& bars) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nl = a.n_lists, nb = a.n_buckets;
+  if (warp == 0) {
+    int carry = 0, fL = -1, fc = 0, fn = 0;
+    for (int l0 = 0; l0 < nl; l0 += 32) {
+      const int L = l0 + lane;
+      int cnt = 0;
+      if (L < nl)
+        for (int k = 0; k < nb; ++k) cnt += __ldg(a.bucket_cnt + k * nl + L);
+      const int nk = (cnt + a.chunk_tokens - 1) / a.chunk_tokens;
+      int incl = nk;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int excl = carry + incl - nk;
+      const unsigned m = __ballot_sync(0xffffffffu, w >= excl && w < excl + nk);
+      if (m) {
+        const int src = __ffs(m) - 1;
+        fL = __shfl_sync(0xffffffffu, L, src);
+        fc = __shfl_sync(0xffffffffu, w - excl, src);
+        fn = __shfl_sync(0xffffffffu, cnt, src);
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      bars.item_L = fL;
+      bars.item_c = fc;
+      bars.item_ntok = fL >= 0 ? min(a.chunk_tokens, fn - fc * a.chunk_tokens) : 0;
+    }
+    if (fL >= 0) {
+      const int v = lane < nb ? __ldg(a.bucket_cnt + lane * nl + fL) : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (lane < nb) {
+        bars.bstart[lane] = incl - v;
+        bars.boff[lane] = __ldg(a.bucket_off + lane * nl + fL);
+      }
+    }
+  }
+  __syncthreads();
+  if (bars.item_L < 0) return;
+  const int lo = bars.item_c * a.chunk_tokens, n = bars.item_ntok;
+  for (int r = threadIdx.x; r < n; r += blockDim.x) {
+    const int R = lo + r;
+    int k = 0;  // the last bucket whose part starts at or before rank R
+    for (int k2 = 1; k2 < nb; ++k2)
+      if (bars.bstart[k2] <= R) k = k2;
+    toks[r] = __ldg(a.entries + k * kBucketSlots + bars.boff[k] + (R - bars.bstart[k]));
+  }
 }
 
 template <int DQK, int DV, bool WITH_DQ>
@@ -82,33 +180,12 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- which work item: (list, chunk) ----
-  const int w = blockIdx.x;
-  if (w >= *a.work_count) return;
-  if (a.status && (*(volatile int*)a.status & kStatusTimeout)) return;  // another CTA gave up
-  int lo = 0, hi = a.n_lists - 1;  // largest list L with chunk_off[L] <= w
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (__ldg(a.chunk_off + mid) <= w) lo = mid; else hi = mid - 1;
-  }
-  const int L = lo;
-  const int chunk = w - __ldg(a.chunk_off + L);
-  // list id = ((batch * nwin + window) * Hkv + kv-head) * nblk + block
-  const int j = L % a.nblk;
-  const int rest = L / a.nblk;
-  const int g = rest % a.Hkv, b = (rest / a.Hkv) / a.nwin;
-  const int list_begin = __ldg(a.list_off + L), list_end = __ldg(a.list_off + L + 1);
-  const int tok0 = list_begin + chunk * a.chunk_tokens;
-  const int ntok = min(a.chunk_tokens, list_end - tok0);
-  const int TPT = a.TPT, RPT = a.RPT;
-  const int ntiles = (ntok + TPT - 1) / TPT;
-  const int* toks = a.entries + tok0;
-
   const uint32_t sQ = smem_u32(smem + PL::oQ), sDO = smem_u32(smem + PL::oDO);
   const uint32_t sK = smem_u32(smem + PL::oK), sV = smem_u32(smem + PL::oV);
   const uint32_t sPS = smem_u32(smem + PL::oPS);
   volatile int* abort_flag = &bars.abort_flag;
 
+  // ---- set-up on shared memory and TMEM only: may overlap the preceding kernel
   // zero the Q / dO stages once: rows no token fills stay finite (0)
   {
     uint4 z = make_uint4(0, 0, 0, 0);
@@ -132,35 +209,71 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
     mbar_init(&bars.dq_full, 1);
     mbar_init(&bars.dq_free, 128);
     mbar_fence_init();
+    tma_prefetch_desc(&mapQ);
+    tma_prefetch_desc(&mapDO);
+    tma_prefetch_desc(&mapK);
+    tma_prefetch_desc(&mapV);
   }
   if (warp == 1) tmem_alloc(&bars.tmem_base, PL::kAlloc);
+
+  // ---- the work item {list, tokens}
+  const int w = blockIdx.x;
+  const int* toks;
+  pdl_wait();  // the index, Delta and the cleared accumulators come from the preceding kernels
+  if (a.n_buckets > 0) {
+    // from the bucketed index: the chunk's token ids land in shared memory
+    kv_bucket_item(a, w, reinterpret_cast<int*>(smem + PL::oTok), bars);
+    toks = reinterpret_cast<const int*>(smem + PL::oTok);
+  } else {
+    // from the work-item table
+    const int4 item = __ldg(a.items + w);  // in bounds (w < max_work); used only when w < work_count
+    const int nwork = __ldg(a.work_count);
+    if (threadIdx.x == 0) {
+      bars.item_L = w < nwork ? item.x : -1;
+      bars.item_ntok = item.z;
+    }
+    toks = a.entries + item.y;
+  }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_trigger();
   const uint32_t tmem = bars.tmem_base;
+  const int L = bars.item_L, ntok = bars.item_ntok;
+  if (L < 0) {  // past the last work item (uniform over the CTA)
+    if (warp == 1) {
+      tmem_dealloc(tmem, PL::kAlloc);
+      tmem_relinquish();
+    }
+    return;
+  }
+  // list id = ((batch * nwin + window) * Hkv + kv-head) * nblk + block
+  const int j = L % a.nblk;
+  const int rest = L / a.nblk;
+  const int g = rest % a.Hkv, b = (rest / a.Hkv) / a.nwin;
+  const int TPT = a.TPT, RPT = a.RPT;
+  const int ntiles = (ntok + TPT - 1) / TPT;
+  if (threadIdx.x == 0) {
+    const int row0 = b * a.S + 64 * j;  // first KV row of block j
+    mbar_arrive_tx(&bars.kv_full, (uint32_t)(64 * (DQK + DV) * 2));
+    for (int s = 0; s < DQK / 64; ++s) tma_load_2d(sK + s * 64 * 128, &mapK, g * DQK + 64 * s, row0, &bars.kv_full);
+    for (int s = 0; s < DV / 64; ++s) tma_load_2d(sV + s * 64 * 128, &mapV, g * DV + 64 * s, row0, &bars.kv_full);
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (whole warp)
     // lane u issues the TMA loads of token u of the tile; the next tile's token
     // ids are fetched while the current stage is being waited for.
-    const int row0 = b * a.S + 64 * j;
-    if (lane == 0) {
-      tma_prefetch_desc(&mapQ);
-      tma_prefetch_desc(&mapDO);
-      mbar_arrive_tx(&bars.kv_full, (uint32_t)(64 * (DQK + DV) * 2));
-      for (int s = 0; s < DQK / 64; ++s) tma_load_2d(sK + s * 64 * 128, &mapK, g * DQK + 64 * s, row0, &bars.kv_full);
-      for (int s = 0; s < DV / 64; ++s) tma_load_2d(sV + s * 64 * 128, &mapV, g * DV + 64 * s, row0, &bars.kv_full);
-    }
     int issued = 0;
-    int tq_next = (lane < TPT && lane < ntok) ? __ldg(toks + lane) : 0;
+    int tq_next = (lane < TPT && lane < ntok) ? toks[lane] : 0;
     for (int i = 0; i < ntiles; ++i) {
       const int st = i & 1;
       const int n = min(TPT, ntok - i * TPT);
       const int tq = tq_next;
       if (i + 1 < ntiles) {
         const int u2 = (i + 1) * TPT + lane;
-        tq_next = (lane < TPT && u2 < ntok) ? __ldg(toks + u2) : 0;
+        tq_next = (lane < TPT && u2 < ntok) ? toks[u2] : 0;
       }
       bool ok = true;
       if (lane == 0 && i >= 2) ok = mbar_wait(&bars.q_empty[st], ((i >> 1) - 1) & 1, abort_flag, a.status);
@@ -226,7 +339,8 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
           const int M = min(128, DQK - 128 * t);
           const uint32_t id = idesc_bf16(M, 64, true, true);
           for (int kk = 0; kk < 8; ++kk)
-            mma_bf16(tmem + PL::cDK + 64 * t, sdesc(q + 2 * t * 16384 + kk * 2048, 16384, 1024),
+            mma_bf16(tmem + ((uint32_t)PL::kDkLane << 16) + PL::cDK + 64 * t,
+                     sdesc(q + 2 * t * 16384 + kk * 2048, 16384, 1024),
                      sdesc(sPS + kk * 2048, 16384, 1024), id, (i > 0 || kk > 0) ? 1u : 0u);
         }
         if (WITH_DQ) {
@@ -260,7 +374,7 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
       lse_n = INFINITY;
       dlt_n = 0.f;
       if (i2 < ntiles && u < n2 && hh < a.G) {
-        tq_n = __ldg(toks + i2 * TPT + u);
+        tq_n = toks[i2 * TPT + u];
         const long long ih = (long long)tq_n * a.Hq + g * a.G + hh;
         lse_n = __ldg(a.lse + ih);
         dlt_n = __ldg(a.delta + ih);
@@ -346,32 +460,44 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
       fence_async_smem();
       mbar_arrive(&bars.ds_full);
     }
-    // ---- epilogue: dV^T and dK^T (scaled) into the fp32 accumulators
+    // ---- epilogue, part 1: dV^T and dK^T from TMEM into shared memory as fp32
+    // [key][dim] rows (the Q / dO stages are idle once acc_done has fired)
     if (ok && mbar_wait(&bars.acc_done, 0, abort_flag, a.status)) {
       tc_fence_after();
-      const long long kv_row0 = (long long)b * a.S + blk_row0;
-      const int nrows = min(64, a.S - blk_row0);
-      for (int which = 0; which < 2; ++which) {
-        const int D = which == 0 ? DV : DQK;
-        const int ntile = which == 0 ? PL::NV : PL::NK;
-        const int cbase = which == 0 ? PL::cDV : PL::cDK;
-        float* acc = which == 0 ? a.dv_acc : a.dk_acc;
-        const float mul = which == 0 ? 1.f : a.scale;
-        for (int t = 0; t < ntile; ++t) {
-          const int M = min(128, D - 128 * t);
-          int dim = -1;
-          if (M == 128) dim = 128 * t + 32 * sub + lane;
-          else if (lane < 16) dim = 128 * t + 16 * sub + lane;
-          for (int c = 0; c < 64; c += 16) {
-            uint32_t v[16];
-            tmem_ld16(lane_base + cbase + 64 * t + c, v);
-            tmem_wait_ld();
-            reg_dep16(v);
-            if (dim >= 0) {
+      float* stV = reinterpret_cast<float*>(smem + PL::oStV);
+      float* stK = reinterpret_cast<float*>(smem + PL::oStK);
+      if constexpr (PL::kPack) {
+        // one pass: lanes 0..15 hold dV^T rows, lanes 16..31 dK^T rows (lane offset 16)
+        float* dst = (lane < 16 ? stV : stK) + 16 * sub + (lane & 15);
 #pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                if (c + e < nrows)
-                  atomicAdd(acc + ((kv_row0 + c + e) * a.Hkv + g) * D + dim, __uint_as_float(v[e]) * mul);
+        for (int c = 0; c < 64; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(lane_base + PL::cDV + c, v);
+          tmem_wait_ld();
+          reg_dep16(v);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) dst[(c + e) * 64] = __uint_as_float(v[e]);
+        }
+      } else {
+        for (int which = 0; which < 2; ++which) {
+          const int D = which == 0 ? DV : DQK;
+          const int ntile = which == 0 ? PL::NV : PL::NK;
+          const int cbase = which == 0 ? PL::cDV : PL::cDK;
+          float* st = which == 0 ? stV : stK;
+          for (int t = 0; t < ntile; ++t) {
+            const int M = min(128, D - 128 * t);
+            int dim = -1;
+            if (M == 128) dim = 128 * t + 32 * sub + lane;
+            else if (lane < 16) dim = 128 * t + 16 * sub + lane;
+#pragma unroll 1
+            for (int c = 0; c < 64; c += 16) {
+              uint32_t v[16];
+              tmem_ld16(lane_base + cbase + 64 * t + c, v);
+              tmem_wait_ld();
+              reg_dep16(v);
+              if (dim >= 0) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) st[(c + e) * D + dim] = __uint_as_float(v[e]);
               }
             }
           }
@@ -387,11 +513,11 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
     const int r = 32 * sub + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * sub) << 16);
     const int u = r / RPT, hh = r - u * RPT;
-    int tq_n = (u < min(TPT, ntok) && hh < a.G) ? __ldg(toks + u) : -1;
+    int tq_n = (u < min(TPT, ntok) && hh < a.G) ? toks[u] : -1;
     for (int i = 0; i < ntiles; ++i) {
       const int tq = tq_n;
       const int n2 = min(TPT, ntok - (i + 1) * TPT);
-      tq_n = (i + 1 < ntiles && u < n2 && hh < a.G) ? __ldg(toks + (i + 1) * TPT + u) : -1;
+      tq_n = (i + 1 < ntiles && u < n2 && hh < a.G) ? toks[(i + 1) * TPT + u] : -1;
       if (!mbar_wait(&bars.dq_full, i & 1, abort_flag, a.status)) break;
       tc_fence_after();
       float* dst = a.dq_acc + ((long long)(tq < 0 ? 0 : tq) * a.Hq + g * a.G + hh) * DQK;
@@ -418,6 +544,32 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
     tmem_dealloc(tmem, PL::kAlloc);
     tmem_relinquish();
   }
+  // ---- epilogue, part 2: every thread adds the staged dV^T / dK^T (scaled) to the
+  // fp32 accumulators, four consecutive dims per vector reduction
+  if (!bars.abort_flag) {
+    // the item again (shared): keeps its fields out of registers through the roles above
+    const int L2 = bars.item_L;
+    const int j2 = L2 % a.nblk, g2 = (L2 / a.nblk) % a.Hkv, b2 = (L2 / a.nblk / a.Hkv) / a.nwin;
+    const long long kv_row0 = (long long)b2 * a.S + 64 * j2;
+    const int nrows = min(64, a.S - 64 * j2);
+    const float4* stV = reinterpret_cast<const float4*>(smem + PL::oStV);
+    const float4* stK = reinterpret_cast<const float4*>(smem + PL::oStK);
+    for (int i = threadIdx.x; i < 16 * DV; i += blockDim.x) {
+      const int key = i / (DV / 4), d4 = i - key * (DV / 4);
+      if (key < nrows) {
+        const float4 x = stV[i];
+        red_add_v4(a.dv_acc + ((kv_row0 + key) * a.Hkv + g2) * DV + 4 * d4, x.x, x.y, x.z, x.w);
+      }
+    }
+    for (int i = threadIdx.x; i < 16 * DQK; i += blockDim.x) {
+      const int key = i / (DQK / 4), d4 = i - key * (DQK / 4);
+      if (key < nrows) {
+        const float4 x = stK[i];
+        red_add_v4(a.dk_acc + ((kv_row0 + key) * a.Hkv + g2) * DQK + 4 * d4, x.x * a.scale, x.y * a.scale,
+                   x.z * a.scale, x.w * a.scale);
+      }
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -425,31 +577,42 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
 // of the window that select the block
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ bool kv_slot_list(const KvIndexArgs& a, long long e, int* list, int* tq_out) {
-  const int slot = (int)(e % a.topk);
-  const long long ug = e / a.topk;
-  const int tq = (int)(ug / a.Hkv), g = (int)(ug - (long long)tq * a.Hkv);
-  if (a.ori_len && slot >= __ldg(a.ori_len + ug)) return false;
-  const int x = __ldg(a.ori_idx + e);
-  if (x < 0) return false;
-  const long long first = (long long)x * 64;
-  if (first >= a.S) return false;
-  const int b = tq / a.S;
-  const int ta = tq - b * a.S;
-  // the block must keep at least one visible row for this token
-  if (a.ori_mask == kMaskCausal && first > ta) return false;
-  if (a.ori_mask == kMaskBand) {
-    long long last = min(first + 63, (long long)a.S - 1);
-    if (first > (long long)ta + a.wr || last < (long long)ta - a.wl) return false;
+  int slot, tq, g;
+  long long ug;
+  if (a.n_slots <= 0x7fffffffll) {  // 32-bit index arithmetic when it fits
+    const int e32 = (int)e, u32 = e32 / a.topk;
+    slot = e32 - u32 * a.topk;
+    tq = u32 / a.Hkv;
+    g = u32 - tq * a.Hkv;
+    ug = u32;
+  } else {
+    slot = (int)(e % a.topk);
+    ug = e / a.topk;
+    tq = (int)(ug / a.Hkv);
+    g = (int)(ug - (long long)tq * a.Hkv);
   }
-  // keyed by the token's window first, so that CTAs launched together add their dQ
-  // contributions to a window of tokens whose fp32 accumulators stay in L2
-  const int win = ta / a.win_tokens;
-  *list = ((b * a.nwin + win) * a.Hkv + g) * a.nblk + x;
+  if (a.ori_len && slot >= __ldg(a.ori_len + ug)) return false;
+  const int b = tq / a.S;
+  const int L = kv_block_list(a, __ldg(a.ori_idx + e), b, tq - b * a.S, g);
+  if (L < 0) return false;
+  *list = L;
   *tq_out = tq;
   return true;
 }
 
+// Small problems (fewer than 2^31 slots): the same with 32-bit index arithmetic only.
+__device__ __forceinline__ int kv_slot_list32(const KvIndexArgs& a, int e, int* tq_out) {
+  const int ug = e / a.topk, slot = e - ug * a.topk;
+  const int tq = ug / a.Hkv, g = ug - tq * a.Hkv;
+  if (a.ori_len && slot >= __ldg(a.ori_len + ug)) return -1;
+  const int b = tq / a.S;
+  *tq_out = tq;
+  return kv_block_list(a, __ldg(a.ori_idx + e), b, tq - b * a.S, g);
+}
+
 __global__ void kv_count_kernel(const KvIndexArgs a) {
+  pdl_wait();
+  pdl_trigger();
   long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= a.n_slots) return;
   int list, tq;
@@ -457,6 +620,8 @@ __global__ void kv_count_kernel(const KvIndexArgs a) {
 }
 
 __global__ void kv_fill_kernel(const KvIndexArgs a) {
+  pdl_wait();
+  pdl_trigger();
   long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= a.n_slots) return;
   int list, tq;
@@ -466,8 +631,10 @@ __global__ void kv_fill_kernel(const KvIndexArgs a) {
   }
 }
 
-// exclusive scans of counts -> list_off, chunk counts -> chunk_off; one CTA of 1024
-__global__ void __launch_bounds__(1024) kv_scan_kernel(const KvIndexArgs a) {
+// Exclusive scans of the list counts -> list offsets, and of the lists' chunk
+// counts -> the work-item table (one item per chunk of a list).  Run by a whole
+// CTA of 1024 threads.
+__device__ void kv_scan_lists(const KvIndexArgs& a, const int* counts) {
   __shared__ int warp_tot[2][32];
   __shared__ int carry[2];
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -475,7 +642,7 @@ __global__ void __launch_bounds__(1024) kv_scan_kernel(const KvIndexArgs a) {
   __syncthreads();
   for (int base = 0; base < a.n_lists; base += 1024) {
     const int i = base + tid;
-    int c = i < a.n_lists ? a.counts[i] : 0;
+    int c = i < a.n_lists ? counts[i] : 0;
     int k = (c + a.chunk_tokens - 1) / a.chunk_tokens;
     int xc = c, xk = k;  // inclusive warp scans
 #pragma unroll
@@ -500,7 +667,11 @@ __global__ void __launch_bounds__(1024) kv_scan_kernel(const KvIndexArgs a) {
     const int pk = (wid ? warp_tot[1][wid - 1] : 0) + xk - k + carry[1];
     if (i < a.n_lists) {
       a.list_off[i] = pc;
-      a.chunk_off[i] = pk;
+      // the list's work items: consecutive chunks of its entries
+      for (int q = 0; q < k; ++q) {
+        const int first = q * a.chunk_tokens;
+        a.items[pk + q] = make_int4(i, pc + first, min(a.chunk_tokens, c - first), 0);
+      }
     }
     __syncthreads();
     if (tid == 1023) { carry[0] = pc + c; carry[1] = pk + k; }
@@ -508,8 +679,72 @@ __global__ void __launch_bounds__(1024) kv_scan_kernel(const KvIndexArgs a) {
   }
   if (tid == 0) {
     a.list_off[a.n_lists] = carry[0];
-    a.chunk_off[a.n_lists] = carry[1];
     *a.work_count = carry[1];
+  }
+}
+
+__global__ void __launch_bounds__(1024) kv_scan_kernel(const KvIndexArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  kv_scan_lists(a, a.counts);
+}
+
+// Small problems: one launch builds the bucketed index, clears the workspace's
+// accumulators and forms Delta = rowsum(dO o O).  CTA b < n_buckets takes slots
+// [b * 512, (b + 1) * 512): it ranks each valid slot within its list in the
+// bucket (shared-memory counters, one atomic per list and warp), lays the
+// bucket's lists out back to back, and publishes their counts and offsets.
+// The other CTAs clear and form Delta.
+__global__ void __launch_bounds__(kBucketSlots) kv_prep_small_kernel(const KvIndexArgs a, const KvPrepArgs p) {
+  pdl_wait();
+  pdl_trigger();
+  if ((int)blockIdx.x < a.n_buckets) {
+    extern __shared__ int sh[];
+    int* cnt = sh;             // [n_lists]
+    int* off = sh + a.n_lists;  // [n_lists]
+    const int nl = a.n_lists, bk = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < nl; i += blockDim.x) cnt[i] = 0;
+    const int e = bk * kBucketSlots + threadIdx.x;
+    int tq = 0;
+    const int L = e < a.n_slots ? kv_slot_list32(a, e, &tq) : -1;
+    __syncthreads();
+    const unsigned peers = __match_any_sync(0xffffffffu, L);
+    const int leader = __ffs(peers) - 1;
+    int rank = 0;
+    if (L >= 0 && lane == leader) rank = atomicAdd(cnt + L, __popc(peers));
+    rank = __shfl_sync(0xffffffffu, rank, leader) + __popc(peers & ((1u << lane) - 1));
+    __syncthreads();
+    if (warp == 0) {
+      int carry = 0;
+      for (int l0 = 0; l0 < nl; l0 += 32) {
+        const int l = l0 + lane;
+        const int c = l < nl ? cnt[l] : 0;
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        if (l < nl) {
+          off[l] = carry + incl - c;
+          a.bucket_cnt[bk * nl + l] = c;
+          a.bucket_off[bk * nl + l] = carry + incl - c;
+        }
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+      }
+    }
+    __syncthreads();
+    if (L >= 0) a.entries[bk * kBucketSlots + off[L] + rank] = tq;
+    if (bk == 0 && threadIdx.x == 0) *p.status = 0;
+    return;
+  }
+  const long long nthreads = (long long)(gridDim.x - a.n_buckets) * blockDim.x;
+  const long long t0 = (long long)(blockIdx.x - a.n_buckets) * blockDim.x + threadIdx.x;
+  for (long long i = t0; i < p.zero_n16; i += nthreads) p.zero[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int lane = threadIdx.x & 31;
+  for (long long row = t0 >> 5; row < p.rows; row += nthreads >> 5) {
+    const float d = warp_row_dot_bf16(p.o + row * p.dv, p.d_o + row * p.dv, p.dv, lane);
+    if (lane == 0) p.delta[row] = d;
   }
 }
 
@@ -535,25 +770,49 @@ static cudaError_t kv_launch_t(const KvLaunch& L, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   if (L.max_work == 0) return cudaSuccess;
   mark_begin(st, kTimeBwdKV);
-  k<<<(unsigned)L.max_work, WITH_DQ ? 320 : 192, PL::kSmem, st>>>(mq, mdo, mk, mv, a);
+  e = launch_pdl(k, (unsigned)L.max_work, WITH_DQ ? 320 : 192, PL::kSmem, st, mq, mdo, mk, mv, a);
   count_launch();
   mark_end(st, kTimeBwdKV);
-  return cudaGetLastError();
+  return e;
+}
+
+int kv_bucket_count(long long n_slots) { return (int)((n_slots + kBucketSlots - 1) / kBucketSlots); }
+
+bool kv_bucketed_fits(long long n_slots, int n_lists, int chunk) {
+  const long long nb = kv_bucket_count(n_slots);
+  return nb >= 1 && nb <= kBucketMax && n_lists <= kBucketMaxLists && nb * n_lists <= kBucketMaxCells &&
+         chunk <= kBucketMaxChunk;
+}
+
+cudaError_t launch_kv_prep_small(const KvIndexArgs& a, const KvPrepArgs& p, cudaStream_t st) {
+  if (a.n_buckets < 1 || !kv_bucketed_fits(a.n_slots, a.n_lists, a.chunk_tokens)) return cudaErrorInvalidValue;
+  long long work = (p.rows + kBucketSlots / 32 - 1) / (kBucketSlots / 32);  // one warp per Delta row
+  long long zw = (p.zero_n16 + kBucketSlots - 1) / kBucketSlots;
+  if (zw > work) work = zw;
+  if (work < 1) work = 1;
+  if (work > 148 - a.n_buckets) work = 148 - a.n_buckets;
+  const size_t shm = sizeof(int) * 2 * (size_t)a.n_lists;
+  cudaError_t e = launch_pdl(kv_prep_small_kernel, (unsigned)(a.n_buckets + work), kBucketSlots, shm, st, a, p);
+  count_launch();
+  return e;
 }
 
 cudaError_t launch_kv_index(const KvIndexArgs& a, cudaStream_t st) {
   // counts and cursor arrive zeroed (cleared with the rest of the workspace)
+  cudaError_t e = cudaSuccess;
   if (a.n_slots > 0) {
-    kv_count_kernel<<<(unsigned)((a.n_slots + 255) / 256), 256, 0, st>>>(a);
+    e = launch_pdl(kv_count_kernel, (unsigned)((a.n_slots + 255) / 256), 256, 0, st, a);
     count_launch();
+    if (e != cudaSuccess) return e;
   }
-  kv_scan_kernel<<<1, 1024, 0, st>>>(a);
+  e = launch_pdl(kv_scan_kernel, 1, 1024, 0, st, a);
   count_launch();
+  if (e != cudaSuccess) return e;
   if (a.n_slots > 0) {
-    kv_fill_kernel<<<(unsigned)((a.n_slots + 255) / 256), 256, 0, st>>>(a);
+    e = launch_pdl(kv_fill_kernel, (unsigned)((a.n_slots + 255) / 256), 256, 0, st, a);
     count_launch();
   }
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_kv_bwd(const KvLaunch& L, bool with_dq, cudaStream_t st) {

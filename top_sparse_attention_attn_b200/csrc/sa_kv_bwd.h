@@ -19,9 +19,15 @@ struct KvIndexArgs {
   int* counts;          // [n_lists]
   int* cursor;          // [n_lists]
   int* list_off;        // [n_lists + 1]
-  int* chunk_off;       // [n_lists + 1]
+  int4* items;          // [max_work] work items {list, first entry, entries, 0}
   int* entries;         // [n_slots] token ids grouped by list
   int* work_count;      // [1]
+  // bucketed index (small problems): bucket b = slots [b * kBucketSlots, ...) keeps
+  // its own inverse index at entries + b * kBucketSlots, lists at bucket_off[b][L],
+  // bucket_cnt[b][L] entries each
+  int n_buckets;
+  int* bucket_cnt;      // [n_buckets][n_lists]
+  int* bucket_off;      // [n_buckets][n_lists]
 };
 
 struct KvArgs {
@@ -29,8 +35,7 @@ struct KvArgs {
   int nwin;
   long long wl, wr;
   float scale, scale_log2;
-  const int* list_off;
-  const int* chunk_off;
+  const int4* items;    // [work_count] {list, first entry, entries, 0}
   const int* entries;
   const int* work_count;
   const float* lse;     // [Tq, Hq]
@@ -39,7 +44,21 @@ struct KvArgs {
   float* dv_acc;        // [Tkv, Hkv, DV]
   float* dq_acc;        // [Tq, Hq, DQK] (dQ in this kernel) or null
   int* status;
+  // bucketed mode (small problems): every CTA derives its work item from the
+  // per-bucket index (items and work_count unused)
+  int n_buckets;
+  const int* bucket_cnt;  // [n_buckets][n_lists]
+  const int* bucket_off;  // [n_buckets][n_lists]
 };
+
+// Bucketed index: buckets of 512 slots, each built by one CTA (512 threads) of
+// the preparation launch; the KV kernel combines at most 32 of them, and a
+// chunk's token ids stay in its shared memory.
+constexpr int kBucketSlots = 512;
+constexpr int kBucketMax = 32;
+constexpr int kBucketMaxLists = 1024;
+constexpr int kBucketMaxCells = 8192;  // n_buckets * n_lists
+constexpr int kBucketMaxChunk = 512;
 
 struct KvLaunch {
   KvArgs args;
@@ -52,7 +71,25 @@ struct KvLaunch {
   long long max_work;   // grid size: an upper bound on the work items
 };
 
+// One-launch preparation for small problems: CTAs [0, n_buckets) build the
+// bucketed index; the others clear [zero, zero + 16 * zero_n16) (a range that
+// must not hold Delta) and form Delta (rows of dv bf16); CTA 0 also clears the
+// status word.
+struct KvPrepArgs {
+  int* status;
+  float4* zero;
+  long long zero_n16;
+  const bf16* o;
+  const bf16* d_o;
+  float* delta;
+  long long rows;
+  int dv;
+};
+
 bool kv_path_built(int dqk, int dv);
+int kv_bucket_count(long long n_slots);
+bool kv_bucketed_fits(long long n_slots, int n_lists, int chunk);
+cudaError_t launch_kv_prep_small(const KvIndexArgs& a, const KvPrepArgs& p, cudaStream_t st);
 cudaError_t launch_kv_index(const KvIndexArgs& a, cudaStream_t st);
 cudaError_t launch_kv_bwd(const KvLaunch& L, bool with_dq, cudaStream_t st);
 

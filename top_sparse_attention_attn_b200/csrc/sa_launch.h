@@ -31,6 +31,25 @@ inline void mark_end(cudaStream_t st, int which) {
   if (g_ev_begin && g_ev_end && which == g_ev_which) cudaEventRecord(g_ev_end, st);
 }
 
+// Launch with programmatic stream serialization (the kernel calls pdl_wait()
+// before it reads or writes global memory); captures into CUDA graphs as a
+// programmatic edge.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // TMA tensor map over a [rows][cols] bf16 matrix (row stride in bytes), boxes
 // of box_rows x 64 columns, 128-byte swizzle, zero fill out of range.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,

@@ -492,25 +492,12 @@ __global__ void __launch_bounds__(128) bwd_kernel(const Prob p, const bf16* __re
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) delta_kernel(const bf16* __restrict__ O, const bf16* __restrict__ dO,
                                                     float* __restrict__ delta, long long rows, int dv) {
+  pdl_wait();
+  pdl_trigger();
   long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   int lane = threadIdx.x & 31;
   if (row >= rows) return;
-  const uint4* o4 = reinterpret_cast<const uint4*>(O + row * dv);
-  const uint4* d4 = reinterpret_cast<const uint4*>(dO + row * dv);
-  float acc = 0.f;
-  for (int i = lane; i < dv / 8; i += 32) {
-    uint4 a = __ldg(o4 + i), b = __ldg(d4 + i);
-    const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
-    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float2 fa = __bfloat1622float2(pa[j]), fb = __bfloat1622float2(pb[j]);
-      acc = fmaf(fa.x, fb.x, acc);
-      acc = fmaf(fa.y, fb.y, acc);
-    }
-  }
-#pragma unroll
-  for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  const float acc = warp_row_dot_bf16(O + row * dv, dO + row * dv, dv, lane);
   if (lane == 0) delta[row] = acc;
 }
 
@@ -536,6 +523,8 @@ struct CvtJobs {
 };
 
 __global__ void __launch_bounds__(256) to_bf16_multi_kernel(const CvtJobs J) {
+  pdl_wait();
+  pdl_trigger();
   const long long total = J.end8[J.n - 1];
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
@@ -666,9 +655,9 @@ cudaError_t launch_bwd_dq(const Prob& p, const bf16* d_o, const float* lse, cons
 cudaError_t launch_delta(const bf16* o, const bf16* d_o, float* delta, long long rows, int dv,
                          cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
-  delta_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(o, d_o, delta, rows, dv);
+  cudaError_t e = launch_pdl(delta_kernel, (unsigned)((rows + 7) / 8), 256, 0, st, o, d_o, delta, rows, dv);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_to_bf16(const float* src, bf16* dst, long long n, cudaStream_t st) {
@@ -695,9 +684,9 @@ cudaError_t launch_to_bf16_multi(const Cvt* jobs, int njobs, cudaStream_t st) {
   if (J.n == 0) return cudaSuccess;
   long long blocks = (acc + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  to_bf16_multi_kernel<<<(unsigned)blocks, 256, 0, st>>>(J);
+  cudaError_t e = launch_pdl(to_bf16_multi_kernel, (unsigned)blocks, 256, 0, st, J);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_check(const Prob& p, cudaStream_t st) {

@@ -14,7 +14,7 @@
 namespace sa {
 
 struct SelftestArgs {
-  int M, N, K, a_mn, b_mn, box_rows;
+  int M, N, K, a_mn, b_mn, box_rows, d_lane;
 };
 
 __global__ void __launch_bounds__(128) selftest_mma_kernel(const __grid_constant__ CUtensorMap mapA,
@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(128) selftest_mma_kernel(const __grid_constant
                              : sdesc(sA + (kk >> 2) * a.M * 128 + (kk & 3) * 32, 16, 1024);
         uint64_t db = a.b_mn ? sdesc(sB + kk * 2048, a.K * 128, 1024)
                              : sdesc(sB + (kk >> 2) * a.N * 128 + (kk & 3) * 32, 16, 1024);
-        mma_bf16(tmem_base, da, db, idesc, kk > 0 ? 1u : 0u);
+        mma_bf16(tmem_base + ((uint32_t)a.d_lane << 16), da, db, idesc, kk > 0 ? 1u : 0u);
       }
       mma_commit(&bar_mma);
     }
@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(128) selftest_mma_kernel(const __grid_constant
     const int sub = warp & 3;
     int m = -1;
     if (a.M == 128) m = 32 * sub + lane;
-    else if (lane < 16) m = 16 * sub + lane;
+    else if (lane >= a.d_lane && lane < a.d_lane + 16) m = 16 * sub + (lane - a.d_lane);
     for (int c = 0; c < a.N; c += 16) {
       uint32_t r[16];
       tmem_ld16(tmem_base + ((uint32_t)(32 * sub) << 16) + c, r);
@@ -103,9 +103,10 @@ __global__ void __launch_bounds__(128) selftest_mma_kernel(const __grid_constant
 }  // namespace sa
 
 extern "C" sa_status sa_selftest_mma(int32_t M, int32_t N, int32_t K, int32_t a_mn, int32_t b_mn,
-                                     int32_t box_rows, const void* A, const void* B, float* D, int32_t* status,
-                                     void* stream) {
+                                     int32_t box_rows, int32_t d_lane, const void* A, const void* B, float* D,
+                                     int32_t* status, void* stream) {
   if (!A || !B || !D || !status) return SA_ERR_NULLPTR;
+  if (d_lane != 0 && !(d_lane == 16 && M == 64)) return SA_ERR_PARAM;
   if ((M != 64 && M != 128) || N < 64 || N > 256 || N % 64 || K < 64 || K > 256 || K % 64) return SA_ERR_PARAM;
   if (box_rows != 8 && box_rows != 16 && box_rows != 32 && box_rows != 64) return SA_ERR_PARAM;
   CUtensorMap ma, mb;
@@ -115,7 +116,7 @@ extern "C" sa_status sa_selftest_mma(int32_t M, int32_t N, int32_t K, int32_t a_
   bool okB = b_mn ? sa::make_tmap_bf16(&mb, B, K, N, (uint64_t)N * 2, box_rows)
                   : sa::make_tmap_bf16(&mb, B, N, K, (uint64_t)K * 2, box_rows);
   if (!okA || !okB) return SA_ERR_PARAM;
-  sa::SelftestArgs args{M, N, K, a_mn, b_mn, box_rows};
+  sa::SelftestArgs args{M, N, K, a_mn, b_mn, box_rows, d_lane};
   const int smem = (M + N) * K * 2 + 1024;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaFuncSetAttribute(sa::selftest_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
