@@ -356,17 +356,33 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
             step()
         stream.wait_stream(side)
         torch.cuda.synchronize()
-        g_fwd, g_bwd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        g_fwd, g_bwd, g_step = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         n0 = L.sa_kernel_launch_count()
         with torch.cuda.graph(g_fwd):
             sa.forward(o, lse, ws_f)
         with torch.cuda.graph(g_bwd):
             sa.backward(o, lse, t["do"], grads, ws_b)
         launches_per_step = L.sa_kernel_launch_count() - n0
+        with torch.cuda.graph(g_step):  # the whole step as one graph
+            step()
         for _ in range(2):
             g_fwd.replay()
             g_bwd.replay()
+            g_step.replay()
         torch.cuda.synchronize()
+
+    def step_graph_pass():
+        """K replays of the one-graph step (forward then backward), L2 flushed before
+        each: the backward's cost inside a step is this minus the forward alone."""
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        torch.cuda.synchronize()
+        for k in range(K):
+            flush.zero_()
+            ev[k][0].record(stream)
+            g_step.replay()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in ev) / K
 
     def timed_pass(which):
         """K steps bracketed by events; optionally times one kernel through the hook."""
@@ -403,7 +419,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     launches0 = L.sa_kernel_launch_count()
     with ClockSampler(local_rank) as clk:
         fwd_ms, bwd_ms, _ = timed_pass(None)
-    launches = L.sa_kernel_launch_count() - launches0
+        launches = L.sa_kernel_launch_count() - launches0
+        step_graph_ms = step_graph_pass() if use_graph else fwd_ms + bwd_ms
     if use_graph:
         launches = launches_per_step * K
     step_ms = fwd_ms + bwd_ms
@@ -411,8 +428,10 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     # hook around the dK/dV kernel and around the separate dQ pass, if any
     fwd_eager_ms, bwd_eager_ms, main_ms = timed_pass(L.TIME_BWD_KV)
     _, _, dq_ms = timed_pass(L.TIME_BWD_DQ) if "dq_separate" in args.flags else (0.0, 0.0, 0.0)
-    fwd_ms, bwd_ms, main_ms, step_ms, dq_ms, fwd_eager_ms, bwd_eager_ms = max_over_ranks(
-        [fwd_ms, bwd_ms, main_ms, step_ms, dq_ms, fwd_eager_ms, bwd_eager_ms], world, dev)
+    fwd_ms, bwd_ms, main_ms, step_ms, dq_ms, fwd_eager_ms, bwd_eager_ms, step_graph_ms = max_over_ranks(
+        [fwd_ms, bwd_ms, main_ms, step_ms, dq_ms, fwd_eager_ms, bwd_eager_ms, step_graph_ms], world, dev)
+    # the backward inside a step: no graph boundary of its own before its first kernel
+    bwd_in_step_ms = max(step_graph_ms - fwd_ms, 1e-6)
 
     # end to end through the public API with host buffers
     e2e = None
@@ -504,6 +523,11 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         # gathered + compulsory bytes at HBM bandwidth
         "bwd_roofline_frac": max(work["bwd_flops"] / (peaks["bf16_tflops"] * 1e12),
                                  work["bwd_main_bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3 / bwd_ms,
+        # the backward as part of a one-graph step (forward then backward), minus the
+        # forward alone: the fixed cost of starting a graph of its own drops out
+        "step_graph_ms": step_graph_ms, "bwd_in_step_ms": bwd_in_step_ms,
+        "bwd_roofline_frac_in_step": max(work["bwd_flops"] / (peaks["bf16_tflops"] * 1e12),
+                                         work["bwd_main_bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3 / bwd_in_step_ms,
         "fwd_roofline_frac": max(work["fwd_flops"] / (peaks["bf16_tflops"] * 1e12),
                                  work["fwd_bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3 / fwd_ms,
         "roofline": roof, "clocks": clk.summary(), "gpu_launches": launches,

@@ -157,7 +157,7 @@ def test_bwd_workspace_size_contract():
     # work count and the entries; a problem this small also takes the bucketed
     # index: per bucket of 512 slots, each list's count and offset
     n_lists, n_slots = 2 * 4 * 2, 2 * 128 * 4 * 4
-    chunk = -(-(-(-n_slots // 148)) // 16) * 16  # G = 4: 8 rows per token, 16 tokens per tile
+    chunk = -(-(-(-n_slots // 148)) // 16) * 16  # whole tiles of 16 (8 rows per token) or 32 tokens
     max_work = -(-n_slots // chunk) + n_lists
     cells = -(-n_slots // 512) * n_lists
     index = (2 * _align(4 * n_lists) + _align(4 * (n_lists + 1)) + _align(16 * max_work) + 256

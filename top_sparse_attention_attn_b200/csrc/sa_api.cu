@@ -192,7 +192,10 @@ struct KvGeom {
 KvGeom kv_geometry(const sa_args* a) {
   KvGeom k;
   const int G = a->n_heads_q / a->n_heads_kv;
-  k.RPT = (G + 7) / 8 * 8;
+  // rows per token in a 128-row tile: G itself for G = 1, 2, 4 (gathered row by
+  // row), else G rounded up to whole 8-row swizzle groups (a TMA box per token)
+  const bool with_dq = !(a->flags & SA_FLAG_DQ_SEPARATE);  // the gather runs in the dQ role
+  k.RPT = with_dq && (G == 1 || G == 2 || G == 4) ? G : (G + 7) / 8 * 8;
   k.TPT = 128 / k.RPT;
   k.nblk = (a->s_kv + 63) / 64;
   // token windows: with dQ added by atomics, a window's fp32 dQ rows (~24 MB) stay
@@ -472,6 +475,10 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
     ka.G = args->n_heads_q / args->n_heads_kv;
     ka.RPT = k.RPT;
     ka.TPT = k.TPT;
+    ka.gather_rows = k.RPT == ka.G ? (k.RPT < 8 ? 1 : 0) : 0;
+    ka.log2_G = ka.G == 4 ? 2 : (ka.G == 2 ? 1 : 0);
+    ka.q = static_cast<const bf16*>(args->q);
+    ka.d_o = static_cast<const bf16*>(io->d_o);
     ka.nblk = k.nblk;
     ka.n_lists = k.n_lists;
     ka.nwin = k.nwin;

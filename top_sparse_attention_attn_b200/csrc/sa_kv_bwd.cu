@@ -105,6 +105,23 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
+// Row gather of one tile by NT threads (t = 0 .. NT-1): rows r = u * G + h of the
+// stage hold head head0 + h of token toks[u]; consecutive threads copy
+// consecutive 16-byte pieces with cp.async into the 128-byte-swizzled slab
+// layout the tensor core reads (64 columns per slab).
+template <int D, int NT>
+__device__ __forceinline__ void kv_gather_rows(uint32_t sbase, const bf16* __restrict__ src, const int* toks,
+                                               int nrows, int lg, int Hq, int head0, int t) {
+  constexpr int CPR = D / 8;  // 16-byte pieces per row
+#pragma unroll 4
+  for (int idx = t; idx < nrows * CPR; idx += NT) {
+    const int r = idx / CPR, c = idx - r * CPR;
+    const int tq = toks[r >> lg];
+    const bf16* p = src + ((long long)tq * Hq + head0 + (r & ((1 << lg) - 1))) * D + c * 8;
+    cp_async16(sbase + (c >> 3) * (128 * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4), p, true);
+  }
+}
+
 // Work item w from the bucketed index (every thread of the CTA).  Warp 0 sums
 // each list's counts over the buckets, turns them into chunk counts, finds the
 // list and chunk of item w, and where each bucket's part of that list starts (in
@@ -185,6 +202,8 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
   const uint32_t sPS = smem_u32(smem + PL::oPS);
   volatile int* abort_flag = &bars.abort_flag;
 
+  const bool gather = WITH_DQ && a.gather_rows;  // Q / dO rows copied by the dQ role
+
   // ---- set-up on shared memory and TMEM only: may overlap the preceding kernel
   // zero the Q / dO stages once: rows no token fills stay finite (0)
   {
@@ -197,7 +216,7 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
     bars.abort_flag = 0;
     mbar_init(&bars.kv_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars.q_full[s], 1);
+      mbar_init(&bars.q_full[s], gather ? 128 : 1);  // row gather: every dQ-role thread arrives
       mbar_init(&bars.q_empty[s], 1);
     }
     mbar_init(&bars.s_full, 1);
@@ -266,8 +285,9 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
     // lane u issues the TMA loads of token u of the tile; the next tile's token
     // ids are fetched while the current stage is being waited for.
     int issued = 0;
-    int tq_next = (lane < TPT && lane < ntok) ? toks[lane] : 0;
-    for (int i = 0; i < ntiles; ++i) {
+    if (gather && lane == 0) mbar_wait_drain(&bars.kv_full, 0);  // the dQ role copies Q / dO
+    int tq_next = (!gather && lane < TPT && lane < ntok) ? toks[lane] : 0;
+    for (int i = 0; !gather && i < ntiles; ++i) {
       const int st = i & 1;
       const int n = min(TPT, ntok - i * TPT);
       const int tq = tq_next;
@@ -294,7 +314,7 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
     }
     // drain: before the CTA can exit, every TMA load it issued must have landed
     // (on an abort some stages are never consumed)
-    if (lane == 0) {
+    if (lane == 0 && !gather) {
       mbar_wait_drain(&bars.kv_full, 0);
       for (int st = 0; st < 2; ++st) {
         int last = -1;
@@ -513,6 +533,33 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
     const int r = 32 * sub + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * sub) << 16);
     const int u = r / RPT, hh = r - u * RPT;
+    // row gather: these threads also copy the tiles' Q / dO rows, two stages ahead;
+    // a stage is announced (128 arrivals) once its copies have landed and are
+    // fenced for the tensor core
+    auto gather_tile = [&](int i2) {
+      const int st = i2 & 1, rows = min(TPT, ntok - i2 * TPT) << a.log2_G;
+      kv_gather_rows<DQK, 128>(sQ + st * PL::kQStage, a.q, toks + i2 * TPT, rows, a.log2_G, a.Hq, g * a.G, r);
+      kv_gather_rows<DV, 128>(sDO + st * PL::kDOStage, a.d_o, toks + i2 * TPT, rows, a.log2_G, a.Hq, g * a.G, r);
+      cp_async_commit();
+    };
+    auto announce = [&](int i2) {
+      fence_async_smem();
+      mbar_arrive(&bars.q_full[i2 & 1]);
+    };
+    if (gather) {
+      if (ntiles > 0) gather_tile(0);
+      if (ntiles > 1) {
+        gather_tile(1);
+        cp_async_wait_prev();
+      } else {
+        cp_async_wait_none();
+      }
+      if (ntiles > 0) announce(0);
+      if (ntiles > 1) {
+        cp_async_wait_none();
+        announce(1);
+      }
+    }
     int tq_n = (u < min(TPT, ntok) && hh < a.G) ? toks[u] : -1;
     for (int i = 0; i < ntiles; ++i) {
       const int tq = tq_n;
@@ -536,7 +583,14 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
       }
       tc_fence_before();
       mbar_arrive(&bars.dq_free);
+      if (gather && i + 2 < ntiles) {
+        // dq_full(i) came after every MMA of tile i: its stage is free
+        gather_tile(i + 2);
+        cp_async_wait_none();
+        announce(i + 2);
+      }
     }
+    cp_async_wait_none();  // nothing in flight when the CTA leaves
   }
   __syncthreads();
   if (warp == 1) {

@@ -44,6 +44,12 @@ struct KvArgs {
   float* dv_acc;        // [Tkv, Hkv, DV]
   float* dq_acc;        // [Tq, Hq, DQK] (dQ in this kernel) or null
   int* status;
+  // row gather (G = 1, 2, 4): a tile packs TPT = 128 / G tokens with no padding
+  // rows, copied row piece by row piece with cp.async instead of a TMA box per
+  // token (TMA boxes must start on 8-row swizzle groups)
+  int gather_rows, log2_G;
+  const bf16* q;        // [Tq, Hq, DQK]
+  const bf16* d_o;      // [Tq, Hq, DV]
   // bucketed mode (small problems): every CTA derives its work item from the
   // per-bucket index (items and work_count unused)
   int n_buckets;
