@@ -41,6 +41,10 @@ SMALL = {
                          seed=31), {}),
     "token_shared_128_nomask": (scaled("cfg3", "nomask", S=333, Hq=16, d_qk=128, d_v=128,
                                        topk=100, ori_mask="none", seed=32), {}),
+    # G = 1 and 2: key-stationary tiles of 128 and 64 tokens with rows gathered one by one
+    "block_g1_d64": (scaled("cfg1", "g1", S=700, Hq=2, Hkv=2, topk=5, seed=33), {}),
+    "block_g2_d128": (scaled("cfg5", "g2", S=1000, Hq=4, Hkv=2, d_qk=128, d_v=128, topk=7, zipf_s=1.2,
+                             p_drop=0.2, seed=34), dict(ori_len_range=(0, 7))),
 }
 
 
@@ -51,7 +55,8 @@ def test_small_workload_all_elements(name):
     run_full_comparison(w, kw)
 
 
-BLOCK_CASES = ["cfg1_full", "cfg2_small", "cfg2_future_len", "cfg5_small", "cfg5_empty_rows", "block_g24_128"]
+BLOCK_CASES = ["cfg1_full", "cfg2_small", "cfg2_future_len", "cfg5_small", "cfg5_empty_rows", "block_g24_128",
+               "block_g1_d64", "block_g2_d128"]
 
 
 @pytest.mark.parametrize("flag", ["dq_separate", "query_stationary"])
