@@ -260,6 +260,13 @@ sa_status sa_selftest_mma(int32_t M, int32_t N, int32_t K, int32_t a_mn, int32_t
                           int32_t d_lane, const void* A, const void* B, float* D, int32_t* status,
                           void* stream);
 
+/* Self-check of the bounded waits every kernel uses: one CTA waits on an
+ * mbarrier that nothing arrives on.  The wait gives up after its poll limit,
+ * the kernel ORs the timeout bit (2) into *status (device int32) and returns
+ * normally, so the context stays usable; *waited (device int32) gets 1 if the
+ * wait (wrongly) completed, else 0.  Asynchronous; takes as long as the limit. */
+sa_status sa_selftest_wait_timeout(int32_t* status, int32_t* waited, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* sa_status_string(int32_t status);
 

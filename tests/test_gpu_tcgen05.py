@@ -40,3 +40,22 @@ def test_tcgen05_mma_matches_matmul(case):
     ref = A.float() @ B.float()
     err = (D - ref).abs().max().item()
     assert err <= 1e-3 * ref.abs().max().item(), f"max err {err}"
+
+
+@pytest.mark.gpu
+def test_bounded_wait_gives_up_and_reports():
+    """A wait on an mbarrier that nothing arrives on gives up after its poll limit: the
+    kernel raises the status word's timeout bit and ends normally, and the context keeps
+    working (a tensor-core self-check right after still computes correctly)."""
+    import time
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    waited = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    t0 = time.time()
+    L.sa_selftest_wait_timeout(status.data_ptr(), waited.data_ptr())
+    torch.cuda.synchronize()
+    elapsed = time.time() - t0
+    assert int(waited.item()) == 0, "the wait completed although nothing arrived"
+    assert int(status.item()) & 2, "the timeout bit was not raised"
+    assert elapsed < 20.0, f"the bounded wait took {elapsed:.1f} s"
+    print(f"bounded wait gave up after {elapsed:.2f} s")
+    test_tcgen05_mma_matches_matmul((128, 64, 64, 0, 0, 64))

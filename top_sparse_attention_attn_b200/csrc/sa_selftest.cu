@@ -100,7 +100,28 @@ __global__ void __launch_bounds__(128) selftest_mma_kernel(const __grid_constant
   }
 }
 
+// Nothing ever arrives on `bar`: the bounded wait gives up and raises the status word.
+__global__ void selftest_wait_kernel(int* status, int* waited) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  const bool ok = mbar_wait(&bar, 0, &abort_flag, status);
+  if (threadIdx.x == 0) *waited = ok ? 1 : 0;
+}
+
 }  // namespace sa
+
+extern "C" sa_status sa_selftest_wait_timeout(int32_t* status, int32_t* waited, void* stream) {
+  if (!status || !waited) return SA_ERR_NULLPTR;
+  sa::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status, waited);
+  sa::count_launch();
+  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
 
 extern "C" sa_status sa_selftest_mma(int32_t M, int32_t N, int32_t K, int32_t a_mn, int32_t b_mn,
                                      int32_t box_rows, int32_t d_lane, const void* A, const void* B, float* D,
