@@ -27,7 +27,7 @@ enum { kMaskNone = 0, kMaskCausal = 1, kMaskBand = 2 };
 enum { kOriNone = 0, kOriBlock = 1, kOriToken = 2, kOriRange = 3 };
 
 // Status bits written by kernels into the workspace status word.
-enum { kStatusIndexRange = 1, kStatusTimeout = 2 };
+enum { kStatusIndexRange = 1, kStatusTimeout = 2, kStatusSmemAlign = 4 };
 
 struct Prob {
   int layout, B, s_q, s_kv;

@@ -49,8 +49,11 @@ struct KvPlan {
   static constexpr int oV = oK + NSQ * 64 * 128;   // NSV slabs of 64 rows
   static constexpr int oPS = oV + NSV * 64 * 128;  // P, then dS: 128 rows x 128 B
   static constexpr int oTok = oPS + 128 * 128;     // bucketed mode: the chunk's token ids
-  static constexpr int kBytes = oTok + kBucketMaxChunk * 4;
-  static constexpr int kSmem = kBytes + 1024;      // + alignment slack
+  static constexpr int oDQS = oTok + kBucketMaxChunk * 4;  // dQ staging: 128 rows x 16 fp32
+  static constexpr int kBytes = oDQS + 128 * 16 * 4;
+  // the dynamic region starts right after the 1024-byte static region (KvBars padded
+  // to the extern array's 1024-byte alignment): no slack, checked at run time
+  static constexpr int kSmem = kBytes;
   static constexpr int NV = (DV + 127) / 128;      // M tiles of dV^T
   static constexpr int NK = (DQK + 127) / 128;     // M tiles of dK^T
   // d_qk = d_v = 64: dV^T and dK^T are both M = 64 accumulators (16 lanes of each
@@ -70,7 +73,7 @@ struct KvPlan {
   static constexpr int oStV = oQ;
   static constexpr int oStK = oStV + 64 * DV * 4 + (kPack ? 64 : 0);
   static_assert(oStK + 64 * DQK * 4 <= oK, "epilogue staging does not fit the Q / dO stages");
-  static_assert(kSmem <= 227 * 1024, "shared memory plan too large");
+  static_assert(kSmem + 1024 <= 227 * 1024, "shared memory plan too large");
 };
 
 struct KvBars {
@@ -98,6 +101,17 @@ __device__ __forceinline__ int kv_block_list(const A& a, int x, int b, int ta, i
   // keyed by the token's window first, so that CTAs launched together add their dQ
   // contributions to a window of tokens whose fp32 accumulators stay in L2
   return ((b * a.nwin + ta / a.win_tokens) * a.Hkv + g) * a.nblk + x;
+}
+
+// AND of `pred` over the 128 threads of the dQ role (named barrier 1).
+__device__ __forceinline__ bool dq_role_all(bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(out)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return out != 0;
 }
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
@@ -194,7 +208,11 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
   using PL = KvPlan<DQK, DV, WITH_DQ>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ KvBars bars;
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_raw;
+  if (smem_u32(smem_raw) & 1023) {  // the swizzled operand layouts need 1024-byte alignment
+    if (threadIdx.x == 0 && a.status) atomicOr(a.status, kStatusSmemAlign);
+    return;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const uint32_t sQ = smem_u32(smem + PL::oQ), sDO = smem_u32(smem + PL::oDO);
@@ -560,29 +578,57 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
         announce(1);
       }
     }
-    int tq_n = (u < min(TPT, ntok) && hh < a.G) ? toks[u] : -1;
+    // The atomics go out coalesced: each 16-column slice of the tile passes through
+    // shared memory, so that a warp's reduction covers 8 rows x 64 contiguous bytes
+    // instead of 32 rows x 16 bytes (a quarter of the L1 / L2 requests).  Thread r
+    // stages row r, then adds 16-byte piece (r & 3) of rows (r >> 2) + 32 k.
+    const uint32_t sq = smem_u32(smem + PL::oDQS);
+    const int pq = r & 3;
+    (void)u;
+    (void)hh;
     for (int i = 0; i < ntiles; ++i) {
-      const int tq = tq_n;
-      const int n2 = min(TPT, ntok - (i + 1) * TPT);
-      tq_n = (i + 1 < ntiles && u < n2 && hh < a.G) ? toks[(i + 1) * TPT + u] : -1;
-      if (!mbar_wait(&bars.dq_full, i & 1, abort_flag, a.status)) break;
+      // every thread of the role votes, so that all of them leave together if any
+      // wait gave up (the named barriers below must be reached by all 128)
+      if (!dq_role_all(mbar_wait(&bars.dq_full, i & 1, abort_flag, a.status))) break;
       tc_fence_after();
-      float* dst = a.dq_acc + ((long long)(tq < 0 ? 0 : tq) * a.Hq + g * a.G + hh) * DQK;
+      const int n = min(TPT, ntok - i * TPT);
+      float* rowp[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int rho = (r >> 2) + 32 * k, uu = rho / RPT, h2 = rho - uu * RPT;
+        rowp[k] = (uu < n && h2 < a.G) ? a.dq_acc + ((long long)toks[i * TPT + uu] * a.Hq + g * a.G + h2) * DQK
+                                       : nullptr;
+      }
 #pragma unroll 1
       for (int c = 0; c < DQK; c += 16) {
         uint32_t v[16];
         tmem_ld16(lane_base + PL::cDQ + c, v);
         tmem_wait_ld();
         reg_dep16(v);
-        if (tq >= 0) {
-#pragma unroll
-          for (int e = 0; e < 16; e += 4)
-            red_add_v4(dst + c + e, __uint_as_float(v[e]) * a.scale, __uint_as_float(v[e + 1]) * a.scale,
-                       __uint_as_float(v[e + 2]) * a.scale, __uint_as_float(v[e + 3]) * a.scale);
+        if (c + 16 == DQK) {  // the accumulator goes back to the MMA warp before the atomics
+          tc_fence_before();
+          mbar_arrive(&bars.dq_free);
         }
+#pragma unroll
+        for (int q2 = 0; q2 < 4; ++q2)
+          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"r"(
+                           sq + r * 64 + ((q2 ^ ((r >> 1) & 3)) << 4)),
+                       "f"(__uint_as_float(v[4 * q2]) * a.scale), "f"(__uint_as_float(v[4 * q2 + 1]) * a.scale),
+                       "f"(__uint_as_float(v[4 * q2 + 2]) * a.scale), "f"(__uint_as_float(v[4 * q2 + 3]) * a.scale)
+                       : "memory");
+        asm volatile("bar.sync 1, 128;\n" ::: "memory");
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int rho = (r >> 2) + 32 * k;
+          float x0, x1, x2, x3;
+          asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];\n"
+                       : "=f"(x0), "=f"(x1), "=f"(x2), "=f"(x3)
+                       : "r"(sq + rho * 64 + ((pq ^ ((rho >> 1) & 3)) << 4))
+                       : "memory");
+          if (rowp[k]) red_add_v4(rowp[k] + c + 4 * pq, x0, x1, x2, x3);
+        }
+        asm volatile("bar.sync 1, 128;\n" ::: "memory");
       }
-      tc_fence_before();
-      mbar_arrive(&bars.dq_free);
       if (gather && i + 2 < ntiles) {
         // dq_full(i) came after every MMA of tile i: its stage is free
         gather_tile(i + 2);
