@@ -103,17 +103,6 @@ __device__ __forceinline__ int kv_block_list(const A& a, int x, int b, int ta, i
   return ((b * a.nwin + ta / a.win_tokens) * a.Hkv + g) * a.nblk + x;
 }
 
-// AND of `pred` over the 128 threads of the dQ role (named barrier 1).
-__device__ __forceinline__ bool dq_role_all(bool pred) {
-  uint32_t out;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-      : "=r"(out)
-      : "r"((uint32_t)pred)
-      : "memory");
-  return out != 0;
-}
-
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
@@ -578,56 +567,86 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
         announce(1);
       }
     }
-    // The atomics go out coalesced: each 16-column slice of the tile passes through
-    // shared memory, so that a warp's reduction covers 8 rows x 64 contiguous bytes
-    // instead of 32 rows x 16 bytes (a quarter of the L1 / L2 requests).  Thread r
-    // stages row r, then adds 16-byte piece (r & 3) of rows (r >> 2) + 32 k.
-    const uint32_t sq = smem_u32(smem + PL::oDQS);
-    const int pq = r & 3;
+    // The atomics go out coalesced: each 16-column slice of a warp's 32 rows passes
+    // through shared memory, so that a reduction covers 8 rows x 64 contiguous bytes
+    // instead of 32 rows x 16 bytes (a quarter of the L1 / L2 requests).  Lane l
+    // stages its row, then adds 16-byte piece (l & 3) of the warp's rows (l >> 2) + 8 k.
+    const uint32_t sq = smem_u32(smem + PL::oDQS) + sub * (32 * 64);
+    const int pq = lane & 3;
     (void)u;
     (void)hh;
     for (int i = 0; i < ntiles; ++i) {
-      // every thread of the role votes, so that all of them leave together if any
-      // wait gave up (the named barriers below must be reached by all 128)
-      if (!dq_role_all(mbar_wait(&bars.dq_full, i & 1, abort_flag, a.status))) break;
+      // the warp leaves together if any lane's wait gave up (the lanes exchange
+      // data below)
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars.dq_full, i & 1, abort_flag, a.status))) break;
       tc_fence_after();
       const int n = min(TPT, ntok - i * TPT);
+      // a CTA with one tile has no next tile to overlap: its lanes add their own rows
+      // directly (shorter latency); otherwise the coalesced slices keep the memory
+      // pipeline free for the next tile's softmax
+      const bool staged = ntiles > 1;
+      float* own = nullptr;
+      {
+        const int u0 = r / RPT, h0 = r - u0 * RPT;
+        if (u0 < n && h0 < a.G) own = a.dq_acc + ((long long)toks[i * TPT + u0] * a.Hq + g * a.G + h0) * DQK;
+      }
       float* rowp[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const int rho = (r >> 2) + 32 * k, uu = rho / RPT, h2 = rho - uu * RPT;
+        const int rho = 32 * sub + (lane >> 2) + 8 * k, uu = rho / RPT, h2 = rho - uu * RPT;
         rowp[k] = (uu < n && h2 < a.G) ? a.dq_acc + ((long long)toks[i * TPT + uu] * a.Hq + g * a.G + h2) * DQK
                                        : nullptr;
       }
-#pragma unroll 1
-      for (int c = 0; c < DQK; c += 16) {
-        uint32_t v[16];
-        tmem_ld16(lane_base + PL::cDQ + c, v);
-        tmem_wait_ld();
-        reg_dep16(v);
-        if (c + 16 == DQK) {  // the accumulator goes back to the MMA warp before the atomics
-          tc_fence_before();
-          mbar_arrive(&bars.dq_free);
+      // one 16-column slice: stage this lane's row, then add 16-byte pieces of four rows
+      auto stage_and_add = [&](int c, const uint32_t (&v)[16]) {
+        if (!staged) {
+          if (own) {
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+              red_add_v4(own + c + e, __uint_as_float(v[e]) * a.scale, __uint_as_float(v[e + 1]) * a.scale,
+                         __uint_as_float(v[e + 2]) * a.scale, __uint_as_float(v[e + 3]) * a.scale);
+          }
+          return;
         }
 #pragma unroll
         for (int q2 = 0; q2 < 4; ++q2)
           asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"r"(
-                           sq + r * 64 + ((q2 ^ ((r >> 1) & 3)) << 4)),
+                           sq + lane * 64 + ((q2 ^ ((lane >> 1) & 3)) << 4)),
                        "f"(__uint_as_float(v[4 * q2]) * a.scale), "f"(__uint_as_float(v[4 * q2 + 1]) * a.scale),
                        "f"(__uint_as_float(v[4 * q2 + 2]) * a.scale), "f"(__uint_as_float(v[4 * q2 + 3]) * a.scale)
                        : "memory");
-        asm volatile("bar.sync 1, 128;\n" ::: "memory");
+        __syncwarp();
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int rho = (r >> 2) + 32 * k;
+          const int rl = (lane >> 2) + 8 * k;  // row within the warp's 32
           float x0, x1, x2, x3;
           asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];\n"
                        : "=f"(x0), "=f"(x1), "=f"(x2), "=f"(x3)
-                       : "r"(sq + rho * 64 + ((pq ^ ((rho >> 1) & 3)) << 4))
+                       : "r"(sq + rl * 64 + ((pq ^ ((rl >> 1) & 3)) << 4))
                        : "memory");
           if (rowp[k]) red_add_v4(rowp[k] + c + 4 * pq, x0, x1, x2, x3);
         }
-        asm volatile("bar.sync 1, 128;\n" ::: "memory");
+        __syncwarp();
+      };
+      // TMEM reads run one slice ahead of the staging; the accumulator goes back to
+      // the MMA warp as soon as its last slice is in registers
+      uint32_t v0[16], v1[16];
+      tmem_ld16(lane_base + PL::cDQ, v0);
+#pragma unroll 1
+      for (int c = 0; c < DQK; c += 32) {
+        tmem_wait_ld();
+        reg_dep16(v0);
+        tmem_ld16(lane_base + PL::cDQ + c + 16, v1);
+        stage_and_add(c, v0);
+        tmem_wait_ld();
+        reg_dep16(v1);
+        if (c + 32 < DQK) {
+          tmem_ld16(lane_base + PL::cDQ + c + 32, v0);
+        } else {
+          tc_fence_before();
+          mbar_arrive(&bars.dq_free);
+        }
+        stage_and_add(c + 16, v1);
       }
       if (gather && i + 2 < ntiles) {
         // dq_full(i) came after every MMA of tile i: its stage is free
