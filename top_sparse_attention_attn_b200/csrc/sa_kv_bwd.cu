@@ -7,7 +7,8 @@
 // the KV block: an inverse index lists, for every (batch, kv-head, block),
 // the query tokens whose selection names the block; one CTA takes a chunk of
 // that list and streams the tokens' query rows through the block in tiles of
-// 128 rows (128 / RPT tokens, RPT = G rounded up to a multiple of 8).
+// 128 rows (128 / RPT tokens: RPT = G for G = 1, 2, 4, rows copied one by one;
+// else G rounded up to a multiple of 8, one TMA box per token).
 //
 // Per tile (tcgen05, bf16 operands, fp32 TMEM accumulators):
 //   S   [128 x 64]  = Q K_j^T             (A = Q K-major, B = K_j K-major)
@@ -16,12 +17,14 @@
 //   dV^T [DV x 64] += dO^T P              (A = dO MN-major, B = P MN-major)
 //   dK^T [DQK x 64] += Q^T dS             (A = Q MN-major, B = dS MN-major)
 //   dQ  [128 x DQK] = dS K_j              (optional; A = dS K-major, B = K_j MN-major),
-//                      added to an fp32 dQ accumulator with vector atomics.
-// At the end dK^T / dV^T (scaled) are added to the fp32 dK / dV accumulators;
-// blocks split into several chunks meet there.
+//                      added to an fp32 dQ accumulator with 16-byte atomics that a
+//                      per-warp shared-memory slice makes contiguous (8 rows x 64 B).
+// At the end dK^T / dV^T (scaled) pass through shared memory and are added to the
+// fp32 dK / dV accumulators; blocks split into several chunks meet there.
 //
 // Warp roles: 0 = TMA producer, 1 = MMA issuer + TMEM owner, 2..5 = softmax /
-// dK-dV epilogue (thread = query row = TMEM lane), 6..9 (with dQ) = dQ epilogue.
+// dK-dV epilogue (thread = query row = TMEM lane), 6..9 (with dQ) = dQ epilogue
+// and, for G = 1, 2, 4, the row gather of the tiles' Q / dO rows.
 // Every wait is bounded (sa_tc.cuh): on timeout the CTA raises the status
 // word, skips the rest of its work, drains and frees TMEM.
 #include <cuda.h>
@@ -539,7 +542,6 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
     const int sub = warp & 3;
     const int r = 32 * sub + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * sub) << 16);
-    const int u = r / RPT, hh = r - u * RPT;
     // row gather: these threads also copy the tiles' Q / dO rows, two stages ahead;
     // a stage is announced (128 arrivals) once its copies have landed and are
     // fenced for the tensor core
@@ -573,8 +575,6 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
     // stages its row, then adds 16-byte piece (l & 3) of the warp's rows (l >> 2) + 8 k.
     const uint32_t sq = smem_u32(smem + PL::oDQS) + sub * (32 * 64);
     const int pq = lane & 3;
-    (void)u;
-    (void)hh;
     for (int i = 0; i < ntiles; ++i) {
       // the warp leaves together if any lane's wait gave up (the lanes exchange
       // data below)
