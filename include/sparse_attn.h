@@ -61,6 +61,17 @@
  * Determinism.  The backward accumulates dK / dV / dKV / dSinks with fp32
  * atomics, so results may differ in the last bits from run to run.
  *
+ * Streams.  Calls only enqueue kernels and memsets on the caller's stream, so
+ * they capture into CUDA graphs.  The backward's kernels are launched with
+ * programmatic dependent launch: each may start its shared-memory and TMEM
+ * set-up while the kernel before it on the stream finishes, and waits for that
+ * kernel's completion before it reads or writes global memory, so stream
+ * order is kept for the caller's own work before and after the call.
+ *
+ * Bounded waits.  The tensor-core kernels' waits give up after about two
+ * seconds; the kernel then raises a timeout bit in the workspace status word
+ * and finishes without completing its work (see sa_selftest_wait_timeout).
+ *
  * Errors.  Every entry point returns an sa_status.  Argument errors are found
  * on the host before anything is enqueued.  CUDA launch errors come back as
  * SA_ERR_CUDA (the library calls cudaGetLastError after its launches).
