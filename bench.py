@@ -274,7 +274,7 @@ def oracle_baseline(w, inputs, budget_s: float = 12.0, seed: int = 0) -> dict:
             flops += oracle.unit_flops(p, tq, g)[1]
         n_units += len(batch)
     return {"value": flops / elapsed / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
-            "kind": "oracle",
+            "kind": "oracle", "elapsed_s": elapsed,
             "sample": f"{n_units} random (token, kv-head) units of {w.name}, float64 NumPy backward "
                       f"({elapsed:.1f} s of CPU time)"}
 
@@ -552,10 +552,17 @@ def run_reference(args, rank: int) -> dict | None:
         oracle_baseline(w, inputs, budget_s=1.0, seed=1)
     vals = [oracle_baseline(w, inputs, budget_s=per_step, seed=100 + k) for k in range(args.steps)]
     v = statistics.mean(x["value"] for x in vals)
+    work = count_work(w, inputs)
     return {"metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "impl": "reference",
+            # a whole backward of the workload at the sampled rate (each timed step is a
+            # bounded sample of it; sample_ms_per_step is its measured length)
+            "ms_per_step": work["bwd_flops"] / (v * 1e12) * 1e3,
+            "sample_ms_per_step": statistics.mean(x["elapsed_s"] for x in vals) * 1e3,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name},
+            "config": {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv,
+                       "d_qk": w.d_qk, "d_v": w.d_v, "block_size": w.block_size, "topk": w.topk,
+                       "parallelism": "replicas1", "l2": "n/a (host cores)", "flags": "default"},
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": vals[0]["cores"],
                              "kind": "oracle", "sample": vals[0]["sample"]},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
