@@ -138,8 +138,55 @@ def count_work(w, inputs) -> dict:
         # query-stationary dQ pass: S, dP, dQ contractions over the gathered rows
         "dq_flops": 2 * (2 * w.d_qk + w.d_v) * triples,
         "dq_bytes": gathered + n_q + n_v + 2 * lse_b + n_q,
+        # fp32 reductions of the fused query-stationary backward: every visible row of
+        # every 16-head slice adds its dK/dV (dKV) row
+        "red_bytes_qs": int(vis.sum()) * ((G + 15) // 16) * (w.d_qk + (0 if w.kv_shared else w.d_v)) * 4,
         "units": T * w.Hkv,
+        "_npair": npair,
     }
+
+
+def kv_reduction_bytes(w, inputs, work: dict) -> int:
+    """fp32 reduction bytes of the key-stationary backward with dQ in the kernel: one
+    dQ row per (token, head, selected block with a visible row) and one dK/dV flush
+    per work item (a chunk of a block's token list), with the work-item sizing the
+    library uses (a model of it: the count is reported, not used for timing)."""
+    G = w.G
+    rpt = G if G in (1, 2, 4) else (G + 7) // 8 * 8
+    tpt = 128 // rpt
+    nblk = (w.S + 63) // 64
+    n_slots = w.B * w.S * w.Hkv * w.topk
+    win = w.S
+    fit = (48 << 20) // (w.Hq * w.d_qk * 4) // 64 * 64
+    need = 128 * nblk // max(1, w.topk)
+    if 64 <= fit < w.S and fit >= need:
+        win = fit
+    want = -(-n_slots // 592)
+    lo, hi = tpt, (512 // tpt) * tpt
+    if want < lo:
+        want = -(-n_slots // 148)
+    want = min(max(want, lo), hi)
+    chunk = -(-want // tpt) * tpt
+    idx = inputs["ori_idx"].reshape(w.B, w.S, w.Hkv, -1).astype(np.int64)
+    slot = np.arange(idx.shape[3])[None, None, None, :]
+    ok = idx >= 0
+    if "ori_topk_len" in inputs:
+        ok &= slot < inputs["ori_topk_len"].reshape(w.B, w.S, w.Hkv)[..., None]
+    ta = np.arange(w.S)[None, :, None, None]
+    ok &= idx * 64 < w.S
+    if w.ori_mask == "causal":
+        ok &= idx * 64 <= ta
+    elif w.ori_mask == "band":
+        last = np.minimum(idx * 64 + 63, w.S - 1)
+        ok &= (idx * 64 <= ta + w.win_right) & (last >= ta - w.win_left)
+    bb = np.broadcast_to(np.arange(w.B)[:, None, None, None], idx.shape)
+    gg = np.broadcast_to(np.arange(w.Hkv)[None, None, :, None], idx.shape)
+    ww = np.broadcast_to(ta // win, idx.shape)
+    lists = ((bb * ((w.S + win - 1) // win) + ww) * w.Hkv + gg) * nblk + np.where(ok, idx, 0)
+    counts = np.bincount(lists[ok].ravel())
+    n_chunks = int((-(-counts // chunk)).sum())
+    dq = int(work["_npair"].sum()) * G * w.d_qk * 4
+    return dq + n_chunks * 64 * (w.d_qk + w.d_v) * 4
 
 
 def load_peaks() -> tuple:
@@ -489,6 +536,17 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         bwd_path = "query-stationary fused (dK/dV scatter-add)"
         kern.append(("bwd_kernel (fused query-stationary backward)", main_ms, work["bwd_flops"],
                      work["bwd_main_bytes"]))
+    # the fp32 scatter-add traffic of the dominant kernel, as achieved GB/s (a
+    # reporting model: a failure here must not cost the measurement)
+    try:
+        if keystat and "dq_separate" not in args.flags:
+            red_bytes = kv_reduction_bytes(w, inputs, work)
+        elif not keystat:
+            red_bytes = work["red_bytes_qs"]
+        else:
+            red_bytes = None
+    except Exception:  # noqa: BLE001
+        red_bytes = None
     name, kms, kflops, kbytes = max(kern, key=lambda x: x[1])
     t_bytes = kbytes / (peaks["hbm_gbs"] * 1e9)
     t_flops = kflops / (peaks["bf16_tflops_sustained"] * 1e12)
@@ -531,6 +589,12 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         "fwd_roofline_frac": max(work["fwd_flops"] / (peaks["bf16_tflops"] * 1e12),
                                  work["fwd_bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3 / fwd_ms,
         "roofline": roof, "clocks": clk.summary(), "gpu_launches": launches,
+        # fp32 dQ / dK / dV reductions (L2 read-modify-writes, not DRAM bytes) of the
+        # dominant backward kernel, over its measured time
+        "reductions": None if red_bytes is None else {
+            "bytes": red_bytes, "achieved_gbs": red_bytes / (main_ms * 1e-3) / 1e9,
+            "model": "dQ row per (token, head, block) + dK/dV flush per work item" if keystat
+                     else "dK/dV (dKV) row per visible row and 16-head slice"},
         "e2e": e2e,
     }
     if world == 1 and not args.no_cpu_baseline:
