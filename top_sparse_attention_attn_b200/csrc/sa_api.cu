@@ -518,6 +518,10 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
       q.dq = static_cast<bf16*>(io->dq);
       e = sa::launch_qb(q, args->k, args->v, true, cs);
     }
+  } else if (sa::tk_path_built(args->d_qk, args->d_v, args->kv_shared, args->n_heads_q / args->n_heads_kv) &&
+             !(args->flags & SA_FLAG_QUERY_STATIONARY_BWD)) {
+    // token-level shared KV (576 / 512): the tcgen05 kernel, 64 heads per CTA
+    e = sa::launch_tk_bwd(p, io->lse, delta, static_cast<const bf16*>(io->d_o), out, cs);
   } else {
     e = sa::launch_bwd(p, static_cast<const bf16*>(io->o), static_cast<const bf16*>(io->d_o), io->lse, delta,
                        out, cs);
