@@ -41,9 +41,11 @@ struct TkPlan {
   static constexpr int oDO = oQ + NSQ * H * 128;         // dO: NSV slabs of 64 rows
   static constexpr int kKVStage = NSQ * NK * 128;        // one KV tile: NSQ slabs of 32 rows
   static constexpr int oKV = oDO + NSV * H * 128;        // 2 stages
-  static constexpr int oP = oKV + 2 * kKVStage;          // P [64 heads][32 keys] bf16, 128-byte rows
-  static constexpr int oDS = oP + H * 128;               // dS (scaled), the same layout
-  static constexpr int oCode = oDS + H * 128;            // row codes of the last 4 tiles
+  // P and dS [64 heads][32 keys] bf16 in the 64-byte swizzle (rows of 64 B): a
+  // K-major A for dQ (K = keys) and an MN-major B of one 32-wide atom for dKV
+  static constexpr int oP = oKV + 2 * kKVStage;
+  static constexpr int oDS = oP + H * 64;
+  static constexpr int oCode = oDS + H * 64;             // row codes of the last 4 tiles
   static constexpr int kSmem = oCode + 4 * NK * 4;
   static_assert(kSmem + 1024 <= 227 * 1024, "shared memory plan too large");
   static_assert(oDO % 1024 == 0 && oKV % 1024 == 0 && kKVStage % 1024 == 0 && oP % 1024 == 0 && oDS % 1024 == 0,
@@ -176,19 +178,19 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
         for (int t = 0; t < 4; ++t) {
           for (int kk = 0; kk < 4; ++kk)
             mma_bf16(tmem + PL::cKV + 32 * t, sdesc(sQ + 2 * t * (PL::H * 128) + kk * 2048, PL::H * 128, 1024),
-                     sdesc(sDS + kk * 2048, PL::H * 128, 1024), idKV, kk > 0);
+                     sdesc64(sDS + kk * 1024, PL::H * 64, 512), idKV, kk > 0);
           for (int kk = 0; kk < 4; ++kk)
             mma_bf16(tmem + PL::cKV + 32 * t, sdesc(sDO + 2 * t * (PL::H * 128) + kk * 2048, PL::H * 128, 1024),
-                     sdesc(sP + kk * 2048, PL::H * 128, 1024), idKV, 1u);
+                     sdesc64(sP + kk * 1024, PL::H * 64, 512), idKV, 1u);
         }
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmem + PL::cKVR, sdesc(sQ + 8 * (PL::H * 128) + kk * 2048, PL::H * 128, 1024),
-                   sdesc(sDS + kk * 2048, PL::H * 128, 1024), idKVR, kk > 0);
+                   sdesc64(sDS + kk * 1024, PL::H * 64, 512), idKVR, kk > 0);
         mma_commit(&bars.dkv_full);
         // dQ += dS KV (KV as an MN-major B: N = dims in 64-wide slabs of 32 rows)
         for (int kk = 0; kk < PL::NK / 16; ++kk) {
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          const uint64_t a = sdesc(sDS + kk * 32, 16, 1024);
+          const uint64_t a = sdesc64(sDS + kk * 32, 16, 512);
           mma_bf16(tmem + PL::cDQ, a, sdesc(kv + kk * 2048, PL::NK * 128, 1024), idDQ, acc);
           mma_bf16(tmem + (16u << 16) + PL::cDQ, a, sdesc(kv + 4 * (PL::NK * 128) + kk * 2048, PL::NK * 128, 1024),
                    idDQ, acc);
@@ -246,10 +248,10 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
         }
         pk[k >> 1] = pack_bf16(a0, a1);
       }
-      const uint32_t rowaddr = (is_s ? sP : sDS) + h * 128;
+      const uint32_t rowaddr = (is_s ? sP : sDS) + h * 64;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(rowaddr + ((c ^ (h & 7)) << 4)),
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(rowaddr + ((c ^ ((h >> 1) & 3)) << 4)),
                      "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
                      : "memory");
       tc_fence_before();
