@@ -360,6 +360,8 @@ sa_status sa_fwd(const sa_args* args, const sa_fwd_out* out, void* ws, size_t ws
     q.lse = out->lse;
     return cuda_status(sa::launch_qb(q, args->k, args->v, false, cs));
   }
+  if (sa::tk_path_built(args->d_qk, args->d_v, args->kv_shared, args->n_heads_q / args->n_heads_kv))
+    return cuda_status(sa::launch_tk_fwd(p, static_cast<bf16*>(out->o), out->lse, cs));
   return cuda_status(sa::launch_fwd(p, static_cast<bf16*>(out->o), out->lse, cs));
 }
 

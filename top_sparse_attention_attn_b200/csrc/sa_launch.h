@@ -71,6 +71,7 @@ cudaError_t launch_to_bf16(const float* src, bf16* dst, long long n, cudaStream_
 bool tk_path_built(int dqk, int dv, int shared, int G);
 cudaError_t launch_tk_bwd(const Prob& p, const float* lse, const float* delta, const bf16* d_o, const BwdOut& out,
                           cudaStream_t st);
+cudaError_t launch_tk_fwd(const Prob& p, bf16* o, float* lse, cudaStream_t st);
 // Up to four fp32 -> bf16 conversions in one launch (each n a multiple of 8).
 struct Cvt {
   const float* src;

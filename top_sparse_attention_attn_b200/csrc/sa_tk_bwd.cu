@@ -354,4 +354,261 @@ cudaError_t launch_tk_bwd(const Prob& p, const float* lse, const float* delta, c
   return e;
 }
 
+
+
+// ---------------------------------------------------------------------------
+// Token-level forward over one shared KV head (576 / 512) on tcgen05, the same
+// unit and tile decomposition: one CTA per (token, kv-head, 64 heads).
+//   S [64 x 32] = Q KV^T (lanes 0..15); online softmax in the softmax warps;
+//   O [64 x 512] += P V: dims 0..255 in lanes 0..15 and 256..511 in lanes 16..31
+//   of TMEM columns [32, 288).  The running maximum moves only when a tile's
+//   maximum exceeds it by more than 8 (a factor of 256 in the exponentials): O and
+//   the running sum are then rescaled once, after the previous P V has landed.
+// Sinks start the running state (m = sink, l = 1).
+// ---------------------------------------------------------------------------
+struct TkFwdPlan {
+  static constexpr int DQK = 576, DV = 512, H = 64, NK = 32;
+  static constexpr int NSQ = DQK / 64;
+  static constexpr int oQ = 0;
+  static constexpr int kKVStage = NSQ * NK * 128;
+  static constexpr int oKV = oQ + NSQ * H * 128;
+  static constexpr int oP = oKV + 2 * kKVStage;  // P [64 heads][32 keys] bf16, 64-byte swizzle
+  static constexpr int oCode = oP + H * 64;
+  static constexpr int kSmem = oCode + 4 * NK * 4;
+  static_assert(kSmem + 1024 <= 227 * 1024, "shared memory plan too large");
+  static constexpr int cS = 0, cO = 32;
+  static constexpr uint32_t kAlloc = 512;
+};
+
+struct TkFwdBars {
+  uint64_t q_full, kv_full[2], kv_empty[2], s_full, p_full, pv_done;
+  uint64_t codes_full[4];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const Prob p,
+                                                        bf16* __restrict__ O, float* __restrict__ LSE) {
+  using PL = TkFwdPlan;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ TkFwdBars bars;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (smem_u32(smem) & 1023) {
+    if (threadIdx.x == 0 && p.status) atomicOr(p.status, kStatusSmemAlign);
+    return;
+  }
+  const int nhs = p.G / PL::H;
+  const int unit = blockIdx.x / nhs, hs = blockIdx.x - unit * nhs;
+  const int tq = unit / p.Hkv, g = unit - tq * p.Hkv;
+  const int head0 = g * p.G + hs * PL::H;
+  const uint32_t sQ = smem_u32(smem + PL::oQ), sKV = smem_u32(smem + PL::oKV), sP = smem_u32(smem + PL::oP);
+  int* codes = reinterpret_cast<int*>(smem + PL::oCode);
+  volatile int* abort_flag = &bars.abort_flag;
+  if (threadIdx.x == 0) {
+    bars.abort_flag = 0;
+    mbar_init(&bars.q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars.kv_full[s], 32);
+      mbar_init(&bars.kv_empty[s], 1);
+    }
+    mbar_init(&bars.s_full, 1);
+    mbar_init(&bars.p_full, 128);
+    mbar_init(&bars.pv_done, 1);
+    for (int s = 0; s < 4; ++s) mbar_init(&bars.codes_full[s], 1);
+    mbar_fence_init();
+    tma_prefetch_desc(&mapQ);
+  }
+  if (warp == 1) tmem_alloc(&bars.tmem_base, PL::kAlloc);
+  pdl_wait();
+  pdl_trigger();
+  const Unit u = make_unit(p, tq, g);
+  const int nsub = 2 * u.n_tiles;
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ loader
+    if (lane == 0) {
+      mbar_arrive_tx(&bars.q_full, (uint32_t)(PL::NSQ * PL::H * 128));
+      for (int s = 0; s < PL::NSQ; ++s)
+        tma_load_2d(sQ + s * PL::H * 128, &mapQ, 64 * s, tq * p.Hq + head0, &bars.q_full);
+    }
+    for (int i = 0; i < nsub; ++i) {
+      const int st = i & 1;
+      bool ok = true;
+      if (lane == 0 && i >= 2) ok = mbar_wait(&bars.kv_empty[st], ((i >> 1) - 1) & 1, abort_flag, p.status);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      int* cd = codes + (i & 3) * PL::NK;
+      cd[lane] = resolve_row(p, u, i >> 1, 32 * (i & 1) + lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.codes_full[i & 3]);
+      const uint32_t stage = sKV + st * PL::kKVStage;
+#pragma unroll 4
+      for (int idx = lane; idx < PL::NK * (PL::DQK / 8); idx += 32) {
+        const int r = idx / (PL::DQK / 8), c = idx - r * (PL::DQK / 8);
+        const int code = cd[r];
+        const bf16* src = code >= 0 ? row_k_ptr(p, code, g) + c * 8 : p.k;
+        cp_async16(tk_kv_addr(stage, r, c), src, code >= 0);
+      }
+      cp_async_commit();
+      cp_async_wait_none();
+      fence_async_smem();
+      mbar_arrive(&bars.kv_full[st]);
+    }
+    cp_async_wait_none();
+    if (lane == 0) mbar_wait_drain(&bars.q_full, 0);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(64, 32, false, false);
+      constexpr uint32_t idPV = idesc_bf16(64, 256, false, true);
+      bool ok = mbar_wait(&bars.q_full, 0, abort_flag, p.status);
+      for (int i = 0; ok && i < nsub; ++i) {
+        const int st = i & 1;
+        if (!mbar_wait(&bars.kv_full[st], (i >> 1) & 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t kv = sKV + st * PL::kKVStage;
+        for (int kk = 0; kk < PL::DQK / 16; ++kk)
+          mma_bf16(tmem + PL::cS, sdesc(sQ + (kk >> 2) * (PL::H * 128) + (kk & 3) * 32, 16, 1024),
+                   sdesc(kv + (kk >> 2) * (PL::NK * 128) + (kk & 3) * 32, 16, 1024), idS, kk > 0);
+        mma_commit(&bars.s_full);
+        if (!mbar_wait(&bars.p_full, i & 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        // O += P V (V = the first 512 dims of the KV rows, an MN-major B)
+        for (int kk = 0; kk < PL::NK / 16; ++kk) {
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          const uint64_t a = sdesc64(sP + kk * 32, 16, 512);
+          mma_bf16(tmem + PL::cO, a, sdesc(kv + kk * 2048, PL::NK * 128, 1024), idPV, acc);
+          mma_bf16(tmem + (16u << 16) + PL::cO, a, sdesc(kv + 4 * (PL::NK * 128) + kk * 2048, PL::NK * 128, 1024),
+                   idPV, acc);
+        }
+        mma_commit(&bars.kv_empty[st]);
+        mma_commit(&bars.pv_done);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + O
+    const int sub = warp & 3;
+    const int h = 16 * sub + (lane & 15);
+    const bool is_s = lane < 16;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * sub) << 16);
+    const long long row = (long long)tq * p.Hq + head0 + h;
+    float m = -INFINITY, l = 0.f;  // running maximum (log2 units) and sum
+    if (p.sinks) {
+      m = __ldg(p.sinks + head0 + h) * kLog2eTk;
+      l = 1.f;
+    }
+    bool ok = true;
+    for (int i = 0; i < nsub; ++i) {
+      if (!mbar_wait(&bars.s_full, i & 1, abort_flag, p.status)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t v[2][16];
+      tmem_ld16(lane_base + PL::cS, v[0]);
+      tmem_ld16(lane_base + PL::cS + 16, v[1]);
+      tmem_wait_ld();
+      reg_dep16(v[0]);
+      reg_dep16(v[1]);
+      if (!mbar_wait(&bars.codes_full[i & 3], (i >> 2) & 1, abort_flag, p.status)) { ok = false; break; }
+      const int* cd = codes + (i & 3) * PL::NK;
+      float sc[32];
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        sc[k] = cd[k] >= 0 ? __uint_as_float(v[k >> 4][k & 15]) * p.scale_log2 : -INFINITY;
+        tmax = fmaxf(tmax, sc[k]);
+      }
+      tmax = __shfl_sync(0xffffffffu, tmax, lane & 15);  // the S lane's maximum for both halves
+      // the previous P V has landed (P buffer free, O stable) before P or O changes
+      if (i > 0 && !mbar_wait(&bars.pv_done, (i - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+      tc_fence_after();
+      const bool grow = tmax > m + 8.f;  // the same decision in both lanes of a head
+      if (__any_sync(0xffffffffu, grow)) {
+        const float mn = grow ? tmax : m;
+        const float f = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+        if (i > 0) {
+          // rescale this lane's half of the head's O row (256 columns)
+          for (int c = 0; c < 256; c += 16) {
+            uint32_t w[16];
+            tmem_ld16(lane_base + PL::cO + c, w);
+            tmem_wait_ld();
+            reg_dep16(w);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * f);
+            tmem_st16(lane_base + PL::cO + c, w);
+          }
+          tmem_wait_st();
+        }
+        l *= f;
+        m = mn;
+      }
+      if (is_s) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          const float a0 = exp2f(sc[k] - m), a1 = exp2f(sc[k + 1] - m);
+          l += a0 + a1;
+          pk[k >> 1] = pack_bf16(a0, a1);
+        }
+        const uint32_t rowaddr = sP + h * 64;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(rowaddr + ((c ^ ((h >> 1) & 3)) << 4)),
+                       "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                       : "memory");
+      }
+      tc_fence_before();
+      fence_async_smem();
+      mbar_arrive(&bars.p_full);
+    }
+    l = __shfl_sync(0xffffffffu, l, lane & 15);  // the S lane holds the sum
+    // O / l to bf16, lse = (m + log2 l) ln 2; a row with nothing visible gets O = 0, lse = +inf
+    if (ok && (nsub == 0 || mbar_wait(&bars.pv_done, (nsub - 1) & 1, abort_flag, p.status))) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      bf16* dst = O + row * PL::DV + (is_s ? 0 : 256);
+      for (int c = 0; c < 256; c += 16) {
+        uint32_t w[16];
+        tmem_ld16(lane_base + PL::cO + c, w);
+        tmem_wait_ld();
+        reg_dep16(w);
+        uint32_t o8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          o8[e] = nsub == 0 ? 0u : pack_bf16(__uint_as_float(w[2 * e]) * inv, __uint_as_float(w[2 * e + 1]) * inv);
+        reinterpret_cast<uint4*>(dst + c)[0] = make_uint4(o8[0], o8[1], o8[2], o8[3]);
+        reinterpret_cast<uint4*>(dst + c)[1] = make_uint4(o8[4], o8[5], o8[6], o8[7]);
+      }
+      if (is_s) LSE[row] = l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : INFINITY;
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, PL::kAlloc);
+    tmem_relinquish();
+  }
+}
+
+cudaError_t launch_tk_fwd(const Prob& p, bf16* o, float* lse, cudaStream_t st) {
+  using PL = TkFwdPlan;
+  if (!tk_path_built(p.dqk, p.dv, p.shared, p.G)) return cudaErrorInvalidValue;
+  const long long grid = (long long)p.Tq * p.Hkv * (p.G / PL::H);
+  if (grid == 0) return cudaSuccess;
+  CUtensorMap mq;
+  if (!make_tmap_bf16(&mq, p.q, (uint64_t)p.Tq * p.Hq, PL::DQK, (uint64_t)PL::DQK * 2, PL::H))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(tk_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kSmem);
+  if (e != cudaSuccess) return e;
+  mark_begin(st, kTimeFwd);
+  e = launch_pdl(tk_fwd_kernel, (unsigned)grid, 192, PL::kSmem, st, mq, p, o, lse);
+  count_launch();
+  mark_end(st, kTimeFwd);
+  return e;
+}
+
 }  // namespace sa
