@@ -271,6 +271,15 @@ sa_status sa_selftest_mma(int32_t M, int32_t N, int32_t K, int32_t a_mn, int32_t
                           int32_t d_lane, const void* A, const void* B, float* D, int32_t* status,
                           void* stream);
 
+/* Self-check of tcgen05 operand layouts written in software: D = A B as in
+ * sa_selftest_mma, but both operands are copied into shared memory by the CTA
+ * (no TMA), each in its own swizzle: a_sw / b_sw = 128 or 64 (bytes per row of
+ * an atom; atoms of 64 or 32 bf16 along the contiguous dimension, which must
+ * hold whole atoms).  M in {64, 128}; N, K multiples of 16 up to 256. */
+sa_status sa_selftest_mma2(int32_t M, int32_t N, int32_t K, int32_t a_mn, int32_t b_mn, int32_t a_sw,
+                           int32_t b_sw, int32_t d_lane, const void* A, const void* B, float* D, int32_t* status,
+                           void* stream);
+
 /* Self-check of the bounded waits every kernel uses: one CTA waits on an
  * mbarrier that nothing arrives on.  The wait gives up after its poll limit,
  * the kernel ORs the timeout bit (2) into *status (device int32) and returns

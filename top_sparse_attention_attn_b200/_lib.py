@@ -80,7 +80,8 @@ _lib = None
 EXPORTS = ["sa_fwd_get_workspace_size", "sa_fwd", "sa_bwd_get_workspace_size", "sa_bwd",
            "sa_softmax_grad_preprocess", "sa_debug_resolve", "sa_status_string", "sa_abi_version",
            "sa_set_timing_events", "sa_kernel_launch_count", "sa_bwd_no_alloc",
-           "sa_bwd_no_alloc_max_workspace", "sa_selftest_mma", "sa_selftest_wait_timeout"]
+           "sa_bwd_no_alloc_max_workspace", "sa_selftest_mma", "sa_selftest_wait_timeout",
+           "sa_selftest_mma2"]
 
 
 def lib() -> ctypes.CDLL:
@@ -110,6 +111,7 @@ def lib() -> ctypes.CDLL:
         L.sa_bwd_no_alloc_max_workspace.restype = ctypes.c_size_t
         L.sa_selftest_mma.argtypes = [ctypes.c_int32] * 7 + [_vp, _vp, _vp, _vp, _vp]
         L.sa_selftest_wait_timeout.argtypes = [_vp, _vp, _vp]
+        L.sa_selftest_mma2.argtypes = [ctypes.c_int32] * 8 + [_vp, _vp, _vp, _vp, _vp]
         for name in EXPORTS:
             if name not in ("sa_status_string", "sa_set_timing_events", "sa_kernel_launch_count",
                             "sa_bwd_no_alloc_max_workspace"):
@@ -162,6 +164,12 @@ def sa_selftest_mma(M: int, N: int, K: int, a_mn: int, b_mn: int, box_rows: int,
                     D: int, status: int, stream: int = 0, d_lane: int = 0) -> None:
     _check(lib().sa_selftest_mma(M, N, K, a_mn, b_mn, box_rows, d_lane, A, B, D, status, stream),
            "sa_selftest_mma")
+
+
+def sa_selftest_mma2(M: int, N: int, K: int, a_mn: int, b_mn: int, a_sw: int, b_sw: int, A: int, B: int,
+                     D: int, status: int, stream: int = 0, d_lane: int = 0) -> None:
+    _check(lib().sa_selftest_mma2(M, N, K, a_mn, b_mn, a_sw, b_sw, d_lane, A, B, D, status, stream),
+           "sa_selftest_mma2")
 
 
 def sa_selftest_wait_timeout(status: int, waited: int, stream: int = 0) -> None:
