@@ -32,7 +32,10 @@
  * sa_fwd_out / sa_bwd_io structs themselves are host memory read during the
  * call only.  `stream` is a cudaStream_t (NULL = the legacy default stream).
  *
- * Layouts (layout = SA_LAYOUT_BSND or SA_LAYOUT_TND, shared by Q and KV):
+ * Layouts (layout_q for q / o / d_o / lse / the index tensors, layout_kv for
+ * k / v / kv / cmp_kv, each SA_LAYOUT_BSND or SA_LAYOUT_TND, as the pages'
+ * layoutQ / layoutKv rows; only equal layouts are built, a mix returns
+ * SA_ERR_UNSUPPORTED):
  *   BSND: q [B, s_q, Hq, d_qk]   k [B, s_kv, Hkv, d_qk]   v [B, s_kv, Hkv, d_v]
  *         kv [B, s_kv, Hkv, d_qk] (K = V)  cmp_kv [B, s_kv / cmp_ratio, Hkv, d_qk]
  *         ori_idx [B, s_q, Hkv, topk]  cmp_idx [B, s_q, Hkv, cmp_topk]
@@ -68,13 +71,24 @@
  * kernel's completion before it reads or writes global memory, so stream
  * order is kept for the caller's own work before and after the call.
  *
+ * Status word.  The first 4 bytes of every forward or backward workspace are a
+ * status word that each call clears before its kernels run and that the
+ * kernels OR bits into:
+ *   1  an index past the end of its sequence was met (it selected nothing);
+ *   2  a bounded device wait gave up (the call's outputs are incomplete);
+ *   4  a kernel found its shared memory misaligned and did nothing.
+ * sa_read_status() synchronises the stream and maps the word to SA_OK,
+ * SA_ERR_TIMEOUT (bit 2), SA_ERR_INDEX (bit 1) or SA_ERR_CUDA (bit 4).
+ *
  * Bounded waits.  The tensor-core kernels' waits give up after about two
- * seconds; the kernel then raises a timeout bit in the workspace status word
- * and finishes without completing its work (see sa_selftest_wait_timeout).
+ * seconds; the kernel then raises the timeout bit in the status word and
+ * finishes without completing its work (see sa_selftest_wait_timeout).
  *
  * Errors.  Every entry point returns an sa_status.  Argument errors are found
  * on the host before anything is enqueued.  CUDA launch errors come back as
  * SA_ERR_CUDA (the library calls cudaGetLastError after its launches).
+ * Device-side conditions (timeouts, out-of-range indices) are read back with
+ * sa_read_status(), or at once with SA_FLAG_CHECK for indices.
  */
 #ifndef SPARSE_ATTN_H_
 #define SPARSE_ATTN_H_
@@ -86,7 +100,7 @@
 extern "C" {
 #endif
 
-#define SA_ABI_VERSION 1
+#define SA_ABI_VERSION 2
 
 typedef enum sa_status {
   SA_OK = 0,
@@ -108,20 +122,40 @@ typedef enum sa_dtype { SA_DTYPE_BF16 = 0, SA_DTYPE_FP16 = 1 } sa_dtype;
                               synchronises `stream` and returns SA_ERR_INDEX if one is
                               past its sequence (nothing else is computed) */
 /* Backward kernel choice (results agree within rounding; the default is the
- * fastest measured).  Block-level selection with block_size 64, BSND, equal
- * query / key lengths, separate K and V and no sinks runs key-stationary by
- * default: one CTA per (kv block, chunk of the tokens that select it)
- * accumulates dK / dV on the tensor cores and adds its dQ contributions to an
- * fp32 accumulator with vector atomics (Tq*Hq*d_qk*4 workspace bytes).
- * Every other problem runs query-stationary. */
-#define SA_FLAG_QUERY_STATIONARY_BWD 2u  /* force the query-stationary backward
+ * fastest measured; sa_plan() reports which kernel a problem gets).
+ * Block-level selection with block_size 64, BSND, equal query / key lengths,
+ * separate K and V and no sinks runs key-stationary by default: one CTA per
+ * (kv block, chunk of the tokens that select it) accumulates dK / dV on the
+ * tensor cores and adds its dQ contributions to an fp32 accumulator with
+ * vector atomics (Tq*Hq*d_qk*4 workspace bytes).  Token-level selection over
+ * one shared KV row of 576 (V = its first 512 columns) with a multiple of 64
+ * query heads per kv-head runs the tensor-core token kernel.  Every other
+ * problem runs the generic query-stationary kernel. */
+#define SA_FLAG_QUERY_STATIONARY_BWD 2u  /* force the generic query-stationary backward
                                             (dK / dV by fp32 scatter-add) */
 #define SA_FLAG_DQ_SEPARATE 4u  /* key-stationary backward: take dQ from a separate
-                                   query-stationary pass instead of atomics */
+                                   query-stationary pass instead of atomics; honoured
+                                   only when topk <= 256 (otherwise ignored) */
+
+/* Kernels reported by sa_plan(). */
+typedef enum sa_kernel {
+  SA_KERNEL_FWD_BLOCK = 1,         /* forward, query-stationary over 64-row blocks (topk <= 256) */
+  SA_KERNEL_FWD_TOKEN_TC = 2,      /* forward, token-level shared KV 576/512 on tcgen05 */
+  SA_KERNEL_FWD_GENERIC = 3,       /* forward, any selection, rows gathered one by one */
+  SA_KERNEL_BWD_KEY_STATIONARY = 4,        /* backward, key-stationary, dQ by atomics */
+  SA_KERNEL_BWD_KEY_STATIONARY_DQ_PASS = 5,/* backward, key-stationary + separate dQ pass */
+  SA_KERNEL_BWD_TOKEN_TC = 6,      /* backward, token-level shared KV 576/512 on tcgen05 */
+  SA_KERNEL_BWD_GENERIC = 7        /* backward, any selection, dK / dV by fp32 scatter-add */
+} sa_kernel;
+
+/* Views of sa_debug_block_index(). */
+#define SA_INDEX_VIEW_QUERY_BLOCKS 0  /* usable slots as the query-stationary block kernels see them */
+#define SA_INDEX_VIEW_KEY_LISTS 1     /* the key-stationary backward's inverse index */
 
 /* The problem description shared by every entry point (host struct). */
 typedef struct sa_args {
-  int32_t layout;          /* sa_layout */
+  int32_t layout_q;        /* sa_layout of q, o, d_o, lse and the index tensors */
+  int32_t layout_kv;       /* sa_layout of k, v, kv and cmp_kv (must equal layout_q) */
   int32_t dtype;           /* sa_dtype; only SA_DTYPE_BF16 is built */
   int32_t batch;           /* B >= 0 */
   int32_t s_q, s_kv;       /* BSND sequence lengths (ignored for TND) */
@@ -211,9 +245,11 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
  * the library until the process exits) and allocates nothing.
  *   - Problems whose sa_bwd_get_workspace_size exceeds that size are rejected
  *     with SA_ERR_WORKSPACE before anything is enqueued.
- *   - The first call on a device (with that device current) resolves the
- *     array's device address once; make that first call before any stream
- *     capture.
+ *   - The first call in a CUDA context (the device's primary context, with
+ *     that device current) resolves the array's device address once; make
+ *     that first call before any stream capture.  A new context on the same
+ *     device (after cudaDeviceReset, or one made current through the driver
+ *     API) resolves it again.
  *   - All calls share the one array: calls whose work overlaps on the GPU
  *     (other streams, other host threads on the same device) race.  Each call
  *     re-zeroes the parts it uses, so nothing carries over between calls.
@@ -271,12 +307,54 @@ sa_status sa_selftest_mma(int32_t M, int32_t N, int32_t K, int32_t a_mn, int32_t
                           int32_t d_lane, const void* A, const void* B, float* D, int32_t* status,
                           void* stream);
 
+/* Self-check of tcgen05 operand layouts written in software: D = A B as in
+ * sa_selftest_mma, but both operands are copied into shared memory by the CTA
+ * (no TMA), each in its own swizzle: a_sw / b_sw = 128 or 64 (bytes per row of
+ * an atom; atoms of 64 or 32 bf16 along the contiguous dimension, which must
+ * hold whole atoms).  M in {64, 128}; N, K multiples of 16 up to 256. */
+sa_status sa_selftest_mma2(int32_t M, int32_t N, int32_t K, int32_t a_mn, int32_t b_mn, int32_t a_sw,
+                           int32_t b_sw, int32_t d_lane, const void* A, const void* B, float* D, int32_t* status,
+                           void* stream);
+
 /* Self-check of the bounded waits every kernel uses: one CTA waits on an
  * mbarrier that nothing arrives on.  The wait gives up after its poll limit,
  * the kernel ORs the timeout bit (2) into *status (device int32) and returns
  * normally, so the context stays usable; *waited (device int32) gets 1 if the
  * wait (wrongly) completed, else 0.  Asynchronous; takes as long as the limit. */
 sa_status sa_selftest_wait_timeout(int32_t* status, int32_t* waited, void* stream);
+
+/* Which kernels sa_fwd and sa_bwd would run for `args` (validated as by
+ * *_get_workspace_size).  Either output pointer may be NULL.  Host only. */
+sa_status sa_plan(const sa_args* args, int32_t* fwd_kernel, int32_t* bwd_kernel);
+
+/* Read back the status word of a forward or backward workspace (device
+ * pointer `ws`, the one the last call on `stream` used): synchronises
+ * `stream`, then returns SA_ERR_TIMEOUT if a bounded wait gave up, else
+ * SA_ERR_INDEX if an index past its sequence was met, else SA_ERR_CUDA if a
+ * kernel could not run, else SA_OK.  The word is left as it is. */
+sa_status sa_read_status(const void* ws, size_t ws_bytes, void* stream);
+
+/* The same for the scratch array behind sa_bwd_no_alloc on the current
+ * device (after its last call on `stream`). */
+sa_status sa_bwd_no_alloc_read_status(void* stream);
+
+/* Block-level index sets exactly as the block kernels build them, for
+ * bit-exact checks (64-row blocks, separate K / V).  Each record is four int32
+ * {unit = token * Hkv + kv-head, block x, lo, hi}: block x contributes rows
+ * [64x + lo, 64x + hi] (sequence-local) to the unit's visible set.
+ *   SA_INDEX_VIEW_QUERY_BLOCKS: one record per usable slot of every unit, from
+ *     the slot rule and in-block row range of the query-stationary block
+ *     kernels (requires SA_KERNEL_FWD_BLOCK for `args`; `ws` unused).
+ *   SA_INDEX_VIEW_KEY_LISTS: builds the key-stationary backward's inverse index
+ *     into `ws` (a backward workspace of sa_bwd_get_workspace_size bytes) the
+ *     way sa_bwd does, then walks every work item as the backward kernel does
+ *     and emits one record per (item, token) with the block's row range for
+ *     that token (requires a key-stationary backward for `args`).
+ * records: device int32 [max_records][4]; *n_records (device int32) receives
+ * the number of records produced (may exceed max_records; only max_records
+ * are written).  Records come in no particular order.  Asynchronous. */
+sa_status sa_debug_block_index(const sa_args* args, int32_t view, void* ws, size_t ws_bytes, int32_t* records,
+                               int64_t max_records, int32_t* n_records, void* stream);
 
 /* Human-readable name of a status code (static string). */
 const char* sa_status_string(int32_t status);

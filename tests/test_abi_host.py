@@ -46,7 +46,7 @@ C_PROBE = r"""
 #define F(S, m) printf("%s.%s %zu\n", #S, #m, offsetof(S, m));
 int main(void) {
   printf("sa_args %zu\nsa_fwd_out %zu\nsa_bwd_io %zu\n", sizeof(sa_args), sizeof(sa_fwd_out), sizeof(sa_bwd_io));
-  F(sa_args, ori_win_left) F(sa_args, scale) F(sa_args, flags) F(sa_args, q) F(sa_args, sinks)
+  F(sa_args, layout_kv) F(sa_args, dtype) F(sa_args, ori_win_left) F(sa_args, scale) F(sa_args, flags) F(sa_args, q) F(sa_args, sinks)
   F(sa_args, cmp_idx) F(sa_args, cu_seqlens_cmp) F(sa_bwd_io, dsinks) F(sa_bwd_io, dcmp_kv)
   return 0;
 }
@@ -80,7 +80,7 @@ FAKE = 0x10000  # 16-byte aligned, never dereferenced: these calls fail validati
 
 def _args(**kw):
     a = L.SaArgs()
-    a.layout = L.SA_LAYOUT_BSND
+    a.layout_q = a.layout_kv = L.SA_LAYOUT_BSND
     a.dtype = L.SA_DTYPE_BF16
     a.batch, a.s_q, a.s_kv = 2, 128, 128
     a.n_heads_q, a.n_heads_kv = 16, 4
@@ -116,13 +116,15 @@ def _ws(a):
     (dict(q=None), L.SA_ERR_NULLPTR),
     (dict(ori_idx=None), L.SA_ERR_NULLPTR),
     (dict(v=None), L.SA_ERR_NULLPTR),
-    (dict(layout=5), L.SA_ERR_PARAM),
+    (dict(layout_q=5, layout_kv=5), L.SA_ERR_PARAM),
+    (dict(layout_kv=5), L.SA_ERR_PARAM),
+    (dict(layout_kv=L.SA_LAYOUT_TND), L.SA_ERR_UNSUPPORTED),                 # mixed layouts are not built
     (dict(ori_mask_mode=L.SA_MASK_BAND, ori_win_left=-1), L.SA_ERR_PARAM),
     (dict(cmp_mask_mode=L.SA_MASK_BAND), L.SA_ERR_PARAM),
     (dict(cmp_ratio=0), L.SA_ERR_PARAM),
     (dict(scale=float("nan")), L.SA_ERR_PARAM),
     (dict(cmp_topk=8, cmp_kv=FAKE, cmp_idx=FAKE), L.SA_ERR_UNSUPPORTED),   # compressed KV needs K = V
-    (dict(layout=L.SA_LAYOUT_TND, t_q=256, t_kv=256), L.SA_ERR_NULLPTR),    # no cu_seqlens
+    (dict(layout_q=L.SA_LAYOUT_TND, layout_kv=L.SA_LAYOUT_TND, t_q=256, t_kv=256), L.SA_ERR_NULLPTR),
     (dict(kv_shared=1, d_qk=128, d_v=128, k=None, v=None), L.SA_ERR_NULLPTR),
     (dict(kv_shared=1, d_qk=128, d_v=128, k=None, v=None, kv=FAKE), L.SA_OK),
     (dict(kv_shared=1, d_qk=128, d_v=256, kv=FAKE), L.SA_ERR_PARAM),
@@ -155,20 +157,21 @@ def test_bwd_workspace_size_contract():
     # counts, cursor, list offsets, work items (16 B each; a small problem gets
     # chunks of ceil(n_slots / 148) tokens rounded up to whole 128-row tiles), the
     # work count and the entries; a problem this small also takes the bucketed
-    # index: per bucket of 512 slots, each list's count and offset
+    # index: per bucket of 512 slots, each list's count and offset, and one flag
     n_lists, n_slots = 2 * 4 * 2, 2 * 128 * 4 * 4
     chunk = -(-(-(-n_slots // 148)) // 16) * 16  # whole tiles of 16 (8 rows per token) or 32 tokens
     max_work = -(-n_slots // chunk) + n_lists
     cells = -(-n_slots // 512) * n_lists
+    n_buckets = -(-n_slots // 512)
     index = (2 * _align(4 * n_lists) + _align(4 * (n_lists + 1)) + _align(16 * max_work) + 256
-             + _align(4 * n_slots) + 2 * _align(4 * cells))
+             + _align(4 * n_slots) + 2 * _align(4 * cells) + _align(4 * n_buckets))
     st, n = _ws(_args(flags=L.SA_FLAG_DQ_SEPARATE))
     assert st == L.SA_OK and n == base + index
     # ... + an fp32 dQ accumulator when dQ is formed in the same kernel (the default)
     st, n = _ws(_args())
     assert st == L.SA_OK and n == base + index + _align(Tq * 16 * 192 * 4)
     a = _args(kv_shared=1, d_qk=576, d_v=512, kv=FAKE, n_heads_q=64, n_heads_kv=1, block_size=1,
-              layout=L.SA_LAYOUT_TND, t_q=1000, t_kv=1000, t_cmp=250, cmp_topk=16, cmp_ratio=4,
+              layout_q=L.SA_LAYOUT_TND, layout_kv=L.SA_LAYOUT_TND, t_q=1000, t_kv=1000, t_cmp=250, cmp_topk=16, cmp_ratio=4,
               cmp_kv=FAKE, cmp_idx=FAKE, cu_seqlens_q=FAKE, cu_seqlens_kv=FAKE, cu_seqlens_cmp=FAKE)
     st, n = _ws(a)
     expect = 256 + _align(1000 * 64 * 4) + _align(1000 * 576 * 4) + _align(250 * 576 * 4)
@@ -215,3 +218,52 @@ def test_no_alloc_rejects_oversized_problem_on_the_host():
     io = L.SaBwdIo(o=FAKE, d_o=FAKE, lse=FAKE, dq=FAKE, dk=FAKE, dv=FAKE)
     assert L.lib().sa_bwd_no_alloc(ctypes.byref(a), ctypes.byref(io), None) == L.SA_ERR_WORKSPACE
     assert L.lib().sa_bwd_no_alloc(ctypes.byref(_args(n_heads_q=15)), ctypes.byref(io), None) == L.SA_ERR_PARAM
+
+
+def _plan(a):
+    return L.sa_plan(a)
+
+
+def test_plan_reports_the_kernel_each_problem_gets():
+    """sa_plan names the forward / backward kernels sa_fwd / sa_bwd dispatch to."""
+    assert _plan(_args()) == (L.SA_KERNEL_FWD_BLOCK, L.SA_KERNEL_BWD_KEY_STATIONARY)
+    assert _plan(_args(flags=L.SA_FLAG_DQ_SEPARATE)) == (L.SA_KERNEL_FWD_BLOCK,
+                                                         L.SA_KERNEL_BWD_KEY_STATIONARY_DQ_PASS)
+    assert _plan(_args(flags=L.SA_FLAG_QUERY_STATIONARY_BWD))[1] == L.SA_KERNEL_BWD_GENERIC
+    # sinks, TND, block sizes other than 64 and unequal lengths leave the key-stationary kernel
+    assert _plan(_args(sinks=FAKE))[1] == L.SA_KERNEL_BWD_GENERIC
+    assert _plan(_args(block_size=16)) == (L.SA_KERNEL_FWD_GENERIC, L.SA_KERNEL_BWD_GENERIC)
+    assert _plan(_args(s_kv=256))[1] == L.SA_KERNEL_BWD_GENERIC
+    # token-level shared KV 576 / 512 with 64 heads per kv-head: the tensor-core token kernels
+    tok = dict(kv_shared=1, d_qk=576, d_v=512, kv=FAKE, k=None, v=None, n_heads_q=64, n_heads_kv=1,
+               block_size=1, topk=32)
+    assert _plan(_args(**tok)) == (L.SA_KERNEL_FWD_TOKEN_TC, L.SA_KERNEL_BWD_TOKEN_TC)
+    assert _plan(_args(**dict(tok, n_heads_q=16))) == (L.SA_KERNEL_FWD_GENERIC, L.SA_KERNEL_BWD_GENERIC)
+    with pytest.raises(L.SaError):
+        _plan(_args(n_heads_q=15))
+
+
+def test_dq_separate_is_ignored_past_the_block_kernels_slot_limit():
+    """The separate dQ pass holds at most 256 usable slots per unit: with more, the flag is
+    ignored (the key-stationary kernel forms dQ), in the plan and in the workspace."""
+    a = _args(topk=300, batch=1, s_q=65536, s_kv=65536)
+    b = _args(topk=300, batch=1, s_q=65536, s_kv=65536, flags=L.SA_FLAG_DQ_SEPARATE)
+    assert _plan(b) == (L.SA_KERNEL_FWD_GENERIC, L.SA_KERNEL_BWD_KEY_STATIONARY)
+    assert _ws(a) == _ws(b)
+
+
+def test_status_and_inspection_calls_validate_on_the_host():
+    assert L.lib().sa_read_status(None, 256, None) == L.SA_ERR_NULLPTR
+    assert L.lib().sa_read_status(FAKE, 0, None) == L.SA_ERR_WORKSPACE
+    n = FAKE
+    dbi = L.lib().sa_debug_block_index
+    assert dbi(ctypes.byref(_args()), 7, None, 0, FAKE, 16, n, None) == L.SA_ERR_PARAM
+    assert dbi(ctypes.byref(_args()), L.SA_INDEX_VIEW_QUERY_BLOCKS, None, 0, FAKE, -1, n, None) == L.SA_ERR_PARAM
+    assert dbi(ctypes.byref(_args()), L.SA_INDEX_VIEW_QUERY_BLOCKS, None, 0, FAKE, 16, None, None) == \
+        L.SA_ERR_NULLPTR
+    # the key-stationary view needs a backward workspace, and a problem that runs key-stationary
+    assert dbi(ctypes.byref(_args()), L.SA_INDEX_VIEW_KEY_LISTS, None, 0, FAKE, 16, n, None) == L.SA_ERR_WORKSPACE
+    assert dbi(ctypes.byref(_args(sinks=FAKE)), L.SA_INDEX_VIEW_KEY_LISTS, FAKE, 1 << 30, FAKE, 16, n, None) == \
+        L.SA_ERR_UNSUPPORTED
+    assert dbi(ctypes.byref(_args(block_size=16)), L.SA_INDEX_VIEW_QUERY_BLOCKS, None, 0, FAKE, 16, n, None) == \
+        L.SA_ERR_UNSUPPORTED

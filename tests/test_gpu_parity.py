@@ -41,6 +41,11 @@ SMALL = {
                          seed=31), {}),
     "token_shared_128_nomask": (scaled("cfg3", "nomask", S=333, Hq=16, d_qk=128, d_v=128,
                                        topk=100, ori_mask="none", seed=32), {}),
+    # token-level shared KV with 64 or 128 heads per KV head: the tcgen05 token kernel
+    "token_h64_topk": (scaled("cfg3", "h64", S=400, Hq=64, topk=256, seed=35), {}),
+    "token_h128_topk": (scaled("cfg3", "h128", S=300, Hq=128, topk=96, seed=36), {}),
+    "swa_cmp_h64": (scaled("cfg4", "h64", seqlens=(100, 300, 37), Hq=64, cmp_topk=64,
+                           cmp_len_range=(16, 64), seed=37), {}),
     # G = 1 and 2: key-stationary tiles of 128 and 64 tokens with rows gathered one by one
     "block_g1_d64": (scaled("cfg1", "g1", S=700, Hq=2, Hkv=2, topk=5, seed=33), {}),
     "block_g2_d128": (scaled("cfg5", "g2", S=1000, Hq=4, Hkv=2, d_qk=128, d_v=128, topk=7, zipf_s=1.2,

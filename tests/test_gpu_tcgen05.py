@@ -58,4 +58,39 @@ def test_bounded_wait_gives_up_and_reports():
     assert int(status.item()) & 2, "the timeout bit was not raised"
     assert elapsed < 20.0, f"the bounded wait took {elapsed:.1f} s"
     print(f"bounded wait gave up after {elapsed:.2f} s")
+    # the word reads back through the ABI as SA_ERR_TIMEOUT (a status word of its own:
+    # sa_read_status reads the first 4 bytes of any workspace)
+    assert L.sa_read_status(status.data_ptr(), 4, torch.cuda.current_stream().cuda_stream) == L.SA_ERR_TIMEOUT
+    status.zero_()
+    assert L.sa_read_status(status.data_ptr(), 4, torch.cuda.current_stream().cuda_stream) == L.SA_OK
     test_tcgen05_mma_matches_matmul((128, 64, 64, 0, 0, 64))
+
+
+CASES2 = [
+    # M, N, K, a_mn, b_mn, a_sw, b_sw[, d_lane]: the token-level kernel's operand shapes
+    (64, 32, 128, 0, 0, 128, 128), (64, 32, 128, 0, 0, 128, 128, 16),   # S / dP: 32-row K-major B
+    (64, 256, 32, 0, 1, 64, 128), (64, 64, 32, 0, 1, 64, 128),          # dQ: 64-byte-swizzle A, K = 32
+    (64, 256, 32, 0, 1, 64, 128, 16),                                   # dQ upper half at lane offset 16
+    (128, 32, 64, 1, 1, 128, 64), (64, 32, 64, 1, 1, 128, 64),          # dKV: MN-major B of one 32-wide atom
+    (128, 64, 128, 0, 0, 128, 128), (128, 128, 64, 1, 1, 128, 128),     # the TMA-loaded cases, loaded in software
+]
+
+
+@pytest.mark.parametrize("case", CASES2, ids=[str(c) for c in CASES2])
+def test_software_layouts_match_matmul(case):
+    M, N, K, a_mn, b_mn, a_sw, b_sw = case[:7]
+    d_lane = case[7] if len(case) > 7 else 0
+    g = torch.Generator(device="cuda").manual_seed(M * 1000 + N * 10 + K + a_sw + b_sw)
+    A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+    B = torch.randn(K, N, device="cuda", generator=g).to(torch.bfloat16)
+    a_store = A.t().contiguous() if a_mn else A.contiguous()
+    b_store = B.contiguous() if b_mn else B.t().contiguous()
+    D = torch.full((M, N), float("nan"), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.sa_selftest_mma2(M, N, K, a_mn, b_mn, a_sw, b_sw, a_store.data_ptr(), b_store.data_ptr(), D.data_ptr(),
+                       status.data_ptr(), torch.cuda.current_stream().cuda_stream, d_lane=d_lane)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ref = A.float() @ B.float()
+    err = (D - ref).abs().max().item()
+    assert err <= 1e-3 * ref.abs().max().item(), f"max err {err}"

@@ -33,6 +33,22 @@ SA_FLAG_CHECK = 1
 SA_FLAG_QUERY_STATIONARY_BWD = 2
 SA_FLAG_DQ_SEPARATE = 4
 
+# sa_kernel (sa_plan)
+SA_KERNEL_FWD_BLOCK = 1
+SA_KERNEL_FWD_TOKEN_TC = 2
+SA_KERNEL_FWD_GENERIC = 3
+SA_KERNEL_BWD_KEY_STATIONARY = 4
+SA_KERNEL_BWD_KEY_STATIONARY_DQ_PASS = 5
+SA_KERNEL_BWD_TOKEN_TC = 6
+SA_KERNEL_BWD_GENERIC = 7
+SA_INDEX_VIEW_QUERY_BLOCKS = 0
+SA_INDEX_VIEW_KEY_LISTS = 1
+
+# status word bits (the first 4 bytes of every workspace)
+SA_STATUS_INDEX = 1
+SA_STATUS_TIMEOUT = 2
+SA_STATUS_SMEM_ALIGN = 4
+
 MASKS = {"none": SA_MASK_NONE, "causal": SA_MASK_CAUSAL, "band": SA_MASK_BAND}
 LAYOUTS = {"BSND": SA_LAYOUT_BSND, "TND": SA_LAYOUT_TND}
 
@@ -43,7 +59,8 @@ _fp = ctypes.POINTER(ctypes.c_float)
 
 class SaArgs(ctypes.Structure):
     _fields_ = [
-        ("layout", ctypes.c_int32), ("dtype", ctypes.c_int32), ("batch", ctypes.c_int32),
+        ("layout_q", ctypes.c_int32), ("layout_kv", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("batch", ctypes.c_int32),
         ("s_q", ctypes.c_int32), ("s_kv", ctypes.c_int32),
         ("t_q", ctypes.c_int32), ("t_kv", ctypes.c_int32), ("t_cmp", ctypes.c_int32),
         ("n_heads_q", ctypes.c_int32), ("n_heads_kv", ctypes.c_int32),
@@ -80,7 +97,9 @@ _lib = None
 EXPORTS = ["sa_fwd_get_workspace_size", "sa_fwd", "sa_bwd_get_workspace_size", "sa_bwd",
            "sa_softmax_grad_preprocess", "sa_debug_resolve", "sa_status_string", "sa_abi_version",
            "sa_set_timing_events", "sa_kernel_launch_count", "sa_bwd_no_alloc",
-           "sa_bwd_no_alloc_max_workspace", "sa_selftest_mma", "sa_selftest_wait_timeout"]
+           "sa_bwd_no_alloc_max_workspace", "sa_selftest_mma", "sa_selftest_wait_timeout",
+           "sa_selftest_mma2", "sa_plan", "sa_read_status", "sa_bwd_no_alloc_read_status",
+           "sa_debug_block_index"]
 
 
 def lib() -> ctypes.CDLL:
@@ -110,6 +129,12 @@ def lib() -> ctypes.CDLL:
         L.sa_bwd_no_alloc_max_workspace.restype = ctypes.c_size_t
         L.sa_selftest_mma.argtypes = [ctypes.c_int32] * 7 + [_vp, _vp, _vp, _vp, _vp]
         L.sa_selftest_wait_timeout.argtypes = [_vp, _vp, _vp]
+        L.sa_selftest_mma2.argtypes = [ctypes.c_int32] * 8 + [_vp, _vp, _vp, _vp, _vp]
+        L.sa_plan.argtypes = [P(SaArgs), _ip, _ip]
+        L.sa_read_status.argtypes = [_vp, ctypes.c_size_t, _vp]
+        L.sa_bwd_no_alloc_read_status.argtypes = [_vp]
+        L.sa_debug_block_index.argtypes = [P(SaArgs), ctypes.c_int32, _vp, ctypes.c_size_t, _vp, ctypes.c_int64,
+                                           _vp, _vp]
         for name in EXPORTS:
             if name not in ("sa_status_string", "sa_set_timing_events", "sa_kernel_launch_count",
                             "sa_bwd_no_alloc_max_workspace"):
@@ -164,6 +189,12 @@ def sa_selftest_mma(M: int, N: int, K: int, a_mn: int, b_mn: int, box_rows: int,
            "sa_selftest_mma")
 
 
+def sa_selftest_mma2(M: int, N: int, K: int, a_mn: int, b_mn: int, a_sw: int, b_sw: int, A: int, B: int,
+                     D: int, status: int, stream: int = 0, d_lane: int = 0) -> None:
+    _check(lib().sa_selftest_mma2(M, N, K, a_mn, b_mn, a_sw, b_sw, d_lane, A, B, D, status, stream),
+           "sa_selftest_mma2")
+
+
 def sa_selftest_wait_timeout(status: int, waited: int, stream: int = 0) -> None:
     _check(lib().sa_selftest_wait_timeout(status, waited, stream), "sa_selftest_wait_timeout")
 
@@ -175,6 +206,28 @@ def sa_softmax_grad_preprocess(args: SaArgs, o: int, d_o: int, delta: int, strea
 
 def sa_debug_resolve(args: SaArgs, rows: int, counts: int, max_rows: int, stream: int = 0) -> None:
     _check(lib().sa_debug_resolve(ctypes.byref(args), rows, counts, max_rows, stream), "sa_debug_resolve")
+
+
+def sa_plan(args: SaArgs) -> tuple:
+    """(forward kernel, backward kernel) as SA_KERNEL_* values."""
+    f, b = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(lib().sa_plan(ctypes.byref(args), ctypes.byref(f), ctypes.byref(b)), "sa_plan")
+    return f.value, b.value
+
+
+def sa_read_status(ws: int, ws_bytes: int, stream: int = 0) -> int:
+    """The workspace status word mapped to an sa_status (synchronises the stream; never raises)."""
+    return int(lib().sa_read_status(ws, ws_bytes, stream))
+
+
+def sa_bwd_no_alloc_read_status(stream: int = 0) -> int:
+    return int(lib().sa_bwd_no_alloc_read_status(stream))
+
+
+def sa_debug_block_index(args: SaArgs, view: int, ws: int, ws_bytes: int, records: int, max_records: int,
+                         n_records: int, stream: int = 0) -> None:
+    _check(lib().sa_debug_block_index(ctypes.byref(args), view, ws, ws_bytes, records, max_records, n_records,
+                                      stream), "sa_debug_block_index")
 
 
 def sa_abi_version() -> int:

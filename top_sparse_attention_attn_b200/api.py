@@ -73,7 +73,8 @@ class SparseAttention:
 
     def args(self) -> L.SaArgs:
         a = L.SaArgs()
-        a.layout = L.LAYOUTS[self.layout]
+        a.layout_q = L.LAYOUTS[self.layout]
+        a.layout_kv = L.LAYOUTS[self.layout]
         a.dtype = L.SA_DTYPE_BF16
         a.batch = self.batch
         a.s_q, a.s_kv = self.s_q, self.s_kv
@@ -167,6 +168,32 @@ class SparseAttention:
         st = torch.cuda.current_stream().cuda_stream if stream is None else stream
         L.sa_debug_resolve(self.args(), _ptr(rows), _ptr(counts), max_rows, st)
         return rows, counts
+
+    def block_index(self, view: int, max_records: int | None = None, stream=None):
+        """Records {unit, block, lo, hi} of the block-level index sets as the block
+        kernels build them (sa_debug_block_index); returns an int32 [n, 4] device tensor."""
+        if max_records is None:
+            max_records = self.n_tokens * self.Hkv * max(self.topk, 1)
+        rec = torch.full((max(max_records, 1), 4), -1, dtype=torch.int32, device=self.q.device)
+        n = torch.zeros(1, dtype=torch.int32, device=self.q.device)
+        ws = self.bwd_workspace() if view == L.SA_INDEX_VIEW_KEY_LISTS else None
+        st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+        L.sa_debug_block_index(self.args(), view, _ptr(ws), 0 if ws is None else ws.numel(), _ptr(rec),
+                               max_records, _ptr(n), st)
+        count = int(n.item())
+        if count > max_records:
+            raise RuntimeError(f"{count} records, room for {max_records}")
+        return rec[:count]
+
+    def plan(self) -> tuple:
+        """(forward kernel, backward kernel) that sa_fwd / sa_bwd run (SA_KERNEL_*)."""
+        return L.sa_plan(self.args())
+
+    @staticmethod
+    def read_status(ws: torch.Tensor, stream=None) -> int:
+        """The status word of a workspace after its last call, as an sa_status."""
+        st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+        return L.sa_read_status(_ptr(ws), ws.numel(), st)
 
     # ---- construction from a workload description ---------------------------
     @classmethod

@@ -16,6 +16,10 @@ namespace {
 using sa::bf16;
 
 constexpr size_t kAlign = 256;
+// BAND windows wider than any sequence change nothing; clamping keeps the
+// kernels' 64-bit window arithmetic far from overflow.
+constexpr long long kWinClamp = 1ll << 40;
+long long clamp_win(long long w) { return w < kWinClamp ? w : kWinClamp; }
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Sizes {
@@ -24,7 +28,7 @@ struct Sizes {
 
 Sizes sizes_of(const sa_args* a) {
   Sizes s;
-  if (a->layout == SA_LAYOUT_BSND) {
+  if (a->layout_q == SA_LAYOUT_BSND) {
     s.Tq = (long long)a->batch * a->s_q;
     s.Tkv = (long long)a->batch * a->s_kv;
     s.Tcmp = a->cmp_topk > 0 ? (long long)a->batch * (a->s_kv / (a->cmp_ratio > 0 ? a->cmp_ratio : 1)) : 0;
@@ -40,9 +44,11 @@ sa_status validate(const sa_args* a) {
   if (!a) return SA_ERR_NULLPTR;
   if (a->dtype == SA_DTYPE_FP16) return SA_ERR_UNSUPPORTED;
   if (a->dtype != SA_DTYPE_BF16) return SA_ERR_PARAM;
-  if (a->layout != SA_LAYOUT_BSND && a->layout != SA_LAYOUT_TND) return SA_ERR_PARAM;
+  if (a->layout_q != SA_LAYOUT_BSND && a->layout_q != SA_LAYOUT_TND) return SA_ERR_PARAM;
+  if (a->layout_kv != SA_LAYOUT_BSND && a->layout_kv != SA_LAYOUT_TND) return SA_ERR_PARAM;
+  if (a->layout_q != a->layout_kv) return SA_ERR_UNSUPPORTED;  // mixed layouts are not built
   if (a->batch < 0) return SA_ERR_PARAM;
-  if (a->layout == SA_LAYOUT_BSND) {
+  if (a->layout_q == SA_LAYOUT_BSND) {
     if (a->s_q < 0 || a->s_kv < 0) return SA_ERR_PARAM;
   } else {
     if (a->t_q < 0 || a->t_kv < 0 || a->t_cmp < 0) return SA_ERR_PARAM;
@@ -68,7 +74,7 @@ sa_status validate(const sa_args* a) {
     if (a->kv_shared ? !a->kv : (!a->k || !a->v)) return SA_ERR_NULLPTR;
     if (a->topk > 0 && !a->ori_idx) return SA_ERR_NULLPTR;
     if (a->cmp_topk > 0 && (!a->cmp_kv || !a->cmp_idx)) return SA_ERR_NULLPTR;
-    if (a->layout == SA_LAYOUT_TND) {
+    if (a->layout_q == SA_LAYOUT_TND) {
       if (!a->cu_seqlens_q || !a->cu_seqlens_kv) return SA_ERR_NULLPTR;
       if (a->cmp_topk > 0 && !a->cu_seqlens_cmp) return SA_ERR_NULLPTR;
       if (a->batch < 1) return SA_ERR_PARAM;
@@ -84,7 +90,7 @@ sa::Prob make_prob(const sa_args* a, int* status) {
   sa::Prob p;
   memset(&p, 0, sizeof(p));
   Sizes s = sizes_of(a);
-  p.layout = a->layout;
+  p.layout = a->layout_q;
   p.B = a->batch;
   p.s_q = a->s_q;
   p.s_kv = a->s_kv;
@@ -103,8 +109,8 @@ sa::Prob make_prob(const sa_args* a, int* status) {
   p.ratio = a->cmp_ratio;
   p.ori_mask = a->ori_mask_mode;
   p.cmp_mask = a->cmp_mask_mode;
-  p.wl = a->ori_win_left;
-  p.wr = a->ori_win_right;
+  p.wl = clamp_win(a->ori_win_left);
+  p.wr = clamp_win(a->ori_win_right);
   p.scale = a->scale;
   p.scale_log2 = a->scale * 1.4426950408889634f;
   p.q = static_cast<const bf16*>(a->q);
@@ -142,22 +148,27 @@ sa_status check_tensor_alignment(const sa_args* a) {
 bool use_kv_path(const sa_args* a) {
   if (a->flags & SA_FLAG_QUERY_STATIONARY_BWD) return false;
   const int G = a->n_heads_q / a->n_heads_kv;
-  return a->layout == SA_LAYOUT_BSND && a->topk > 0 && a->block_size == 64 && a->s_q == a->s_kv &&
+  return a->layout_q == SA_LAYOUT_BSND && a->topk > 0 && a->block_size == 64 && a->s_q == a->s_kv &&
          !a->kv_shared && a->cmp_topk == 0 && a->sinks == nullptr && G <= 128 &&
          sa::kv_path_built(a->d_qk, a->d_v);
 }
 
 // Query-stationary block kernels (TMA-fed): 64-row blocks, separate K / V, no compressed KV.
 bool use_qb_path(const sa_args* a) {
-  return a->topk > 0 && a->topk <= 256 && a->block_size == 64 && !a->kv_shared && a->cmp_topk == 0 &&
+  return a->topk > 0 && a->topk <= sa::kQbMaxSlots && a->block_size == 64 && !a->kv_shared && a->cmp_topk == 0 &&
          sa::qb_path_built(a->d_qk, a->d_v);
 }
+
+// SA_FLAG_DQ_SEPARATE applies only where the query-stationary block kernels do
+// (they hold at most kQbMaxSlots usable slots per unit); elsewhere the
+// key-stationary kernel forms dQ with atomics as by default.
+bool dq_separate(const sa_args* a) { return (a->flags & SA_FLAG_DQ_SEPARATE) && use_qb_path(a); }
 
 sa::QbArgs make_qb_args(const sa_args* a, int* status) {
   sa::QbArgs q;
   memset(&q, 0, sizeof(q));
   Sizes s = sizes_of(a);
-  q.layout = a->layout;
+  q.layout = a->layout_q;
   q.B = a->batch;
   q.s_q = a->s_q;
   q.s_kv = a->s_kv;
@@ -170,8 +181,8 @@ sa::QbArgs make_qb_args(const sa_args* a, int* status) {
   q.dv = a->d_v;
   q.topk = a->topk;
   q.ori_mask = a->ori_mask_mode;
-  q.wl = a->ori_win_left;
-  q.wr = a->ori_win_right;
+  q.wl = clamp_win(a->ori_win_left);
+  q.wr = clamp_win(a->ori_win_right);
   q.scale = a->scale;
   q.scale_log2 = a->scale * 1.4426950408889634f;
   q.q = static_cast<const bf16*>(a->q);
@@ -194,7 +205,7 @@ KvGeom kv_geometry(const sa_args* a) {
   const int G = a->n_heads_q / a->n_heads_kv;
   // rows per token in a 128-row tile: G itself for G = 1, 2, 4 (gathered row by
   // row), else G rounded up to whole 8-row swizzle groups (a TMA box per token)
-  const bool with_dq = !(a->flags & SA_FLAG_DQ_SEPARATE);  // the gather runs in the dQ role
+  const bool with_dq = !dq_separate(a);  // the gather runs in the dQ role
   k.RPT = with_dq && (G == 1 || G == 2 || G == 4) ? G : (G + 7) / 8 * 8;
   k.TPT = 128 / k.RPT;
   k.nblk = (a->s_kv + 63) / 64;
@@ -204,7 +215,7 @@ KvGeom kv_geometry(const sa_args* a) {
   // (window, block) cell still holds enough tokens (>= 128 on average) that the
   // extra dK / dV flushes stay cheap; otherwise one window spans the sequence.
   k.win_tokens = a->s_q > 0 ? a->s_q : 1;
-  if (!(a->flags & SA_FLAG_DQ_SEPARATE) && a->topk > 0) {
+  if (with_dq && a->topk > 0) {
     long long fit = (48ll << 20) / ((long long)a->n_heads_q * a->d_qk * 4);
     fit = fit / 64 * 64;
     const long long need = 128ll * k.nblk / a->topk;
@@ -230,10 +241,12 @@ KvGeom kv_geometry(const sa_args* a) {
 
 // Workspace: [status word][delta][dK or dKV acc][dV acc][dCmp acc]
 //            + key-stationary path: [dQ acc][counts][cursor] | [list_off][items][work][entries]
-// Everything before `zero_end` is cleared at the start of each call with one memset.
+//              [bucket counts][bucket offsets][bucket flags]
+// Everything before `zero_end` is cleared at the start of each call with one memset
+// (the bucketed preparation launch clears it instead).
 struct BwdWs {
   size_t status, delta, dk, dv, dcmp;
-  size_t dq, counts, cursor, list_off, items, work, entries, bucket_cnt, bucket_off;
+  size_t dq, counts, cursor, list_off, items, work, entries, bucket_cnt, bucket_off, bucket_flag;
   size_t zero_end, total;
 };
 
@@ -257,7 +270,7 @@ BwdWs bwd_ws_layout(const sa_args* a) {
   off += align_up((size_t)s.Tcmp * a->n_heads_kv * a->d_qk * sizeof(float));
   if (use_kv_path(a)) {
     KvGeom k = kv_geometry(a);
-    if (!(a->flags & SA_FLAG_DQ_SEPARATE)) {
+    if (!dq_separate(a)) {
       w.dq = off;
       off += align_up((size_t)s.Tq * a->n_heads_q * a->d_qk * sizeof(float));
     }
@@ -275,11 +288,14 @@ BwdWs bwd_ws_layout(const sa_args* a) {
     w.entries = off;
     off += align_up(sizeof(int) * (size_t)k.n_slots);
     if (kv_bucketed(a, k)) {
-      const size_t cells = (size_t)sa::kv_bucket_count(k.n_slots) * k.n_lists;
+      const size_t nb = (size_t)sa::kv_bucket_count(k.n_slots);
+      const size_t cells = nb * k.n_lists;
       w.bucket_cnt = off;
       off += align_up(sizeof(int) * cells);
       w.bucket_off = off;
       off += align_up(sizeof(int) * cells);
+      w.bucket_flag = off;
+      off += align_up(sizeof(int) * nb);
     }
   } else {
     w.zero_end = off;
@@ -290,6 +306,14 @@ BwdWs bwd_ws_layout(const sa_args* a) {
 
 sa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
 
+// Status word bits -> sa_status (the first that applies).
+sa_status status_of_bits(int bits) {
+  if (bits & sa::kStatusTimeout) return SA_ERR_TIMEOUT;
+  if (bits & sa::kStatusIndexRange) return SA_ERR_INDEX;
+  if (bits & sa::kStatusSmemAlign) return SA_ERR_CUDA;
+  return SA_OK;
+}
+
 // SA_FLAG_CHECK: validate every usable index on the device, synchronously.
 sa_status run_check(const sa_args* a, int* status, cudaStream_t st) {
   sa::Prob p = make_prob(a, status);
@@ -299,6 +323,132 @@ sa_status run_check(const sa_args* a, int* status, cudaStream_t st) {
   if (cudaMemcpyAsync(&host, status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SA_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return SA_ERR_CUDA;
   return (host & sa::kStatusIndexRange) ? SA_ERR_INDEX : SA_OK;
+}
+
+// Kernel choices (sa_plan reports them; sa_fwd / sa_bwd dispatch on them).
+bool tk_path(const sa_args* a) {
+  return sa::tk_path_built(a->d_qk, a->d_v, a->kv_shared, a->n_heads_q / a->n_heads_kv);
+}
+
+int32_t fwd_choice(const sa_args* a) {
+  if (use_qb_path(a)) return SA_KERNEL_FWD_BLOCK;
+  if (tk_path(a)) return SA_KERNEL_FWD_TOKEN_TC;
+  return SA_KERNEL_FWD_GENERIC;
+}
+
+int32_t bwd_choice(const sa_args* a) {
+  if (use_kv_path(a)) return dq_separate(a) ? SA_KERNEL_BWD_KEY_STATIONARY_DQ_PASS : SA_KERNEL_BWD_KEY_STATIONARY;
+  if (tk_path(a) && !(a->flags & SA_FLAG_QUERY_STATIONARY_BWD)) return SA_KERNEL_BWD_TOKEN_TC;
+  return SA_KERNEL_BWD_GENERIC;
+}
+
+// The key-stationary inverse index of one backward call, built into the workspace
+// exactly as sa_bwd builds it: the bucketed preparation launch (which also clears
+// the accumulators and, when o / d_o are given, forms Delta), or a memset of
+// [0, zero_end) then the count / scan / fill launches.
+struct KvIndexBuild {
+  KvGeom k;
+  sa::KvIndexArgs ia;
+  bool bucketed;
+};
+
+sa_status build_kv_index(const sa_args* args, const BwdWs& w, char* base, const void* o, const void* d_o,
+                         cudaStream_t cs, KvIndexBuild* out) {
+  Sizes s = sizes_of(args);
+  KvIndexBuild& r = *out;
+  memset(&r, 0, sizeof(r));
+  r.k = kv_geometry(args);
+  r.bucketed = kv_bucketed(args, r.k);
+  int* status = reinterpret_cast<int*>(base + w.status);
+  float* delta = reinterpret_cast<float*>(base + w.delta);
+  sa::KvIndexArgs& ia = r.ia;
+  ia.ori_idx = args->ori_idx;
+  ia.ori_len = args->ori_topk_len;
+  ia.n_slots = r.k.n_slots;
+  ia.topk = args->topk;
+  ia.Hkv = args->n_heads_kv;
+  ia.S = args->s_q;
+  ia.nblk = r.k.nblk;
+  ia.n_lists = r.k.n_lists;
+  ia.nwin = r.k.nwin;
+  ia.win_tokens = r.k.win_tokens;
+  ia.chunk_tokens = r.k.chunk;
+  ia.ori_mask = args->ori_mask_mode;
+  ia.wl = clamp_win(args->ori_win_left);
+  ia.wr = clamp_win(args->ori_win_right);
+  ia.counts = reinterpret_cast<int*>(base + w.counts);
+  ia.cursor = reinterpret_cast<int*>(base + w.cursor);
+  ia.list_off = reinterpret_cast<int*>(base + w.list_off);
+  ia.items = reinterpret_cast<int4*>(base + w.items);
+  ia.entries = reinterpret_cast<int*>(base + w.entries);
+  ia.work_count = reinterpret_cast<int*>(base + w.work);
+  ia.status = status;
+  if (r.bucketed) {
+    ia.n_buckets = sa::kv_bucket_count(r.k.n_slots);
+    ia.bucket_cnt = reinterpret_cast<int*>(base + w.bucket_cnt);
+    ia.bucket_off = reinterpret_cast<int*>(base + w.bucket_off);
+    ia.bucket_flag = reinterpret_cast<int*>(base + w.bucket_flag);
+    sa::KvPrepArgs pa;
+    // the accumulators and counters after Delta (Delta is formed in the same launch)
+    pa.status = status;
+    pa.zero = reinterpret_cast<float4*>(base + w.dk);
+    pa.zero_n16 = (long long)((w.zero_end - w.dk) / 16);
+    pa.o = static_cast<const bf16*>(o);
+    pa.d_o = static_cast<const bf16*>(d_o);
+    pa.delta = delta;
+    pa.rows = (o && d_o) ? s.Tq * args->n_heads_q : 0;
+    pa.dv = args->d_v;
+    return cuda_status(sa::launch_kv_prep_small(ia, pa, cs));
+  }
+  // zero the accumulators and the index counters (one memset), then Delta
+  if (cudaMemsetAsync(base, 0, w.zero_end, cs) != cudaSuccess) return SA_ERR_CUDA;
+  if (o && d_o) {
+    if (sa::launch_delta(static_cast<const bf16*>(o), static_cast<const bf16*>(d_o), delta, s.Tq * args->n_heads_q,
+                         args->d_v, cs) != cudaSuccess)
+      return SA_ERR_CUDA;
+  }
+  return cuda_status(sa::launch_kv_index(ia, cs));
+}
+
+// The key-stationary kernel's arguments for an index built by build_kv_index.
+sa::KvArgs kv_args(const sa_args* args, const KvIndexBuild& r, const BwdWs& w, char* base, const void* d_o,
+                   const float* lse, float* dk_acc, float* dv_acc) {
+  sa::KvArgs ka;
+  memset(&ka, 0, sizeof(ka));
+  const KvGeom& k = r.k;
+  ka.S = args->s_q;
+  ka.Hq = args->n_heads_q;
+  ka.Hkv = args->n_heads_kv;
+  ka.G = args->n_heads_q / args->n_heads_kv;
+  ka.RPT = k.RPT;
+  ka.TPT = k.TPT;
+  ka.gather_rows = k.RPT == ka.G ? (k.RPT < 8 ? 1 : 0) : 0;
+  ka.log2_G = ka.G == 4 ? 2 : (ka.G == 2 ? 1 : 0);
+  ka.q = static_cast<const bf16*>(args->q);
+  ka.d_o = static_cast<const bf16*>(d_o);
+  ka.nblk = k.nblk;
+  ka.n_lists = k.n_lists;
+  ka.nwin = k.nwin;
+  ka.chunk_tokens = k.chunk;
+  ka.ori_mask = args->ori_mask_mode;
+  ka.wl = clamp_win(args->ori_win_left);
+  ka.wr = clamp_win(args->ori_win_right);
+  ka.scale = args->scale;
+  ka.scale_log2 = args->scale * 1.4426950408889634f;
+  ka.items = r.ia.items;
+  ka.entries = r.ia.entries;
+  ka.work_count = r.ia.work_count;
+  ka.lse = lse;
+  ka.delta = reinterpret_cast<float*>(base + w.delta);
+  ka.dk_acc = dk_acc;
+  ka.dv_acc = dv_acc;
+  ka.dq_acc = w.dq ? reinterpret_cast<float*>(base + w.dq) : nullptr;
+  ka.status = reinterpret_cast<int*>(base + w.status);
+  ka.n_buckets = r.ia.n_buckets;
+  ka.bucket_cnt = r.ia.bucket_cnt;
+  ka.bucket_off = r.ia.bucket_off;
+  ka.bucket_flag = r.ia.bucket_flag;
+  return ka;
 }
 
 }  // namespace
@@ -354,12 +504,15 @@ sa_status sa_fwd(const sa_args* args, const sa_fwd_out* out, void* ws, size_t ws
   }
   sa::Prob p = make_prob(args, status);
   if (cudaMemsetAsync(status, 0, sizeof(int), cs) != cudaSuccess) return SA_ERR_CUDA;
-  if (use_qb_path(args)) {
+  const int32_t choice = fwd_choice(args);
+  if (choice == SA_KERNEL_FWD_BLOCK) {
     sa::QbArgs q = make_qb_args(args, status);
     q.o = static_cast<bf16*>(out->o);
     q.lse = out->lse;
     return cuda_status(sa::launch_qb(q, args->k, args->v, false, cs));
   }
+  if (choice == SA_KERNEL_FWD_TOKEN_TC)
+    return cuda_status(sa::launch_tk_fwd(p, static_cast<bf16*>(out->o), out->lse, cs));
   return cuda_status(sa::launch_fwd(p, static_cast<bf16*>(out->o), out->lse, cs));
 }
 
@@ -406,15 +559,15 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
   const long long nk = s.Tkv * args->n_heads_kv * args->d_qk;
   const long long nv = s.Tkv * args->n_heads_kv * args->d_v;
   const long long nc = s.Tcmp * args->n_heads_kv * args->d_qk;
-  KvGeom k;
-  memset(&k, 0, sizeof(k));
-  if (w.counts) k = kv_geometry(args);
-  // small key-stationary problems: one launch clears, forms Delta and builds the index
-  // small problems: one launch builds a bucketed index, clears and forms Delta
-  const bool prep_small = w.counts && kv_bucketed(args, k);
+  const int32_t choice = bwd_choice(args);
   cudaError_t e = cudaSuccess;
-  if (!prep_small) {
-    // zero the accumulators and the index counters (one memset), then Delta
+  KvIndexBuild kib;
+  if (w.counts) {
+    // key-stationary: the inverse index (with the cleared accumulators and Delta)
+    st = build_kv_index(args, w, base, io->o, io->d_o, cs, &kib);
+    if (st != SA_OK) return st;
+  } else {
+    // zero the accumulators and the status word (one memset), then Delta
     if (cudaMemsetAsync(base, 0, w.zero_end, cs) != cudaSuccess) return SA_ERR_CUDA;
     e = sa::launch_delta(static_cast<const bf16*>(io->o), static_cast<const bf16*>(io->d_o), delta,
                          s.Tq * args->n_heads_q, args->d_v, cs);
@@ -423,83 +576,10 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
   if (sinks && cudaMemsetAsync(io->dsinks, 0, sizeof(float) * args->n_heads_q, cs) != cudaSuccess)
     return SA_ERR_CUDA;
   if (w.counts) {
-    // key-stationary: inverse index, then dK / dV per KV block (+ dQ)
-    sa::KvIndexArgs ia;
-    memset(&ia, 0, sizeof(ia));
-    ia.ori_idx = args->ori_idx;
-    ia.ori_len = args->ori_topk_len;
-    ia.n_slots = k.n_slots;
-    ia.topk = args->topk;
-    ia.Hkv = args->n_heads_kv;
-    ia.S = args->s_q;
-    ia.nblk = k.nblk;
-    ia.n_lists = k.n_lists;
-    ia.nwin = k.nwin;
-    ia.win_tokens = k.win_tokens;
-    ia.chunk_tokens = k.chunk;
-    ia.ori_mask = args->ori_mask_mode;
-    ia.wl = args->ori_win_left;
-    ia.wr = args->ori_win_right;
-    ia.counts = reinterpret_cast<int*>(base + w.counts);
-    ia.cursor = reinterpret_cast<int*>(base + w.cursor);
-    ia.list_off = reinterpret_cast<int*>(base + w.list_off);
-    ia.items = reinterpret_cast<int4*>(base + w.items);
-    ia.entries = reinterpret_cast<int*>(base + w.entries);
-    ia.work_count = reinterpret_cast<int*>(base + w.work);
-    if (prep_small) {
-      ia.n_buckets = sa::kv_bucket_count(k.n_slots);
-      ia.bucket_cnt = reinterpret_cast<int*>(base + w.bucket_cnt);
-      ia.bucket_off = reinterpret_cast<int*>(base + w.bucket_off);
-    }
-    if (prep_small) {
-      sa::KvPrepArgs pa;
-      // the accumulators and counters after Delta (Delta is formed in the same launch)
-      pa.status = status;
-      pa.zero = reinterpret_cast<float4*>(base + w.dk);
-      pa.zero_n16 = (long long)((w.zero_end - w.dk) / 16);
-      pa.o = static_cast<const bf16*>(io->o);
-      pa.d_o = static_cast<const bf16*>(io->d_o);
-      pa.delta = delta;
-      pa.rows = s.Tq * args->n_heads_q;
-      pa.dv = args->d_v;
-      if (sa::launch_kv_prep_small(ia, pa, cs) != cudaSuccess) return SA_ERR_CUDA;
-    } else if (sa::launch_kv_index(ia, cs) != cudaSuccess) {
-      return SA_ERR_CUDA;
-    }
+    // dK / dV per KV block (+ dQ)
     sa::KvLaunch kl;
     memset(&kl, 0, sizeof(kl));
-    sa::KvArgs& ka = kl.args;
-    ka.S = args->s_q;
-    ka.Hq = args->n_heads_q;
-    ka.Hkv = args->n_heads_kv;
-    ka.G = args->n_heads_q / args->n_heads_kv;
-    ka.RPT = k.RPT;
-    ka.TPT = k.TPT;
-    ka.gather_rows = k.RPT == ka.G ? (k.RPT < 8 ? 1 : 0) : 0;
-    ka.log2_G = ka.G == 4 ? 2 : (ka.G == 2 ? 1 : 0);
-    ka.q = static_cast<const bf16*>(args->q);
-    ka.d_o = static_cast<const bf16*>(io->d_o);
-    ka.nblk = k.nblk;
-    ka.n_lists = k.n_lists;
-    ka.nwin = k.nwin;
-    ka.chunk_tokens = k.chunk;
-    ka.ori_mask = args->ori_mask_mode;
-    ka.wl = args->ori_win_left;
-    ka.wr = args->ori_win_right;
-    ka.scale = args->scale;
-    ka.scale_log2 = args->scale * 1.4426950408889634f;
-    ka.items = ia.items;
-    ka.entries = ia.entries;
-    ka.work_count = ia.work_count;
-    ka.lse = io->lse;
-    ka.delta = delta;
-    ka.dk_acc = out.dk_acc;
-    ka.dv_acc = out.dv_acc;
-    ka.dq_acc = w.dq ? reinterpret_cast<float*>(base + w.dq) : nullptr;
-    ka.status = status;
-    ka.n_buckets = ia.n_buckets;
-    ka.bucket_cnt = ia.bucket_cnt;
-    ka.bucket_off = ia.bucket_off;
+    kl.args = kv_args(args, kib, w, base, io->d_o, io->lse, out.dk_acc, out.dv_acc);
     kl.q = args->q;
     kl.d_o = io->d_o;
     kl.k = args->k;
@@ -508,7 +588,7 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
     kl.Tkv = s.Tkv;
     kl.dqk = args->d_qk;
     kl.dv = args->d_v;
-    kl.max_work = k.max_work;
+    kl.max_work = kib.k.max_work;
     if (sa::launch_kv_bwd(kl, w.dq != 0, cs) != cudaSuccess) return SA_ERR_CUDA;
     if (!w.dq) {
       sa::QbArgs q = make_qb_args(args, status);
@@ -518,6 +598,9 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
       q.dq = static_cast<bf16*>(io->dq);
       e = sa::launch_qb(q, args->k, args->v, true, cs);
     }
+  } else if (choice == SA_KERNEL_BWD_TOKEN_TC) {
+    // token-level shared KV (576 / 512): the tcgen05 kernel, 64 heads per CTA
+    e = sa::launch_tk_bwd(p, io->lse, delta, static_cast<const bf16*>(io->d_o), out, cs);
   } else {
     e = sa::launch_bwd(p, static_cast<const bf16*>(io->o), static_cast<const bf16*>(io->d_o), io->lse, delta,
                        out, cs);
@@ -561,6 +644,51 @@ sa_status sa_debug_resolve(const sa_args* args, int32_t* rows, int32_t* counts, 
   if (!counts || (max_rows > 0 && !rows)) return SA_ERR_NULLPTR;
   sa::Prob p = make_prob(args, nullptr);
   return cuda_status(sa::launch_debug_resolve(p, rows, counts, max_rows, static_cast<cudaStream_t>(stream)));
+}
+
+sa_status sa_plan(const sa_args* args, int32_t* fwd_kernel, int32_t* bwd_kernel) {
+  sa_status st = validate(args);
+  if (st != SA_OK) return st;
+  if (fwd_kernel) *fwd_kernel = fwd_choice(args);
+  if (bwd_kernel) *bwd_kernel = bwd_choice(args);
+  return SA_OK;
+}
+
+sa_status sa_read_status(const void* ws, size_t ws_bytes, void* stream) {
+  if (!ws) return SA_ERR_NULLPTR;
+  if (ws_bytes < sizeof(int)) return SA_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int host = 0;
+  if (cudaMemcpyAsync(&host, ws, sizeof(int), cudaMemcpyDeviceToHost, cs) != cudaSuccess) return SA_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return SA_ERR_CUDA;
+  return status_of_bits(host);
+}
+
+sa_status sa_debug_block_index(const sa_args* args, int32_t view, void* ws, size_t ws_bytes, int32_t* records,
+                               int64_t max_records, int32_t* n_records, void* stream) {
+  sa_status st = validate(args);
+  if (st != SA_OK) return st;
+  if (!n_records || (max_records > 0 && !records)) return SA_ERR_NULLPTR;
+  if (max_records < 0) return SA_ERR_PARAM;
+  if (view != SA_INDEX_VIEW_QUERY_BLOCKS && view != SA_INDEX_VIEW_KEY_LISTS) return SA_ERR_PARAM;
+  if (view == SA_INDEX_VIEW_QUERY_BLOCKS && !use_qb_path(args)) return SA_ERR_UNSUPPORTED;
+  if (view == SA_INDEX_VIEW_KEY_LISTS && !use_kv_path(args)) return SA_ERR_UNSUPPORTED;
+  BwdWs w = bwd_ws_layout(args);
+  if (view == SA_INDEX_VIEW_KEY_LISTS && (!ws || ws_bytes < w.total)) return SA_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(n_records, 0, sizeof(int32_t), cs) != cudaSuccess) return SA_ERR_CUDA;
+  if (sizes_of(args).Tq == 0) return SA_OK;
+  int4* rec = reinterpret_cast<int4*>(records);
+  if (view == SA_INDEX_VIEW_QUERY_BLOCKS) {
+    sa::QbArgs q = make_qb_args(args, nullptr);
+    return cuda_status(sa::launch_qb_debug_slots(q, rec, max_records, n_records, cs));
+  }
+  char* base = static_cast<char*>(ws);
+  KvIndexBuild kib;
+  st = build_kv_index(args, w, base, nullptr, nullptr, cs, &kib);
+  if (st != SA_OK) return st;
+  sa::KvArgs ka = kv_args(args, kib, w, base, nullptr, nullptr, nullptr, nullptr);
+  return cuda_status(sa::launch_kv_debug_walk(ka, kib.k.max_work, rec, max_records, n_records, cs));
 }
 
 }  // extern "C"

@@ -139,6 +139,50 @@ __device__ __forceinline__ Unit make_unit(const Prob& p, int tq, int g) {
   return u;
 }
 
+// ---------------------------------------------------------------------------
+// Block-level selection with 64-row blocks (aclnnSparseFlashAttentionGrad,
+// "Formula": each of the selectBlockCount indices names 64 contiguous rows).
+// The slot rule and the in-block row range below are the only definitions the
+// block kernels, the key-stationary inverse index and the inspection entry
+// point use, so what the inspection returns is what the kernels compute.
+// A query row sits at sequence-local position ta (aligned bottom-right) over a
+// key sequence of Lk rows; wl / wr are the BAND window (host-clamped to 2^40).
+// ---------------------------------------------------------------------------
+
+// Slot naming block x is usable: x >= 0, the block starts inside the sequence,
+// and at least one of its rows survives the ori mask.
+__device__ __forceinline__ bool blk_usable(int x, int Lk, int ta, int mask, long long wl, long long wr) {
+  if (x < 0) return false;
+  const long long first = (long long)x * kTileRows;
+  if (first >= Lk) return false;
+  if (mask == kMaskCausal) return first <= ta;
+  if (mask == kMaskBand) {
+    const long long last = min(first + kTileRows - 1, (long long)Lk - 1);
+    return first <= (long long)ta + wr && last >= (long long)ta - wl;
+  }
+  return true;
+}
+
+// Visible rows of block x for the same query row, as offsets [*lo, *hi] within
+// the block (0..63); *lo > *hi when none.  Non-empty whenever blk_usable holds.
+__device__ __forceinline__ void blk_rows(int x, int Lk, int ta, int mask, long long wl, long long wr, int* lo,
+                                         int* hi) {
+  const long long first = (long long)x * kTileRows;
+  long long l = 0, h = min((long long)kTileRows - 1, (long long)Lk - 1 - first);
+  if (mask == kMaskCausal) {
+    h = min(h, (long long)ta - first);
+  } else if (mask == kMaskBand) {
+    h = min(h, (long long)ta + wr - first);
+    l = max(l, (long long)ta - wl - first);
+  }
+  if (h < l) {
+    l = 0;
+    h = -1;
+  }
+  *lo = (int)l;
+  *hi = (int)h;
+}
+
 __device__ __forceinline__ bool ori_mask_ok(const Prob& p, const Unit& u, int r) {
   if (p.ori_mask == kMaskCausal) return r <= u.ta;
   if (p.ori_mask == kMaskBand) return (long long)r >= (long long)u.ta - p.wl && (long long)r <= (long long)u.ta + p.wr;

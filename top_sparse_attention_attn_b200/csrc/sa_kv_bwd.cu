@@ -79,13 +79,20 @@ struct KvPlan {
   static_assert(kSmem + 1024 <= 227 * 1024, "shared memory plan too large");
 };
 
+// A CTA's work item: list L (-1 past the last item), chunk c of the list and its
+// ntok tokens; bucketed mode also keeps where each bucket's part of the list
+// starts (in rank order) and sits.
+struct KvItem {
+  int L, c, ntok;
+  int bstart[kBucketMax];
+  int boff[kBucketMax];
+};
+
 struct KvBars {
   uint64_t kv_full, q_full[2], q_empty[2], s_full, p_full, p_free, ds_full, tile_done, acc_done, dq_full, dq_free;
   uint32_t tmem_base;
   int abort_flag;
-  int item_L, item_c, item_ntok;  // the work item: list, chunk of the list, tokens
-  int bstart[kBucketMax];         // bucketed mode: first rank of each bucket in the list
-  int boff[kBucketMax];           // bucketed mode: the list's offset within each bucket
+  KvItem item;
 };
 
 // The list that block x of one token's selections joins: (batch b, token window,
@@ -93,14 +100,7 @@ struct KvBars {
 // row for the token (offset ta within its sequence).  A is KvArgs or KvIndexArgs.
 template <class A>
 __device__ __forceinline__ int kv_block_list(const A& a, int x, int b, int ta, int g) {
-  if (x < 0) return -1;
-  const long long first = (long long)x * 64;
-  if (first >= a.S) return -1;
-  if (a.ori_mask == kMaskCausal && first > ta) return -1;
-  if (a.ori_mask == kMaskBand) {
-    const long long last = min(first + 63, (long long)a.S - 1);
-    if (first > (long long)ta + a.wr || last < (long long)ta - a.wl) return -1;
-  }
+  if (!blk_usable(x, a.S, ta, a.ori_mask, a.wl, a.wr)) return -1;
   // keyed by the token's window first, so that CTAs launched together add their dQ
   // contributions to a window of tokens whose fp32 accumulators stay in L2
   return ((b * a.nwin + ta / a.win_tokens) * a.Hkv + g) * a.nblk + x;
@@ -132,11 +132,13 @@ __device__ __forceinline__ void kv_gather_rows(uint32_t sbase, const bf16* __res
 // each list's counts over the buckets, turns them into chunk counts, finds the
 // list and chunk of item w, and where each bucket's part of that list starts (in
 // rank order) and sits; then the CTA gathers the chunk's token ids into `toks`.
-// Fills bars.item_* (item_L = -1 past the last item).
-__device__ void kv_bucket_item(const KvArgs& a, int w, int* toks, KvBars& bars) {
+// Fills `it` (it.L = -1 past the last item).
+__device__ void kv_bucket_item(const KvArgs& a, int w, int* toks, KvItem& it) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nl = a.n_lists, nb = a.n_buckets;
   if (warp == 0) {
+    // indices past their sequence, seen by the preparation launch, reach the status word
+    if (w == 0 && lane < nb && __ldg(a.bucket_flag + lane) && a.status) atomicOr(a.status, kStatusIndexRange);
     int carry = 0, fL = -1, fc = 0, fn = 0;
     for (int l0 = 0; l0 < nl; l0 += 32) {
       const int L = l0 + lane;
@@ -161,9 +163,9 @@ __device__ void kv_bucket_item(const KvArgs& a, int w, int* toks, KvBars& bars) 
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) {
-      bars.item_L = fL;
-      bars.item_c = fc;
-      bars.item_ntok = fL >= 0 ? min(a.chunk_tokens, fn - fc * a.chunk_tokens) : 0;
+      it.L = fL;
+      it.c = fc;
+      it.ntok = fL >= 0 ? min(a.chunk_tokens, fn - fc * a.chunk_tokens) : 0;
     }
     if (fL >= 0) {
       const int v = lane < nb ? __ldg(a.bucket_cnt + lane * nl + fL) : 0;
@@ -174,21 +176,47 @@ __device__ void kv_bucket_item(const KvArgs& a, int w, int* toks, KvBars& bars) 
         if (lane >= o) incl += y;
       }
       if (lane < nb) {
-        bars.bstart[lane] = incl - v;
-        bars.boff[lane] = __ldg(a.bucket_off + lane * nl + fL);
+        it.bstart[lane] = incl - v;
+        it.boff[lane] = __ldg(a.bucket_off + lane * nl + fL);
       }
     }
   }
   __syncthreads();
-  if (bars.item_L < 0) return;
-  const int lo = bars.item_c * a.chunk_tokens, n = bars.item_ntok;
+  if (it.L < 0) return;
+  const int lo = it.c * a.chunk_tokens, n = it.ntok;
   for (int r = threadIdx.x; r < n; r += blockDim.x) {
     const int R = lo + r;
     int k = 0;  // the last bucket whose part starts at or before rank R
     for (int k2 = 1; k2 < nb; ++k2)
-      if (bars.bstart[k2] <= R) k = k2;
-    toks[r] = __ldg(a.entries + k * kBucketSlots + bars.boff[k] + (R - bars.bstart[k]));
+      if (it.bstart[k2] <= R) k = k2;
+    toks[r] = __ldg(a.entries + k * kBucketSlots + it.boff[k] + (R - it.bstart[k]));
   }
+}
+
+// Work item w of either index (every thread of the CTA calls it): its token ids
+// are returned (shared memory `toks_smem` in bucketed mode, the entries array
+// otherwise) and `it` is filled by the time of the caller's next __syncthreads.
+__device__ __forceinline__ const int* kv_get_item(const KvArgs& a, int w, int* toks_smem, KvItem& it) {
+  if (a.n_buckets > 0) {
+    kv_bucket_item(a, w, toks_smem, it);
+    return toks_smem;
+  }
+  const int4 item = __ldg(a.items + w);  // in bounds (w < max_work); used only when w < work_count
+  const int nwork = __ldg(a.work_count);
+  if (threadIdx.x == 0) {
+    it.L = w < nwork ? item.x : -1;
+    it.c = 0;
+    it.ntok = item.z;
+  }
+  return a.entries + item.y;
+}
+
+// List id = ((batch * nwin + window) * Hkv + kv-head) * nblk + block.
+__device__ __forceinline__ void kv_list_decode(const KvArgs& a, int L, int* b, int* g, int* j) {
+  *j = L % a.nblk;
+  const int rest = L / a.nblk;
+  *g = rest % a.Hkv;
+  *b = (rest / a.Hkv) / a.nwin;
 }
 
 template <int DQK, int DV, bool WITH_DQ>
@@ -202,6 +230,7 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
   __shared__ KvBars bars;
   uint8_t* smem = smem_raw;
   if (smem_u32(smem_raw) & 1023) {  // the swizzled operand layouts need 1024-byte alignment
+    pdl_wait();  // the status word is cleared by a preceding launch
     if (threadIdx.x == 0 && a.status) atomicOr(a.status, kStatusSmemAlign);
     return;
   }
@@ -247,29 +276,15 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
 
   // ---- the work item {list, tokens}
   const int w = blockIdx.x;
-  const int* toks;
   pdl_wait();  // the index, Delta and the cleared accumulators come from the preceding kernels
-  if (a.n_buckets > 0) {
-    // from the bucketed index: the chunk's token ids land in shared memory
-    kv_bucket_item(a, w, reinterpret_cast<int*>(smem + PL::oTok), bars);
-    toks = reinterpret_cast<const int*>(smem + PL::oTok);
-  } else {
-    // from the work-item table
-    const int4 item = __ldg(a.items + w);  // in bounds (w < max_work); used only when w < work_count
-    const int nwork = __ldg(a.work_count);
-    if (threadIdx.x == 0) {
-      bars.item_L = w < nwork ? item.x : -1;
-      bars.item_ntok = item.z;
-    }
-    toks = a.entries + item.y;
-  }
+  const int* toks = kv_get_item(a, w, reinterpret_cast<int*>(smem + PL::oTok), bars.item);
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   pdl_trigger();
   const uint32_t tmem = bars.tmem_base;
-  const int L = bars.item_L, ntok = bars.item_ntok;
+  const int L = bars.item.L, ntok = bars.item.ntok;
   if (L < 0) {  // past the last work item (uniform over the CTA)
     if (warp == 1) {
       tmem_dealloc(tmem, PL::kAlloc);
@@ -277,10 +292,8 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
     }
     return;
   }
-  // list id = ((batch * nwin + window) * Hkv + kv-head) * nblk + block
-  const int j = L % a.nblk;
-  const int rest = L / a.nblk;
-  const int g = rest % a.Hkv, b = (rest / a.Hkv) / a.nwin;
+  int b, g, j;
+  kv_list_decode(a, L, &b, &g, &j);
   const int TPT = a.TPT, RPT = a.RPT;
   const int ntiles = (ntok + TPT - 1) / TPT;
   if (threadIdx.x == 0) {
@@ -393,7 +406,6 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
     const int r = 32 * sub + lane;  // query row of the tile = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(32 * sub) << 16);
     const int u = r / RPT, hh = r - u * RPT;
-    const int blk_row0 = 64 * j;
     bool ok = true;
     // row metadata of tile i (token, lse, Delta), fetched one tile ahead
     int tq_n = 0;
@@ -419,18 +431,9 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
       const float lse2 = vrow ? lse_n * kLog2eKv : INFINITY;
       const float dlt = vrow ? dlt_n : 0.f;
       fetch(i + 1);
-      // visible key rows of this block for this query row
+      // visible key rows of this block for this query row (blk_rows)
       int vlo = 0, vhi = -1;
-      if (vrow) {
-        vlo = 0;
-        vhi = min(63, a.S - 1 - blk_row0);
-        if (a.ori_mask == kMaskCausal) {
-          vhi = min(vhi, ta - blk_row0);
-        } else if (a.ori_mask == kMaskBand) {
-          vhi = (int)min((long long)vhi, (long long)ta + a.wr - blk_row0);
-          vlo = (int)max((long long)vlo, (long long)ta - a.wl - blk_row0);
-        }
-      }
+      if (vrow) blk_rows(j, a.S, ta, a.ori_mask, a.wl, a.wr, &vlo, &vhi);
       if (!mbar_wait(&bars.s_full, i & 1, abort_flag, a.status)) { ok = false; break; }
       tc_fence_after();
       // The P / dS buffer is free once the previous tile's dK^T and dQ MMAs are
@@ -667,8 +670,8 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
   // fp32 accumulators, four consecutive dims per vector reduction
   if (!bars.abort_flag) {
     // the item again (shared): keeps its fields out of registers through the roles above
-    const int L2 = bars.item_L;
-    const int j2 = L2 % a.nblk, g2 = (L2 / a.nblk) % a.Hkv, b2 = (L2 / a.nblk / a.Hkv) / a.nwin;
+    int b2, g2, j2;
+    kv_list_decode(a, bars.item.L, &b2, &g2, &j2);
     const long long kv_row0 = (long long)b2 * a.S + 64 * j2;
     const int nrows = min(64, a.S - 64 * j2);
     const float4* stV = reinterpret_cast<const float4*>(smem + PL::oStV);
@@ -695,7 +698,9 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
 // inverse index: for every (batch, token window, kv-head, block) the tokens
 // of the window that select the block
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ bool kv_slot_list(const KvIndexArgs& a, long long e, int* list, int* tq_out) {
+// The list that slot e joins (false when the slot is unusable); *oor is raised
+// when the slot is usable by length but names a block past its sequence.
+__device__ __forceinline__ bool kv_slot_list(const KvIndexArgs& a, long long e, int* list, int* tq_out, bool* oor) {
   int slot, tq, g;
   long long ug;
   if (a.n_slots <= 0x7fffffffll) {  // 32-bit index arithmetic when it fits
@@ -712,7 +717,9 @@ __device__ __forceinline__ bool kv_slot_list(const KvIndexArgs& a, long long e, 
   }
   if (a.ori_len && slot >= __ldg(a.ori_len + ug)) return false;
   const int b = tq / a.S;
-  const int L = kv_block_list(a, __ldg(a.ori_idx + e), b, tq - b * a.S, g);
+  const int x = __ldg(a.ori_idx + e);
+  if (x >= 0 && (long long)x * kTileRows >= a.S) *oor = true;
+  const int L = kv_block_list(a, x, b, tq - b * a.S, g);
   if (L < 0) return false;
   *list = L;
   *tq_out = tq;
@@ -720,13 +727,15 @@ __device__ __forceinline__ bool kv_slot_list(const KvIndexArgs& a, long long e, 
 }
 
 // Small problems (fewer than 2^31 slots): the same with 32-bit index arithmetic only.
-__device__ __forceinline__ int kv_slot_list32(const KvIndexArgs& a, int e, int* tq_out) {
+__device__ __forceinline__ int kv_slot_list32(const KvIndexArgs& a, int e, int* tq_out, bool* oor) {
   const int ug = e / a.topk, slot = e - ug * a.topk;
   const int tq = ug / a.Hkv, g = ug - tq * a.Hkv;
   if (a.ori_len && slot >= __ldg(a.ori_len + ug)) return -1;
   const int b = tq / a.S;
   *tq_out = tq;
-  return kv_block_list(a, __ldg(a.ori_idx + e), b, tq - b * a.S, g);
+  const int x = __ldg(a.ori_idx + e);
+  if (x >= 0 && (long long)x * kTileRows >= a.S) *oor = true;
+  return kv_block_list(a, x, b, tq - b * a.S, g);
 }
 
 __global__ void kv_count_kernel(const KvIndexArgs a) {
@@ -735,7 +744,9 @@ __global__ void kv_count_kernel(const KvIndexArgs a) {
   long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= a.n_slots) return;
   int list, tq;
-  if (kv_slot_list(a, e, &list, &tq)) atomicAdd(a.counts + list, 1);
+  bool oor = false;
+  if (kv_slot_list(a, e, &list, &tq, &oor)) atomicAdd(a.counts + list, 1);
+  if (oor && a.status) atomicOr(a.status, kStatusIndexRange);
 }
 
 __global__ void kv_fill_kernel(const KvIndexArgs a) {
@@ -744,7 +755,8 @@ __global__ void kv_fill_kernel(const KvIndexArgs a) {
   long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= a.n_slots) return;
   int list, tq;
-  if (kv_slot_list(a, e, &list, &tq)) {
+  bool oor = false;
+  if (kv_slot_list(a, e, &list, &tq, &oor)) {
     int pos = atomicAdd(a.cursor + list, 1);
     a.entries[__ldg(a.list_off + list) + pos] = tq;
   }
@@ -825,8 +837,12 @@ __global__ void __launch_bounds__(kBucketSlots) kv_prep_small_kernel(const KvInd
     for (int i = threadIdx.x; i < nl; i += blockDim.x) cnt[i] = 0;
     const int e = bk * kBucketSlots + threadIdx.x;
     int tq = 0;
-    const int L = e < a.n_slots ? kv_slot_list32(a, e, &tq) : -1;
-    __syncthreads();
+    bool oor = false;
+    const int L = e < a.n_slots ? kv_slot_list32(a, e, &tq, &oor) : -1;
+    // the bucket's out-of-range flag, written whole every call (the status word itself
+    // is cleared by CTA 0 below, so the main kernel folds the flags into it)
+    const int any_oor = __syncthreads_or(oor);
+    if (threadIdx.x == 0) a.bucket_flag[bk] = any_oor;
     const unsigned peers = __match_any_sync(0xffffffffu, L);
     const int leader = __ffs(peers) - 1;
     int rank = 0;
@@ -864,6 +880,27 @@ __global__ void __launch_bounds__(kBucketSlots) kv_prep_small_kernel(const KvInd
   for (long long row = t0 >> 5; row < p.rows; row += nthreads >> 5) {
     const float d = warp_row_dot_bf16(p.o + row * p.dv, p.d_o + row * p.dv, p.dv, lane);
     if (lane == 0) p.delta[row] = d;
+  }
+}
+
+// Inspection: walks every work item exactly as kv_bwd_kernel does (kv_get_item,
+// kv_list_decode) and records, per (item, token), the block and its visible row
+// range (blk_rows): {token * Hkv + kv-head, block, lo, hi}.
+__global__ void __launch_bounds__(128) kv_debug_walk_kernel(const KvArgs a, int4* rec, long long max_rec,
+                                                            int* n_rec) {
+  __shared__ KvItem item;
+  __shared__ int toks_smem[kBucketMaxChunk];
+  const int* toks = kv_get_item(a, blockIdx.x, toks_smem, item);
+  __syncthreads();
+  if (item.L < 0) return;
+  int b, g, j;
+  kv_list_decode(a, item.L, &b, &g, &j);
+  for (int r = threadIdx.x; r < item.ntok; r += blockDim.x) {
+    const int tq = toks[r];
+    int lo, hi;
+    blk_rows(j, a.S, tq - b * a.S, a.ori_mask, a.wl, a.wr, &lo, &hi);
+    const int k = atomicAdd(n_rec, 1);
+    if (k < max_rec) rec[k] = make_int4(tq * a.Hkv + g, j, lo, hi);
   }
 }
 
@@ -932,6 +969,14 @@ cudaError_t launch_kv_index(const KvIndexArgs& a, cudaStream_t st) {
     count_launch();
   }
   return e;
+}
+
+cudaError_t launch_kv_debug_walk(const KvArgs& a, long long max_work, int4* rec, long long max_rec, int* n_rec,
+                                 cudaStream_t st) {
+  if (max_work == 0) return cudaSuccess;
+  kv_debug_walk_kernel<<<(unsigned)max_work, 128, 0, st>>>(a, rec, max_rec, n_rec);
+  count_launch();
+  return cudaGetLastError();
 }
 
 cudaError_t launch_kv_bwd(const KvLaunch& L, bool with_dq, cudaStream_t st) {

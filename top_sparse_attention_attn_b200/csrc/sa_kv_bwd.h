@@ -28,6 +28,8 @@ struct KvIndexArgs {
   int n_buckets;
   int* bucket_cnt;      // [n_buckets][n_lists]
   int* bucket_off;      // [n_buckets][n_lists]
+  int* bucket_flag;     // [n_buckets]: the bucket held an index past its sequence
+  int* status;          // status word (index bit), cleared before the index is built
 };
 
 struct KvArgs {
@@ -55,6 +57,7 @@ struct KvArgs {
   int n_buckets;
   const int* bucket_cnt;  // [n_buckets][n_lists]
   const int* bucket_off;  // [n_buckets][n_lists]
+  const int* bucket_flag; // [n_buckets]
 };
 
 // Bucketed index: buckets of 512 slots, each built by one CTA (512 threads) of
@@ -98,5 +101,8 @@ bool kv_bucketed_fits(long long n_slots, int n_lists, int chunk);
 cudaError_t launch_kv_prep_small(const KvIndexArgs& a, const KvPrepArgs& p, cudaStream_t st);
 cudaError_t launch_kv_index(const KvIndexArgs& a, cudaStream_t st);
 cudaError_t launch_kv_bwd(const KvLaunch& L, bool with_dq, cudaStream_t st);
+// Inspection walk over the work items (grid max_work), after the index is built.
+cudaError_t launch_kv_debug_walk(const KvArgs& a, long long max_work, int4* rec, long long max_rec, int* n_rec,
+                                 cudaStream_t st);
 
 }  // namespace sa

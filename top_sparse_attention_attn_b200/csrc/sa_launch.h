@@ -66,6 +66,12 @@ cudaError_t launch_delta(const bf16* o, const bf16* d_o, float* delta, long long
 cudaError_t launch_bwd(const Prob& p, const bf16* o, const bf16* d_o, const float* lse,
                        const float* delta, const BwdOut& out, cudaStream_t st);
 cudaError_t launch_to_bf16(const float* src, bf16* dst, long long n, cudaStream_t st);
+// Token-level backward over one shared KV head (d 576 / 512) on tcgen05: dQ to
+// bf16 directly, dKV (dCmpKv) into the fp32 accumulators, dSinks accumulated.
+bool tk_path_built(int dqk, int dv, int shared, int G);
+cudaError_t launch_tk_bwd(const Prob& p, const float* lse, const float* delta, const bf16* d_o, const BwdOut& out,
+                          cudaStream_t st);
+cudaError_t launch_tk_fwd(const Prob& p, bf16* o, float* lse, cudaStream_t st);
 // Up to four fp32 -> bf16 conversions in one launch (each n a multiple of 8).
 struct Cvt {
   const float* src;

@@ -62,8 +62,10 @@ struct QbBars {
   int abort_flag;
 };
 
-// Warp-collective: the usable slots of a work item (valid, in range, not fully
-// masked), in slot order, written to xs (shared); returns their number.
+// Warp-collective: the usable slots of a work item (blk_usable: valid, in range,
+// not fully masked), in slot order, written to xs (shared, kQbMaxSlots entries);
+// returns their number.  An index past the end of its sequence raises the
+// status word's index bit.  The host routes only topk <= kQbMaxSlots here.
 __device__ __forceinline__ int qb_slots(const QbArgs& a, const Unit& u, int* xs, int lane) {
   const long long ug = (long long)u.tq * a.Hkv + u.g;
   int n = a.topk;
@@ -75,20 +77,16 @@ __device__ __forceinline__ int qb_slots(const QbArgs& a, const Unit& u, int* xs,
     int x = -1;
     if (s < n) {
       x = __ldg(a.ori_idx + ug * a.topk + s);
-      const long long first = (long long)x * 64;
-      ok = x >= 0 && first < u.Lk;
-      if (a.ori_mask == kMaskCausal) ok = ok && first <= u.ta;
-      if (a.ori_mask == kMaskBand) {
-        const long long last = min(first + 63, (long long)u.Lk - 1);
-        ok = ok && first <= (long long)u.ta + a.wr && last >= (long long)u.ta - a.wl;
-      }
+      ok = blk_usable(x, u.Lk, u.ta, a.ori_mask, a.wl, a.wr);
+      if (x >= 0 && (long long)x * kTileRows >= u.Lk && a.status) atomicOr(a.status, kStatusIndexRange);
     }
     const unsigned m = __ballot_sync(0xffffffffu, ok);
-    if (ok) xs[cnt + __popc(m & ((1u << lane) - 1u))] = x;
+    const int pos = cnt + __popc(m & ((1u << lane) - 1u));
+    if (ok && pos < kQbMaxSlots) xs[pos] = x;
     cnt += __popc(m);
   }
   __syncwarp();
-  return cnt;
+  return min(cnt, kQbMaxSlots);
 }
 
 __device__ __forceinline__ Unit qb_unit(const QbArgs& a, int tq, int g) {
@@ -122,7 +120,7 @@ __global__ void __launch_bounds__(160, NCTA) qb_kernel(const __grid_constant__ C
   constexpr int NV = DV / 16;    // k steps over d_v
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ QbBars bars;
-  __shared__ int slot_x[5][256];  // per warp: the current item's usable block indices
+  __shared__ int slot_x[5][kQbMaxSlots];  // per warp: the current item's usable block indices
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t ring = smem_u32(smem + PL::oRing);
@@ -261,19 +259,16 @@ __global__ void __launch_bounds__(160, NCTA) qb_kernel(const __grid_constant__ C
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
           for (int j = 0; j < 4; ++j) s[nt][j] += s2[nt][j];
-        // visibility of the warp's block rows for this query token
-        const int rbase = 64 * x + 16 * warp;
+        // visibility of the warp's block rows for this query token (blk_rows)
+        int vlo, vhi;
+        blk_rows(x, u.Lk, u.ta, a.ori_mask, a.wl, a.wr, &vlo, &vhi);
         bool vis[2][2];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int rr = rbase + 8 * nt + cq + e;
-            bool v = rr < u.Lk;
-            if (a.ori_mask == kMaskCausal) v = v && rr <= u.ta;
-            else if (a.ori_mask == kMaskBand)
-              v = v && (long long)rr >= (long long)u.ta - a.wl && (long long)rr <= (long long)u.ta + a.wr;
-            vis[nt][e] = v;
+            const int off = 16 * warp + 8 * nt + cq + e;
+            vis[nt][e] = off >= vlo && off <= vhi;
           }
         uint32_t pa[4];  // P (forward) or dS (dQ pass) as an A fragment over the 16 block rows
         if (!DQ) {
@@ -440,6 +435,35 @@ __global__ void __launch_bounds__(160, NCTA) qb_kernel(const __grid_constant__ C
     }
     (void)W;
   }
+}
+
+// Inspection: one warp per (token, kv-head) unit runs qb_unit / qb_slots /
+// blk_rows exactly as qb_kernel does and records every usable slot as
+// {unit, block, lo, hi}.
+__global__ void __launch_bounds__(128) qb_debug_slots_kernel(const QbArgs a, int4* rec, long long max_rec,
+                                                             int* n_rec) {
+  __shared__ int xs_all[4][kQbMaxSlots];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long unit = (long long)blockIdx.x * 4 + warp;
+  if (unit >= (long long)a.Tq * a.Hkv) return;  // whole warps leave together
+  const int tq = (int)(unit / a.Hkv), g = (int)(unit - (long long)tq * a.Hkv);
+  const Unit u = qb_unit(a, tq, g);
+  int* xs = xs_all[warp];
+  const int n = qb_slots(a, u, xs, lane);
+  for (int i = lane; i < n; i += 32) {
+    int lo, hi;
+    blk_rows(xs[i], u.Lk, u.ta, a.ori_mask, a.wl, a.wr, &lo, &hi);
+    const int k = atomicAdd(n_rec, 1);
+    if (k < max_rec) rec[k] = make_int4((int)unit, xs[i], lo, hi);
+  }
+}
+
+cudaError_t launch_qb_debug_slots(const QbArgs& a, int4* rec, long long max_rec, int* n_rec, cudaStream_t st) {
+  const long long units = (long long)a.Tq * a.Hkv;
+  if (units == 0) return cudaSuccess;
+  qb_debug_slots_kernel<<<(unsigned)((units + 3) / 4), 128, 0, st>>>(a, rec, max_rec, n_rec);
+  count_launch();
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------

@@ -8,6 +8,9 @@
 
 namespace sa {
 
+// Most usable slots per work item the query-stationary block kernels hold.
+constexpr int kQbMaxSlots = 256;
+
 struct QbArgs {
   int layout, B, s_q, s_kv, Tq, Tkv, Hq, Hkv, G, dqk, dv, topk, ori_mask;
   long long wl, wr;
@@ -28,5 +31,7 @@ struct QbArgs {
 
 bool qb_path_built(int dqk, int dv);
 cudaError_t launch_qb(const QbArgs& a, const void* k, const void* v, bool dq, cudaStream_t st);
+// Inspection: the usable slots and row ranges of every unit as the block kernels see them.
+cudaError_t launch_qb_debug_slots(const QbArgs& a, int4* rec, long long max_rec, int* n_rec, cudaStream_t st);
 
 }  // namespace sa

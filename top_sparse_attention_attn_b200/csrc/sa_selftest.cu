@@ -100,6 +100,101 @@ __global__ void __launch_bounds__(128) selftest_mma_kernel(const __grid_constant
   }
 }
 
+// Operand layouts written in software: a matrix X[R][C] (R rows, C contiguous)
+// in atoms of W = sw / 2 elements along C, rows of sw bytes, the 16-byte piece
+// index XOR (r & 7) for the 128-byte swizzle or ((r >> 1) & 3) for the 64-byte one.
+__device__ __forceinline__ uint32_t sw_offset(int r, int c, int R, int sw) {
+  const int W = sw / 2;
+  const int a = c / W, w = c - a * W;
+  const int piece = (w * 2) >> 4, sub = (w * 2) & 15;
+  const int x = sw == 128 ? (r & 7) : ((r >> 1) & 3);
+  return (uint32_t)(a * (R * sw) + r * sw + ((piece ^ x) << 4) + sub);
+}
+
+struct Selftest2Args {
+  int M, N, K, a_mn, b_mn, a_sw, b_sw, d_lane;
+};
+
+// D = A B with both operands copied into shared memory in software (any of the
+// K-major / MN-major orientations, 128- or 64-byte swizzle), one CTA of 128.
+__global__ void __launch_bounds__(128) selftest_mma2_kernel(const bf16* __restrict__ A, const bf16* __restrict__ B,
+                                                            const Selftest2Args a, float* __restrict__ D,
+                                                            int* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t bar_mma;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // A: K-major [M][K] (rows M) or MN-major [K][M] (rows K); B: K-major [N][K] or MN-major [K][N]
+  const int aR = a.a_mn ? a.K : a.M, aC = a.a_mn ? a.M : a.K;
+  const int bR = a.b_mn ? a.K : a.N, bC = a.b_mn ? a.N : a.K;
+  const int aBytes = aR * aC * 2;
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + ((aBytes + 1023) & ~1023);
+  for (int i = threadIdx.x; i < aR * aC; i += blockDim.x) {
+    const int r = i / aC, c = i - r * aC;
+    *reinterpret_cast<bf16*>(sA + sw_offset(r, c, aR, a.a_sw)) = A[i];
+  }
+  for (int i = threadIdx.x; i < bR * bC; i += blockDim.x) {
+    const int r = i / bC, c = i - r * bC;
+    *reinterpret_cast<bf16*>(sB + sw_offset(r, c, bR, a.b_sw)) = B[i];
+  }
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar_mma, 1);
+    mbar_fence_init();
+  }
+  const uint32_t ncols = a.N <= 32 ? 32 : (a.N <= 64 ? 64 : (a.N <= 128 ? 128 : 256));
+  if (warp == 0) tmem_alloc(&tmem_base, ncols);
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t uA = smem_u32(sA), uB = smem_u32(sB);
+  auto desc = [](uint32_t base, bool mn, int R, int sw, int kk) -> uint64_t {
+    const int W = sw / 2;
+    if (!mn) {  // K-major: a K step of 16 moves 32 bytes inside an atom
+      const uint32_t addr = base + ((kk * 16) / W) * (R * sw) + ((kk * 16) % W) * 2;
+      return sw == 128 ? sdesc(addr, 16, 1024) : sdesc64(addr, 16, 512);
+    }
+    // MN-major: a K step of 16 rows; atoms of W elements along M / N, R * sw bytes apart
+    const uint32_t addr = base + kk * 16 * sw;
+    return sw == 128 ? sdesc(addr, R * sw, 1024) : sdesc64(addr, R * sw, 512);
+  };
+  if (threadIdx.x == 0) {
+    const uint32_t idesc = idesc_bf16(a.M, a.N, a.a_mn != 0, a.b_mn != 0);
+    for (int kk = 0; kk < a.K / 16; ++kk)
+      mma_bf16(tmem_base + ((uint32_t)a.d_lane << 16), desc(uA, a.a_mn != 0, aR, a.a_sw, kk),
+               desc(uB, a.b_mn != 0, bR, a.b_sw, kk), idesc, kk > 0 ? 1u : 0u);
+    mma_commit(&bar_mma);
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(&bar_mma, 0, &abort_flag, status);
+  tc_fence_after();
+  if (ok) {
+    const int sub = warp & 3;
+    int m = -1;
+    if (a.M == 128) m = 32 * sub + lane;
+    else if (lane >= a.d_lane && lane < a.d_lane + 16) m = 16 * sub + (lane - a.d_lane);
+    for (int c = 0; c < a.N; c += 16) {
+      uint32_t r[16];
+      tmem_ld16(tmem_base + ((uint32_t)(32 * sub) << 16) + c, r);
+      tmem_wait_ld();
+      reg_dep16(r);
+      if (m >= 0)
+        for (int i = 0; i < 16; ++i) D[(long long)m * a.N + c + i] = __uint_as_float(r[i]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, ncols);
+    tmem_relinquish();
+  }
+}
+
 // Nothing ever arrives on `bar`: the bounded wait gives up and raises the status word.
 __global__ void selftest_wait_kernel(int* status, int* waited) {
   __shared__ uint64_t bar;
@@ -115,6 +210,28 @@ __global__ void selftest_wait_kernel(int* status, int* waited) {
 }
 
 }  // namespace sa
+
+extern "C" sa_status sa_selftest_mma2(int32_t M, int32_t N, int32_t K, int32_t a_mn, int32_t b_mn, int32_t a_sw,
+                                      int32_t b_sw, int32_t d_lane, const void* A, const void* B, float* D,
+                                      int32_t* status, void* stream) {
+  if (!A || !B || !D || !status) return SA_ERR_NULLPTR;
+  if ((M != 64 && M != 128) || N < 16 || N > 256 || N % 16 || K < 16 || K > 256 || K % 16) return SA_ERR_PARAM;
+  if ((a_sw != 64 && a_sw != 128) || (b_sw != 64 && b_sw != 128)) return SA_ERR_PARAM;
+  if (d_lane != 0 && !(d_lane == 16 && M == 64)) return SA_ERR_PARAM;
+  // every operand extent along its contiguous dimension must fill whole atoms
+  const int aC = a_mn ? M : K, bC = b_mn ? N : K;
+  if (aC % (a_sw / 2) || bC % (b_sw / 2)) return SA_ERR_PARAM;
+  sa::Selftest2Args args{M, N, K, a_mn, b_mn, a_sw, b_sw, d_lane};
+  const int smem = ((M * K * 2 + 1023) & ~1023) + N * K * 2 + 1024;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaFuncSetAttribute(sa::selftest_mma2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return SA_ERR_CUDA;
+  sa::selftest_mma2_kernel<<<1, 128, smem, st>>>(static_cast<const sa::bf16*>(A), static_cast<const sa::bf16*>(B), args,
+                                                 D, status);
+  sa::count_launch();
+  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
 
 extern "C" sa_status sa_selftest_wait_timeout(int32_t* status, int32_t* waited, void* stream) {
   if (!status || !waited) return SA_ERR_NULLPTR;
