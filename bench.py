@@ -141,6 +141,8 @@ def count_work(w, inputs) -> dict:
         # fp32 reductions of the fused query-stationary backward: every visible row of
         # every 16-head slice adds its dK/dV (dKV) row
         "red_bytes_qs": int(vis.sum()) * ((G + 15) // 16) * (w.d_qk + (0 if w.kv_shared else w.d_v)) * 4,
+        # ... of the token-level tensor-core backward: one dKV row per visible row and 64-head slice
+        "red_bytes_tk": int(vis.sum()) * ((G + 63) // 64) * w.d_qk * 4,
         "units": T * w.Hkv,
         "_npair": npair,
     }
@@ -358,46 +360,85 @@ def aggregate_rate(units_per_rank: float, world: int, max_ms: float) -> float:
     return world * units_per_rank / (max_ms * 1e-3)
 
 
-def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
-    import torch
-    from gen.torch_io import to_torch
-    from top_sparse_attention_attn_b200 import SparseAttention
-    from top_sparse_attention_attn_b200 import _lib as L
+KERNEL_NAMES = {
+    1: "qb_kernel (query-stationary block forward)",
+    2: "tk_fwd_kernel (token-level tcgen05 forward)",
+    3: "fwd_kernel (generic forward)",
+    4: "kv_bwd_kernel (key-stationary dK/dV/dQ, dQ by fp32 atomics)",
+    5: "kv_bwd_kernel (key-stationary dK/dV) + qb_kernel<dQ> pass",
+    6: "tk_bwd_kernel (token-level tcgen05 backward)",
+    7: "bwd_kernel (generic fused backward)",
+}
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    w = workload_of(args)
-    inputs = make_inputs(w)
+
+def compulsory_bytes(w, work) -> dict:
+    """Bytes any implementation moves at least once: the forward reads Q and K/V (or
+    the shared KV and cmp_kv) and writes O and lse; the backward reads Q, K/V, dO, O
+    and lse and writes dQ and dK/dV (dKV, dCmpKv) in bf16."""
+    T = w.T
+    q = T * w.Hq * w.d_qk * 2
+    o = T * w.Hq * w.d_v * 2
+    lse = T * w.Hq * 4
+    kv = T * w.Hkv * (w.d_qk + (0 if w.kv_shared else w.d_v)) * 2
+    if w.cmp_topk:
+        kv += sum(L // w.cmp_ratio for L in w.seq_lengths) * w.Hkv * w.d_qk * 2
+    return {"fwd": q + kv + o + lse, "bwd": q + kv + 2 * o + lse + q + kv}
+
+
+def fractions(work, comp, peaks, fwd_ms, bwd_ms) -> dict:
+    """Roofline fractions (burst tensor peak, measured HBM bandwidth):
+    the benchmark spec -- the slower of FLOPs at the tensor peak and gathered + compulsory
+                  bytes at HBM bandwidth, over the measured time;
+    tensor     -- the slower of FLOPs at the tensor peak and compulsory bytes only
+                  (the stricter figure: gathers that hit L2 or are avoided do not count).
+    A fraction above 1 means that model does not bind (the kernel beat it)."""
+    P, BW = peaks["bf16_tflops"] * 1e12, peaks["hbm_gbs"] * 1e9
+    out = {}
+    for side, ms, flops, gbytes in (("fwd", fwd_ms, work["fwd_flops"], work["fwd_bytes"]),
+                                    ("bwd", bwd_ms, work["bwd_flops"], work["bwd_main_bytes"])):
+        ns = max(flops / P, gbytes / BW) * 1e3 / ms
+        tc = max(flops / P, comp[side] / BW) * 1e3 / ms
+        out[f"{side}_north_star_frac"] = ns
+        out[f"{side}_tensor_frac"] = tc
+        out[f"{side}_north_star_binding"] = ns <= 1.0
+    return out
+
+
+def setup_problem(w, dev, flags: int, host_dense: bool):
+    """Inputs, accounting and the SparseAttention object of one workload.  The index
+    sets come from the NumPy generator; the dense tensors from the GPU generator
+    (same recipe, torch's Philox stream) unless host_dense asks for the NumPy ones."""
+    from gen.torch_io import dense_on_device, to_torch
+    from top_sparse_attention_attn_b200 import SparseAttention
+    inputs = make_inputs(w, dense=host_dense)
     work = count_work(w, inputs)
     t = to_torch(inputs, dev)
-    flags = 0
-    for f in filter(None, args.flags.split(",")):
-        flags |= {"dq_separate": L.SA_FLAG_DQ_SEPARATE, "query_stationary": L.SA_FLAG_QUERY_STATIONARY_BWD}[f]
-    sa = SparseAttention.from_workload(w, t, flags=flags)
-    stream = torch.cuda.current_stream(dev)
+    if not host_dense:
+        t.update(dense_on_device(w, dev))
+    return SparseAttention.from_workload(w, t, flags=flags), t, inputs, work
+
+
+def measure(sa, t, K: int, warmup: int, use_graph: bool, flush, stream, world: int, hook_passes=True) -> dict:
+    """Forward and backward times of one problem: K steps, L2 flushed before each,
+    CUDA events on the launching stream.  With graphs the timed steps replay a graph
+    of each call; a third graph holds the whole step (forward then backward), whose
+    replay time minus the forward's is the backward inside a step."""
+    import torch
+    from top_sparse_attention_attn_b200 import _lib as L
     o, lse = sa.alloc_fwd()
     grads = sa.alloc_bwd()
-    ws_f = sa.fwd_workspace()
-    ws_b = sa.bwd_workspace()
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    ws_f, ws_b = sa.fwd_workspace(), sa.bwd_workspace()
 
     def step():
         sa.forward(o, lse, ws_f)
         sa.backward(o, lse, t["do"], grads, ws_b)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
-
-    K = args.steps
-    # The timed steps replay a CUDA graph of each call (forward, backward) unless
-    # --no-graph: the calls enqueue only kernels and memsets on the stream, so they
-    # capture as they are, and replays drop the host-side launch gaps that would
-    # otherwise dominate small problems.
-    use_graph = not args.no_graph
     launches_per_step = None
     if use_graph:
-        side = torch.cuda.Stream(dev)
+        side = torch.cuda.Stream(stream.device)
         side.wait_stream(stream)
         with torch.cuda.stream(side):
             step()
@@ -410,7 +451,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         with torch.cuda.graph(g_bwd):
             sa.backward(o, lse, t["do"], grads, ws_b)
         launches_per_step = L.sa_kernel_launch_count() - n0
-        with torch.cuda.graph(g_step):  # the whole step as one graph
+        with torch.cuda.graph(g_step):
             step()
         for _ in range(2):
             g_fwd.replay()
@@ -418,21 +459,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
             g_step.replay()
         torch.cuda.synchronize()
 
-    def step_graph_pass():
-        """K replays of the one-graph step (forward then backward), L2 flushed before
-        each: the backward's cost inside a step is this minus the forward alone."""
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-        torch.cuda.synchronize()
-        for k in range(K):
-            flush.zero_()
-            ev[k][0].record(stream)
-            g_step.replay()
-            ev[k][1].record(stream)
-        torch.cuda.synchronize()
-        return sum(a.elapsed_time(b) for a, b in ev) / K
-
     def timed_pass(which):
-        """K steps bracketed by events; optionally times one kernel through the hook."""
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
         for e in ev:  # materialise the raw cudaEvent_t handles
             for x in e:
@@ -450,9 +477,12 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
                 e1.record(stream)
                 g_bwd.replay()
             else:
+                if which == L.TIME_FWD:
+                    L.sa_set_timing_events(mb.cuda_event, me.cuda_event, which)
                 sa.forward(o, lse, ws_f)
+                L.sa_set_timing_events(None, None, -1)
                 e1.record(stream)
-                if which is not None:
+                if which is not None and which != L.TIME_FWD:
                     L.sa_set_timing_events(mb.cuda_event, me.cuda_event, which)
                 sa.backward(o, lse, t["do"], grads, ws_b)
                 L.sa_set_timing_events(None, None, -1)
@@ -460,25 +490,108 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         torch.cuda.synchronize()
         fwd = sum(e[0].elapsed_time(e[1]) for e in ev) / K
         bwd = sum(e[1].elapsed_time(e[2]) for e in ev) / K
-        kern = sum(e[3].elapsed_time(e[4]) for e in ev) / K
+        kern = sum(e[3].elapsed_time(e[4]) for e in ev) / K if which is not None else 0.0
         return fwd, bwd, kern
 
-    launches0 = L.sa_kernel_launch_count()
+    def step_graph_pass():
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        torch.cuda.synchronize()
+        for k in range(K):
+            flush.zero_()
+            ev[k][0].record(stream)
+            g_step.replay()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in ev) / K
+
+    r = {}
+    n0 = L.sa_kernel_launch_count()
+    r["fwd_ms"], r["bwd_ms"], _ = timed_pass(None)
+    r["launches"] = launches_per_step * K if use_graph else L.sa_kernel_launch_count() - n0
+    r["step_graph_ms"] = step_graph_pass() if use_graph else r["fwd_ms"] + r["bwd_ms"]
+    r["bwd_in_step_ms"] = max(r["step_graph_ms"] - r["fwd_ms"], 1e-6)
+    if hook_passes:
+        # attribution passes (eager calls, not part of the timed steps): the timing hook
+        # around the backward's main kernel, the separate dQ pass, the forward kernel
+        r["fwd_eager_ms"], r["bwd_eager_ms"], r["bwd_kernel_ms"] = timed_pass(L.TIME_BWD_KV)
+        r["dq_kernel_ms"] = timed_pass(L.TIME_BWD_DQ)[2]
+        r["fwd_kernel_ms"] = timed_pass(L.TIME_FWD)[2]
+    r["_bufs"] = (o, lse, grads, ws_f, ws_b)
+    return r
+
+
+def dominant_kernel_roofline(w, work, comp, peaks, peak_src, plan, m) -> dict:
+    """Roofline of the longest kernel: its FLOPs at the burst tensor peak against its
+    compulsory bytes at HBM bandwidth (whichever is slower sets the bound), over its
+    CUDA-event time; plus the spec fraction of the same kernel and the DRAM
+    bytes of its committed ncu capture (null when the sources changed since)."""
+    fwd_k, bwd_k = plan
+    cands = [(KERNEL_NAMES[bwd_k], m.get("bwd_kernel_ms", 0.0), "bwd"),
+             (KERNEL_NAMES[fwd_k], m.get("fwd_kernel_ms", 0.0), "fwd")]
+    if m.get("dq_kernel_ms"):
+        cands.append(("qb_kernel<dQ> (query-stationary dQ pass)", m["dq_kernel_ms"], "bwd"))
+    name, kms, side = max(cands, key=lambda c: c[1])
+    if side == "bwd" and bwd_k == 5:  # split backward: each kernel carries its own contractions
+        flops = work["dq_flops"] if name.startswith("qb_kernel") else work["kv_flops"]
+    else:
+        flops = work[f"{side}_flops"]
+    cbytes = comp[side]
+    gbytes = work["fwd_bytes"] if side == "fwd" else work["bwd_main_bytes"]
+    P, BW = peaks["bf16_tflops"] * 1e12, peaks["hbm_gbs"] * 1e9
+    t_f, t_b = flops / P, cbytes / BW
+    bound = "tensor" if t_f >= t_b else "hbm"
+    if bound == "tensor":
+        achieved, peak, unit = flops / (kms * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    else:
+        achieved, peak, unit = cbytes / (kms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
+    traffic = load_traffic(name.split(" ")[0], w.name)
+    ns = max(t_f, gbytes / BW) * 1e3 / kms
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+            "traffic": traffic, "kernel": name, "kernel_ms": kms,
+            "algorithmic_flops": flops, "algorithmic_bytes": cbytes,
+            "peak_source": ("measured MEASURED_PEAKS.json (bf16 burst; HBM copy)" if peak_src == "measured"
+                            else "fallback"),
+            "t_roof_ms": max(t_f, t_b) * 1e3,
+            "north_star_frac": ns, "north_star_binding": ns <= 1.0,
+            "dram_over_compulsory": None if traffic is None else traffic / cbytes}
+
+
+def config_of(w, work, world: int, flags: str) -> dict:
+    return {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv,
+            "d_qk": w.d_qk, "d_v": w.d_v, "block_size": w.block_size, "topk": w.topk,
+            "parallelism": f"replicas{world}", "flags": flags or "default",
+            "visible_triples": work["triples"], "gathered_bytes": work["gathered_bytes"]}
+
+
+PER_WORKLOAD = (("cfg1", 20), ("cfg5", 5), ("cfg4", 5), ("cfg3", 3))
+
+
+def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
+    import torch
+    from top_sparse_attention_attn_b200 import _lib as L
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workload_of(args)
+    flags = 0
+    for f in filter(None, args.flags.split(",")):
+        flags |= {"dq_separate": L.SA_FLAG_DQ_SEPARATE, "query_stationary": L.SA_FLAG_QUERY_STATIONARY_BWD}[f]
+    sa, t, inputs, work = setup_problem(w, dev, flags, host_dense=False)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    use_graph = not args.no_graph
+    K = args.steps
+    plan = sa.plan()
+
     with ClockSampler(local_rank) as clk:
-        fwd_ms, bwd_ms, _ = timed_pass(None)
-        launches = L.sa_kernel_launch_count() - launches0
-        step_graph_ms = step_graph_pass() if use_graph else fwd_ms + bwd_ms
-    if use_graph:
-        launches = launches_per_step * K
-    step_ms = fwd_ms + bwd_ms
-    # attribution passes (not part of the timed steps): eager calls with the timing
-    # hook around the dK/dV kernel and around the separate dQ pass, if any
-    fwd_eager_ms, bwd_eager_ms, main_ms = timed_pass(L.TIME_BWD_KV)
-    _, _, dq_ms = timed_pass(L.TIME_BWD_DQ) if "dq_separate" in args.flags else (0.0, 0.0, 0.0)
-    fwd_ms, bwd_ms, main_ms, step_ms, dq_ms, fwd_eager_ms, bwd_eager_ms, step_graph_ms = max_over_ranks(
-        [fwd_ms, bwd_ms, main_ms, step_ms, dq_ms, fwd_eager_ms, bwd_eager_ms, step_graph_ms], world, dev)
-    # the backward inside a step: no graph boundary of its own before its first kernel
-    bwd_in_step_ms = max(step_graph_ms - fwd_ms, 1e-6)
+        m = measure(sa, t, K, args.warmup, use_graph, flush, stream, world)
+    keys = ["fwd_ms", "bwd_ms", "bwd_kernel_ms", "dq_kernel_ms", "fwd_kernel_ms", "fwd_eager_ms",
+            "bwd_eager_ms", "step_graph_ms"]
+    for k_, v in zip(keys, max_over_ranks([m[k_] for k_ in keys], world, dev)):
+        m[k_] = v
+    m["bwd_in_step_ms"] = max(m["step_graph_ms"] - m["fwd_ms"], 1e-6)
+    o, lse, grads, ws_f, ws_b = m.pop("_bufs")
+    step_ms = m["fwd_ms"] + m["bwd_ms"]
 
     # end to end through the public API with host buffers
     e2e = None
@@ -516,88 +629,99 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
                "ms_per_step": e2e_ms.item(),
                "note": "bwd FLOPs over the whole step: H2D of inputs, forward, backward, D2H of gradients"}
 
+    # the other workloads, measured in the same run (every rank runs them: the
+    # barriers inside the timed passes stay matched); fewer steps for the long ones
+    per_workload = {}
+    if not args.no_per_workload and args.override is None:
+        for name, k_steps in PER_WORKLOAD:
+            w2 = get_workload(name)
+            if w2.name == w.name:
+                continue
+            sa2, t2, _, work2 = setup_problem(w2, dev, 0, host_dense=False)
+            with ClockSampler(local_rank) as clk2:
+                m2 = measure(sa2, t2, k_steps, 2, use_graph, flush, stream, world)
+            m2.pop("_bufs")
+            ks = ["fwd_ms", "bwd_ms", "bwd_kernel_ms", "fwd_kernel_ms", "step_graph_ms", "dq_kernel_ms"]
+            for k_, v in zip(ks, max_over_ranks([m2[k_] for k_ in ks], world, dev)):
+                m2[k_] = v
+            m2["bwd_in_step_ms"] = max(m2["step_graph_ms"] - m2["fwd_ms"], 1e-6)
+            if rank == 0:
+                peaks2, src2 = load_peaks()
+                comp2 = compulsory_bytes(w2, work2)
+                plan2 = sa2.plan()
+                fr = fractions(work2, comp2, peaks2, m2["fwd_ms"], m2["bwd_ms"])
+                fr_step = fractions(work2, comp2, peaks2, m2["fwd_ms"], m2["bwd_in_step_ms"])
+                roof2 = dominant_kernel_roofline(w2, work2, comp2, peaks2, src2, plan2, m2)
+                per_workload[name] = {
+                    "workload": w2.name, "steps": k_steps,
+                    "fwd_ms": m2["fwd_ms"], "bwd_ms": m2["bwd_ms"], "bwd_in_step_ms": m2["bwd_in_step_ms"],
+                    "fwd_tflops": work2["fwd_flops"] / (m2["fwd_ms"] * 1e-3) / 1e12,
+                    "bwd_tflops": work2["bwd_flops"] / (m2["bwd_ms"] * 1e-3) / 1e12,
+                    "fwd_kernel": KERNEL_NAMES[plan2[0]], "bwd_kernel": KERNEL_NAMES[plan2[1]],
+                    **fr,
+                    "bwd_north_star_frac_in_step": fr_step["bwd_north_star_frac"],
+                    "bwd_tensor_frac_in_step": fr_step["bwd_tensor_frac"],
+                    "roofline": roof2, "clocks": clk2.summary(),
+                    "config": config_of(w2, work2, world, "")}
+            del sa2, t2
+            torch.cuda.empty_cache()
+
     if rank != 0:
         return None
     peaks, peak_src = load_peaks()
-    bwd_tflops = aggregate_rate(work["bwd_flops"], world, bwd_ms) / 1e12
-    fwd_tflops = aggregate_rate(work["fwd_flops"], world, fwd_ms) / 1e12
-    # roofline of the dominant backward kernel
-    kern = []
-    keystat = (w.mode == "block" and w.block_size == 64 and w.layout == "BSND" and not w.sinks
-               and "query_stationary" not in args.flags)
-    if keystat and "dq_separate" in args.flags:
-        bwd_path = "key-stationary dK/dV + query-stationary dQ pass"
-        kern.append(("kv_bwd_kernel (key-stationary dK/dV)", main_ms, work["kv_flops"], work["kv_bytes"]))
-        kern.append(("qb_kernel<dQ> (query-stationary dQ pass)", dq_ms, work["dq_flops"], work["dq_bytes"]))
-    elif keystat:
-        bwd_path = "key-stationary dK/dV/dQ (dQ by fp32 atomics)"
-        kern.append(("kv_bwd_kernel (key-stationary dK/dV/dQ)", main_ms, work["kvq_flops"], work["kvq_bytes"]))
-    else:
-        bwd_path = "query-stationary fused (dK/dV scatter-add)"
-        kern.append(("bwd_kernel (fused query-stationary backward)", main_ms, work["bwd_flops"],
-                     work["bwd_main_bytes"]))
-    # the fp32 scatter-add traffic of the dominant kernel, as achieved GB/s (a
+    comp = compulsory_bytes(w, work)
+    bwd_tflops = aggregate_rate(work["bwd_flops"], world, m["bwd_ms"]) / 1e12
+    fwd_tflops = aggregate_rate(work["fwd_flops"], world, m["fwd_ms"]) / 1e12
+    roof = dominant_kernel_roofline(w, work, comp, peaks, peak_src, plan, m)
+    fr = fractions(work, comp, peaks, m["fwd_ms"], m["bwd_ms"])
+    fr_step = fractions(work, comp, peaks, m["fwd_ms"], m["bwd_in_step_ms"])
+    # the fp32 reduction traffic of the backward's main kernel, as achieved GB/s (a
     # reporting model: a failure here must not cost the measurement)
     try:
-        if keystat and "dq_separate" not in args.flags:
+        if plan[1] == 4:
             red_bytes = kv_reduction_bytes(w, inputs, work)
-        elif not keystat:
+            red_model = "dQ row per (token, head, block) + dK/dV flush per work item"
+        elif plan[1] == 6:
+            red_bytes = work["red_bytes_tk"]
+            red_model = "dKV row per visible row and 64-head slice"
+        elif plan[1] == 7:
             red_bytes = work["red_bytes_qs"]
+            red_model = "dK/dV (dKV) row per visible row and 16-head slice"
         else:
-            red_bytes = None
+            red_bytes, red_model = None, None
     except Exception:  # noqa: BLE001
-        red_bytes = None
-    name, kms, kflops, kbytes = max(kern, key=lambda x: x[1])
-    t_bytes = kbytes / (peaks["hbm_gbs"] * 1e9)
-    t_flops = kflops / (peaks["bf16_tflops_sustained"] * 1e12)
-    bound = "hbm" if t_bytes >= t_flops else "tensor"
-    if bound == "hbm":
-        achieved = kbytes / (kms * 1e-3) / 1e9
-        peak, unit = peaks["hbm_gbs"], "GB/s"
-    else:
-        achieved = kflops / (kms * 1e-3) / 1e12
-        peak, unit = peaks["bf16_tflops_sustained"], "TFLOP/s"
-    roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-            "frac": achieved / peak, "traffic": load_traffic(name.split(" ")[0], w.name),
-            "kernel": name, "kernel_ms": kms,
-            "algorithmic_bytes": kbytes, "algorithmic_flops": kflops,
-            "peak_source": f"{peak_src} MEASURED_PEAKS.json" if peak_src == "measured" else "fallback",
-            "t_roof_ms": max(t_bytes, t_flops) * 1e3,
-            "kernels_ms": {k_[0]: k_[1] for k_ in kern}}
+        red_bytes, red_model = None, None
     line = {
         "metric": METRIC, "value": bwd_tflops, "unit": "TFLOP/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv,
-                   "d_qk": w.d_qk, "d_v": w.d_v, "block_size": w.block_size, "topk": w.topk,
-                   "parallelism": f"replicas{world}", "l2": "flushed between timed steps",
-                   "flags": args.flags or "default",
-                   "visible_triples": work["triples"], "gathered_bytes": work["gathered_bytes"]},
-        "fwd_tflops": fwd_tflops, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+        "config": config_of(w, work, world, args.flags),
+        "l2": "flushed between timed steps (a 2x L2 write before each)",
+        "fwd_tflops": fwd_tflops, "fwd_ms": m["fwd_ms"], "bwd_ms": m["bwd_ms"],
         "timing": "CUDA-graph replays" if use_graph else "eager calls",
-        "fwd_eager_ms": fwd_eager_ms, "bwd_eager_ms": bwd_eager_ms,
-        "bwd_path": bwd_path,
-        # the benchmark spec's roofline for the whole backward: the slower of tensor peak and
-        # gathered + compulsory bytes at HBM bandwidth
-        "bwd_roofline_frac": max(work["bwd_flops"] / (peaks["bf16_tflops"] * 1e12),
-                                 work["bwd_main_bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3 / bwd_ms,
+        "fwd_eager_ms": m["fwd_eager_ms"], "bwd_eager_ms": m["bwd_eager_ms"],
+        "fwd_kernel": KERNEL_NAMES[plan[0]], "bwd_path": KERNEL_NAMES[plan[1]],
+        **fr,
         # the backward as part of a one-graph step (forward then backward), minus the
         # forward alone: the fixed cost of starting a graph of its own drops out
-        "step_graph_ms": step_graph_ms, "bwd_in_step_ms": bwd_in_step_ms,
-        "bwd_roofline_frac_in_step": max(work["bwd_flops"] / (peaks["bf16_tflops"] * 1e12),
-                                         work["bwd_main_bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3 / bwd_in_step_ms,
-        "fwd_roofline_frac": max(work["fwd_flops"] / (peaks["bf16_tflops"] * 1e12),
-                                 work["fwd_bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3 / fwd_ms,
-        "roofline": roof, "clocks": clk.summary(), "gpu_launches": launches,
+        "step_graph_ms": m["step_graph_ms"], "bwd_in_step_ms": m["bwd_in_step_ms"],
+        "bwd_north_star_frac_in_step": fr_step["bwd_north_star_frac"],
+        "bwd_tensor_frac_in_step": fr_step["bwd_tensor_frac"],
+        "roofline": roof, "clocks": clk.summary(), "gpu_launches": m["launches"],
         # fp32 dQ / dK / dV reductions (L2 read-modify-writes, not DRAM bytes) of the
-        # dominant backward kernel, over its measured time
+        # backward's main kernel, over its measured time
         "reductions": None if red_bytes is None else {
-            "bytes": red_bytes, "achieved_gbs": red_bytes / (main_ms * 1e-3) / 1e9,
-            "model": "dQ row per (token, head, block) + dK/dV flush per work item" if keystat
-                     else "dK/dV (dKV) row per visible row and 16-head slice"},
+            "bytes": red_bytes, "achieved_gbs": red_bytes / (m["bwd_kernel_ms"] * 1e-3) / 1e9,
+            "model": red_model},
         "e2e": e2e,
+        "per_workload": per_workload,
     }
     if world == 1 and not args.no_cpu_baseline:
+        # the oracle reads the same dense tensors the GPU ran on (host copies of the bits)
+        from gen.torch_io import bf16_bits
+        for k_ in ("q", "k", "v", "kv", "do", "cmp_kv"):
+            if k_ in t:
+                inputs[k_] = bf16_bits(t[k_])
         line["cpu_baseline"] = oracle_baseline(w, inputs)
     return line
 
@@ -617,16 +741,17 @@ def run_reference(args, rank: int) -> dict | None:
     vals = [oracle_baseline(w, inputs, budget_s=per_step, seed=100 + k) for k in range(args.steps)]
     v = statistics.mean(x["value"] for x in vals)
     work = count_work(w, inputs)
+    sample_ms = statistics.mean(x["elapsed_s"] for x in vals) * 1e3
     return {"metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "impl": "reference",
-            # a whole backward of the workload at the sampled rate (each timed step is a
-            # bounded sample of it; sample_ms_per_step is its measured length)
-            "ms_per_step": work["bwd_flops"] / (v * 1e12) * 1e3,
-            "sample_ms_per_step": statistics.mean(x["elapsed_s"] for x in vals) * 1e3,
+            # each timed step is a bounded sample of the workload's backward (random
+            # units); ms_per_step is that measured sample, and a whole backward at the
+            # sampled rate is reported beside it
+            "ms_per_step": sample_ms,
+            "whole_backward_ms_at_sampled_rate": work["bwd_flops"] / (v * 1e12) * 1e3,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv,
-                       "d_qk": w.d_qk, "d_v": w.d_v, "block_size": w.block_size, "topk": w.topk,
-                       "parallelism": "replicas1", "l2": "n/a (host cores)", "flags": "default"},
+            "config": config_of(w, work, 1, ""),
+            "l2": "n/a (host cores)",
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": vals[0]["cores"],
                              "kind": "oracle", "sample": vals[0]["sample"]},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -643,6 +768,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager calls instead of CUDA-graph replays")
+    ap.add_argument("--no-per-workload", action="store_true", help="skip the other workloads' figures")
     ap.add_argument("--flags", default="", help="backward variant for measurements: dq_separate | query_stationary")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -130,7 +130,7 @@ def _cmp_indices(rng, w: Workload, S: int, any_pos: bool) -> np.ndarray:
 
 
 def make_inputs(w: Workload, *, allow_future: bool = False, cmp_any: bool = False,
-                ori_len_range: tuple | None = None) -> dict:
+                ori_len_range: tuple | None = None, dense: bool = True) -> dict:
     """Draw every input of workload ``w``.
 
     Returns a dict of numpy arrays.  bf16 tensors are uint16 bit patterns with
@@ -141,6 +141,11 @@ def make_inputs(w: Workload, *, allow_future: bool = False, cmp_any: bool = Fals
     the diagonal (the causal mask must then hide them); ``cmp_any`` draws cmp
     indices from all compressed rows; ``ori_len_range`` adds a per-row ori topk
     length drawn uniformly from the inclusive range.
+
+    ``dense=False`` skips q, k / kv, v, dO and cmp_kv (the stream then serves
+    the sinks and the index sets only): the benchmark draws those dense
+    tensors on the GPU instead (``gen.torch_io.dense_on_device``), which the
+    long-sequence workloads need to start within seconds.
     """
     rng = np.random.Generator(np.random.PCG64(w.seed))
     lens = w.seq_lengths
@@ -148,13 +153,14 @@ def make_inputs(w: Workload, *, allow_future: bool = False, cmp_any: bool = Fals
     lead = (w.B, w.S) if w.layout == "BSND" else (T,)
     out: dict = {}
 
-    out["q"] = _normal_bf16(rng, lead + (w.Hq, w.d_qk))
-    if w.kv_shared:
-        out["kv"] = _normal_bf16(rng, lead + (w.Hkv, w.d_qk))
-    else:
-        out["k"] = _normal_bf16(rng, lead + (w.Hkv, w.d_qk))
-        out["v"] = _normal_bf16(rng, lead + (w.Hkv, w.d_v))
-    out["do"] = _normal_bf16(rng, lead + (w.Hq, w.d_v), mul=w.do_scale)
+    if dense:
+        out["q"] = _normal_bf16(rng, lead + (w.Hq, w.d_qk))
+        if w.kv_shared:
+            out["kv"] = _normal_bf16(rng, lead + (w.Hkv, w.d_qk))
+        else:
+            out["k"] = _normal_bf16(rng, lead + (w.Hkv, w.d_qk))
+            out["v"] = _normal_bf16(rng, lead + (w.Hkv, w.d_v))
+        out["do"] = _normal_bf16(rng, lead + (w.Hq, w.d_v), mul=w.do_scale)
     if w.sinks:
         out["sinks"] = rng.standard_normal(w.Hq, dtype=np.float32)
 
@@ -173,16 +179,17 @@ def make_inputs(w: Workload, *, allow_future: bool = False, cmp_any: bool = Fals
         out["ori_idx"] = idx.reshape(lead + (w.Hkv, w.topk))
 
     if w.cmp_topk > 0:
-        kvkey = "kv" if w.kv_shared else "k"
-        src = out[kvkey].reshape((T, w.Hkv, w.d_qk))
-        cmp_parts, cmp_lens = [], []
-        for b, L in enumerate(lens):
-            Tc = L // w.cmp_ratio
-            seg = f32_from_bf16_bits(src[starts[b]:starts[b] + Tc * w.cmp_ratio]).astype(np.float64)
-            pooled = seg.reshape(Tc, w.cmp_ratio, w.Hkv, w.d_qk).mean(axis=1)
-            cmp_parts.append(bf16_bits_from_f32(pooled.astype(np.float32)))
-            cmp_lens.append(Tc)
-        out["cmp_kv"] = np.concatenate(cmp_parts, axis=0)
+        cmp_lens = [L // w.cmp_ratio for L in lens]
+        if dense:
+            kvkey = "kv" if w.kv_shared else "k"
+            src = out[kvkey].reshape((T, w.Hkv, w.d_qk))
+            cmp_parts = []
+            for b, L in enumerate(lens):
+                Tc = L // w.cmp_ratio
+                seg = f32_from_bf16_bits(src[starts[b]:starts[b] + Tc * w.cmp_ratio]).astype(np.float64)
+                pooled = seg.reshape(Tc, w.cmp_ratio, w.Hkv, w.d_qk).mean(axis=1)
+                cmp_parts.append(bf16_bits_from_f32(pooled.astype(np.float32)))
+            out["cmp_kv"] = np.concatenate(cmp_parts, axis=0)
         out["cu_seqlens_cmp"] = np.concatenate([[0], np.cumsum(cmp_lens)]).astype(np.int32)
         out["cmp_residual"] = np.array([L % w.cmp_ratio for L in lens], dtype=np.int32)
         cidx = np.concatenate([_cmp_indices(rng, w, L, cmp_any) for L in lens], axis=0)

@@ -316,6 +316,15 @@ sa_status sa_selftest_mma2(int32_t M, int32_t N, int32_t K, int32_t a_mn, int32_
                            int32_t b_sw, int32_t d_lane, const void* A, const void* B, float* D, int32_t* status,
                            void* stream);
 
+/* Self-check of the TMA row gather the token-level kernels use: n rows (n a
+ * multiple of 4, <= 32) of src, a bf16 [rows][cols] matrix (cols a multiple of
+ * 64, <= 576), named by row_idx (device int32 [n], each in [0, rows)), are
+ * loaded by tile::gather4 copies into 128-byte-swizzled shared memory and
+ * written back un-swizzled to out, bf16 [n][cols] (device).  *status (device
+ * int32) gets the timeout bit if the wait gives up.  Asynchronous. */
+sa_status sa_selftest_gather4(const void* src, int32_t rows, int32_t cols, const int32_t* row_idx, int32_t n,
+                              void* out, int32_t* status, void* stream);
+
 /* Self-check of the bounded waits every kernel uses: one CTA waits on an
  * mbarrier that nothing arrives on.  The wait gives up after its poll limit,
  * the kernel ORs the timeout bit (2) into *status (device int32) and returns

@@ -57,3 +57,36 @@ def test_reference_arm_line():
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     assert bench.run_reference(A(), rank=1) is None
+
+
+def test_reference_arm_reports_the_sample_and_the_gpu_arms_config():
+    """ms_per_step is the measured sample; the config dict is the GPU arm's (same keys
+    and values for the same workload), so the two arms compare like for like."""
+    class A:
+        workload = "cfg1"
+        override = None
+        steps = 2
+        warmup = 0
+        step_budget = 0.5
+    line = bench.run_reference(A(), rank=0)
+    w = get_workload("cfg1")
+    work = bench.count_work(w, make_inputs(w))
+    assert line["config"] == bench.config_of(w, work, 1, "")
+    assert 400.0 <= line["ms_per_step"] <= 5000.0          # the ~0.5 s sample, not an extrapolation
+    assert line["whole_backward_ms_at_sampled_rate"] > 0
+
+
+def test_roofline_fractions():
+    """The tensor fraction uses compulsory bytes only, so it never exceeds the
+    spec fraction (whose byte count adds the gathered rows)."""
+    w = get_workload("cfg1")
+    work = bench.count_work(w, make_inputs(w))
+    comp = bench.compulsory_bytes(w, work)
+    assert comp["fwd"] < work["fwd_bytes"] and comp["bwd"] < work["bwd_main_bytes"] + comp["bwd"]
+    peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}
+    fr = bench.fractions(work, comp, peaks, fwd_ms=0.05, bwd_ms=0.05)
+    assert fr["fwd_tensor_frac"] <= fr["fwd_north_star_frac"]
+    assert fr["bwd_tensor_frac"] <= fr["bwd_north_star_frac"]
+    # a time at exactly the north-star roofline is a fraction of one
+    t_ns = max(work["bwd_flops"] / 1e15, work["bwd_main_bytes"] / 5e12) * 1e3
+    assert abs(bench.fractions(work, comp, peaks, 1.0, t_ns)["bwd_north_star_frac"] - 1.0) < 1e-9

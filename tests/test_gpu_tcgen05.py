@@ -73,6 +73,10 @@ CASES2 = [
     (64, 256, 32, 0, 1, 64, 128, 16),                                   # dQ upper half at lane offset 16
     (128, 32, 64, 1, 1, 128, 64), (64, 32, 64, 1, 1, 128, 64),          # dKV: MN-major B of one 32-wide atom
     (128, 64, 128, 0, 0, 128, 128), (128, 128, 64, 1, 1, 128, 128),     # the TMA-loaded cases, loaded in software
+    # the block forward's transposed operands: S^T = K Q^T (M = 64 keys, N = 16 heads, at
+    # lane offsets 0 and 16) and O^T += V^T P^T (M = d_v as an MN-major A, P^T K-major)
+    (64, 16, 192, 0, 0, 128, 128), (64, 16, 128, 0, 0, 128, 128, 16), (64, 16, 64, 0, 0, 128, 128),
+    (128, 16, 64, 1, 0, 128, 128), (64, 16, 64, 1, 0, 128, 128),
 ]
 
 
@@ -94,3 +98,26 @@ def test_software_layouts_match_matmul(case):
     ref = A.float() @ B.float()
     err = (D - ref).abs().max().item()
     assert err <= 1e-3 * ref.abs().max().item(), f"max err {err}"
+
+
+@pytest.mark.parametrize("cols,n", [(576, 32), (128, 8), (64, 4)])
+def test_tma_row_gather_matches_index_select(cols, n):
+    """tile::gather4 copies land each named row in the 128-byte-swizzled slab layout the
+    tensor-core operands use (rows repeated and row 0 included)."""
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA GPU is required for -m gpu tests")
+    rows = 1000
+    g = torch.Generator(device="cuda").manual_seed(cols + n)
+    src = torch.randn(rows, cols, device="cuda", generator=g).to(torch.bfloat16)
+    idx = torch.randint(0, rows, (n,), device="cuda", generator=g, dtype=torch.int32)
+    idx[0] = 0
+    idx[-1] = rows - 1
+    if n >= 8:
+        idx[3] = idx[2]
+    out = torch.full((n, cols), float("nan"), device="cuda").to(torch.bfloat16)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.sa_selftest_gather4(src.data_ptr(), rows, cols, idx.data_ptr(), n, out.data_ptr(), status.data_ptr(),
+                          torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.equal(out.view(torch.int16), src[idx.long()].view(torch.int16))

@@ -30,9 +30,10 @@ def _io(o, lse, d_o, g):
 
 
 @pytest.mark.parametrize("w", [
-    get_workload("cfg1"),
+    get_workload("cfg1"),                                                    # bucketed key-stationary index
+    scaled("cfg2", "noalloc", S=700, Hq=32, Hkv=2, seed=42),                 # count / scan / fill index
     scaled("cfg4", "noalloc", seqlens=(100, 60), Hq=16, cmp_topk=32, cmp_len_range=(8, 32), seed=41),
-], ids=["cfg1", "cfg4_small"])
+], ids=["cfg1", "cfg2_small", "cfg4_small"])
 def test_no_alloc_backward_matches_workspace_backward(w):
     if not torch.cuda.is_available():
         pytest.fail("a CUDA GPU is required for -m gpu tests")
@@ -49,6 +50,7 @@ def test_no_alloc_backward_matches_workspace_backward(w):
             v.fill_(float("nan"))                            # every output must be overwritten
         L.sa_bwd_no_alloc(sa.args(), _io(o, lse, t["do"], g), stream)
         torch.cuda.synchronize()
+        assert L.sa_bwd_no_alloc_read_status(stream) == L.SA_OK
         got = grads_to_host(g)
         assert set(got) == set(ref)
         for key in ref:

@@ -99,7 +99,7 @@ EXPORTS = ["sa_fwd_get_workspace_size", "sa_fwd", "sa_bwd_get_workspace_size", "
            "sa_set_timing_events", "sa_kernel_launch_count", "sa_bwd_no_alloc",
            "sa_bwd_no_alloc_max_workspace", "sa_selftest_mma", "sa_selftest_wait_timeout",
            "sa_selftest_mma2", "sa_plan", "sa_read_status", "sa_bwd_no_alloc_read_status",
-           "sa_debug_block_index"]
+           "sa_debug_block_index", "sa_selftest_gather4"]
 
 
 def lib() -> ctypes.CDLL:
@@ -131,6 +131,7 @@ def lib() -> ctypes.CDLL:
         L.sa_selftest_wait_timeout.argtypes = [_vp, _vp, _vp]
         L.sa_selftest_mma2.argtypes = [ctypes.c_int32] * 8 + [_vp, _vp, _vp, _vp, _vp]
         L.sa_plan.argtypes = [P(SaArgs), _ip, _ip]
+        L.sa_selftest_gather4.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, _vp, ctypes.c_int32, _vp, _vp, _vp]
         L.sa_read_status.argtypes = [_vp, ctypes.c_size_t, _vp]
         L.sa_bwd_no_alloc_read_status.argtypes = [_vp]
         L.sa_debug_block_index.argtypes = [P(SaArgs), ctypes.c_int32, _vp, ctypes.c_size_t, _vp, ctypes.c_int64,
@@ -193,6 +194,11 @@ def sa_selftest_mma2(M: int, N: int, K: int, a_mn: int, b_mn: int, a_sw: int, b_
                      D: int, status: int, stream: int = 0, d_lane: int = 0) -> None:
     _check(lib().sa_selftest_mma2(M, N, K, a_mn, b_mn, a_sw, b_sw, d_lane, A, B, D, status, stream),
            "sa_selftest_mma2")
+
+
+def sa_selftest_gather4(src: int, rows: int, cols: int, row_idx: int, n: int, out: int, status: int,
+                        stream: int = 0) -> None:
+    _check(lib().sa_selftest_gather4(src, rows, cols, row_idx, n, out, status, stream), "sa_selftest_gather4")
 
 
 def sa_selftest_wait_timeout(status: int, waited: int, stream: int = 0) -> None:

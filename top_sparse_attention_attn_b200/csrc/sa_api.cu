@@ -327,7 +327,8 @@ sa_status run_check(const sa_args* a, int* status, cudaStream_t st) {
 
 // Kernel choices (sa_plan reports them; sa_fwd / sa_bwd dispatch on them).
 bool tk_path(const sa_args* a) {
-  return sa::tk_path_built(a->d_qk, a->d_v, a->kv_shared, a->n_heads_q / a->n_heads_kv);
+  // the row gathers need at least one KV row to point at (an empty KV takes the generic path)
+  return sa::tk_path_built(a->d_qk, a->d_v, a->kv_shared, a->n_heads_q / a->n_heads_kv) && sizes_of(a).Tkv >= 1;
 }
 
 int32_t fwd_choice(const sa_args* a) {
@@ -509,7 +510,7 @@ sa_status sa_fwd(const sa_args* args, const sa_fwd_out* out, void* ws, size_t ws
     sa::QbArgs q = make_qb_args(args, status);
     q.o = static_cast<bf16*>(out->o);
     q.lse = out->lse;
-    return cuda_status(sa::launch_qb(q, args->k, args->v, false, cs));
+    return cuda_status(sa::launch_bq_fwd(q, args->k, args->v, cs));
   }
   if (choice == SA_KERNEL_FWD_TOKEN_TC)
     return cuda_status(sa::launch_tk_fwd(p, static_cast<bf16*>(out->o), out->lse, cs));

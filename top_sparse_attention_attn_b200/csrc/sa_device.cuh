@@ -200,13 +200,31 @@ __device__ __forceinline__ bool tile_is_empty_slot(const Prob& p, const Unit& u,
   return false;
 }
 
-// Resolve row r (0..63) of tile `tile` of unit u to a global row code, or -1.
-__device__ __forceinline__ int resolve_row(const Prob& p, const Unit& u, int tile, int r) {
+// The raw index row r (0..63) of tile `tile` of unit u reads: its slot's ori or
+// cmp index, -1 for a slot past the unit's count, 0 for the window (range) mode,
+// which reads none.  Split from resolve_row so that a kernel can issue the load
+// early (the token-level kernels prefetch the next tile's indices).
+__device__ __forceinline__ int slot_index(const Prob& p, const Unit& u, int tile, int r) {
+  const long long ug = (long long)u.tq * p.Hkv + u.g;
   if (tile < u.n_ori_tiles) {
-    const long long ug = (long long)u.tq * p.Hkv + u.g;
+    if (u.ori_mode == kOriBlock) return __ldg(p.ori_idx + ug * p.topk + tile / u.tps);
+    if (u.ori_mode == kOriToken) {
+      const int s = tile * kTileRows + r;
+      return s < u.n_ori_slots ? __ldg(p.ori_idx + ug * p.topk + s) : -1;
+    }
+    return 0;
+  }
+  const int s = (tile - u.n_ori_tiles) * kTileRows + r;
+  return s < u.n_cmp_slots ? __ldg(p.cmp_idx + ug * p.cmp_topk + s) : -1;
+}
+
+// Resolve row r (0..63) of tile `tile` of unit u, whose slot holds index x (from
+// slot_index), to a global row code, or -1.  An index past the end of its
+// sequence selects nothing and raises the status word's index bit.
+__device__ __forceinline__ int resolve_row_x(const Prob& p, const Unit& u, int tile, int r, int x) {
+  if (tile < u.n_ori_tiles) {
     if (u.ori_mode == kOriBlock) {
-      int s = tile / u.tps, sub = tile - s * u.tps;
-      int x = __ldg(p.ori_idx + ug * p.topk + s);
+      const int sub = tile - (tile / u.tps) * u.tps;
       if (x < 0) return -1;
       int within = sub * kTileRows + r;
       if (within >= p.bs) return -1;
@@ -219,9 +237,6 @@ __device__ __forceinline__ int resolve_row(const Prob& p, const Unit& u, int til
       if (row >= u.Lk || !ori_mask_ok(p, u, (int)row)) return -1;
       return u.kv0 + (int)row;
     } else if (u.ori_mode == kOriToken) {
-      int s = tile * kTileRows + r;
-      if (s >= u.n_ori_slots) return -1;
-      int x = __ldg(p.ori_idx + ug * p.topk + s);
       if (x < 0) return -1;
       if (x >= u.Lk) {
         if (p.status) atomicOr(p.status, kStatusIndexRange);
@@ -235,10 +250,7 @@ __device__ __forceinline__ int resolve_row(const Prob& p, const Unit& u, int til
       return u.kv0 + row;
     }
   }
-  int s = (tile - u.n_ori_tiles) * kTileRows + r;
-  if (s >= u.n_cmp_slots) return -1;
-  const long long ug = (long long)u.tq * p.Hkv + u.g;
-  int c = __ldg(p.cmp_idx + ug * p.cmp_topk + s);
+  const int c = x;
   if (c < 0) return -1;
   if (c >= u.Lc) {
     if (p.status) atomicOr(p.status, kStatusIndexRange);
@@ -246,6 +258,11 @@ __device__ __forceinline__ int resolve_row(const Prob& p, const Unit& u, int til
   }
   if (p.cmp_mask == kMaskCausal && (long long)(c + 1) * p.ratio - 1 > u.ta) return -1;
   return kCmpFlag | (u.cmp0 + c);
+}
+
+// Resolve row r (0..63) of tile `tile` of unit u to a global row code, or -1.
+__device__ __forceinline__ int resolve_row(const Prob& p, const Unit& u, int tile, int r) {
+  return resolve_row_x(p, u, tile, r, slot_index(p, u, tile, r));
 }
 
 // Element offsets of a row's K and V vectors (kv-head g) for a row code >= 0.

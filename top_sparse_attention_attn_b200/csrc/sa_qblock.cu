@@ -437,6 +437,509 @@ __global__ void __launch_bounds__(160, NCTA) qb_kernel(const __grid_constant__ C
   }
 }
 
+// ---------------------------------------------------------------------------
+// Forward for 64-row blocks on tcgen05 (aclnnNsaSelectedAttentionInfer,
+// "Formula": O = Softmax(Q K_sel^T scale) V_sel, lse with the sink).
+// Persistent: one CTA per SM walks work items (query token, kv-head, slice of
+// up to 16 heads).  Transposed so that the tensor-core M dimension is keys or
+// value dims, which a 16-head slice could not fill:
+//   S_b^T [64 keys x 16 heads] = K_b Q^T   block b of a chunk of up to 16 usable
+//                                          blocks, M = 64 accumulators paired at
+//                                          TMEM lane offsets 0 / 16 (128 columns,
+//                                          two buffers)
+//   softmax over the chunk's keys per head (cross-warp reductions of the
+//   running maximum and sum; a later chunk of the same item rescales O^T)
+//   O^T [d_v x 16] += V_b^T P_b^T          V_b as an MN-major A, P_b^T [16][64]
+//                                          (two buffers, one per item in flight)
+// The producer warp streams through one ring of TMA-loaded stages, in the order
+// K(chunk c), V(chunk c - 1): the scores of a chunk are formed while the
+// previous chunk's softmax runs, and the ring keeps loading across items.  An
+// item without usable blocks flushes the pending V chunk (in the producer and
+// the MMA warp alike), so a chunk's V never waits behind a later item.  The
+// usable slots and each block's visible rows are qb_slots / blk_rows, as in every
+// block kernel.
+// ---------------------------------------------------------------------------
+template <int DQK, int DV>
+struct BqPlan {
+  static constexpr int NH = 16;   // heads per item: the N of every MMA
+  static constexpr int CH = 16;   // blocks per chunk: their scores fill 128 TMEM columns
+  static constexpr int NIT = 3;   // item descriptors in flight
+  static constexpr int kStage = 64 * (DQK > DV ? DQK : DV) * 2;
+  static constexpr int kQ = (DQK / 64) * NH * 128;              // one Q slice
+  static constexpr int oQ = 0;                                  // two Q slices
+  static constexpr int oP = (2 * kQ + 1023) / 1024 * 1024;      // CH blocks of P^T [16][64] bf16
+  static constexpr int oRedM = oP + CH * NH * 128;              // [4 warps][16] maxima
+  static constexpr int oRedL = oRedM + 4 * NH * 4;              // [4 warps][16] sums
+  static constexpr int oInfo = oRedL + 4 * NH * 4;              // NIT x (count + usable block indices)
+  static constexpr int kInfo = (1 + kQbMaxSlots) * 4;
+  static constexpr int oRing = (oInfo + NIT * kInfo + 1023) / 1024 * 1024;
+  static constexpr int kBudget = 225 * 1024;
+  static constexpr int NST0 = (kBudget - oRing) / kStage;
+  static constexpr int NST = NST0 > 12 ? 12 : NST0;
+  static constexpr int kSmem = oRing + NST * kStage;
+  static constexpr int cS = 0, cO = 256;                        // S: 2 x 128 columns; O: 2 x 16
+  static constexpr uint32_t kAlloc = 512;
+  static_assert(NST >= 4, "ring too small");
+  static_assert(kStage % 1024 == 0 && oP % 1024 == 0 && oRing % 1024 == 0, "swizzle alignment");
+  static_assert(kSmem + 1024 <= 227 * 1024, "shared memory plan too large");
+};
+
+struct BqBars {
+  uint64_t info_full[3], info_free[3], q_full[2], q_empty[2], kv_full[12], kv_empty[12];
+  uint64_t s_full[2], s_free[2], p_full, pv_done, o_free[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// The chunk walk shared by the three roles: item k's n usable blocks split into
+// chunks of at most CH; an item with n = 0 has none.
+struct BqWalk {
+  int k, slot, n, nch, c_in;  // item (local index), its info slot, count, chunks, chunk within the item
+};
+
+template <int DQK, int DV>
+__global__ void __launch_bounds__(192, 1) bq_fwd_kernel(const __grid_constant__ CUtensorMap mapQ,
+                                                        const __grid_constant__ CUtensorMap mapK,
+                                                        const __grid_constant__ CUtensorMap mapV, const QbArgs a) {
+  using PL = BqPlan<DQK, DV>;
+  constexpr int NST = PL::NST, CH = PL::CH, NIT = PL::NIT;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ BqBars bars;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (smem_u32(smem) & 1023) {
+    if (threadIdx.x == 0 && a.status) atomicOr(a.status, kStatusSmemAlign);
+    return;
+  }
+  const int n_hsl = (a.G + 15) >> 4;
+  const long long n_items = (long long)a.Tq * a.Hkv * n_hsl;
+  const uint32_t sQ = smem_u32(smem + PL::oQ), sRing = smem_u32(smem + PL::oRing), sP = smem_u32(smem + PL::oP);
+  float* redm = reinterpret_cast<float*>(smem + PL::oRedM);
+  float* redl = reinterpret_cast<float*>(smem + PL::oRedL);
+  volatile int* abort_flag = &bars.abort_flag;
+  auto info_n = [&](int slot) -> volatile int* { return reinterpret_cast<volatile int*>(smem + PL::oInfo + slot * PL::kInfo); };
+  auto info_xs = [&](int slot) -> int* { return reinterpret_cast<int*>(smem + PL::oInfo + slot * PL::kInfo + 4); };
+  // item k of this CTA -> (token, kv-head, first head, heads)
+  auto item_of = [&](int k, int* tq, int* g, int* h0, int* nh) -> bool {
+    const long long it = blockIdx.x + (long long)k * gridDim.x;
+    if (it >= n_items) return false;
+    const int unit = (int)(it / n_hsl), hsl = (int)(it - (long long)unit * n_hsl);
+    *tq = unit / a.Hkv;
+    *g = unit - *tq * a.Hkv;
+    *h0 = *g * a.G + hsl * 16;
+    *nh = min(16, a.G - hsl * 16);
+    return true;
+  };
+
+  if (threadIdx.x == 0) {
+    bars.abort_flag = 0;
+    for (int s = 0; s < NIT; ++s) {
+      mbar_init(&bars.info_full[s], 32);
+      mbar_init(&bars.info_free[s], 1 + 128);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars.q_full[s], 1);
+      mbar_init(&bars.q_empty[s], 1);
+      mbar_init(&bars.s_full[s], 1);
+      mbar_init(&bars.s_free[s], 128);
+      mbar_init(&bars.o_free[s], 128);
+    }
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&bars.kv_full[s], 1);
+      mbar_init(&bars.kv_empty[s], 1);
+    }
+    mbar_init(&bars.p_full, 128);
+    mbar_init(&bars.pv_done, 1);
+    mbar_fence_init();
+    tma_prefetch_desc(&mapQ);
+    tma_prefetch_desc(&mapK);
+    tma_prefetch_desc(&mapV);
+  }
+  if (warp == 1) tmem_alloc(&bars.tmem_base, PL::kAlloc);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (whole warp)
+    // items in order: the usable slots to the info ring, the Q slice, then the
+    // blocks in the order K(chunk c), V(chunk c - 1)
+    int t = 0, qk = 0;
+    bool ok = true;
+    int pv_slot = -1, pv_first = 0, pv_nb = 0, pv_row0 = 0, pv_g = 0;  // the chunk whose V is pending
+    auto load_blocks = [&](bool is_v, int slot, int first, int nb, int kv0, int g) {
+      for (int b = 0; ok && b < nb; ++b, ++t) {
+        const int st = t % NST;
+        if (lane == 0) {
+          if (t >= NST && !mbar_wait(&bars.kv_empty[st], ((t / NST) - 1) & 1, abort_flag, a.status)) {
+            ok = false;
+          } else {
+            const uint32_t stage = sRing + st * PL::kStage;
+            const int row = kv0 + 64 * info_xs(slot)[first + b];
+            if (!is_v) {
+              mbar_arrive_tx(&bars.kv_full[st], (uint32_t)(64 * DQK * 2));
+              for (int s = 0; s < DQK / 64; ++s) tma_load_2d(stage + s * 8192, &mapK, g * DQK + 64 * s, row, &bars.kv_full[st]);
+            } else {
+              mbar_arrive_tx(&bars.kv_full[st], (uint32_t)(64 * DV * 2));
+              for (int s = 0; s < DV / 64; ++s) tma_load_2d(stage + s * 8192, &mapV, g * DV + 64 * s, row, &bars.kv_full[st]);
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
+    };
+    for (int k = 0; ok; ++k) {
+      int tq, g, h0, nh;
+      const bool have = item_of(k, &tq, &g, &h0, &nh);
+      const int slot = k % NIT;
+      if (k >= NIT) {
+        bool w = lane != 0 || mbar_wait(&bars.info_free[slot], ((k / NIT) - 1) & 1, abort_flag, a.status);
+        ok = __shfl_sync(0xffffffffu, w, 0);
+        if (!ok) break;
+      }
+      int n = -1;  // -1: no more items
+      if (have) {
+        const Unit u = qb_unit(a, tq, g);
+        n = qb_slots(a, u, info_xs(slot), lane);
+        if (lane == 0) *info_n(slot) = n;
+        __syncwarp();
+        mbar_arrive(&bars.info_full[slot]);
+        if (n == 0 && pv_slot >= 0) {
+          // an item without blocks: the pending V chunk goes now (the MMA warp issues its
+          // P V at the same point), before its slot list can be reused
+          load_blocks(true, pv_slot, pv_first, pv_nb, pv_row0, pv_g);
+          pv_slot = -1;
+        }
+        if (n > 0) {
+          const int qs = qk & 1;
+          if (lane == 0) {
+            if (qk >= 2 && !mbar_wait(&bars.q_empty[qs], ((qk >> 1) - 1) & 1, abort_flag, a.status)) {
+              ok = false;
+            } else {
+              mbar_arrive_tx(&bars.q_full[qs], (uint32_t)(PL::NH * DQK * 2));
+              for (int s = 0; s < DQK / 64; ++s)
+                tma_load_2d(sQ + qs * PL::kQ + s * (PL::NH * 128), &mapQ, 64 * s, tq * a.Hq + h0, &bars.q_full[qs]);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ++qk;
+          const int nch = (n + CH - 1) / CH;
+          for (int c = 0; ok && c < nch; ++c) {
+            const int nb = min(CH, n - c * CH);
+            load_blocks(false, slot, c * CH, nb, u.kv0, g);
+            if (pv_slot >= 0) load_blocks(true, pv_slot, pv_first, pv_nb, pv_row0, pv_g);
+            pv_slot = slot;
+            pv_first = c * CH;
+            pv_nb = nb;
+            pv_row0 = u.kv0;
+            pv_g = g;
+          }
+        }
+      } else {
+        if (lane == 0) *info_n(slot) = -1;
+        __syncwarp();
+        mbar_arrive(&bars.info_full[slot]);
+        break;
+      }
+    }
+    if (ok && pv_slot >= 0) load_blocks(true, pv_slot, pv_first, pv_nb, pv_row0, pv_g);
+    // drain: every issued load lands before the CTA exits
+    if (lane == 0) {
+      for (int k2 = t > NST ? t - NST : 0; k2 < t; ++k2) mbar_wait_drain(&bars.kv_full[k2 % NST], (k2 / NST) & 1);
+      for (int q2 = qk > 2 ? qk - 2 : 0; q2 < qk; ++q2) mbar_wait_drain(&bars.q_full[q2 & 1], (q2 >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(64, PL::NH, false, false);
+      constexpr uint32_t idO = idesc_bf16(DV >= 128 ? 128 : 64, PL::NH, true, false);
+      int t = 0, c = 0, qk = 0, ok_items = 0;
+      bool ok = true;
+      // the chunk whose P V is pending: its chunk number, blocks, O buffer and whether it opens its item
+      int pv_c = -1, pv_nb = 0, pv_ob = 0;
+      bool pv_first = false;
+      auto issue_pv = [&]() {
+        if (!mbar_wait(&bars.p_full, pv_c & 1, abort_flag, a.status)) { ok = false; return; }
+        tc_fence_after();
+        for (int b = 0; ok && b < pv_nb; ++b, ++t) {
+          const int st = t % NST;
+          if (!mbar_wait(&bars.kv_full[st], (t / NST) & 1, abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t stage = sRing + st * PL::kStage;
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + PL::cO + 16 * pv_ob, sdesc(stage + kk * 2048, 8192, 1024),
+                     sdesc(sP + b * 2048 + kk * 32, 16, 1024), idO, (!pv_first || b > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bars.kv_empty[st]);
+        }
+        if (ok) mma_commit(&bars.pv_done);
+      };
+      for (int k = 0; ok; ++k) {
+        const int slot = k % NIT;
+        if (!mbar_wait(&bars.info_full[slot], (k / NIT) & 1, abort_flag, a.status)) break;
+        const int n = *info_n(slot);
+        mbar_arrive(&bars.info_free[slot]);
+        if (n < 0) break;
+        if (n == 0) {
+          if (pv_c >= 0) issue_pv();  // mirrors the producer: the pending V chunk comes now
+          pv_c = -1;
+          continue;
+        }
+        const int qs = qk & 1, ob = ok_items & 1;
+        if (!mbar_wait(&bars.q_full[qs], (qk >> 1) & 1, abort_flag, a.status)) break;
+        // the O buffer of this item was read by the epilogue of item ok_items - 2
+        if (ok_items >= 2 && !mbar_wait(&bars.o_free[ob], ((ok_items >> 1) - 1) & 1, abort_flag, a.status)) break;
+        const int nch = (n + CH - 1) / CH;
+        for (int cc = 0; ok && cc < nch; ++cc, ++c) {
+          const int nb = min(CH, n - cc * CH);
+          const int sb = c & 1;
+          if (c >= 2 && !mbar_wait(&bars.s_free[sb], ((c >> 1) - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+          for (int b = 0; b < nb; ++b, ++t) {
+            const int st = t % NST;
+            if (!mbar_wait(&bars.kv_full[st], (t / NST) & 1, abort_flag, a.status)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t stage = sRing + st * PL::kStage;
+            const uint32_t d = tmem + PL::cS + 128 * sb + 16 * (b >> 1) + ((uint32_t)(16 * (b & 1)) << 16);
+            for (int kk = 0; kk < DQK / 16; ++kk)
+              mma_bf16(d, sdesc(stage + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                       sdesc(sQ + qs * PL::kQ + (kk >> 2) * (PL::NH * 128) + (kk & 3) * 32, 16, 1024), idS, kk > 0);
+            mma_commit(&bars.kv_empty[st]);
+          }
+          if (!ok) break;
+          if (cc == nch - 1) mma_commit(&bars.q_empty[qs]);
+          mma_commit(&bars.s_full[sb]);
+          if (pv_c >= 0) issue_pv();
+          pv_c = c;
+          pv_nb = nb;
+          pv_ob = ob;
+          pv_first = cc == 0;
+        }
+        ++qk;
+        ++ok_items;
+      }
+      if (ok && pv_c >= 0) issue_pv();
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    // Every chunk runs both named barriers in all four warps, also after a wait gave
+    // up (the work is skipped, the barriers are not), so no warp is left at one.
+    const int sub = warp & 3;
+    const int par = lane >> 4, key = (lane & 15) + 16 * sub;  // block parity and key of this TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * sub) << 16);
+    const int tid = threadIdx.x - 64;
+    int c = 0, ok_items = 0;
+    bool ok = true;
+    for (int k = 0;; ++k) {
+      const int slot = k % NIT;
+      if (!mbar_wait(&bars.info_full[slot], (k / NIT) & 1, abort_flag, a.status)) break;
+      const int n = *info_n(slot);
+      if (n < 0) break;
+      int tq, g, h0, nh;
+      item_of(k, &tq, &g, &h0, &nh);
+      const Unit u = qb_unit(a, tq, g);
+      const int* xs = info_xs(slot);
+      const int ob = ok_items & 1;
+      float m[16], l[16];
+#pragma unroll
+      for (int h = 0; h < 16; ++h) {
+        const bool sk = a.sinks && h < nh;
+        m[h] = sk ? __ldg(a.sinks + h0 + h) * kLog2eQb : -INFINITY;
+        l[h] = sk ? 1.f : 0.f;
+      }
+      const int nch = (n + CH - 1) / CH;
+      for (int cc = 0; cc < nch; ++cc, ++c) {
+        const int nb = min(CH, n - cc * CH);
+        const int sb = c & 1;
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars.s_full[sb], (c >> 1) & 1, abort_flag, a.status));
+        tc_fence_after();
+        unsigned vis = 0;  // bit j: this thread's key of block 2j + par is visible
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int b = 2 * j + par;
+          if (b < nb) {
+            int lo, hi;
+            blk_rows(xs[cc * CH + b], u.Lk, u.ta, a.ori_mask, a.wl, a.wr, &lo, &hi);
+            if (key >= lo && key <= hi) vis |= 1u << j;
+          }
+        }
+        // pass 1 over the scores (TMEM): the chunk's maximum per head
+        float mx[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) mx[h] = -INFINITY;
+#pragma unroll 1
+        for (int j = 0; ok && j < 8; ++j) {
+          if (2 * j >= nb) break;  // uniform over the CTA
+          uint32_t v[16];
+          tmem_ld16(lane_base + PL::cS + 128 * sb + 16 * j, v);
+          tmem_wait_ld();
+          reg_dep16(v);
+          if ((vis >> j) & 1u) {
+#pragma unroll
+            for (int h = 0; h < 16; ++h) mx[h] = fmaxf(mx[h], __uint_as_float(v[h]) * a.scale_log2);
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+#pragma unroll
+          for (int o = 16; o; o >>= 1) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], o));
+        }
+        if (lane < 16) {
+          float mine = mx[0];
+#pragma unroll
+          for (int h = 1; h < 16; ++h) mine = lane == h ? mx[h] : mine;
+          redm[sub * 16 + lane] = mine;
+        }
+        asm volatile("bar.sync 1, 128;\n" ::: "memory");
+        bool grow = false;
+        float* f = mx;  // the rescale factors replace the maxima
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+          const float cm = fmaxf(fmaxf(redm[h], redm[16 + h]), fmaxf(redm[32 + h], redm[48 + h]));
+          const float mn = fmaxf(m[h], cm);
+          f[h] = (m[h] == -INFINITY) ? 0.f : exp2f(m[h] - mn);
+          grow |= (cc > 0) && (mn > m[h]);
+          m[h] = mn;
+          l[h] *= f[h];
+        }
+        // the single P buffer and O^T: the previous chunk's P V has landed
+        if (c >= 1) ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars.pv_done, (c - 1) & 1, abort_flag, a.status));
+        if (ok && __any_sync(0xffffffffu, grow)) {
+          // a later chunk of the item raised a maximum: rescale O^T columns
+          tc_fence_after();
+          uint32_t w[16];
+          tmem_ld16(lane_base + PL::cO + 16 * ob, w);
+          tmem_wait_ld();
+          reg_dep16(w);
+#pragma unroll
+          for (int h = 0; h < 16; ++h) w[h] = __float_as_uint(__uint_as_float(w[h]) * f[h]);
+          tmem_st16(lane_base + PL::cO + 16 * ob, w);
+          tmem_wait_st();
+        }
+        // pass 2: P = exp2(s - m) to the P^T buffers (row = head, 64 keys per block)
+        float sm[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) sm[h] = 0.f;
+#pragma unroll 1
+        for (int j = 0; ok && j < 8; ++j) {
+          if (2 * j >= nb) break;
+          uint32_t v[16];
+          tmem_ld16(lane_base + PL::cS + 128 * sb + 16 * j, v);
+          tmem_wait_ld();
+          reg_dep16(v);
+          const int b = 2 * j + par;
+          if (b < nb) {
+            const bool on = (vis >> j) & 1u;
+            const uint32_t pb = sP + b * 2048 + (key & 7) * 2;
+#pragma unroll
+            for (int h = 0; h < 16; ++h) {
+              const float pv = on ? exp2f(__uint_as_float(v[h]) * a.scale_log2 - m[h]) : 0.f;
+              sm[h] += pv;
+              const __nv_bfloat16 pbf = __float2bfloat16_rn(pv);
+              const uint16_t bits = *reinterpret_cast<const uint16_t*>(&pbf);
+              asm volatile("st.shared.b16 [%0], %1;\n" ::"r"(pb + h * 128 + ((((key >> 3) ^ h) & 7) << 4)),
+                           "h"(bits)
+                           : "memory");
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&bars.s_free[sb]);
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+#pragma unroll
+          for (int o = 16; o; o >>= 1) sm[h] += __shfl_xor_sync(0xffffffffu, sm[h], o);
+        }
+        if (lane < 16) {
+          float mine = sm[0];
+#pragma unroll
+          for (int h = 1; h < 16; ++h) mine = lane == h ? sm[h] : mine;
+          redl[sub * 16 + lane] = mine;
+        }
+        fence_async_smem();
+        mbar_arrive(&bars.p_full);
+        asm volatile("bar.sync 1, 128;\n" ::: "memory");
+#pragma unroll
+        for (int h = 0; h < 16; ++h) l[h] += (redl[h] + redl[16 + h]) + (redl[32 + h] + redl[48 + h]);
+      }
+      // epilogue: O = O^T / l (this thread's value dim, every head), lse per head
+      bool have_o = n == 0;
+      if (n > 0) have_o = __all_sync(0xffffffffu, ok && mbar_wait(&bars.pv_done, (c - 1) & 1, abort_flag, a.status));
+      if (have_o) {
+        tc_fence_after();
+        uint32_t w[16];
+        if (n > 0) {
+          tmem_ld16(lane_base + PL::cO + 16 * ob, w);
+          tmem_wait_ld();
+          reg_dep16(w);
+        }
+        // O^T rows: M = 128 puts value dim d in lane d; M = 64 puts it in lane (d % 16) + 32 (d / 16)
+        const int dvi = DV >= 128 ? 32 * sub + lane : (lane < 16 ? 16 * sub + lane : -1);
+        if (dvi >= 0) {
+#pragma unroll
+          for (int h = 0; h < 16; ++h) {
+            if (h < nh) {
+              const float val = (n == 0 || l[h] <= 0.f) ? 0.f : __uint_as_float(w[h]) / l[h];
+              a.o[((long long)tq * a.Hq + h0 + h) * DV + dvi] = __float2bfloat16_rn(val);
+            }
+          }
+        }
+        if (tid < nh) {
+          float lt = l[0], mt = m[0];
+#pragma unroll
+          for (int h = 1; h < 16; ++h) {
+            lt = tid == h ? l[h] : lt;
+            mt = tid == h ? m[h] : mt;
+          }
+          a.lse[(long long)tq * a.Hq + h0 + tid] = lt > 0.f ? (mt + log2f(lt)) * kLn2Qb : INFINITY;
+        }
+      }
+      if (n > 0) {
+        tc_fence_before();
+        mbar_arrive(&bars.o_free[ob]);
+        ++ok_items;
+      }
+      mbar_arrive(&bars.info_free[slot]);
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, PL::kAlloc);
+    tmem_relinquish();
+  }
+}
+
+template <int DQK, int DV>
+static cudaError_t bq_launch_t(const QbArgs& a, const void* k, const void* v, cudaStream_t st) {
+  using PL = BqPlan<DQK, DV>;
+  CUtensorMap mq, mk, mv;
+  if (!make_tmap_bf16(&mq, a.q, (uint64_t)a.Tq * a.Hq, DQK, (uint64_t)DQK * 2, PL::NH) ||
+      !make_tmap_bf16(&mk, k, (uint64_t)a.Tkv, (uint64_t)a.Hkv * DQK, (uint64_t)a.Hkv * DQK * 2, 64) ||
+      !make_tmap_bf16(&mv, v, (uint64_t)a.Tkv, (uint64_t)a.Hkv * DV, (uint64_t)a.Hkv * DV * 2, 64))
+    return cudaErrorInvalidValue;
+  auto kern = bq_fwd_kernel<DQK, DV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kSmem);
+  if (e != cudaSuccess) return e;
+  const long long items = (long long)a.Tq * a.Hkv * ((a.G + 15) / 16);
+  if (items == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long grid = items < sms ? items : sms;
+  mark_begin(st, kTimeFwd);
+  kern<<<(unsigned)grid, 192, PL::kSmem, st>>>(mq, mk, mv, a);
+  count_launch();
+  mark_end(st, kTimeFwd);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bq_fwd(const QbArgs& a, const void* k, const void* v, cudaStream_t st) {
+  if (a.dqk == 64 && a.dv == 64) return bq_launch_t<64, 64>(a, k, v, st);
+  if (a.dqk == 128 && a.dv == 128) return bq_launch_t<128, 128>(a, k, v, st);
+  if (a.dqk == 192 && a.dv == 128) return bq_launch_t<192, 128>(a, k, v, st);
+  return cudaErrorInvalidValue;
+}
+
 // Inspection: one warp per (token, kv-head) unit runs qb_unit / qb_slots /
 // blk_rows exactly as qb_kernel does and records every usable slot as
 // {unit, block, lo, hi}.
@@ -498,14 +1001,12 @@ static cudaError_t qb_launch_t(const QbArgs& a, const void* k, const void* v, cu
   return cudaGetLastError();
 }
 
+// The dQ pass (the forward runs on bq_fwd_kernel).
 cudaError_t launch_qb(const QbArgs& a, const void* k, const void* v, bool dq, cudaStream_t st) {
-  const int tid = dq ? kTimeBwdDQ : kTimeFwd;
-  if (a.dqk == 64 && a.dv == 64)
-    return dq ? qb_launch_t<64, 64, true>(a, k, v, st, tid) : qb_launch_t<64, 64, false>(a, k, v, st, tid);
-  if (a.dqk == 128 && a.dv == 128)
-    return dq ? qb_launch_t<128, 128, true>(a, k, v, st, tid) : qb_launch_t<128, 128, false>(a, k, v, st, tid);
-  if (a.dqk == 192 && a.dv == 128)
-    return dq ? qb_launch_t<192, 128, true>(a, k, v, st, tid) : qb_launch_t<192, 128, false>(a, k, v, st, tid);
+  if (!dq) return cudaErrorInvalidValue;
+  if (a.dqk == 64 && a.dv == 64) return qb_launch_t<64, 64, true>(a, k, v, st, kTimeBwdDQ);
+  if (a.dqk == 128 && a.dv == 128) return qb_launch_t<128, 128, true>(a, k, v, st, kTimeBwdDQ);
+  if (a.dqk == 192 && a.dv == 128) return qb_launch_t<192, 128, true>(a, k, v, st, kTimeBwdDQ);
   return cudaErrorInvalidValue;
 }
 

@@ -31,6 +31,8 @@ struct QbArgs {
 
 bool qb_path_built(int dqk, int dv);
 cudaError_t launch_qb(const QbArgs& a, const void* k, const void* v, bool dq, cudaStream_t st);
+// Forward on tcgen05 (64-row blocks, 16-head slices, scores held transposed in TMEM).
+cudaError_t launch_bq_fwd(const QbArgs& a, const void* k, const void* v, cudaStream_t st);
 // Inspection: the usable slots and row ranges of every unit as the block kernels see them.
 cudaError_t launch_qb_debug_slots(const QbArgs& a, int4* rec, long long max_rec, int* n_rec, cudaStream_t st);
 

@@ -195,6 +195,47 @@ __global__ void __launch_bounds__(128) selftest_mma2_kernel(const bf16* __restri
   }
 }
 
+// TMA row gather: n rows (n a multiple of 4, <= 32) of a [rows][cols] bf16 matrix
+// (cols a multiple of 64, <= 576) named by row_idx land by tile::gather4 loads in
+// shared memory as slabs of n rows x 128 bytes (128-byte swizzle), exactly where
+// the token-level kernels read them; the CTA then writes them back un-swizzled
+// to out [n][cols].
+__global__ void __launch_bounds__(128) selftest_gather4_kernel(const __grid_constant__ CUtensorMap map,
+                                                               const int* __restrict__ row_idx, int n, int cols,
+                                                               bf16* __restrict__ out, int* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t base = smem_u32(smem);
+  const int nslab = cols / 64;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_tx(&bar, (uint32_t)(n * cols * 2));
+    for (int q = 0; q < n / 4; ++q)
+      for (int s = 0; s < nslab; ++s)
+        tma_gather4(base + s * (n * 128) + q * 4 * 128, &map, 64 * s, __ldg(row_idx + 4 * q),
+                    __ldg(row_idx + 4 * q + 1), __ldg(row_idx + 4 * q + 2), __ldg(row_idx + 4 * q + 3), &bar);
+  }
+  const bool ok = mbar_wait(&bar, 0, &abort_flag, status);
+  if (!ok) {
+    if (threadIdx.x == 0) mbar_wait_drain(&bar, 0);
+    return;
+  }
+  for (int i = threadIdx.x; i < n * cols / 8; i += blockDim.x) {
+    const int r = i / (cols / 8), c = i - r * (cols / 8);  // 16-byte piece c of row r
+    const uint32_t a = base + (c >> 3) * (n * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    reinterpret_cast<uint4*>(out + (long long)r * cols)[c] = v;
+  }
+}
+
 // Nothing ever arrives on `bar`: the bounded wait gives up and raises the status word.
 __global__ void selftest_wait_kernel(int* status, int* waited) {
   __shared__ uint64_t bar;
@@ -229,6 +270,22 @@ extern "C" sa_status sa_selftest_mma2(int32_t M, int32_t N, int32_t K, int32_t a
     return SA_ERR_CUDA;
   sa::selftest_mma2_kernel<<<1, 128, smem, st>>>(static_cast<const sa::bf16*>(A), static_cast<const sa::bf16*>(B), args,
                                                  D, status);
+  sa::count_launch();
+  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+extern "C" sa_status sa_selftest_gather4(const void* src, int32_t rows, int32_t cols, const int32_t* row_idx,
+                                         int32_t n, void* out, int32_t* status, void* stream) {
+  if (!src || !row_idx || !out || !status) return SA_ERR_NULLPTR;
+  if (rows < 1 || cols < 64 || cols > 576 || cols % 64 || n < 4 || n > 32 || n % 4) return SA_ERR_PARAM;
+  CUtensorMap map;
+  if (!sa::make_tmap_bf16(&map, src, (uint64_t)rows, (uint64_t)cols, (uint64_t)cols * 2, 1)) return SA_ERR_PARAM;
+  const int smem = n * cols * 2 + 1024;
+  if (cudaFuncSetAttribute(sa::selftest_gather4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return SA_ERR_CUDA;
+  sa::selftest_gather4_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(
+      map, row_idx, n, cols, static_cast<sa::bf16*>(out), status);
   sa::count_launch();
   return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }

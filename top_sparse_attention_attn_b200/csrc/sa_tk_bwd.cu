@@ -1,25 +1,43 @@
-// sa_tk_bwd.cu -- token-level backward over one shared latent KV head (K = V,
-// d_qk = 576, d_v = 512) on tcgen05, query-stationary: one CTA takes one
-// (token, kv-head) unit and 64 of its query heads, and streams the unit's
-// selected KV rows through in tiles of 32 rows.
+// sa_tk_bwd.cu -- token-level selection over one shared latent KV head (K = V,
+// d_qk = 576, d_v = 512: the first 512 columns of each KV row are V) on tcgen05,
+// query-stationary: one CTA takes one (query token, kv-head) unit and 64 of its
+// query heads, and streams the unit's selected KV rows through in sub-tiles of
+// 32 rows.
 //
-// SparseFlashMlaGrad "Computation formula" Stages 2-3 (P recomputed from lse,
-// dP = dO V^T, dS = P o (dP - Delta), dQ = dS K scale, dKV = dS^T Q scale + P^T dO).
+// Selection: SparseFlashMlaGrad "Computation formula" Stage 1 (ori rows through
+// token indices or the sliding window, concatenated with gathered cmpKv rows),
+// resolved row by row with resolve_row_x.  The rows of a sub-tile arrive by TMA
+// row gathers (tile::gather4, four rows per copy) into 128-byte-swizzled shared
+// memory; a lane of the loader warp resolves each row, and the next sub-tile's
+// indices are loaded while the current one is issued.
 //
-// Per 32-row tile (bf16 operands, fp32 TMEM accumulators; M = 64 heads):
-//   S    [64 x 32]   = Q KV^T            lanes 0..15 of each sub-partition
-//   dP   [64 x 32]   = dO V^T            lanes 16..31, the same columns
-//   P, dS (scaled)                        softmax warps, to shared memory
-//   dKV^T [576 x 32] = Q^T dS + dO^T P   (the P^T dO term on dims 0..511),
-//                                          added to the fp32 dKV accumulator
-//   dQ   [64 x 576] += dS KV              accumulated in TMEM over every tile
-// TMEM columns: [0, 32) S / dP; [32, 288) dQ dims 0..255 (lanes 0..15) and
-// 256..511 (lanes 16..31); [288, 352) dQ dims 512..575; [352, 480) dKV^T dims
-// 0..511 as four M = 128 tiles; [480, 512) dKV^T dims 512..575 (M = 64).
+// Forward (aclnnNsaSelectedAttentionInfer "Formula"; SparseFlashMlaGrad Stage 2
+// for lse), per sub-tile i (bf16 operands, fp32 TMEM accumulators, M = 64 heads):
+//   S_i [64 x 32] = Q KV_i^T               two TMEM buffers (lanes 0..15 of each
+//                                           sub-partition)
+//   online softmax in the softmax warps     P_i to one of two shared buffers
+//   O   [64 x 512] += P_i V_i              dims 0..255 in lanes 0..15, 256..511 in
+//                                           lanes 16..31
+// The MMA warp issues S_{i+1} before P_i V_i, so the softmax of one sub-tile
+// overlaps the tensor work of its neighbours (three KV stages in flight).  The
+// running maximum moves only when a sub-tile's maximum exceeds it by more than 8
+// (a factor of 256 in the exponentials): O and the running sum are then rescaled
+// once, after the previous P V has landed.  Sinks start the running state.
 //
-// Warp roles: 0 = loader (Q / dO by TMA, KV rows by cp.async), 1 = MMA issuer
-// + TMEM owner, 2..5 = softmax and the final dQ store, 6..9 = dKV reductions.
-// Every wait is bounded (sa_tc.cuh).
+// Backward (SparseFlashMlaGrad Stages 2-3: P recomputed from lse, dP = dO V^T,
+// dS = P o (dP - Delta), dQ = dS K scale, dKV = dS^T Q scale + P^T dO), per
+// sub-tile:
+//   S  [64 x 32] = Q KV^T   (lanes 0..15)   dP [64 x 32] = dO V^T (lanes 16..31)
+//   P, dS (scaled) by the softmax warps, to shared memory
+//   dKV^T [576 x 32] = Q^T dS + dO^T P      (the P^T dO term on dims 0..511),
+//                                           added to the fp32 dKV accumulator by
+//                                           the reduction warps (one 128-byte
+//                                           warp-wide reduction per row and 32 dims)
+//   dQ [64 x 576] += dS KV                  accumulated in TMEM over every sub-tile
+//
+// Warp roles: 0 = loader (Q / dO box loads, row codes, KV row gathers), 1 = MMA
+// issuer + TMEM owner, 2..5 = softmax (and the final O or dQ store), 6..9
+// (backward) = dKV reductions.  Every wait is bounded (sa_tc.cuh).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -32,56 +50,116 @@ namespace sa {
 
 constexpr float kLog2eTk = 1.4426950408889634f;
 
-struct TkPlan {
-  static constexpr int DQK = 576, DV = 512;
-  static constexpr int H = 64;     // query heads per CTA
-  static constexpr int NK = 32;    // KV rows per tile
-  static constexpr int NSQ = DQK / 64, NSV = DV / 64;
-  static constexpr int oQ = 0;                           // Q: NSQ slabs of 64 rows x 128 B
-  static constexpr int oDO = oQ + NSQ * H * 128;         // dO: NSV slabs of 64 rows
-  static constexpr int kKVStage = NSQ * NK * 128;        // one KV tile: NSQ slabs of 32 rows
-  static constexpr int oKV = oDO + NSV * H * 128;        // 2 stages
-  // P and dS [64 heads][32 keys] bf16 in the 64-byte swizzle (rows of 64 B): a
-  // K-major A for dQ (K = keys) and an MN-major B of one 32-wide atom for dKV
-  static constexpr int oP = oKV + 2 * kKVStage;
-  static constexpr int oDS = oP + H * 64;
-  static constexpr int oCode = oDS + H * 64;             // row codes of the last 4 tiles
-  static constexpr int kSmem = oCode + 4 * NK * 4;
+namespace tk {
+constexpr int DQK = 576, DV = 512;
+constexpr int H = 64;                    // query heads per CTA
+constexpr int NK = 32;                   // KV rows per sub-tile
+constexpr int NSQ = DQK / 64, NSV = DV / 64;
+constexpr int kKVStage = NSQ * NK * 128; // one sub-tile: NSQ slabs of 32 rows x 128 B
+constexpr int kQBytes = NSQ * H * 128;   // Q: NSQ slabs of 64 rows
+constexpr int kDOBytes = NSV * H * 128;  // dO: NSV slabs of 64 rows
+constexpr int kPBytes = H * 64;          // P or dS [64 heads][32 keys] bf16, 64-byte swizzle
+}  // namespace tk
+
+// 16-byte piece index XOR for a [64][32] bf16 operand in the 64-byte swizzle.
+__device__ __forceinline__ uint32_t tk_p_addr(uint32_t base, int h, int c) {
+  return base + h * 64 + ((c ^ ((h >> 1) & 3)) << 4);
+}
+
+// Loader (warp 0, every lane): the row codes of each 32-row sub-tile (lane = row)
+// into the 4-deep codes ring, then the rows themselves by TMA row gathers into
+// stage i % NST.  Stage reuse waits for kv_empty; on abort the warp stops issuing.
+// Before returning it waits (bounded) for every gather it issued to land.
+template <int NST>
+__device__ void tk_load_rows(const Prob& p, const Unit& u, int g, int nsub, uint32_t sKV, int* codes,
+                             const CUtensorMap* mapKV, const CUtensorMap* mapCmp, bool has_cmp, uint64_t* kv_full,
+                             uint64_t* kv_empty, uint64_t* codes_full, volatile int* abort_flag, int lane) {
+  int x_next = nsub > 0 ? slot_index(p, u, 0, lane) : -1;
+  int issued = 0;
+  for (int i = 0; i < nsub; ++i) {
+    const int st = i % NST, tile = i >> 1, r = 32 * (i & 1) + lane;
+    const int x = x_next;
+    if (i + 1 < nsub) x_next = slot_index(p, u, (i + 1) >> 1, 32 * ((i + 1) & 1) + lane);  // prefetch
+    bool ok = true;
+    if (lane == 0 && i >= NST) ok = mbar_wait(&kv_empty[st], ((i / NST) - 1) & 1, abort_flag, p.status);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) break;
+    const int code = resolve_row_x(p, u, tile, r, x);
+    codes[(i & 3) * tk::NK + lane] = code;
+    const bool cmp_tile = tile >= u.n_ori_tiles && has_cmp;
+    const int y = code >= 0 ? (code & ~kCmpFlag) : 0;  // invisible rows load row 0 (masked later)
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&codes_full[i & 3]);
+      mbar_arrive_tx(&kv_full[st], (uint32_t)tk::kKVStage);
+    }
+    __syncwarp();
+    const int q4 = lane & 7;
+    const int y0 = __shfl_sync(0xffffffffu, y, 4 * q4), y1 = __shfl_sync(0xffffffffu, y, 4 * q4 + 1);
+    const int y2 = __shfl_sync(0xffffffffu, y, 4 * q4 + 2), y3 = __shfl_sync(0xffffffffu, y, 4 * q4 + 3);
+    if (lane < 8) {
+      const CUtensorMap* map = cmp_tile ? mapCmp : mapKV;
+      const uint32_t dst = sKV + st * tk::kKVStage + q4 * 4 * 128;
+#pragma unroll
+      for (int s = 0; s < tk::NSQ; ++s) tma_gather4(dst + s * (tk::NK * 128), map, g * tk::DQK + 64 * s, y0, y1, y2, y3, &kv_full[st]);
+    }
+    issued = i + 1;
+  }
+  if (lane == 0)
+    for (int i = issued > NST ? issued - NST : 0; i < issued; ++i) mbar_wait_drain(&kv_full[i % NST], (i / NST) & 1);
+}
+
+// ===========================================================================
+// backward
+// ===========================================================================
+struct TkBwdPlan {
+  static constexpr int NST = 2;
+  static constexpr int oQ = 0;
+  static constexpr int oDO = oQ + tk::kQBytes;
+  static constexpr int oKV = oDO + tk::kDOBytes;
+  static constexpr int oP = oKV + NST * tk::kKVStage;
+  static constexpr int oDS = oP + tk::kPBytes;
+  static constexpr int oCode = oDS + tk::kPBytes;  // row codes of the last 4 sub-tiles
+  static constexpr int kSmem = oCode + 4 * tk::NK * 4;
   static_assert(kSmem + 1024 <= 227 * 1024, "shared memory plan too large");
-  static_assert(oDO % 1024 == 0 && oKV % 1024 == 0 && kKVStage % 1024 == 0 && oP % 1024 == 0 && oDS % 1024 == 0,
+  static_assert(oDO % 1024 == 0 && oKV % 1024 == 0 && tk::kKVStage % 1024 == 0 && oP % 1024 == 0 &&
+                    oDS % 1024 == 0,
                 "swizzled operands need 1024-byte alignment");
+  // TMEM columns: [0, 32) S (lanes 0..15) / dP (lanes 16..31); [32, 288) dQ dims
+  // 0..255 (lanes 0..15) and 256..511 (lanes 16..31); [288, 352) dQ dims 512..575
+  // (lanes 0..15); [352, 480) dKV^T dims 0..511 as four M = 128 tiles; [480, 512)
+  // dKV^T dims 512..575 (M = 64).
   static constexpr int cS = 0, cDQ = 32, cDQR = 288, cKV = 352, cKVR = 480;
   static constexpr uint32_t kAlloc = 512;
 };
 
-struct TkBars {
-  uint64_t q_full, kv_full[2], kv_empty[2], s_full, pds_full, pds_free, dkv_full, dkv_free, dq_done;
-  uint64_t codes_full[4];  // a tile's row codes are in shared memory (ring of 4 tiles)
+struct TkBwdBars {
+  uint64_t q_full, kv_full[TkBwdPlan::NST], kv_empty[TkBwdPlan::NST], s_full, pds_full, pds_free, kvq_done,
+      dkv_free, dq_done;
+  uint64_t codes_full[4];  // a sub-tile's row codes are in shared memory (ring of 4)
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// 16-byte piece c (0..71) of a 576-wide bf16 row r of a 32-row KV tile
-__device__ __forceinline__ uint32_t tk_kv_addr(uint32_t stage, int r, int c) {
-  return stage + (c >> 3) * (TkPlan::NK * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-}
-
 __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ CUtensorMap mapQ,
-                                                         const __grid_constant__ CUtensorMap mapDO, const Prob p,
-                                                         const float* __restrict__ LSE,
+                                                         const __grid_constant__ CUtensorMap mapDO,
+                                                         const __grid_constant__ CUtensorMap mapKV,
+                                                         const __grid_constant__ CUtensorMap mapCmp, const int has_cmp,
+                                                         const Prob p, const float* __restrict__ LSE,
                                                          const float* __restrict__ Delta, BwdOut out) {
-  using PL = TkPlan;
+  using PL = TkBwdPlan;
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ TkBars bars;
+  __shared__ TkBwdBars bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {
+    pdl_wait();
     if (threadIdx.x == 0 && p.status) atomicOr(p.status, kStatusSmemAlign);
     return;
   }
-  const int nhs = p.G / PL::H;  // head slices per unit
+  const int nhs = p.G / tk::H;  // head slices per unit
   const int unit = blockIdx.x / nhs, hs = blockIdx.x - unit * nhs;
   const int tq = unit / p.Hkv, g = unit - tq * p.Hkv;
-  const int head0 = g * p.G + hs * PL::H;  // first query head of the CTA
+  const int head0 = g * p.G + hs * tk::H;  // first query head of the CTA
   const uint32_t sQ = smem_u32(smem + PL::oQ), sDO = smem_u32(smem + PL::oDO);
   const uint32_t sKV = smem_u32(smem + PL::oKV), sP = smem_u32(smem + PL::oP), sDS = smem_u32(smem + PL::oDS);
   int* codes = reinterpret_cast<int*>(smem + PL::oCode);
@@ -90,26 +168,28 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
   if (threadIdx.x == 0) {
     bars.abort_flag = 0;
     mbar_init(&bars.q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars.kv_full[s], 32);
+    for (int s = 0; s < PL::NST; ++s) {
+      mbar_init(&bars.kv_full[s], 1);
       mbar_init(&bars.kv_empty[s], 1);
     }
     mbar_init(&bars.s_full, 1);
     mbar_init(&bars.pds_full, 128);
     mbar_init(&bars.pds_free, 1);
-    mbar_init(&bars.dkv_full, 1);
+    mbar_init(&bars.kvq_done, 1);
     mbar_init(&bars.dkv_free, 128);
     mbar_init(&bars.dq_done, 1);
     for (int s = 0; s < 4; ++s) mbar_init(&bars.codes_full[s], 1);
     mbar_fence_init();
     tma_prefetch_desc(&mapQ);
     tma_prefetch_desc(&mapDO);
+    tma_prefetch_desc(&mapKV);
+    tma_prefetch_desc(&mapCmp);
   }
   if (warp == 1) tmem_alloc(&bars.tmem_base, PL::kAlloc);
   pdl_wait();
   pdl_trigger();
   const Unit u = make_unit(p, tq, g);
-  const int nsub = 2 * u.n_tiles;  // 32-row tiles
+  const int nsub = 2 * u.n_tiles;  // 32-row sub-tiles
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -119,35 +199,13 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
   if (warp == 0) {
     // ------------------------------------------------------------ loader
     if (lane == 0) {
-      mbar_arrive_tx(&bars.q_full, (uint32_t)((PL::NSQ + PL::NSV) * PL::H * 128));
+      mbar_arrive_tx(&bars.q_full, (uint32_t)(tk::kQBytes + tk::kDOBytes));
       const int row = tq * p.Hq + head0;
-      for (int s = 0; s < PL::NSQ; ++s) tma_load_2d(sQ + s * PL::H * 128, &mapQ, 64 * s, row, &bars.q_full);
-      for (int s = 0; s < PL::NSV; ++s) tma_load_2d(sDO + s * PL::H * 128, &mapDO, 64 * s, row, &bars.q_full);
+      for (int s = 0; s < tk::NSQ; ++s) tma_load_2d(sQ + s * tk::H * 128, &mapQ, 64 * s, row, &bars.q_full);
+      for (int s = 0; s < tk::NSV; ++s) tma_load_2d(sDO + s * tk::H * 128, &mapDO, 64 * s, row, &bars.q_full);
     }
-    for (int i = 0; i < nsub; ++i) {
-      const int st = i & 1;
-      bool ok = true;
-      if (lane == 0 && i >= 2) ok = mbar_wait(&bars.kv_empty[st], ((i >> 1) - 1) & 1, abort_flag, p.status);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      int* cd = codes + (i & 3) * PL::NK;
-      cd[lane] = resolve_row(p, u, i >> 1, 32 * (i & 1) + lane);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.codes_full[i & 3]);
-      const uint32_t stage = sKV + st * PL::kKVStage;
-#pragma unroll 4
-      for (int idx = lane; idx < PL::NK * (PL::DQK / 8); idx += 32) {
-        const int r = idx / (PL::DQK / 8), c = idx - r * (PL::DQK / 8);
-        const int code = cd[r];
-        const bf16* src = code >= 0 ? row_k_ptr(p, code, g) + c * 8 : p.k;
-        cp_async16(tk_kv_addr(stage, r, c), src, code >= 0);
-      }
-      cp_async_commit();
-      cp_async_wait_none();
-      fence_async_smem();
-      mbar_arrive(&bars.kv_full[st]);
-    }
-    cp_async_wait_none();
+    tk_load_rows<PL::NST>(p, u, g, nsub, sKV, codes, &mapKV, &mapCmp, has_cmp != 0, bars.kv_full, bars.kv_empty,
+                          bars.codes_full, abort_flag, lane);
     if (lane == 0) mbar_wait_drain(&bars.q_full, 0);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -159,44 +217,45 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
       constexpr uint32_t idDQR = idesc_bf16(64, 64, false, true);
       bool ok = mbar_wait(&bars.q_full, 0, abort_flag, p.status);
       for (int i = 0; ok && i < nsub; ++i) {
-        const int st = i & 1;
-        if (!mbar_wait(&bars.kv_full[st], (i >> 1) & 1, abort_flag, p.status)) break;
+        const int st = i % PL::NST;
+        if (!mbar_wait(&bars.kv_full[st], (i / PL::NST) & 1, abort_flag, p.status)) break;
         tc_fence_after();
-        const uint32_t kv = sKV + st * PL::kKVStage;
+        const uint32_t kv = sKV + st * tk::kKVStage;
         // S = Q KV^T (lanes 0..15), dP = dO V^T (lanes 16..31)
-        for (int kk = 0; kk < PL::DQK / 16; ++kk)
-          mma_bf16(tmem + PL::cS, sdesc(sQ + (kk >> 2) * (PL::H * 128) + (kk & 3) * 32, 16, 1024),
-                   sdesc(kv + (kk >> 2) * (PL::NK * 128) + (kk & 3) * 32, 16, 1024), idS, kk > 0);
-        for (int kk = 0; kk < PL::DV / 16; ++kk)
-          mma_bf16(tmem + (16u << 16) + PL::cS, sdesc(sDO + (kk >> 2) * (PL::H * 128) + (kk & 3) * 32, 16, 1024),
-                   sdesc(kv + (kk >> 2) * (PL::NK * 128) + (kk & 3) * 32, 16, 1024), idS, kk > 0);
+        for (int kk = 0; kk < tk::DQK / 16; ++kk)
+          mma_bf16(tmem + PL::cS, sdesc(sQ + (kk >> 2) * (tk::H * 128) + (kk & 3) * 32, 16, 1024),
+                   sdesc(kv + (kk >> 2) * (tk::NK * 128) + (kk & 3) * 32, 16, 1024), idS, kk > 0);
+        for (int kk = 0; kk < tk::DV / 16; ++kk)
+          mma_bf16(tmem + (16u << 16) + PL::cS, sdesc(sDO + (kk >> 2) * (tk::H * 128) + (kk & 3) * 32, 16, 1024),
+                   sdesc(kv + (kk >> 2) * (tk::NK * 128) + (kk & 3) * 32, 16, 1024), idS, kk > 0);
         mma_commit(&bars.s_full);
         if (!mbar_wait(&bars.pds_full, i & 1, abort_flag, p.status)) break;
         if (i > 0 && !mbar_wait(&bars.dkv_free, (i - 1) & 1, abort_flag, p.status)) break;
         tc_fence_after();
-        // dKV^T = Q^T dS + dO^T P over the 64 heads (fresh for every tile)
+        // dKV^T = Q^T dS + dO^T P over the 64 heads (fresh for every sub-tile)
         for (int t = 0; t < 4; ++t) {
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + PL::cKV + 32 * t, sdesc(sQ + 2 * t * (PL::H * 128) + kk * 2048, PL::H * 128, 1024),
-                     sdesc64(sDS + kk * 1024, PL::H * 64, 512), idKV, kk > 0);
+            mma_bf16(tmem + PL::cKV + 32 * t, sdesc(sQ + 2 * t * (tk::H * 128) + kk * 2048, tk::H * 128, 1024),
+                     sdesc64(sDS + kk * 1024, tk::H * 64, 512), idKV, kk > 0);
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + PL::cKV + 32 * t, sdesc(sDO + 2 * t * (PL::H * 128) + kk * 2048, PL::H * 128, 1024),
-                     sdesc64(sP + kk * 1024, PL::H * 64, 512), idKV, 1u);
+            mma_bf16(tmem + PL::cKV + 32 * t, sdesc(sDO + 2 * t * (tk::H * 128) + kk * 2048, tk::H * 128, 1024),
+                     sdesc64(sP + kk * 1024, tk::H * 64, 512), idKV, 1u);
         }
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + PL::cKVR, sdesc(sQ + 8 * (PL::H * 128) + kk * 2048, PL::H * 128, 1024),
-                   sdesc64(sDS + kk * 1024, PL::H * 64, 512), idKVR, kk > 0);
-        mma_commit(&bars.dkv_full);
+          mma_bf16(tmem + PL::cKVR, sdesc(sQ + 8 * (tk::H * 128) + kk * 2048, tk::H * 128, 1024),
+                   sdesc64(sDS + kk * 1024, tk::H * 64, 512), idKVR, kk > 0);
         // dQ += dS KV (KV as an MN-major B: N = dims in 64-wide slabs of 32 rows)
-        for (int kk = 0; kk < PL::NK / 16; ++kk) {
+        for (int kk = 0; kk < tk::NK / 16; ++kk) {
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
           const uint64_t a = sdesc64(sDS + kk * 32, 16, 512);
-          mma_bf16(tmem + PL::cDQ, a, sdesc(kv + kk * 2048, PL::NK * 128, 1024), idDQ, acc);
-          mma_bf16(tmem + (16u << 16) + PL::cDQ, a, sdesc(kv + 4 * (PL::NK * 128) + kk * 2048, PL::NK * 128, 1024),
+          mma_bf16(tmem + PL::cDQ, a, sdesc(kv + kk * 2048, tk::NK * 128, 1024), idDQ, acc);
+          mma_bf16(tmem + (16u << 16) + PL::cDQ, a, sdesc(kv + 4 * (tk::NK * 128) + kk * 2048, tk::NK * 128, 1024),
                    idDQ, acc);
-          mma_bf16(tmem + PL::cDQR, a, sdesc(kv + 8 * (PL::NK * 128) + kk * 2048, PL::NK * 128, 1024), idDQR, acc);
+          mma_bf16(tmem + PL::cDQR, a, sdesc(kv + 8 * (tk::NK * 128) + kk * 2048, tk::NK * 128, 1024), idDQR, acc);
         }
-        mma_commit(&bars.kv_empty[st]);
+        // the stage is released by the reduction warps, which stage dKV^T in it once
+        // every MMA of the sub-tile (dKV^T included) has completed
+        mma_commit(&bars.kvq_done);
         mma_commit(&bars.pds_free);
       }
       mma_commit(&bars.dq_done);
@@ -223,7 +282,7 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
       reg_dep16(v[0]);
       reg_dep16(v[1]);
       if (!mbar_wait(&bars.codes_full[i & 3], (i >> 2) & 1, abort_flag, p.status)) { ok = false; break; }
-      const int* cd = codes + (i & 3) * PL::NK;
+      const int* cd = codes + (i & 3) * tk::NK;
       float own[32], oth[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
@@ -232,7 +291,7 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
       }
 #pragma unroll
       for (int k = 0; k < 32; ++k) oth[k] = __shfl_xor_sync(0xffffffffu, own[k], 16);
-      // the P / dS buffers are free once the previous tile's dKV and dQ MMAs are done
+      // the P / dS buffers are free once the previous sub-tile's dKV and dQ MMAs are done
       if (i > 0 && !mbar_wait(&bars.pds_free, (i - 1) & 1, abort_flag, p.status)) { ok = false; break; }
       uint32_t pk[16];
 #pragma unroll
@@ -248,11 +307,11 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
         }
         pk[k >> 1] = pack_bf16(a0, a1);
       }
-      const uint32_t rowaddr = (is_s ? sP : sDS) + h * 64;
+      const uint32_t rb = is_s ? sP : sDS;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(rowaddr + ((c ^ ((h >> 1) & 3)) << 4)),
-                     "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(tk_p_addr(rb, h, c)), "r"(pk[4 * c]),
+                     "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
                      : "memory");
       tc_fence_before();
       fence_async_smem();
@@ -267,14 +326,14 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
     // lanes 16..31 dims 256..511
     if (ok && (nsub == 0 || mbar_wait(&bars.dq_done, 0, abort_flag, p.status))) {
       tc_fence_after();
-      bf16* dst = out.dq + row * PL::DQK + (is_s ? 0 : 256);
+      bf16* dst = out.dq + row * tk::DQK + (is_s ? 0 : 256);
       for (int c = 0; c < 256 + 64; c += 16) {
         uint32_t v[16];
         tmem_ld16(lane_base + PL::cDQ + c, v);
         tmem_wait_ld();
         reg_dep16(v);
         if (c >= 256 && !is_s) continue;  // dims 512..575 live in lanes 0..15 only
-        bf16* d = c < 256 ? dst + c : out.dq + row * PL::DQK + 512 + (c - 256);
+        bf16* d = c < 256 ? dst + c : out.dq + row * tk::DQK + 512 + (c - 256);
         uint32_t w[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e)
@@ -286,42 +345,71 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
     tc_fence_before();
   } else {
     // ------------------------------------------------------------ dKV reductions
-    const int sub = warp & 3;
+    // dKV^T leaves through the TMA engine: once every MMA of sub-tile i is done (the
+    // KV stage and dKV^T are then both free), the four warps copy dKV^T from TMEM
+    // into the KV stage as fp32 [key][dim] rows, 256 dims at a time (then the 64
+    // rope dims), and each warp's lane 0 adds eight of the key rows to the fp32
+    // accumulator with bulk reductions (cp.reduce.async.bulk ... .add.f32).  After
+    // the last pass the stage goes back to the loader.  Bulk reductions keep many
+    // bytes in flight per issuing thread, where per-thread atomics were limited by
+    // the few warps issuing them.
+    const int sub = warp & 3, rw = warp - 6;  // sub-partition; warp within the role (0..3)
     const uint32_t lane_base = tmem + ((uint32_t)(32 * sub) << 16);
     for (int i = 0; i < nsub; ++i) {
-      if (!mbar_wait(&bars.dkv_full, i & 1, abort_flag, p.status)) break;
-      if (!mbar_wait(&bars.codes_full[i & 3], (i >> 2) & 1, abort_flag, p.status)) break;
+      const int st = i % PL::NST;
+      bool ok = mbar_wait(&bars.kvq_done, i & 1, abort_flag, p.status) &&
+                mbar_wait(&bars.codes_full[i & 3], (i >> 2) & 1, abort_flag, p.status);
+      ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      const int* cd = codes + (i & 3) * PL::NK;
-      float* rowp[PL::NK];
-#pragma unroll
-      for (int k = 0; k < PL::NK; ++k) {
-        const int code = cd[k];
-        rowp[k] = code < 0 ? nullptr
-                           : ((code & kCmpFlag) ? out.dcmp_acc + ((long long)(code & ~kCmpFlag) * p.Hkv + g) * PL::DQK
-                                                : out.dk_acc + ((long long)code * p.Hkv + g) * PL::DQK);
-      }
-      // four M = 128 tiles (dims 128 t + 32 sub + lane) and the rope tile (dims
-      // 512 + 16 sub + lane, lanes 0..15)
+      const int* cd = codes + (i & 3) * tk::NK;
+      const uint32_t stage = sKV + st * tk::kKVStage;
 #pragma unroll 1
-      for (int t = 0; t < 5; ++t) {
-        uint32_t v[2][16];
-        tmem_ld16(lane_base + PL::cKV + 32 * t, v[0]);
-        tmem_ld16(lane_base + PL::cKV + 32 * t + 16, v[1]);
-        tmem_wait_ld();
-        reg_dep16(v[0]);
-        reg_dep16(v[1]);
-        if (t == 4) {
-          tc_fence_before();
-          mbar_arrive(&bars.dkv_free);  // the accumulators go back before the reductions
-        }
-        const int dim = t < 4 ? 128 * t + 32 * sub + lane : 512 + 16 * sub + lane;
-        if (t == 4 && lane >= 16) continue;
+      for (int pass = 0; pass < 3; ++pass) {
+        const int w = pass < 2 ? 256 : 64;  // dims in this pass; rows of w fp32 in the stage
+        if (ok) {
+#pragma unroll 1
+          for (int tt = 0; tt < (pass < 2 ? 2 : 1); ++tt) {
+            const int t = pass < 2 ? 2 * pass + tt : 4;
+            uint32_t v[2][16];
+            tmem_ld16(lane_base + PL::cKV + 32 * t, v[0]);
+            tmem_ld16(lane_base + PL::cKV + 32 * t + 16, v[1]);
+            tmem_wait_ld();
+            reg_dep16(v[0]);
+            reg_dep16(v[1]);
+            // this lane's dim within the pass: M = 128 tiles 128 tt + 32 sub + lane; the
+            // rope tile (M = 64) 16 sub + lane for lanes 0..15
+            const int dl = pass < 2 ? 128 * tt + 32 * sub + lane : 16 * sub + lane;
+            if (pass < 2 || lane < 16) {
 #pragma unroll
-        for (int k = 0; k < PL::NK; ++k)
-          if (rowp[k]) atomicAdd(rowp[k] + dim, __uint_as_float(v[k >> 4][k & 15]));
+              for (int k = 0; k < tk::NK; ++k)
+                asm volatile("st.shared.f32 [%0], %1;\n" ::"r"(stage + k * (w * 4) + dl * 4),
+                             "f"(__uint_as_float(v[k >> 4][k & 15]))
+                             : "memory");
+            }
+          }
+        }
+        if (pass == 2) {
+          tc_fence_before();
+          mbar_arrive(&bars.dkv_free);  // dKV^T has been read out of TMEM
+        }
+        fence_async_smem();
+        asm volatile("bar.sync 2, 128;\n" ::: "memory");
+        if (ok && lane == 0) {
+          for (int k = 8 * rw; k < 8 * rw + 8; ++k) {
+            const int code = cd[k];
+            if (code < 0) continue;
+            float* rp = (code & kCmpFlag) ? out.dcmp_acc + ((long long)(code & ~kCmpFlag) * p.Hkv + g) * tk::DQK
+                                          : out.dk_acc + ((long long)code * p.Hkv + g) * tk::DQK;
+            bulk_reduce_add_f32(rp + 256 * pass, stage + k * (w * 4), (uint32_t)(w * 4));
+          }
+          bulk_commit();
+          bulk_wait_read_all();  // the stage may be overwritten once these reads are done
+        }
+        asm volatile("bar.sync 2, 128;\n" ::: "memory");
       }
+      if (rw == 0 && lane == 0) mbar_arrive(&bars.kv_empty[st]);  // the stage goes back to the loader
     }
+    if (lane == 0) bulk_wait_all();  // every bulk reduction complete before the CTA leaves
   }
   __syncthreads();
   if (warp == 1) {
@@ -331,92 +419,70 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
   }
 }
 
-bool tk_path_built(int dqk, int dv, int shared, int G) {
-  return dqk == TkPlan::DQK && dv == TkPlan::DV && shared && G % TkPlan::H == 0;
-}
-
-cudaError_t launch_tk_bwd(const Prob& p, const float* lse, const float* delta, const bf16* d_o, const BwdOut& out,
-                          cudaStream_t st) {
-  using PL = TkPlan;
-  if (!tk_path_built(p.dqk, p.dv, p.shared, p.G)) return cudaErrorInvalidValue;
-  const long long grid = (long long)p.Tq * p.Hkv * (p.G / PL::H);
-  if (grid == 0) return cudaSuccess;
-  CUtensorMap mq, mdo;
-  if (!make_tmap_bf16(&mq, p.q, (uint64_t)p.Tq * p.Hq, PL::DQK, (uint64_t)PL::DQK * 2, PL::H) ||
-      !make_tmap_bf16(&mdo, d_o, (uint64_t)p.Tq * p.Hq, PL::DV, (uint64_t)PL::DV * 2, PL::H))
-    return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(tk_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kSmem);
-  if (e != cudaSuccess) return e;
-  mark_begin(st, kTimeBwdKV);
-  e = launch_pdl(tk_bwd_kernel, (unsigned)grid, 320, PL::kSmem, st, mq, mdo, p, lse, delta, out);
-  count_launch();
-  mark_end(st, kTimeBwdKV);
-  return e;
-}
-
-
-
-// ---------------------------------------------------------------------------
-// Token-level forward over one shared KV head (576 / 512) on tcgen05, the same
-// unit and tile decomposition: one CTA per (token, kv-head, 64 heads).
-//   S [64 x 32] = Q KV^T (lanes 0..15); online softmax in the softmax warps;
-//   O [64 x 512] += P V: dims 0..255 in lanes 0..15 and 256..511 in lanes 16..31
-//   of TMEM columns [32, 288).  The running maximum moves only when a tile's
-//   maximum exceeds it by more than 8 (a factor of 256 in the exponentials): O and
-//   the running sum are then rescaled once, after the previous P V has landed.
-// Sinks start the running state (m = sink, l = 1).
-// ---------------------------------------------------------------------------
+// ===========================================================================
+// forward
+// ===========================================================================
 struct TkFwdPlan {
-  static constexpr int DQK = 576, DV = 512, H = 64, NK = 32;
-  static constexpr int NSQ = DQK / 64;
+  static constexpr int NST = 3;
   static constexpr int oQ = 0;
-  static constexpr int kKVStage = NSQ * NK * 128;
-  static constexpr int oKV = oQ + NSQ * H * 128;
-  static constexpr int oP = oKV + 2 * kKVStage;  // P [64 heads][32 keys] bf16, 64-byte swizzle
-  static constexpr int oCode = oP + H * 64;
-  static constexpr int kSmem = oCode + 4 * NK * 4;
+  static constexpr int oKV = oQ + tk::kQBytes;
+  static constexpr int oP = oKV + NST * tk::kKVStage;  // two P buffers
+  static constexpr int oCode = oP + 2 * tk::kPBytes;
+  static constexpr int kSmem = oCode + 4 * tk::NK * 4;
   static_assert(kSmem + 1024 <= 227 * 1024, "shared memory plan too large");
-  static constexpr int cS = 0, cO = 32;
+  static_assert(oKV % 1024 == 0 && oP % 1024 == 0, "swizzled operands need 1024-byte alignment");
+  // TMEM columns: S buffers [0, 32) and [32, 64) (lanes 0..15); O [64, 320): dims
+  // 0..255 in lanes 0..15, 256..511 in lanes 16..31.
+  static constexpr int cS0 = 0, cO = 64;
   static constexpr uint32_t kAlloc = 512;
 };
 
 struct TkFwdBars {
-  uint64_t q_full, kv_full[2], kv_empty[2], s_full, p_full, pv_done;
+  uint64_t q_full, kv_full[TkFwdPlan::NST], kv_empty[TkFwdPlan::NST], s_full[2], s_free[2], p_full[2],
+      pv_done[2];
   uint64_t codes_full[4];
   uint32_t tmem_base;
   int abort_flag;
 };
 
-__global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const Prob p,
-                                                        bf16* __restrict__ O, float* __restrict__ LSE) {
+__global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ CUtensorMap mapQ,
+                                                        const __grid_constant__ CUtensorMap mapKV,
+                                                        const __grid_constant__ CUtensorMap mapCmp, const int has_cmp,
+                                                        const Prob p, bf16* __restrict__ O, float* __restrict__ LSE) {
   using PL = TkFwdPlan;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ TkFwdBars bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {
+    pdl_wait();
     if (threadIdx.x == 0 && p.status) atomicOr(p.status, kStatusSmemAlign);
     return;
   }
-  const int nhs = p.G / PL::H;
+  const int nhs = p.G / tk::H;
   const int unit = blockIdx.x / nhs, hs = blockIdx.x - unit * nhs;
   const int tq = unit / p.Hkv, g = unit - tq * p.Hkv;
-  const int head0 = g * p.G + hs * PL::H;
+  const int head0 = g * p.G + hs * tk::H;
   const uint32_t sQ = smem_u32(smem + PL::oQ), sKV = smem_u32(smem + PL::oKV), sP = smem_u32(smem + PL::oP);
   int* codes = reinterpret_cast<int*>(smem + PL::oCode);
   volatile int* abort_flag = &bars.abort_flag;
   if (threadIdx.x == 0) {
     bars.abort_flag = 0;
     mbar_init(&bars.q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars.kv_full[s], 32);
+    for (int s = 0; s < PL::NST; ++s) {
+      mbar_init(&bars.kv_full[s], 1);
       mbar_init(&bars.kv_empty[s], 1);
     }
-    mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.p_full, 128);
-    mbar_init(&bars.pv_done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars.s_full[b], 1);
+      mbar_init(&bars.s_free[b], 128);
+      mbar_init(&bars.p_full[b], 128);
+      mbar_init(&bars.pv_done[b], 1);
+    }
     for (int s = 0; s < 4; ++s) mbar_init(&bars.codes_full[s], 1);
     mbar_fence_init();
     tma_prefetch_desc(&mapQ);
+    tma_prefetch_desc(&mapKV);
+    tma_prefetch_desc(&mapCmp);
   }
   if (warp == 1) tmem_alloc(&bars.tmem_base, PL::kAlloc);
   pdl_wait();
@@ -432,62 +498,48 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
   if (warp == 0) {
     // ------------------------------------------------------------ loader
     if (lane == 0) {
-      mbar_arrive_tx(&bars.q_full, (uint32_t)(PL::NSQ * PL::H * 128));
-      for (int s = 0; s < PL::NSQ; ++s)
-        tma_load_2d(sQ + s * PL::H * 128, &mapQ, 64 * s, tq * p.Hq + head0, &bars.q_full);
+      mbar_arrive_tx(&bars.q_full, (uint32_t)tk::kQBytes);
+      for (int s = 0; s < tk::NSQ; ++s)
+        tma_load_2d(sQ + s * tk::H * 128, &mapQ, 64 * s, tq * p.Hq + head0, &bars.q_full);
     }
-    for (int i = 0; i < nsub; ++i) {
-      const int st = i & 1;
-      bool ok = true;
-      if (lane == 0 && i >= 2) ok = mbar_wait(&bars.kv_empty[st], ((i >> 1) - 1) & 1, abort_flag, p.status);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      int* cd = codes + (i & 3) * PL::NK;
-      cd[lane] = resolve_row(p, u, i >> 1, 32 * (i & 1) + lane);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.codes_full[i & 3]);
-      const uint32_t stage = sKV + st * PL::kKVStage;
-#pragma unroll 4
-      for (int idx = lane; idx < PL::NK * (PL::DQK / 8); idx += 32) {
-        const int r = idx / (PL::DQK / 8), c = idx - r * (PL::DQK / 8);
-        const int code = cd[r];
-        const bf16* src = code >= 0 ? row_k_ptr(p, code, g) + c * 8 : p.k;
-        cp_async16(tk_kv_addr(stage, r, c), src, code >= 0);
-      }
-      cp_async_commit();
-      cp_async_wait_none();
-      fence_async_smem();
-      mbar_arrive(&bars.kv_full[st]);
-    }
-    cp_async_wait_none();
+    tk_load_rows<PL::NST>(p, u, g, nsub, sKV, codes, &mapKV, &mapCmp, has_cmp != 0, bars.kv_full, bars.kv_empty,
+                          bars.codes_full, abort_flag, lane);
     if (lane == 0) mbar_wait_drain(&bars.q_full, 0);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // order: S_0, then for each i: S_{i+1} (when it exists) before P_i V_i
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(64, 32, false, false);
       constexpr uint32_t idPV = idesc_bf16(64, 256, false, true);
       bool ok = mbar_wait(&bars.q_full, 0, abort_flag, p.status);
-      for (int i = 0; ok && i < nsub; ++i) {
-        const int st = i & 1;
-        if (!mbar_wait(&bars.kv_full[st], (i >> 1) & 1, abort_flag, p.status)) break;
-        tc_fence_after();
-        const uint32_t kv = sKV + st * PL::kKVStage;
-        for (int kk = 0; kk < PL::DQK / 16; ++kk)
-          mma_bf16(tmem + PL::cS, sdesc(sQ + (kk >> 2) * (PL::H * 128) + (kk & 3) * 32, 16, 1024),
-                   sdesc(kv + (kk >> 2) * (PL::NK * 128) + (kk & 3) * 32, 16, 1024), idS, kk > 0);
-        mma_commit(&bars.s_full);
-        if (!mbar_wait(&bars.p_full, i & 1, abort_flag, p.status)) break;
-        tc_fence_after();
-        // O += P V (V = the first 512 dims of the KV rows, an MN-major B)
-        for (int kk = 0; kk < PL::NK / 16; ++kk) {
-          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          const uint64_t a = sdesc64(sP + kk * 32, 16, 512);
-          mma_bf16(tmem + PL::cO, a, sdesc(kv + kk * 2048, PL::NK * 128, 1024), idPV, acc);
-          mma_bf16(tmem + (16u << 16) + PL::cO, a, sdesc(kv + 4 * (PL::NK * 128) + kk * 2048, PL::NK * 128, 1024),
-                   idPV, acc);
+      for (int i = 0; ok && i <= nsub; ++i) {
+        if (i < nsub) {
+          const int st = i % PL::NST;
+          if (!mbar_wait(&bars.kv_full[st], (i / PL::NST) & 1, abort_flag, p.status)) break;
+          if (i >= 2 && !mbar_wait(&bars.s_free[i & 1], ((i - 2) >> 1) & 1, abort_flag, p.status)) break;
+          tc_fence_after();
+          const uint32_t kv = sKV + st * tk::kKVStage;
+          for (int kk = 0; kk < tk::DQK / 16; ++kk)
+            mma_bf16(tmem + PL::cS0 + 32 * (i & 1), sdesc(sQ + (kk >> 2) * (tk::H * 128) + (kk & 3) * 32, 16, 1024),
+                     sdesc(kv + (kk >> 2) * (tk::NK * 128) + (kk & 3) * 32, 16, 1024), idS, kk > 0);
+          mma_commit(&bars.s_full[i & 1]);
         }
-        mma_commit(&bars.kv_empty[st]);
-        mma_commit(&bars.pv_done);
+        if (i >= 1) {
+          const int j = i - 1, stj = j % PL::NST;
+          if (!mbar_wait(&bars.p_full[j & 1], (j >> 1) & 1, abort_flag, p.status)) break;
+          tc_fence_after();
+          // O += P_j V_j (V = the first 512 dims of the KV rows, an MN-major B)
+          const uint32_t kv = sKV + stj * tk::kKVStage, pb = sP + (j & 1) * tk::kPBytes;
+          for (int kk = 0; kk < tk::NK / 16; ++kk) {
+            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t a = sdesc64(pb + kk * 32, 16, 512);
+            mma_bf16(tmem + PL::cO, a, sdesc(kv + kk * 2048, tk::NK * 128, 1024), idPV, acc);
+            mma_bf16(tmem + (16u << 16) + PL::cO, a, sdesc(kv + 4 * (tk::NK * 128) + kk * 2048, tk::NK * 128, 1024),
+                     idPV, acc);
+          }
+          mma_commit(&bars.kv_empty[stj]);
+          mma_commit(&bars.pv_done[j & 1]);
+        }
       }
     }
   } else {
@@ -504,16 +556,18 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
     }
     bool ok = true;
     for (int i = 0; i < nsub; ++i) {
-      if (!mbar_wait(&bars.s_full, i & 1, abort_flag, p.status)) { ok = false; break; }
+      if (!mbar_wait(&bars.s_full[i & 1], (i >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
       tc_fence_after();
       uint32_t v[2][16];
-      tmem_ld16(lane_base + PL::cS, v[0]);
-      tmem_ld16(lane_base + PL::cS + 16, v[1]);
+      tmem_ld16(lane_base + PL::cS0 + 32 * (i & 1), v[0]);
+      tmem_ld16(lane_base + PL::cS0 + 32 * (i & 1) + 16, v[1]);
       tmem_wait_ld();
       reg_dep16(v[0]);
       reg_dep16(v[1]);
+      tc_fence_before();
+      mbar_arrive(&bars.s_free[i & 1]);  // the S buffer may take S_{i+2}
       if (!mbar_wait(&bars.codes_full[i & 3], (i >> 2) & 1, abort_flag, p.status)) { ok = false; break; }
-      const int* cd = codes + (i & 3) * PL::NK;
+      const int* cd = codes + (i & 3) * tk::NK;
       float sc[32];
       float tmax = -INFINITY;
 #pragma unroll
@@ -522,14 +576,18 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
         tmax = fmaxf(tmax, sc[k]);
       }
       tmax = __shfl_sync(0xffffffffu, tmax, lane & 15);  // the S lane's maximum for both halves
-      // the previous P V has landed (P buffer free, O stable) before P or O changes
-      if (i > 0 && !mbar_wait(&bars.pv_done, (i - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-      tc_fence_after();
+      // P buffer i & 1 is free once P_{i-2} V_{i-2} has landed
+      if (i >= 2 && !mbar_wait(&bars.pv_done[i & 1], ((i - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
       const bool grow = tmax > m + 8.f;  // the same decision in both lanes of a head
       if (__any_sync(0xffffffffu, grow)) {
         const float mn = grow ? tmax : m;
         const float f = (m == -INFINITY) ? 0.f : exp2f(m - mn);
-        if (i > 0) {
+        if (i >= 1) {
+          // O must be stable: P_{i-1} V_{i-1} has landed (and no P V is in flight)
+          if (!mbar_wait(&bars.pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, p.status)) { ok = false; }
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
           // rescale this lane's half of the head's O row (256 columns)
           for (int c = 0; c < 256; c += 16) {
             uint32_t w[16];
@@ -549,27 +607,29 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 32; k += 2) {
-          const float a0 = exp2f(sc[k] - m), a1 = exp2f(sc[k + 1] - m);
+          const float a0 = sc[k] == -INFINITY ? 0.f : exp2f(sc[k] - m);
+          const float a1 = sc[k + 1] == -INFINITY ? 0.f : exp2f(sc[k + 1] - m);
           l += a0 + a1;
           pk[k >> 1] = pack_bf16(a0, a1);
         }
-        const uint32_t rowaddr = sP + h * 64;
+        const uint32_t pb = sP + (i & 1) * tk::kPBytes;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(rowaddr + ((c ^ ((h >> 1) & 3)) << 4)),
-                       "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(tk_p_addr(pb, h, c)), "r"(pk[4 * c]),
+                       "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
                        : "memory");
       }
       tc_fence_before();
       fence_async_smem();
-      mbar_arrive(&bars.p_full);
+      mbar_arrive(&bars.p_full[i & 1]);
     }
     l = __shfl_sync(0xffffffffu, l, lane & 15);  // the S lane holds the sum
     // O / l to bf16, lse = (m + log2 l) ln 2; a row with nothing visible gets O = 0, lse = +inf
-    if (ok && (nsub == 0 || mbar_wait(&bars.pv_done, (nsub - 1) & 1, abort_flag, p.status))) {
+    const int last = nsub - 1;
+    if (ok && (nsub == 0 || mbar_wait(&bars.pv_done[last & 1], (last >> 1) & 1, abort_flag, p.status))) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      bf16* dst = O + row * PL::DV + (is_s ? 0 : 256);
+      bf16* dst = O + row * tk::DV + (is_s ? 0 : 256);
       for (int c = 0; c < 256; c += 16) {
         uint32_t w[16];
         tmem_ld16(lane_base + PL::cO + c, w);
@@ -594,18 +654,64 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
   }
 }
 
+// ===========================================================================
+// host side
+// ===========================================================================
+bool tk_path_built(int dqk, int dv, int shared, int G) {
+  return dqk == tk::DQK && dv == tk::DV && shared && G % tk::H == 0;
+}
+
+// Row-gather maps over the shared KV and cmp_kv ([rows][Hkv * 576], boxes of one
+// row x 64 columns); without compressed rows the cmp map repeats the KV map.
+static bool tk_row_maps(const Prob& p, CUtensorMap* mkv, CUtensorMap* mcmp, int* has_cmp) {
+  if (p.Tkv < 1) return false;
+  if (!make_tmap_bf16(mkv, p.k, (uint64_t)p.Tkv, (uint64_t)p.Hkv * tk::DQK, (uint64_t)p.Hkv * tk::DQK * 2, 1))
+    return false;
+  *has_cmp = 0;
+  *mcmp = *mkv;
+  if (p.cmp_topk > 0 && p.cmpk && p.Tcmp > 0) {
+    if (!make_tmap_bf16(mcmp, p.cmpk, (uint64_t)p.Tcmp, (uint64_t)p.Hkv * tk::DQK, (uint64_t)p.Hkv * tk::DQK * 2, 1))
+      return false;
+    *has_cmp = 1;
+  }
+  return true;
+}
+
+cudaError_t launch_tk_bwd(const Prob& p, const float* lse, const float* delta, const bf16* d_o, const BwdOut& out,
+                          cudaStream_t st) {
+  using PL = TkBwdPlan;
+  if (!tk_path_built(p.dqk, p.dv, p.shared, p.G)) return cudaErrorInvalidValue;
+  const long long grid = (long long)p.Tq * p.Hkv * (p.G / tk::H);
+  if (grid == 0) return cudaSuccess;
+  CUtensorMap mq, mdo, mkv, mcmp;
+  int has_cmp = 0;
+  if (!make_tmap_bf16(&mq, p.q, (uint64_t)p.Tq * p.Hq, tk::DQK, (uint64_t)tk::DQK * 2, tk::H) ||
+      !make_tmap_bf16(&mdo, d_o, (uint64_t)p.Tq * p.Hq, tk::DV, (uint64_t)tk::DV * 2, tk::H) ||
+      !tk_row_maps(p, &mkv, &mcmp, &has_cmp))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(tk_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kSmem);
+  if (e != cudaSuccess) return e;
+  mark_begin(st, kTimeBwdKV);
+  e = launch_pdl(tk_bwd_kernel, (unsigned)grid, 320, PL::kSmem, st, mq, mdo, mkv, mcmp, has_cmp, p, lse, delta, out);
+  count_launch();
+  mark_end(st, kTimeBwdKV);
+  return e;
+}
+
 cudaError_t launch_tk_fwd(const Prob& p, bf16* o, float* lse, cudaStream_t st) {
   using PL = TkFwdPlan;
   if (!tk_path_built(p.dqk, p.dv, p.shared, p.G)) return cudaErrorInvalidValue;
-  const long long grid = (long long)p.Tq * p.Hkv * (p.G / PL::H);
+  const long long grid = (long long)p.Tq * p.Hkv * (p.G / tk::H);
   if (grid == 0) return cudaSuccess;
-  CUtensorMap mq;
-  if (!make_tmap_bf16(&mq, p.q, (uint64_t)p.Tq * p.Hq, PL::DQK, (uint64_t)PL::DQK * 2, PL::H))
+  CUtensorMap mq, mkv, mcmp;
+  int has_cmp = 0;
+  if (!make_tmap_bf16(&mq, p.q, (uint64_t)p.Tq * p.Hq, tk::DQK, (uint64_t)tk::DQK * 2, tk::H) ||
+      !tk_row_maps(p, &mkv, &mcmp, &has_cmp))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(tk_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kSmem);
   if (e != cudaSuccess) return e;
   mark_begin(st, kTimeFwd);
-  e = launch_pdl(tk_fwd_kernel, (unsigned)grid, 192, PL::kSmem, st, mq, p, o, lse);
+  e = launch_pdl(tk_fwd_kernel, (unsigned)grid, 192, PL::kSmem, st, mq, mkv, mcmp, has_cmp, p, o, lse);
   count_launch();
   mark_end(st, kTimeFwd);
   return e;
