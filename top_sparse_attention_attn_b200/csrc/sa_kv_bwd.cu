@@ -466,7 +466,7 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
             for (int q2 = 0; q2 < 2; ++q2) {
               const int col = 32 * half + 16 * c + e + q2;
               const bool vis = col >= vlo && col <= vhi;
-              const float p = vis ? exp2f(__uint_as_float(sr[c][e + q2]) * a.scale_log2 - lse2) : 0.f;
+              const float p = vis ? ex2_approx(__uint_as_float(sr[c][e + q2]) * a.scale_log2 - lse2) : 0.f;
               pv[q2] = p;
               dsv[q2] = p * (__uint_as_float(dr[c][e + q2]) - dlt);
             }

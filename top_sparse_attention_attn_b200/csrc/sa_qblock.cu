@@ -443,9 +443,9 @@ __global__ void __launch_bounds__(160, NCTA) qb_kernel(const __grid_constant__ C
 // Persistent: one CTA per SM walks work items (query token, kv-head, slice of
 // up to 16 heads).  Transposed so that the tensor-core M dimension is keys or
 // value dims, which a 16-head slice could not fill:
-//   S_b^T [64 keys x 16 heads] = K_b Q^T   block b of a chunk of up to 16 usable
-//                                          blocks, M = 64 accumulators paired at
-//                                          TMEM lane offsets 0 / 16 (128 columns,
+//   S_j^T [128 keys x 16 heads] = K_j Q^T  pair j of blocks (2j, 2j + 1) of a chunk
+//                                          of up to 16 usable blocks, stacked in one
+//                                          ring stage (M = 128; 128 columns per chunk,
 //                                          two buffers)
 //   softmax over the chunk's keys per head (cross-warp reductions of the
 //   running maximum and sum; a later chunk of the same item rescales O^T)
@@ -464,7 +464,7 @@ struct BqPlan {
   static constexpr int NH = 16;   // heads per item: the N of every MMA
   static constexpr int CH = 16;   // blocks per chunk: their scores fill 128 TMEM columns
   static constexpr int NIT = 3;   // item descriptors in flight
-  static constexpr int kStage = 64 * (DQK > DV ? DQK : DV) * 2;
+  static constexpr int kStage = 128 * (DQK > DV ? DQK : DV) * 2;  // a pair of blocks
   static constexpr int kQ = (DQK / 64) * NH * 128;              // one Q slice
   static constexpr int oQ = 0;                                  // two Q slices
   static constexpr int oP = (2 * kQ + 1023) / 1024 * 1024;      // CH blocks of P^T [16][64] bf16
@@ -475,18 +475,19 @@ struct BqPlan {
   static constexpr int oRing = (oInfo + NIT * kInfo + 1023) / 1024 * 1024;
   static constexpr int kBudget = 225 * 1024;
   static constexpr int NST0 = (kBudget - oRing) / kStage;
-  static constexpr int NST = NST0 > 12 ? 12 : NST0;
+  static constexpr int NST = NST0 > 8 ? 8 : NST0;
   static constexpr int kSmem = oRing + NST * kStage;
   static constexpr int cS = 0, cO = 256;                        // S: 2 x 128 columns; O: 2 x 16
   static constexpr uint32_t kAlloc = 512;
-  static_assert(NST >= 4, "ring too small");
+  static_assert(NST >= 3, "ring too small");
   static_assert(kStage % 1024 == 0 && oP % 1024 == 0 && oRing % 1024 == 0, "swizzle alignment");
   static_assert(kSmem + 1024 <= 227 * 1024, "shared memory plan too large");
 };
 
 struct BqBars {
-  uint64_t info_full[3], info_free[3], q_full[2], q_empty[2], kv_full[12], kv_empty[12];
-  uint64_t s_full[2], s_free[2], p_full, pv_done, o_free[2];
+  uint64_t info_full[3], info_free[3], q_full[2], q_empty[2], kv_full[8], kv_empty[8];
+  uint64_t s_full[2], s_free[2], p_full, pv_done, o_full[2], o_free[2], stats_full[2];
+  float stat_m[2][16], stat_l[2][16];  // an item's running maximum and sum per head, softmax -> epilogue
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -498,7 +499,7 @@ struct BqWalk {
 };
 
 template <int DQK, int DV>
-__global__ void __launch_bounds__(192, 1) bq_fwd_kernel(const __grid_constant__ CUtensorMap mapQ,
+__global__ void __launch_bounds__(320, 1) bq_fwd_kernel(const __grid_constant__ CUtensorMap mapQ,
                                                         const __grid_constant__ CUtensorMap mapK,
                                                         const __grid_constant__ CUtensorMap mapV, const QbArgs a) {
   using PL = BqPlan<DQK, DV>;
@@ -534,14 +535,16 @@ __global__ void __launch_bounds__(192, 1) bq_fwd_kernel(const __grid_constant__ 
     bars.abort_flag = 0;
     for (int s = 0; s < NIT; ++s) {
       mbar_init(&bars.info_full[s], 32);
-      mbar_init(&bars.info_free[s], 1 + 128);
+      mbar_init(&bars.info_free[s], 1 + 128 + 128);  // MMA thread, softmax and epilogue warps
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.q_full[s], 1);
       mbar_init(&bars.q_empty[s], 1);
       mbar_init(&bars.s_full[s], 1);
       mbar_init(&bars.s_free[s], 128);
+      mbar_init(&bars.o_full[s], 1);
       mbar_init(&bars.o_free[s], 128);
+      mbar_init(&bars.stats_full[s], 128);
     }
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bars.kv_full[s], 1);
@@ -568,20 +571,24 @@ __global__ void __launch_bounds__(192, 1) bq_fwd_kernel(const __grid_constant__ 
     bool ok = true;
     int pv_slot = -1, pv_first = 0, pv_nb = 0, pv_row0 = 0, pv_g = 0;  // the chunk whose V is pending
     auto load_blocks = [&](bool is_v, int slot, int first, int nb, int kv0, int g) {
-      for (int b = 0; ok && b < nb; ++b, ++t) {
-        const int st = t % NST;
+      // pairs of blocks: block 2j in rows 0..63 of the stage's slabs, 2j + 1 in rows 64..127
+      for (int j = 0; ok && 2 * j < nb; ++j, ++t) {
+        const int st = t % NST, nbp = min(2, nb - 2 * j);
         if (lane == 0) {
           if (t >= NST && !mbar_wait(&bars.kv_empty[st], ((t / NST) - 1) & 1, abort_flag, a.status)) {
             ok = false;
           } else {
             const uint32_t stage = sRing + st * PL::kStage;
-            const int row = kv0 + 64 * info_xs(slot)[first + b];
-            if (!is_v) {
-              mbar_arrive_tx(&bars.kv_full[st], (uint32_t)(64 * DQK * 2));
-              for (int s = 0; s < DQK / 64; ++s) tma_load_2d(stage + s * 8192, &mapK, g * DQK + 64 * s, row, &bars.kv_full[st]);
-            } else {
-              mbar_arrive_tx(&bars.kv_full[st], (uint32_t)(64 * DV * 2));
-              for (int s = 0; s < DV / 64; ++s) tma_load_2d(stage + s * 8192, &mapV, g * DV + 64 * s, row, &bars.kv_full[st]);
+            const int D = is_v ? DV : DQK;
+            mbar_arrive_tx(&bars.kv_full[st], (uint32_t)(nbp * 64 * D * 2));
+            for (int e = 0; e < nbp; ++e) {
+              const int row = kv0 + 64 * info_xs(slot)[first + 2 * j + e];
+              for (int s = 0; s < D / 64; ++s) {
+                if (is_v)
+                  tma_load_2d(stage + s * 16384 + e * 8192, &mapV, g * DV + 64 * s, row, &bars.kv_full[st]);
+                else
+                  tma_load_2d(stage + s * 16384 + e * 8192, &mapK, g * DQK + 64 * s, row, &bars.kv_full[st]);
+              }
             }
           }
         }
@@ -651,27 +658,33 @@ __global__ void __launch_bounds__(192, 1) bq_fwd_kernel(const __grid_constant__ 
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(64, PL::NH, false, false);
+      constexpr uint32_t idS = idesc_bf16(128, PL::NH, false, false);
       constexpr uint32_t idO = idesc_bf16(DV >= 128 ? 128 : 64, PL::NH, true, false);
       int t = 0, c = 0, qk = 0, ok_items = 0;
       bool ok = true;
       // the chunk whose P V is pending: its chunk number, blocks, O buffer and whether it opens its item
       int pv_c = -1, pv_nb = 0, pv_ob = 0;
-      bool pv_first = false;
+      bool pv_first = false, pv_last = false;
       auto issue_pv = [&]() {
         if (!mbar_wait(&bars.p_full, pv_c & 1, abort_flag, a.status)) { ok = false; return; }
         tc_fence_after();
-        for (int b = 0; ok && b < pv_nb; ++b, ++t) {
+        for (int j = 0; ok && 2 * j < pv_nb; ++j, ++t) {
           const int st = t % NST;
           if (!mbar_wait(&bars.kv_full[st], (t / NST) & 1, abort_flag, a.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t stage = sRing + st * PL::kStage;
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + PL::cO + 16 * pv_ob, sdesc(stage + kk * 2048, 8192, 1024),
-                     sdesc(sP + b * 2048 + kk * 32, 16, 1024), idO, (!pv_first || b > 0 || kk > 0) ? 1u : 0u);
+          for (int e = 0; e < 2 && 2 * j + e < pv_nb; ++e) {
+            const int b = 2 * j + e;
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(tmem + PL::cO + 16 * pv_ob, sdesc(stage + e * 8192 + kk * 2048, 16384, 1024),
+                       sdesc(sP + b * 2048 + kk * 32, 16, 1024), idO, (!pv_first || b > 0 || kk > 0) ? 1u : 0u);
+          }
           mma_commit(&bars.kv_empty[st]);
         }
-        if (ok) mma_commit(&bars.pv_done);
+        if (ok) {
+          mma_commit(&bars.pv_done);
+          if (pv_last) mma_commit(&bars.o_full[pv_ob]);  // the item's O^T is final
+        }
       };
       for (int k = 0; ok; ++k) {
         const int slot = k % NIT;
@@ -693,14 +706,14 @@ __global__ void __launch_bounds__(192, 1) bq_fwd_kernel(const __grid_constant__ 
           const int nb = min(CH, n - cc * CH);
           const int sb = c & 1;
           if (c >= 2 && !mbar_wait(&bars.s_free[sb], ((c >> 1) - 1) & 1, abort_flag, a.status)) { ok = false; break; }
-          for (int b = 0; b < nb; ++b, ++t) {
+          for (int j = 0; 2 * j < nb; ++j, ++t) {
             const int st = t % NST;
             if (!mbar_wait(&bars.kv_full[st], (t / NST) & 1, abort_flag, a.status)) { ok = false; break; }
             tc_fence_after();
             const uint32_t stage = sRing + st * PL::kStage;
-            const uint32_t d = tmem + PL::cS + 128 * sb + 16 * (b >> 1) + ((uint32_t)(16 * (b & 1)) << 16);
+            const uint32_t d = tmem + PL::cS + 128 * sb + 16 * j;
             for (int kk = 0; kk < DQK / 16; ++kk)
-              mma_bf16(d, sdesc(stage + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+              mma_bf16(d, sdesc(stage + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                        sdesc(sQ + qs * PL::kQ + (kk >> 2) * (PL::NH * 128) + (kk & 3) * 32, 16, 1024), idS, kk > 0);
             mma_commit(&bars.kv_empty[st]);
           }
@@ -712,18 +725,20 @@ __global__ void __launch_bounds__(192, 1) bq_fwd_kernel(const __grid_constant__ 
           pv_nb = nb;
           pv_ob = ob;
           pv_first = cc == 0;
+          pv_last = cc == nch - 1;
         }
         ++qk;
         ++ok_items;
       }
       if (ok && pv_c >= 0) issue_pv();
     }
-  } else {
-    // ------------------------------------------------------------ softmax + epilogue
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ softmax
     // Every chunk runs both named barriers in all four warps, also after a wait gave
     // up (the work is skipped, the barriers are not), so no warp is left at one.
     const int sub = warp & 3;
-    const int par = lane >> 4, key = (lane & 15) + 16 * sub;  // block parity and key of this TMEM lane
+    // TMEM lane 32 sub + lane holds key (32 sub + lane) of a pair: block 2j + par, key
+    const int par = sub >> 1, key = 32 * (sub & 1) + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * sub) << 16);
     const int tid = threadIdx.x - 64;
     int c = 0, ok_items = 0;
@@ -831,7 +846,7 @@ __global__ void __launch_bounds__(192, 1) bq_fwd_kernel(const __grid_constant__ 
             const uint32_t pb = sP + b * 2048 + (key & 7) * 2;
 #pragma unroll
             for (int h = 0; h < 16; ++h) {
-              const float pv = on ? exp2f(__uint_as_float(v[h]) * a.scale_log2 - m[h]) : 0.f;
+              const float pv = on ? ex2_approx(fmaf(__uint_as_float(v[h]), a.scale_log2, -m[h])) : 0.f;
               sm[h] += pv;
               const __nv_bfloat16 pbf = __float2bfloat16_rn(pv);
               const uint16_t bits = *reinterpret_cast<const uint16_t*>(&pbf);
@@ -860,37 +875,79 @@ __global__ void __launch_bounds__(192, 1) bq_fwd_kernel(const __grid_constant__ 
 #pragma unroll
         for (int h = 0; h < 16; ++h) l[h] += (redl[h] + redl[16 + h]) + (redl[32 + h] + redl[48 + h]);
       }
-      // epilogue: O = O^T / l (this thread's value dim, every head), lse per head
-      bool have_o = n == 0;
-      if (n > 0) have_o = __all_sync(0xffffffffu, ok && mbar_wait(&bars.pv_done, (c - 1) & 1, abort_flag, a.status));
-      if (have_o) {
-        tc_fence_after();
-        uint32_t w[16];
-        if (n > 0) {
-          tmem_ld16(lane_base + PL::cO + 16 * ob, w);
-          tmem_wait_ld();
-          reg_dep16(w);
-        }
-        // O^T rows: M = 128 puts value dim d in lane d; M = 64 puts it in lane (d % 16) + 32 (d / 16)
-        const int dvi = DV >= 128 ? 32 * sub + lane : (lane < 16 ? 16 * sub + lane : -1);
-        if (dvi >= 0) {
-#pragma unroll
-          for (int h = 0; h < 16; ++h) {
-            if (h < nh) {
-              const float val = (n == 0 || l[h] <= 0.f) ? 0.f : __uint_as_float(w[h]) / l[h];
-              a.o[((long long)tq * a.Hq + h0 + h) * DV + dvi] = __float2bfloat16_rn(val);
-            }
-          }
-        }
-        if (tid < nh) {
+      // the item's per-head maximum and sum go to the epilogue warps
+      if (n > 0) {
+        if (tid < 16) {
           float lt = l[0], mt = m[0];
 #pragma unroll
           for (int h = 1; h < 16; ++h) {
             lt = tid == h ? l[h] : lt;
             mt = tid == h ? m[h] : mt;
           }
-          a.lse[(long long)tq * a.Hq + h0 + tid] = lt > 0.f ? (mt + log2f(lt)) * kLn2Qb : INFINITY;
+          bars.stat_m[ob][tid] = mt;
+          bars.stat_l[ob][tid] = lt;
         }
+        mbar_arrive(&bars.stats_full[ob]);
+        ++ok_items;
+      }
+      mbar_arrive(&bars.info_free[slot]);
+    }
+    tc_fence_before();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 6..9)
+    // O = O^T / l for this thread's value dim and every head, lse per head; items
+    // without blocks get O = 0 and the sink-only lse.  Runs beside the softmax of the
+    // next item.
+    const int sub = warp & 3;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * sub) << 16);
+    const int tid = threadIdx.x - 192;
+    // O^T rows: M = 128 puts value dim d in lane d; M = 64 puts it in lane (d % 16) + 32 (d / 16)
+    const int dvi = DV >= 128 ? 32 * sub + lane : (lane < 16 ? 16 * sub + lane : -1);
+    int ok_items = 0;
+    bool ok = true;
+    for (int k = 0;; ++k) {
+      const int slot = k % NIT;
+      if (!mbar_wait(&bars.info_full[slot], (k / NIT) & 1, abort_flag, a.status)) break;
+      const int n = *info_n(slot);
+      if (n < 0) break;
+      int tq, g, h0, nh;
+      item_of(k, &tq, &g, &h0, &nh);
+      const int ob = ok_items & 1;
+      float w[16], mt = -INFINITY, lt = 0.f;
+      if (n > 0) {
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars.o_full[ob], (ok_items >> 1) & 1, abort_flag, a.status) &&
+                                         mbar_wait(&bars.stats_full[ob], (ok_items >> 1) & 1, abort_flag, a.status));
+        if (ok) {
+          tc_fence_after();
+          uint32_t v[16];
+          tmem_ld16(lane_base + PL::cO + 16 * ob, v);
+          tmem_wait_ld();
+          reg_dep16(v);
+#pragma unroll
+          for (int h = 0; h < 16; ++h) {
+            const float lh = bars.stat_l[ob][h];
+            w[h] = lh > 0.f ? __uint_as_float(v[h]) / lh : 0.f;
+          }
+          if (tid < nh) {
+            mt = bars.stat_m[ob][tid];
+            lt = bars.stat_l[ob][tid];
+          }
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < 16; ++h) w[h] = 0.f;
+        if (tid < nh && a.sinks) {
+          mt = __ldg(a.sinks + h0 + tid) * kLog2eQb;
+          lt = 1.f;
+        }
+      }
+      if (ok) {
+        if (dvi >= 0) {
+#pragma unroll
+          for (int h = 0; h < 16; ++h)
+            if (h < nh) a.o[((long long)tq * a.Hq + h0 + h) * DV + dvi] = __float2bfloat16_rn(w[h]);
+        }
+        if (tid < nh) a.lse[(long long)tq * a.Hq + h0 + tid] = lt > 0.f ? (mt + log2f(lt)) * kLn2Qb : INFINITY;
       }
       if (n > 0) {
         tc_fence_before();
@@ -927,7 +984,7 @@ static cudaError_t bq_launch_t(const QbArgs& a, const void* k, const void* v, cu
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long grid = items < sms ? items : sms;
   mark_begin(st, kTimeFwd);
-  kern<<<(unsigned)grid, 192, PL::kSmem, st>>>(mq, mk, mv, a);
+  kern<<<(unsigned)grid, 320, PL::kSmem, st>>>(mq, mk, mv, a);
   count_launch();
   mark_end(st, kTimeFwd);
   return cudaGetLastError();

@@ -66,14 +66,27 @@ __device__ __forceinline__ uint32_t tk_p_addr(uint32_t base, int h, int c) {
   return base + h * 64 + ((c ^ ((h >> 1) & 3)) << 4);
 }
 
+// 16-byte piece c (0..71) of row r of a 32-row sub-tile stage: NSQ slabs of 32
+// rows x 128 bytes, 128-byte swizzle (the layout a TMA box or gather writes).
+__device__ __forceinline__ uint32_t tk_kv_addr(uint32_t stage, int r, int c) {
+  return stage + (c >> 3) * (tk::NK * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+}
+
 // Loader (warp 0, every lane): the row codes of each 32-row sub-tile (lane = row)
-// into the 4-deep codes ring, then the rows themselves by TMA row gathers into
-// stage i % NST.  Stage reuse waits for kv_empty; on abort the warp stops issuing.
-// Before returning it waits (bounded) for every gather it issued to land.
-template <int NST>
+// into the 4-deep codes ring, then the rows themselves into stage i % NST.  The
+// first TMA_SLABS 64-column slabs of every row arrive by TMA row gathers
+// (tile::gather4, four rows per copy, 512 bytes each); the rest by 16-byte
+// cp.async copies through the load/store path.  The TMA engine handles about one
+// gather per 70 cycles, so splitting the slabs keeps both paths busy.  kv_full
+// expects the gathered bytes (one arrival) plus one arrival per lane once its
+// copies have landed (TMA_SLABS < NSQ).  The next sub-tile's indices are loaded
+// while the current one is issued.  Stage reuse waits for kv_empty; on abort the
+// warp stops issuing.  Before returning it waits (bounded) for every copy to land.
+template <int NST, int TMA_SLABS>
 __device__ void tk_load_rows(const Prob& p, const Unit& u, int g, int nsub, uint32_t sKV, int* codes,
                              const CUtensorMap* mapKV, const CUtensorMap* mapCmp, bool has_cmp, uint64_t* kv_full,
                              uint64_t* kv_empty, uint64_t* codes_full, volatile int* abort_flag, int lane) {
+  constexpr int CP_PIECES = (tk::NSQ - TMA_SLABS) * 8;  // 16-byte pieces of a row copied by cp.async
   int x_next = nsub > 0 ? slot_index(p, u, 0, lane) : -1;
   int issued = 0;
   for (int i = 0; i < nsub; ++i) {
@@ -86,27 +99,45 @@ __device__ void tk_load_rows(const Prob& p, const Unit& u, int g, int nsub, uint
     if (!ok) break;
     const int code = resolve_row_x(p, u, tile, r, x);
     codes[(i & 3) * tk::NK + lane] = code;
-    const bool cmp_tile = tile >= u.n_ori_tiles && has_cmp;
-    const int y = code >= 0 ? (code & ~kCmpFlag) : 0;  // invisible rows load row 0 (masked later)
     __syncwarp();
-    if (lane == 0) {
-      mbar_arrive(&codes_full[i & 3]);
-      mbar_arrive_tx(&kv_full[st], (uint32_t)tk::kKVStage);
-    }
-    __syncwarp();
-    const int q4 = lane & 7;
-    const int y0 = __shfl_sync(0xffffffffu, y, 4 * q4), y1 = __shfl_sync(0xffffffffu, y, 4 * q4 + 1);
-    const int y2 = __shfl_sync(0xffffffffu, y, 4 * q4 + 2), y3 = __shfl_sync(0xffffffffu, y, 4 * q4 + 3);
-    if (lane < 8) {
-      const CUtensorMap* map = cmp_tile ? mapCmp : mapKV;
-      const uint32_t dst = sKV + st * tk::kKVStage + q4 * 4 * 128;
+    if (lane == 0) mbar_arrive(&codes_full[i & 3]);
+    const uint32_t stage = sKV + st * tk::kKVStage;
+    if (TMA_SLABS > 0) {
+      const bool cmp_tile = tile >= u.n_ori_tiles && has_cmp;
+      const int y = code >= 0 ? (code & ~kCmpFlag) : 0;  // invisible rows load row 0 (masked later)
+      if (lane == 0) mbar_arrive_tx(&kv_full[st], (uint32_t)(TMA_SLABS * tk::NK * 128));
+      __syncwarp();
+      const int q4 = lane & 7;
+      const int y0 = __shfl_sync(0xffffffffu, y, 4 * q4), y1 = __shfl_sync(0xffffffffu, y, 4 * q4 + 1);
+      const int y2 = __shfl_sync(0xffffffffu, y, 4 * q4 + 2), y3 = __shfl_sync(0xffffffffu, y, 4 * q4 + 3);
+      if (lane < 8) {
+        const CUtensorMap* map = cmp_tile ? mapCmp : mapKV;
+        const uint32_t dst = stage + q4 * 4 * 128;
 #pragma unroll
-      for (int s = 0; s < tk::NSQ; ++s) tma_gather4(dst + s * (tk::NK * 128), map, g * tk::DQK + 64 * s, y0, y1, y2, y3, &kv_full[st]);
+        for (int s = 0; s < TMA_SLABS; ++s)
+          tma_gather4(dst + s * (tk::NK * 128), map, g * tk::DQK + 64 * s, y0, y1, y2, y3, &kv_full[st]);
+      }
+    }
+    if (CP_PIECES > 0) {
+      // lanes take consecutive 16-byte pieces of one row; invisible rows are zero-filled
+      const int* cd = codes + (i & 3) * tk::NK;
+#pragma unroll 4
+      for (int idx = lane; idx < tk::NK * CP_PIECES; idx += 32) {
+        const int rr = idx / CP_PIECES, c = TMA_SLABS * 8 + (idx - rr * CP_PIECES);
+        const int cr = cd[rr];
+        const bf16* src = cr >= 0 ? row_k_ptr(p, cr, g) + c * 8 : p.k;
+        cp_async16(tk_kv_addr(stage, rr, c), src, cr >= 0);
+      }
+      cp_async_commit();
+      cp_async_wait_none();
+      fence_async_smem();  // the copies -> visible to the tensor core
+      mbar_arrive(&kv_full[st]);
     }
     issued = i + 1;
   }
-  if (lane == 0)
+  if (TMA_SLABS > 0 && lane == 0)
     for (int i = issued > NST ? issued - NST : 0; i < issued; ++i) mbar_wait_drain(&kv_full[i % NST], (i / NST) & 1);
+  if (CP_PIECES > 0) cp_async_wait_none();
 }
 
 // ===========================================================================
@@ -114,6 +145,9 @@ __device__ void tk_load_rows(const Prob& p, const Unit& u, int g, int nsub, uint
 // ===========================================================================
 struct TkBwdPlan {
   static constexpr int NST = 2;
+  // slabs of each KV row by TMA gather (the rest by cp.async); the TMA engine also
+  // carries the Q / dO boxes and the dKV bulk reductions
+  static constexpr int kTmaSlabs = 9;
   static constexpr int oQ = 0;
   static constexpr int oDO = oQ + tk::kQBytes;
   static constexpr int oKV = oDO + tk::kDOBytes;
@@ -169,7 +203,7 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
     bars.abort_flag = 0;
     mbar_init(&bars.q_full, 1);
     for (int s = 0; s < PL::NST; ++s) {
-      mbar_init(&bars.kv_full[s], 1);
+      mbar_init(&bars.kv_full[s], (PL::kTmaSlabs > 0 ? 1 : 0) + (PL::kTmaSlabs < tk::NSQ ? 32 : 0));
       mbar_init(&bars.kv_empty[s], 1);
     }
     mbar_init(&bars.s_full, 1);
@@ -204,8 +238,8 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
       for (int s = 0; s < tk::NSQ; ++s) tma_load_2d(sQ + s * tk::H * 128, &mapQ, 64 * s, row, &bars.q_full);
       for (int s = 0; s < tk::NSV; ++s) tma_load_2d(sDO + s * tk::H * 128, &mapDO, 64 * s, row, &bars.q_full);
     }
-    tk_load_rows<PL::NST>(p, u, g, nsub, sKV, codes, &mapKV, &mapCmp, has_cmp != 0, bars.kv_full, bars.kv_empty,
-                          bars.codes_full, abort_flag, lane);
+    tk_load_rows<PL::NST, PL::kTmaSlabs>(p, u, g, nsub, sKV, codes, &mapKV, &mapCmp, has_cmp != 0, bars.kv_full,
+                                          bars.kv_empty, bars.codes_full, abort_flag, lane);
     if (lane == 0) mbar_wait_drain(&bars.q_full, 0);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -282,12 +316,24 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
       reg_dep16(v[0]);
       reg_dep16(v[1]);
       if (!mbar_wait(&bars.codes_full[i & 3], (i >> 2) & 1, abort_flag, p.status)) { ok = false; break; }
-      const int* cd = codes + (i & 3) * tk::NK;
+      // the sub-tile's visible keys as a bit mask (eight 16-byte reads of the codes)
+      unsigned visk = 0;
+      {
+        const int4* cd4 = reinterpret_cast<const int4*>(codes + (i & 3) * tk::NK);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int4 c4 = cd4[q];
+          visk |= (c4.x >= 0 ? 1u : 0u) << (4 * q);
+          visk |= (c4.y >= 0 ? 1u : 0u) << (4 * q + 1);
+          visk |= (c4.z >= 0 ? 1u : 0u) << (4 * q + 2);
+          visk |= (c4.w >= 0 ? 1u : 0u) << (4 * q + 3);
+        }
+      }
       float own[32], oth[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
         const float x = __uint_as_float(v[k >> 4][k & 15]);
-        own[k] = is_s ? (cd[k] >= 0 ? exp2f(x * p.scale_log2 - lse2) : 0.f) : x;  // P or dP
+        own[k] = is_s ? (((visk >> k) & 1u) ? ex2_approx(fmaf(x, p.scale_log2, -lse2)) : 0.f) : x;  // P or dP
       }
 #pragma unroll
       for (int k = 0; k < 32; ++k) oth[k] = __shfl_xor_sync(0xffffffffu, own[k], 16);
@@ -347,9 +393,9 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
     // ------------------------------------------------------------ dKV reductions
     // dKV^T leaves through the TMA engine: once every MMA of sub-tile i is done (the
     // KV stage and dKV^T are then both free), the four warps copy dKV^T from TMEM
-    // into the KV stage as fp32 [key][dim] rows, 256 dims at a time (then the 64
-    // rope dims), and each warp's lane 0 adds eight of the key rows to the fp32
-    // accumulator with bulk reductions (cp.reduce.async.bulk ... .add.f32).  After
+    // into the KV stage as fp32 [key][dim] rows, 288 dims at a time (a full stage),
+    // and each warp's lane 0 adds eight of the key rows to the fp32 accumulator with
+    // bulk reductions (cp.reduce.async.bulk ... .add.f32).  After
     // the last pass the stage goes back to the loader.  Bulk reductions keep many
     // bytes in flight per issuing thread, where per-thread atomics were limited by
     // the few warps issuing them.
@@ -364,31 +410,32 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
       const int* cd = codes + (i & 3) * tk::NK;
       const uint32_t stage = sKV + st * tk::kKVStage;
 #pragma unroll 1
-      for (int pass = 0; pass < 3; ++pass) {
-        const int w = pass < 2 ? 256 : 64;  // dims in this pass; rows of w fp32 in the stage
+      for (int pass = 0; pass < 2; ++pass) {
+        // pass 0: dims 0..287 (tiles 0, 1 and the first 32 dims of tile 2); pass 1: dims
+        // 288..575 (the rest of tile 2, tile 3 and the rope tile); rows of 288 fp32
         if (ok) {
 #pragma unroll 1
-          for (int tt = 0; tt < (pass < 2 ? 2 : 1); ++tt) {
-            const int t = pass < 2 ? 2 * pass + tt : 4;
+          for (int t = 2 * pass; t < 2 * pass + 3; ++t) {
             uint32_t v[2][16];
             tmem_ld16(lane_base + PL::cKV + 32 * t, v[0]);
             tmem_ld16(lane_base + PL::cKV + 32 * t + 16, v[1]);
             tmem_wait_ld();
             reg_dep16(v[0]);
             reg_dep16(v[1]);
-            // this lane's dim within the pass: M = 128 tiles 128 tt + 32 sub + lane; the
-            // rope tile (M = 64) 16 sub + lane for lanes 0..15
-            const int dl = pass < 2 ? 128 * tt + 32 * sub + lane : 16 * sub + lane;
-            if (pass < 2 || lane < 16) {
+            // this lane's dim: M = 128 tiles 128 t + 32 sub + lane; the rope tile (M = 64)
+            // 512 + 16 sub + lane for lanes 0..15
+            const int dim = t < 4 ? 128 * t + 32 * sub + lane : (lane < 16 ? 512 + 16 * sub + lane : -1);
+            const int dl = dim - 288 * pass;
+            if (dl >= 0 && dl < 288) {
 #pragma unroll
               for (int k = 0; k < tk::NK; ++k)
-                asm volatile("st.shared.f32 [%0], %1;\n" ::"r"(stage + k * (w * 4) + dl * 4),
+                asm volatile("st.shared.f32 [%0], %1;\n" ::"r"(stage + k * (288 * 4) + dl * 4),
                              "f"(__uint_as_float(v[k >> 4][k & 15]))
                              : "memory");
             }
           }
         }
-        if (pass == 2) {
+        if (pass == 1) {
           tc_fence_before();
           mbar_arrive(&bars.dkv_free);  // dKV^T has been read out of TMEM
         }
@@ -400,7 +447,7 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
             if (code < 0) continue;
             float* rp = (code & kCmpFlag) ? out.dcmp_acc + ((long long)(code & ~kCmpFlag) * p.Hkv + g) * tk::DQK
                                           : out.dk_acc + ((long long)code * p.Hkv + g) * tk::DQK;
-            bulk_reduce_add_f32(rp + 256 * pass, stage + k * (w * 4), (uint32_t)(w * 4));
+            bulk_reduce_add_f32(rp + 288 * pass, stage + k * (288 * 4), 288 * 4);
           }
           bulk_commit();
           bulk_wait_read_all();  // the stage may be overwritten once these reads are done
@@ -424,6 +471,7 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
 // ===========================================================================
 struct TkFwdPlan {
   static constexpr int NST = 3;
+  static constexpr int kTmaSlabs = 9;  // every slab by TMA gather (measured faster than a cp.async share)
   static constexpr int oQ = 0;
   static constexpr int oKV = oQ + tk::kQBytes;
   static constexpr int oP = oKV + NST * tk::kKVStage;  // two P buffers
@@ -469,7 +517,7 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
     bars.abort_flag = 0;
     mbar_init(&bars.q_full, 1);
     for (int s = 0; s < PL::NST; ++s) {
-      mbar_init(&bars.kv_full[s], 1);
+      mbar_init(&bars.kv_full[s], (PL::kTmaSlabs > 0 ? 1 : 0) + (PL::kTmaSlabs < tk::NSQ ? 32 : 0));
       mbar_init(&bars.kv_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -502,8 +550,8 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
       for (int s = 0; s < tk::NSQ; ++s)
         tma_load_2d(sQ + s * tk::H * 128, &mapQ, 64 * s, tq * p.Hq + head0, &bars.q_full);
     }
-    tk_load_rows<PL::NST>(p, u, g, nsub, sKV, codes, &mapKV, &mapCmp, has_cmp != 0, bars.kv_full, bars.kv_empty,
-                          bars.codes_full, abort_flag, lane);
+    tk_load_rows<PL::NST, PL::kTmaSlabs>(p, u, g, nsub, sKV, codes, &mapKV, &mapCmp, has_cmp != 0, bars.kv_full,
+                                          bars.kv_empty, bars.codes_full, abort_flag, lane);
     if (lane == 0) mbar_wait_drain(&bars.q_full, 0);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -607,8 +655,8 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 32; k += 2) {
-          const float a0 = sc[k] == -INFINITY ? 0.f : exp2f(sc[k] - m);
-          const float a1 = sc[k + 1] == -INFINITY ? 0.f : exp2f(sc[k + 1] - m);
+          const float a0 = sc[k] == -INFINITY ? 0.f : ex2_approx(sc[k] - m);
+          const float a1 = sc[k + 1] == -INFINITY ? 0.f : ex2_approx(sc[k + 1] - m);
           l += a0 + a1;
           pk[k >> 1] = pack_bf16(a0, a1);
         }
