@@ -361,13 +361,14 @@ def aggregate_rate(units_per_rank: float, world: int, max_ms: float) -> float:
 
 
 KERNEL_NAMES = {
-    1: "qb_kernel (query-stationary block forward)",
+    1: "qb_kernel (query-stationary block forward, TMA-fed, mma.sync tiles)",
     2: "tk_fwd_kernel (token-level tcgen05 forward)",
     3: "fwd_kernel (generic forward)",
     4: "kv_bwd_kernel (key-stationary dK/dV/dQ, dQ by fp32 atomics)",
     5: "kv_bwd_kernel (key-stationary dK/dV) + qb_kernel<dQ> pass",
     6: "tk_bwd_kernel (token-level tcgen05 backward)",
     7: "bwd_kernel (generic fused backward)",
+    8: "bq_fwd_kernel (block forward on tcgen05)",
 }
 
 
@@ -575,7 +576,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     w = workload_of(args)
     flags = 0
     for f in filter(None, args.flags.split(",")):
-        flags |= {"dq_separate": L.SA_FLAG_DQ_SEPARATE, "query_stationary": L.SA_FLAG_QUERY_STATIONARY_BWD}[f]
+        flags |= {"dq_separate": L.SA_FLAG_DQ_SEPARATE, "query_stationary": L.SA_FLAG_QUERY_STATIONARY_BWD,
+                  "fwd_block_tc": L.SA_FLAG_FWD_BLOCK_TC}[f]
     sa, t, inputs, work = setup_problem(w, dev, flags, host_dense=False)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
@@ -769,7 +771,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager calls instead of CUDA-graph replays")
     ap.add_argument("--no-per-workload", action="store_true", help="skip the other workloads' figures")
-    ap.add_argument("--flags", default="", help="backward variant for measurements: dq_separate | query_stationary")
+    ap.add_argument("--flags", default="", help="kernel variants for measurements: dq_separate | query_stationary | fwd_block_tc")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -136,16 +136,26 @@ typedef enum sa_dtype { SA_DTYPE_BF16 = 0, SA_DTYPE_FP16 = 1 } sa_dtype;
 #define SA_FLAG_DQ_SEPARATE 4u  /* key-stationary backward: take dQ from a separate
                                    query-stationary pass instead of atomics; honoured
                                    only when topk <= 256 (otherwise ignored) */
+/* Forward kernel choice for block-level selection (64-row blocks, BSND, equal
+ * lengths, separate K and V, no sinks, topk <= 256).  The default is the
+ * TMA-fed query-stationary kernel with mma.sync tiles: that forward is bound by
+ * gathering the selected blocks from L2 (every 16-head item streams its blocks'
+ * K and V once), which the warp-level MMAs keep up with.  This flag selects the
+ * tcgen05 version instead (scores and output in TMEM, M = 128 key pairs against
+ * the 16 heads of an item); it computes the same result and measured slower. */
+#define SA_FLAG_FWD_BLOCK_TC 8u
 
 /* Kernels reported by sa_plan(). */
 typedef enum sa_kernel {
-  SA_KERNEL_FWD_BLOCK = 1,         /* forward, query-stationary over 64-row blocks (topk <= 256) */
+  SA_KERNEL_FWD_BLOCK = 1,         /* forward, query-stationary over 64-row blocks (topk <= 256),
+                                      TMA-fed, mma.sync tiles */
   SA_KERNEL_FWD_TOKEN_TC = 2,      /* forward, token-level shared KV 576/512 on tcgen05 */
   SA_KERNEL_FWD_GENERIC = 3,       /* forward, any selection, rows gathered one by one */
   SA_KERNEL_BWD_KEY_STATIONARY = 4,        /* backward, key-stationary, dQ by atomics */
   SA_KERNEL_BWD_KEY_STATIONARY_DQ_PASS = 5,/* backward, key-stationary + separate dQ pass */
   SA_KERNEL_BWD_TOKEN_TC = 6,      /* backward, token-level shared KV 576/512 on tcgen05 */
-  SA_KERNEL_BWD_GENERIC = 7        /* backward, any selection, dK / dV by fp32 scatter-add */
+  SA_KERNEL_BWD_GENERIC = 7,       /* backward, any selection, dK / dV by fp32 scatter-add */
+  SA_KERNEL_FWD_BLOCK_TC = 8       /* forward, the same block problems on tcgen05 (SA_FLAG_FWD_BLOCK_TC) */
 } sa_kernel;
 
 /* Views of sa_debug_block_index(). */

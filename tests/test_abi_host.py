@@ -230,6 +230,9 @@ def test_plan_reports_the_kernel_each_problem_gets():
     assert _plan(_args(flags=L.SA_FLAG_DQ_SEPARATE)) == (L.SA_KERNEL_FWD_BLOCK,
                                                          L.SA_KERNEL_BWD_KEY_STATIONARY_DQ_PASS)
     assert _plan(_args(flags=L.SA_FLAG_QUERY_STATIONARY_BWD))[1] == L.SA_KERNEL_BWD_GENERIC
+    assert _plan(_args(flags=L.SA_FLAG_FWD_BLOCK_TC)) == (L.SA_KERNEL_FWD_BLOCK_TC, L.SA_KERNEL_BWD_KEY_STATIONARY)
+    # the flag touches block problems only
+    assert _plan(_args(block_size=16, flags=L.SA_FLAG_FWD_BLOCK_TC))[0] == L.SA_KERNEL_FWD_GENERIC
     # sinks, TND, block sizes other than 64 and unequal lengths leave the key-stationary kernel
     assert _plan(_args(sinks=FAKE))[1] == L.SA_KERNEL_BWD_GENERIC
     assert _plan(_args(block_size=16)) == (L.SA_KERNEL_FWD_GENERIC, L.SA_KERNEL_BWD_GENERIC)

@@ -76,6 +76,15 @@ def test_block_level_backward_variants(name, flag):
     run_full_comparison(w, kw, flags=flags)
 
 
+@pytest.mark.parametrize("name", BLOCK_CASES)
+def test_block_level_forward_on_tcgen05(name):
+    """The block-level workloads through the tcgen05 forward (SA_FLAG_FWD_BLOCK_TC)."""
+    _need_gpu()
+    from top_sparse_attention_attn_b200 import _lib as L
+    w, kw = SMALL[name]
+    run_full_comparison(w, kw, flags=L.SA_FLAG_FWD_BLOCK_TC)
+
+
 @pytest.mark.parametrize("cfg", ["cfg2", "cfg1", "cfg5", "cfg4", "cfg3"])
 def test_full_size_sampled(cfg):
     _need_gpu()

@@ -32,6 +32,7 @@ SA_DTYPE_FP16 = 1
 SA_FLAG_CHECK = 1
 SA_FLAG_QUERY_STATIONARY_BWD = 2
 SA_FLAG_DQ_SEPARATE = 4
+SA_FLAG_FWD_BLOCK_TC = 8
 
 # sa_kernel (sa_plan)
 SA_KERNEL_FWD_BLOCK = 1
@@ -41,6 +42,7 @@ SA_KERNEL_BWD_KEY_STATIONARY = 4
 SA_KERNEL_BWD_KEY_STATIONARY_DQ_PASS = 5
 SA_KERNEL_BWD_TOKEN_TC = 6
 SA_KERNEL_BWD_GENERIC = 7
+SA_KERNEL_FWD_BLOCK_TC = 8
 SA_INDEX_VIEW_QUERY_BLOCKS = 0
 SA_INDEX_VIEW_KEY_LISTS = 1
 

@@ -332,7 +332,7 @@ bool tk_path(const sa_args* a) {
 }
 
 int32_t fwd_choice(const sa_args* a) {
-  if (use_qb_path(a)) return SA_KERNEL_FWD_BLOCK;
+  if (use_qb_path(a)) return (a->flags & SA_FLAG_FWD_BLOCK_TC) ? SA_KERNEL_FWD_BLOCK_TC : SA_KERNEL_FWD_BLOCK;
   if (tk_path(a)) return SA_KERNEL_FWD_TOKEN_TC;
   return SA_KERNEL_FWD_GENERIC;
 }
@@ -506,11 +506,12 @@ sa_status sa_fwd(const sa_args* args, const sa_fwd_out* out, void* ws, size_t ws
   sa::Prob p = make_prob(args, status);
   if (cudaMemsetAsync(status, 0, sizeof(int), cs) != cudaSuccess) return SA_ERR_CUDA;
   const int32_t choice = fwd_choice(args);
-  if (choice == SA_KERNEL_FWD_BLOCK) {
+  if (choice == SA_KERNEL_FWD_BLOCK || choice == SA_KERNEL_FWD_BLOCK_TC) {
     sa::QbArgs q = make_qb_args(args, status);
     q.o = static_cast<bf16*>(out->o);
     q.lse = out->lse;
-    return cuda_status(sa::launch_bq_fwd(q, args->k, args->v, cs));
+    if (choice == SA_KERNEL_FWD_BLOCK_TC) return cuda_status(sa::launch_bq_fwd(q, args->k, args->v, cs));
+    return cuda_status(sa::launch_qb(q, args->k, args->v, false, cs));
   }
   if (choice == SA_KERNEL_FWD_TOKEN_TC)
     return cuda_status(sa::launch_tk_fwd(p, static_cast<bf16*>(out->o), out->lse, cs));

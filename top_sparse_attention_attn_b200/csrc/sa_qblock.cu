@@ -1058,12 +1058,17 @@ static cudaError_t qb_launch_t(const QbArgs& a, const void* k, const void* v, cu
   return cudaGetLastError();
 }
 
-// The dQ pass (the forward runs on bq_fwd_kernel).
+// The forward (dq = false) or the separate dQ pass (dq = true).
 cudaError_t launch_qb(const QbArgs& a, const void* k, const void* v, bool dq, cudaStream_t st) {
-  if (!dq) return cudaErrorInvalidValue;
-  if (a.dqk == 64 && a.dv == 64) return qb_launch_t<64, 64, true>(a, k, v, st, kTimeBwdDQ);
-  if (a.dqk == 128 && a.dv == 128) return qb_launch_t<128, 128, true>(a, k, v, st, kTimeBwdDQ);
-  if (a.dqk == 192 && a.dv == 128) return qb_launch_t<192, 128, true>(a, k, v, st, kTimeBwdDQ);
+  if (dq) {
+    if (a.dqk == 64 && a.dv == 64) return qb_launch_t<64, 64, true>(a, k, v, st, kTimeBwdDQ);
+    if (a.dqk == 128 && a.dv == 128) return qb_launch_t<128, 128, true>(a, k, v, st, kTimeBwdDQ);
+    if (a.dqk == 192 && a.dv == 128) return qb_launch_t<192, 128, true>(a, k, v, st, kTimeBwdDQ);
+  } else {
+    if (a.dqk == 64 && a.dv == 64) return qb_launch_t<64, 64, false>(a, k, v, st, kTimeFwd);
+    if (a.dqk == 128 && a.dv == 128) return qb_launch_t<128, 128, false>(a, k, v, st, kTimeFwd);
+    if (a.dqk == 192 && a.dv == 128) return qb_launch_t<192, 128, false>(a, k, v, st, kTimeFwd);
+  }
   return cudaErrorInvalidValue;
 }
 

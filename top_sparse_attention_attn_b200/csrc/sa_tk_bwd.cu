@@ -29,10 +29,12 @@
 // sub-tile:
 //   S  [64 x 32] = Q KV^T   (lanes 0..15)   dP [64 x 32] = dO V^T (lanes 16..31)
 //   P, dS (scaled) by the softmax warps, to shared memory
-//   dKV^T [576 x 32] = Q^T dS + dO^T P      (the P^T dO term on dims 0..511),
-//                                           added to the fp32 dKV accumulator by
-//                                           the reduction warps (one 128-byte
-//                                           warp-wide reduction per row and 32 dims)
+//   dKV^T [576 x 32] = Q^T dS + dO^T P      (the P^T dO term on dims 0..511);
+//                                           the reduction warps stage it as fp32
+//                                           key rows over the sub-tile's KV stage
+//                                           (two passes of 288 dims) and add each
+//                                           row to the fp32 dKV accumulator with
+//                                           one TMA bulk reduction
 //   dQ [64 x 576] += dS KV                  accumulated in TMEM over every sub-tile
 //
 // Warp roles: 0 = loader (Q / dO box loads, row codes, KV row gathers), 1 = MMA
