@@ -46,6 +46,9 @@ SMALL = {
     "token_h128_topk": (scaled("cfg3", "h128", S=300, Hq=128, topk=96, seed=36), {}),
     "swa_cmp_h64": (scaled("cfg4", "h64", seqlens=(100, 300, 37), Hq=64, cmp_topk=64,
                            cmp_len_range=(16, 64), seed=37), {}),
+    # 128 heads per KV head: the dim-split CTA pair (window + compressed rows + sinks)
+    "swa_cmp_h128": (scaled("cfg4", "h128", seqlens=(100, 300, 37), Hq=128, cmp_topk=64,
+                            cmp_len_range=(16, 64), seed=38), {}),
     # G = 1 and 2: key-stationary tiles of 128 and 64 tokens with rows gathered one by one
     "block_g1_d64": (scaled("cfg1", "g1", S=700, Hq=2, Hkv=2, topk=5, seed=33), {}),
     "block_g2_d128": (scaled("cfg5", "g2", S=1000, Hq=4, Hkv=2, d_qk=128, d_v=128, topk=7, zipf_s=1.2,
