@@ -4,9 +4,9 @@ TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the
 CPU-baseline leg of the benchmark; never by the CUDA product path.
 """
 
-from .sparse_attn_ref import (Problem, backward, forward, round_to_bf16_bits,
-                              unit_backward, unit_flops, unit_forward,
+from .sparse_attn_ref import (Problem, backward, forward, round_to_bf16_bits, softmax_l1norm,
+                              unit_backward, unit_flops, unit_forward, unit_softmax_l1norm,
                               visible_rows, widen_bf16)
 
-__all__ = ["Problem", "backward", "forward", "round_to_bf16_bits", "unit_backward",
-           "unit_flops", "unit_forward", "visible_rows", "widen_bf16"]
+__all__ = ["Problem", "backward", "forward", "round_to_bf16_bits", "softmax_l1norm", "unit_backward",
+           "unit_flops", "unit_forward", "unit_softmax_l1norm", "visible_rows", "widen_bf16"]

@@ -26,6 +26,11 @@ What it computes is the plain definition, one query token at a time, in float64
       dS = P o (dP - rowsum(dO o O))          (o = elementwise product)
       dQ = dS K scale,  dK = dS^T Q scale,  dV = P^T dO  (dKV = dK + dV if K = V)
       dSinks = sum over rows of -P_sink * sum_j P_j dP_j,  P_sink = exp(sink - lse)
+* SoftmaxL1Norm outputs.  SparseFlashMlaGrad, "Parameter Description"
+  (oriSoftmaxL1NormOptional / cmpSoftmaxL1NormOptional) with the target
+  distribution of aclnnSparseLightningIndexerGradKLLoss, "Formula": P summed over
+  the heads of a kv-head and over each slot's visible rows, L1-normalised along
+  that output's slots.
 
 Readings taken where the pages are silent or garbled (each is listed with its
 reason in the design notes of this repository):
@@ -41,7 +46,10 @@ reason in the design notes of this repository):
   - a row with no visible key and no sink has lse = +inf and O = 0, and gives
     zero gradients;
   - with K = V, V is the first d_v columns of the shared KV row;
-  - TND indices are positions local to their own sequence, like BSND.
+  - TND indices are positions local to their own sequence, like BSND;
+  - each SoftmaxL1Norm output is normalised over its own slots (ori and cmp
+    separately), the sink is no slot, and an output exists only where its index
+    list does.
 """
 
 from __future__ import annotations
@@ -57,6 +65,8 @@ __all__ = [
     "unit_backward",
     "forward",
     "backward",
+    "unit_softmax_l1norm",
+    "softmax_l1norm",
     "unit_flops",
 ]
 
@@ -417,6 +427,111 @@ def backward(p: Problem, O, lse, dO, units=None, rounded: bool = True):
             else:
                 res[key] = round_to_bf16_bits(res[key])
     return res
+
+
+# ----------------------------------------------------------------------------
+# The SoftmaxL1Norm outputs (the indexer loss's target distribution)
+# ----------------------------------------------------------------------------
+
+def _slot_rows(p: Problem, tq: int, g: int, kind: str):
+    """For each ori (kind "ori") or cmp slot of unit (tq, g): the rows it selects that
+    survive the masks (sequence-local, possibly empty), by the same rules as
+    visible_rows, slot by slot."""
+    b = p.batch_of(tq)
+    t = tq - int(p.q_start[b])
+    Lk = int(p.kv_len[b])
+    ta = t + (Lk - int(p.q_len[b]))
+    out = []
+    if kind == "ori":
+        n_all = p.ori_idx.shape[2]
+        n = n_all if p.ori_topk_len is None else max(0, min(n_all, int(p.ori_topk_len[tq, g])))
+        bs = p.block_size
+        for s in range(n_all):
+            x = int(p.ori_idx[tq, g, s])
+            if s >= n or x < 0:
+                out.append(np.zeros(0, dtype=np.int64))
+                continue
+            if x * bs >= Lk:
+                raise IndexError(f"ori index out of range at token {tq}, kv-head {g}")
+            rows = x * bs + np.arange(bs)
+            rows = rows[rows < Lk]
+            if p.ori_mask == "causal":
+                rows = rows[rows <= ta]
+            elif p.ori_mask == "band":
+                rows = rows[(rows >= ta - p.win_left) & (rows <= ta + p.win_right)]
+            out.append(rows)
+    else:
+        n_all = p.cmp_idx.shape[2]
+        n = n_all if p.cmp_topk_len is None else max(0, min(n_all, int(p.cmp_topk_len[tq, g])))
+        for s in range(n_all):
+            c = int(p.cmp_idx[tq, g, s])
+            if s >= n or c < 0:
+                out.append(np.zeros(0, dtype=np.int64))
+                continue
+            if c >= int(p.cmp_len[b]):
+                raise IndexError(f"cmp index out of range at token {tq}, kv-head {g}")
+            ok = p.cmp_mask != "causal" or (c + 1) * p.cmp_ratio - 1 <= ta
+            out.append(np.array([c] if ok else [], dtype=np.int64))
+    return out
+
+
+def unit_softmax_l1norm(p: Problem, tq: int, g: int, lse, normalize: bool = True):
+    """oriSoftmaxL1Norm / cmpSoftmaxL1Norm of query token tq under kv-head g.
+
+    SparseFlashMlaGrad, "Parameter Description": two FLOAT32 outputs, the softmax
+    result computed from the query and the original (resp. compressed) KV.
+    aclnnSparseLightningIndexerGradKLLoss, "Formula": the indexer's target
+    distribution p is the main attention scores summed over all heads, then
+    L1-normalised along the context.  Here P = exp(scale q.k - lse) is the
+    backward's recomputed softmax (``lse`` [G] of this unit, sink included; the
+    sink is no context position).  Entry s of an output sums P over the G heads of
+    kv-head g and over the visible rows its slot selects; each output is then
+    divided by its own sum (all zeros when that sum is 0).
+
+    Returns (ori [topk] or None, cmp [cmp_topk] or None), float64; None where the
+    problem has no index list of that kind.
+    """
+    hs = slice(g * p.G, (g + 1) * p.G)
+    Q = as_f64(p.q[tq, hs])
+    lse = np.asarray(lse, dtype=np.float64)
+    b = p.batch_of(tq)
+    res = []
+    for kind in ("ori", "cmp"):
+        if (kind == "ori" and p.ori_idx is None) or (kind == "cmp" and (p.cmp_idx is None or not p.has_cmp)):
+            res.append(None)
+            continue
+        slots = _slot_rows(p, tq, g, kind)
+        a = np.zeros(len(slots))
+        for s, rows in enumerate(slots):
+            if len(rows) == 0:
+                continue
+            if kind == "ori":
+                K = as_f64(p.k_ori[p.kv_start[b] + rows, g])
+            else:
+                K = as_f64(p.k_cmp[p.cmp_start[b] + rows, g])
+            P = np.exp(p.scale * (Q @ K.T) - lse[:, None])   # [G, rows of the slot]
+            a[s] = P.sum()
+        if normalize:
+            tot = a.sum()
+            a = a / tot if tot > 0 else np.zeros_like(a)
+        res.append(a)
+    return tuple(res)
+
+
+def softmax_l1norm(p: Problem, lse, units=None):
+    """Both outputs over every unit: (ori [T, Hkv, topk] or None, cmp [T, Hkv, cmp_topk]
+    or None), float64, from ``lse`` [T, Hq] (float32 or float64).  With ``units`` only
+    those units are filled (the rest stay zero)."""
+    ori = None if p.ori_idx is None else np.zeros((p.T, p.Hkv, p.ori_idx.shape[2]))
+    cmp = None if (p.cmp_idx is None or not p.has_cmp) else np.zeros((p.T, p.Hkv, p.cmp_idx.shape[2]))
+    for tq, g in (p.all_units() if units is None else units):
+        hs = slice(g * p.G, (g + 1) * p.G)
+        o, c = unit_softmax_l1norm(p, tq, g, np.asarray(lse, dtype=np.float64)[tq, hs])
+        if ori is not None:
+            ori[tq, g] = o
+        if cmp is not None:
+            cmp[tq, g] = c
+    return ori, cmp
 
 
 def unit_flops(p: Problem, tq: int, g: int) -> tuple:
