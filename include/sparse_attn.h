@@ -269,6 +269,26 @@ sa_status sa_bwd_no_alloc(const sa_args* args, const sa_bwd_io* io, void* stream
 /* Size in bytes of the scratch array behind sa_bwd_no_alloc. */
 size_t sa_bwd_no_alloc_max_workspace(void);
 
+/* The SoftmaxL1Norm outputs of SparseFlashMlaGrad ("Parameter Description":
+ * oriSoftmaxL1NormOptional, cmpSoftmaxL1NormOptional, FLOAT32): the target
+ * distribution of the indexer loss (aclnnSparseLightningIndexerGradKLLoss,
+ * "Formula": the attention scores summed over all heads, then L1-normalised along
+ * the context).  With P = exp(scale q.k - lse), the softmax the backward
+ * recomputes (sink included in lse; the sink is no slot):
+ *   ori_out[token, kv-head, s] = sum over the kv-head's query heads and over the
+ *                                visible rows of ori slot s of P, divided by the
+ *                                sum of that row over all its ori slots;
+ *   cmp_out likewise over the cmp slots (each output is normalised on its own).
+ * Empty slots (index < 0, slot >= the topk length, no visible row) hold 0; a row
+ * with no visible slot is all 0.  An index past its sequence selects nothing.
+ * lse fp32 [.., Hq] from sa_fwd (device).  ori_out fp32 [.., Hkv, topk] (needs ori
+ * indices: topk > 0) and cmp_out fp32 [.., Hkv, cmp_topk] (needs cmp indices), both
+ * device buffers the call overwrites; either may be NULL, not both.  Needs no
+ * workspace.  Errors: SA_ERR_NULLPTR (no output, or no lse), SA_ERR_PARAM (an
+ * output without its index list, misaligned tensors), validation errors as for
+ * sa_fwd.  Asynchronous. */
+sa_status sa_softmax_l1norm(const sa_args* args, const float* lse, float* ori_out, float* cmp_out, void* stream);
+
 /* rowsum(dO o O) alone -- the "FlashSoftmaxGrad(dO, O)" / "SoftmaxGrad(dO, O)"
  * term of aclnnSparseFlashAttentionGrad Phase 2 and SparseFlashMlaGrad Stage 2:
  * delta[token, h] = sum_c d_o[token, h, c] * o[token, h, c] in fp32.

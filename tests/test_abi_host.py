@@ -255,6 +255,18 @@ def test_dq_separate_is_ignored_past_the_block_kernels_slot_limit():
     assert _ws(a) == _ws(b)
 
 
+def test_softmax_l1norm_validates_on_the_host():
+    """sa_softmax_l1norm needs an output, its index list, and the forward's lse; all
+    checked before any device work (no GPU here)."""
+    f = L.lib().sa_softmax_l1norm
+    assert f(ctypes.byref(_args()), FAKE, None, None, None) == L.SA_ERR_NULLPTR
+    assert f(ctypes.byref(_args()), None, FAKE, None, None) == L.SA_ERR_NULLPTR          # no lse
+    assert f(ctypes.byref(_args(topk=0, ori_idx=None)), FAKE, FAKE, None, None) == L.SA_ERR_PARAM  # no ori indices
+    assert f(ctypes.byref(_args()), FAKE, None, FAKE, None) == L.SA_ERR_PARAM             # no cmp indices
+    assert f(ctypes.byref(_args(n_heads_q=15)), FAKE, FAKE, None, None) == L.SA_ERR_PARAM
+    assert f(ctypes.byref(_args(s_q=0, s_kv=0)), None, FAKE, None, None) == L.SA_OK       # empty query
+
+
 def test_status_and_inspection_calls_validate_on_the_host():
     assert L.lib().sa_read_status(None, 256, None) == L.SA_ERR_NULLPTR
     assert L.lib().sa_read_status(FAKE, 0, None) == L.SA_ERR_WORKSPACE

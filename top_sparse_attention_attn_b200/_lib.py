@@ -101,7 +101,7 @@ EXPORTS = ["sa_fwd_get_workspace_size", "sa_fwd", "sa_bwd_get_workspace_size", "
            "sa_set_timing_events", "sa_kernel_launch_count", "sa_bwd_no_alloc",
            "sa_bwd_no_alloc_max_workspace", "sa_selftest_mma", "sa_selftest_wait_timeout",
            "sa_selftest_mma2", "sa_plan", "sa_read_status", "sa_bwd_no_alloc_read_status",
-           "sa_debug_block_index", "sa_selftest_gather4"]
+           "sa_debug_block_index", "sa_selftest_gather4", "sa_softmax_l1norm"]
 
 
 def lib() -> ctypes.CDLL:
@@ -118,6 +118,7 @@ def lib() -> ctypes.CDLL:
         L.sa_bwd_get_workspace_size.argtypes = [P(SaArgs), P(ctypes.c_size_t)]
         L.sa_bwd.argtypes = [P(SaArgs), P(SaBwdIo), _vp, ctypes.c_size_t, _vp]
         L.sa_softmax_grad_preprocess.argtypes = [P(SaArgs), _vp, _vp, _vp, _vp]
+        L.sa_softmax_l1norm.argtypes = [P(SaArgs), _vp, _vp, _vp, _vp]
         L.sa_debug_resolve.argtypes = [P(SaArgs), _vp, _vp, ctypes.c_int32, _vp]
         L.sa_status_string.argtypes = [ctypes.c_int32]
         L.sa_status_string.restype = ctypes.c_char_p
@@ -210,6 +211,10 @@ def sa_selftest_wait_timeout(status: int, waited: int, stream: int = 0) -> None:
 def sa_softmax_grad_preprocess(args: SaArgs, o: int, d_o: int, delta: int, stream: int = 0) -> None:
     _check(lib().sa_softmax_grad_preprocess(ctypes.byref(args), o, d_o, delta, stream),
            "sa_softmax_grad_preprocess")
+
+
+def sa_softmax_l1norm(args: SaArgs, lse: int, ori_out, cmp_out, stream: int = 0) -> None:
+    _check(lib().sa_softmax_l1norm(ctypes.byref(args), lse, ori_out, cmp_out, stream), "sa_softmax_l1norm")
 
 
 def sa_debug_resolve(args: SaArgs, rows: int, counts: int, max_rows: int, stream: int = 0) -> None:

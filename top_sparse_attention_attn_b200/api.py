@@ -161,6 +161,18 @@ class SparseAttention:
         L.sa_softmax_grad_preprocess(self.args(), _ptr(o), _ptr(d_o), _ptr(out), st)
         return out
 
+    def softmax_l1norm(self, lse, ori: bool = True, cmp: bool = True, stream=None):
+        """The SoftmaxL1Norm outputs (sa_softmax_l1norm): (ori [.., Hkv, topk] or None,
+        cmp [.., Hkv, cmp_topk] or None), fp32, for the index lists this problem has."""
+        ori_out = cmp_out = None
+        if ori and self.topk > 0:
+            ori_out = torch.empty(self._lead() + (self.Hkv, self.topk), dtype=torch.float32, device=self.q.device)
+        if cmp and self.cmp_topk > 0 and self.cmp_kv is not None:
+            cmp_out = torch.empty(self._lead() + (self.Hkv, self.cmp_topk), dtype=torch.float32, device=self.q.device)
+        st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+        L.sa_softmax_l1norm(self.args(), _ptr(lse), _ptr(ori_out), _ptr(cmp_out), st)
+        return ori_out, cmp_out
+
     def debug_resolve(self, max_rows: int, stream=None):
         n_units = self.n_tokens * self.Hkv
         rows = torch.full((n_units, max(max_rows, 1)), -1, dtype=torch.int32, device=self.q.device)

@@ -637,6 +637,22 @@ sa_status sa_softmax_grad_preprocess(const sa_args* args, const void* o, const v
                                       s.Tq * args->n_heads_q, args->d_v, static_cast<cudaStream_t>(stream)));
 }
 
+sa_status sa_softmax_l1norm(const sa_args* args, const float* lse, float* ori_out, float* cmp_out, void* stream) {
+  sa_status st = validate(args);
+  if (st != SA_OK) return st;
+  if (!ori_out && !cmp_out) return SA_ERR_NULLPTR;
+  // each output needs its index list: ori indices (token or block selection), cmp indices
+  if (ori_out && args->topk <= 0) return SA_ERR_PARAM;
+  if (cmp_out && (args->cmp_topk <= 0 || !args->cmp_kv)) return SA_ERR_PARAM;
+  Sizes s = sizes_of(args);
+  if (s.Tq == 0) return SA_OK;
+  if (!lse) return SA_ERR_NULLPTR;
+  if (check_tensor_alignment(args) != SA_OK) return SA_ERR_PARAM;
+  if (!sa::kernels_built(args->d_qk, args->d_v, args->kv_shared != 0)) return SA_ERR_UNSUPPORTED;
+  sa::Prob p = make_prob(args, nullptr);
+  return cuda_status(sa::launch_softmax_l1norm(p, lse, ori_out, cmp_out, static_cast<cudaStream_t>(stream)));
+}
+
 sa_status sa_debug_resolve(const sa_args* args, int32_t* rows, int32_t* counts, int32_t max_rows, void* stream) {
   sa_status st = validate(args);
   if (st != SA_OK) return st;

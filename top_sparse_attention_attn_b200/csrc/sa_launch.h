@@ -80,6 +80,9 @@ struct Cvt {
 };
 cudaError_t launch_to_bf16_multi(const Cvt* jobs, int njobs, cudaStream_t st);
 cudaError_t launch_check(const Prob& p, cudaStream_t st);
+// SoftmaxL1Norm outputs: ori_out [Tq, Hkv, topk] and / or cmp_out [Tq, Hkv,
+// cmp_topk] fp32 (either may be null), from the forward's lse.
+cudaError_t launch_softmax_l1norm(const Prob& p, const float* lse, float* ori_out, float* cmp_out, cudaStream_t st);
 cudaError_t launch_debug_resolve(const Prob& p, int* rows, int* counts, int max_rows,
                                  cudaStream_t st);
 

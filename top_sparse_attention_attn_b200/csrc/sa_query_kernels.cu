@@ -252,6 +252,140 @@ __global__ void __launch_bounds__(128) fwd_kernel(const Prob p, bf16* __restrict
 }
 
 // ---------------------------------------------------------------------------
+// SoftmaxL1Norm outputs (SparseFlashMlaGrad "Parameter Description":
+// oriSoftmaxL1NormOptional / cmpSoftmaxL1NormOptional, the target distribution of
+// aclnnSparseLightningIndexerGradKLLoss "Formula": attention probabilities summed
+// over the heads, L1-normalised along the context).  The backward's P = exp(S -
+// lse) is recomputed tile by tile as in the forward, summed over the CTA's heads
+// for every tile row, and added to the row's slot of the unit's output (fp32
+// atomics: the 16-head slices of a unit share its output row).  l1_norm_kernel
+// then divides every output row by its sum.
+// ---------------------------------------------------------------------------
+template <int DQK>
+__device__ __forceinline__ void issue_k_tile(const Prob& p, int g, const int* rc, uint32_t sK, int tid) {
+  constexpr int KCH = DQK / 8;
+  for (int i = tid; i < kTileRows * KCH; i += 128) {
+    int r = i / KCH, c = i - r * KCH;
+    int code = rc[r];
+    const bf16* src = code >= 0 ? row_k_ptr(p, code, g) + c * 8 : p.q;
+    cp_async16(swz<DQK>(sK, r, c), src, code >= 0);
+  }
+}
+
+template <int DQK, int DV, bool SHARED>
+__global__ void __launch_bounds__(128) l1_sum_kernel(const Prob p, const float* __restrict__ LSE,
+                                                     float* __restrict__ ori_out, float* __restrict__ cmp_out) {
+  using PL = Plan<DQK, DV, SHARED>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_hsl = (p.G + 15) >> 4;
+  const int unit = blockIdx.x / n_hsl, hsl = blockIdx.x - unit * n_hsl;
+  const int tq = unit / p.Hkv, g = unit - tq * p.Hkv;
+  const Unit u = make_unit(p, tq, g);
+  const int h0 = g * p.G + hsl * 16;
+  const int nh = min(16, p.G - hsl * 16);
+  const long long ug = (long long)tq * p.Hkv + g;
+  const uint32_t sbuf = smem_u32(smem + PL::oBuf);
+  const uint32_t sQ = smem_u32(smem + PL::oQ);
+  int* rowc = reinterpret_cast<int*>(smem + PL::oRow);
+
+  load_rows16<DQK>(p.q + ((long long)tq * p.Hq + h0) * DQK, nh, sQ, tid);
+  cp_async_commit();
+  if (tid < 64 && u.n_tiles > 0) rowc[tid] = resolve_row(p, u, 0, tid);
+  __syncthreads();
+  if (u.n_tiles > 0) {
+    issue_k_tile<DQK>(p, g, rowc, sbuf, tid);
+    cp_async_commit();
+  }
+  // this thread's score rows r0 and r0 + 8 are heads h0 + r0, h0 + r0 + 8
+  const int r0 = lane >> 2;
+  float lse2[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int row = r0 + 8 * r;
+    lse2[r] = row < nh ? __ldg(LSE + (long long)tq * p.Hq + h0 + row) * kLog2e : INFINITY;  // P = 0 past nh
+  }
+  for (int it = 0; it < u.n_tiles; ++it) {
+    const int cur = it % 3;
+    const uint32_t bK = sbuf + (it & 1) * PL::kBuf;
+    if (tid < 64 && it + 1 < u.n_tiles) rowc[((it + 1) % 3) * 64 + tid] = resolve_row(p, u, it + 1, tid);
+    cp_async_wait_all();
+    __syncthreads();
+    if (it + 1 < u.n_tiles) {
+      issue_k_tile<DQK>(p, g, rowc + ((it + 1) % 3) * 64, sbuf + ((it + 1) & 1) * PL::kBuf, tid);
+      cp_async_commit();
+    }
+    // S_w = Q K_w^T over the warp's 16 tile rows (columns of s)
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll 4
+    for (int kc = 0; kc < DQK / 8; kc += 2) {
+      uint32_t a[4], b[4];
+      load_a<DQK>(a, sQ, 0, kc, lane);
+      load_b_nk<DQK>(b, bK, warp * 16, kc, lane);
+      mma16816(s[0], a, b[0], b[1]);
+      mma16816(s[1], a, b[2], b[3]);
+    }
+    const int* rc = rowc + cur * 64 + warp * 16;
+    // P summed over this thread's two heads, then over the 8 row groups of the warp
+    float cs[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int col = nt * 8 + 2 * (lane & 3) + e;
+        float v = 0.f;
+        if (rc[col] >= 0) v = exp2f(fmaf(s[nt][e], p.scale_log2, -lse2[0])) + exp2f(fmaf(s[nt][2 + e], p.scale_log2, -lse2[1]));
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        cs[nt][e] = v;
+      }
+    if (lane < 4) {
+      if (it < u.n_ori_tiles) {
+        if (ori_out && u.ori_mode == kOriToken) {
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int col = nt * 8 + 2 * lane + e;
+              if (rc[col] >= 0) atomicAdd(ori_out + ug * p.topk + it * kTileRows + warp * 16 + col, cs[nt][e]);
+            }
+        } else if (ori_out && u.ori_mode == kOriBlock) {
+          // every row of the tile belongs to one slot
+          const float t = (cs[0][0] + cs[0][1]) + (cs[1][0] + cs[1][1]);
+          if (t != 0.f) atomicAdd(ori_out + ug * p.topk + it / u.tps, t);
+        }
+      } else if (cmp_out) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = nt * 8 + 2 * lane + e;
+            if (rc[col] >= 0)
+              atomicAdd(cmp_out + ug * p.cmp_topk + (it - u.n_ori_tiles) * kTileRows + warp * 16 + col, cs[nt][e]);
+          }
+      }
+    }
+  }
+  cp_async_wait_all();
+}
+
+// Each of `rows` rows of `width` floats divided by its sum (left at zero when 0);
+// one warp per row.
+__global__ void __launch_bounds__(256) l1_norm_kernel(float* __restrict__ out, long long rows, int width) {
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float* r = out + row * width;
+  float sum = 0.f;
+  for (int i = lane; i < width; i += 32) sum += r[i];
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float inv = sum > 0.f ? 1.f / sum : 0.f;
+  for (int i = lane; i < width; i += 32) r[i] *= inv;
+}
+
+// ---------------------------------------------------------------------------
 // fused backward: dQ accumulated in the CTA, dK / dV (dKV) scattered with
 // fp32 vector atomics, dSinks partial sums
 // ---------------------------------------------------------------------------
@@ -623,6 +757,40 @@ static cudaError_t bwd_t(const Prob& p, const bf16* d_o, const float* lse, const
   count_launch();
   mark_end(st, which);
   return cudaGetLastError();
+}
+
+template <int DQK, int DV, bool SHARED>
+static cudaError_t l1_t(const Prob& p, const float* lse, float* ori_out, float* cmp_out, cudaStream_t st) {
+  using PL = Plan<DQK, DV, SHARED>;
+  auto k = l1_sum_kernel<DQK, DV, SHARED>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kBytes);
+  if (e != cudaSuccess) return e;
+  const long long units = (long long)p.Tq * p.Hkv;
+  if (ori_out && cudaMemsetAsync(ori_out, 0, (size_t)units * p.topk * sizeof(float), st) != cudaSuccess)
+    return cudaGetLastError();
+  if (cmp_out && cudaMemsetAsync(cmp_out, 0, (size_t)units * p.cmp_topk * sizeof(float), st) != cudaSuccess)
+    return cudaGetLastError();
+  const long long grid = units * ((p.G + 15) / 16);
+  k<<<(unsigned)grid, 128, PL::kBytes, st>>>(p, lse, ori_out, cmp_out);
+  count_launch();
+  const unsigned ng = (unsigned)((units + 7) / 8);
+  if (ori_out) {
+    l1_norm_kernel<<<ng, 256, 0, st>>>(ori_out, units, p.topk);
+    count_launch();
+  }
+  if (cmp_out) {
+    l1_norm_kernel<<<ng, 256, 0, st>>>(cmp_out, units, p.cmp_topk);
+    count_launch();
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_softmax_l1norm(const Prob& p, const float* lse, float* ori_out, float* cmp_out, cudaStream_t st) {
+#define X(A, B, C) \
+  if (p.dqk == A && p.dv == B && (bool)p.shared == C) return l1_t<A, B, C>(p, lse, ori_out, cmp_out, st);
+  SA_FOR_EACH_SHAPE(X)
+#undef X
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_fwd(const Prob& p, bf16* o, float* lse, cudaStream_t st) {
