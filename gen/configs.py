@@ -37,6 +37,7 @@ class Workload:
     select: str = "none"           # "diag_uniform" | "zipf" | "token_uniform" | "none"
     cmp_ratio: int = 1
     cmp_topk: int = 0              # slots of cmp indices per (token, kv-head); 0 = none
+    cmp_all: bool = False          # compressed KV without indices: every compressed row (CFA)
     cmp_len_range: tuple = (0, 0)  # inclusive range of the per-row cmp topk length
     ori_mask: str = "causal"       # "none" | "causal" | "band"
     cmp_mask: str = "causal"       # "none" | "causal"

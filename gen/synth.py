@@ -178,7 +178,7 @@ def make_inputs(w: Workload, *, allow_future: bool = False, cmp_any: bool = Fals
         idx = np.concatenate(parts, axis=0)
         out["ori_idx"] = idx.reshape(lead + (w.Hkv, w.topk))
 
-    if w.cmp_topk > 0:
+    if w.cmp_topk > 0 or w.cmp_all:
         cmp_lens = [L // w.cmp_ratio for L in lens]
         if dense:
             kvkey = "kv" if w.kv_shared else "k"
@@ -192,8 +192,9 @@ def make_inputs(w: Workload, *, allow_future: bool = False, cmp_any: bool = Fals
             out["cmp_kv"] = np.concatenate(cmp_parts, axis=0)
         out["cu_seqlens_cmp"] = np.concatenate([[0], np.cumsum(cmp_lens)]).astype(np.int32)
         out["cmp_residual"] = np.array([L % w.cmp_ratio for L in lens], dtype=np.int32)
-        cidx = np.concatenate([_cmp_indices(rng, w, L, cmp_any) for L in lens], axis=0)
-        out["cmp_idx"] = cidx.reshape(lead + (w.Hkv, w.cmp_topk))
+        if w.cmp_topk > 0:
+            cidx = np.concatenate([_cmp_indices(rng, w, L, cmp_any) for L in lens], axis=0)
+            out["cmp_idx"] = cidx.reshape(lead + (w.Hkv, w.cmp_topk))
 
     if ori_len_range is not None and w.topk > 0:
         lo, hi = ori_len_range

@@ -11,7 +11,8 @@ What it computes is the plain definition, one query token at a time, in float64
   = Gather(key/value, topkIndices[i]) for 0 <= i < selectBlockCount, each index
   naming a block of contiguous rows.  SparseFlashMlaGrad, "Computation formula",
   Stage 1: cmp_ratio = 1 (SWA) selects the original KV, cmp_ratio = 4 (SCFA)
-  concatenates the original KV with Gather(cmpKv, topkIndices[i]); the
+  concatenates the original KV with Gather(cmpKv, topkIndices[i]), any other
+  ratio (CFA) concatenates the original KV with all of cmpKv; the
   "Parameter Description" table adds oriSparseIndices (token rows of the
   original KV), oriTopkLength / cmpTopkLength (usable slots per query row),
   oriMaskMode / cmpMaskMode and oriWinLeft / oriWinRight.
@@ -47,6 +48,8 @@ reason in the design notes of this repository):
     zero gradients;
   - with K = V, V is the first d_v columns of the shared KV row;
   - TND indices are positions local to their own sequence, like BSND;
+  - the compressed rows are gathered through cmp indices when there are any
+    (SCFA); a compressed KV without indices contributes all its rows (CFA);
   - each SoftmaxL1Norm output is normalised over its own slots (ori and cmp
     separately), the sink is no slot, and an output exists only where its index
     list does.
@@ -202,8 +205,9 @@ class Problem:
         if "cmp_kv" in inp:
             ck = inp["cmp_kv"].reshape(-1, w.Hkv, w.d_qk)
             kw.update(k_cmp=ck, v_cmp=ck[..., :w.d_v],
-                      cmp_lens=np.diff(inp["cu_seqlens_cmp"]),
-                      cmp_idx=inp["cmp_idx"].reshape(T, w.Hkv, -1))
+                      cmp_lens=np.diff(inp["cu_seqlens_cmp"]))
+            if "cmp_idx" in inp:
+                kw["cmp_idx"] = inp["cmp_idx"].reshape(T, w.Hkv, -1)
             if "cmp_topk_len" in inp:
                 kw["cmp_topk_len"] = inp["cmp_topk_len"].reshape(T, w.Hkv)
         if "sinks" in inp:
@@ -267,7 +271,13 @@ def visible_rows(p: Problem, tq: int, g: int):
             raise ValueError(p.cmp_mask)
         cmp = c
     elif p.has_cmp:
-        raise NotImplementedError("compressed KV without cmp indices (CFA)")
+        # CFA (Stage 1, the "else" case): every compressed row of the sequence
+        c = np.arange(int(p.cmp_len[b]), dtype=np.int64)
+        if p.cmp_mask == "causal":
+            c = c[(c + 1) * p.cmp_ratio - 1 <= ta]
+        elif p.cmp_mask != "none":
+            raise ValueError(p.cmp_mask)
+        cmp = c
     return ori, cmp
 
 

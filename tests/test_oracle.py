@@ -81,6 +81,17 @@ def _tiny_params(mode: str, seed: int, dup: bool = False):
                     ori_len=None, ori_mask="band", win_left=3, win_right=1, cmp_lens=clens,
                     cmp_idx=cidx, cmp_len=rng.integers(0, ctopk + 1, (T, Hkv)), ratio=ratio,
                     scale=0.5)
+    elif mode == "cfa":
+        # SparseFlashMlaGrad Stage 1, "else" (CFA): the window over the original KV
+        # concatenated with every compressed row (no cmp indices)
+        lens, Hq, Hkv, dqk, dv, ratio = (14, 10), 4, 1, 6, 4, 3
+        T = sum(lens)
+        clens = tuple(L // ratio for L in lens)
+        par = dict(q=rng.standard_normal((T, Hq, dqk)), kv=rng.standard_normal((T, Hkv, dqk)),
+                   cmp_kv=rng.standard_normal((sum(clens), Hkv, dqk)), sinks=rng.standard_normal(Hq))
+        meta = dict(lens=lens, Hq=Hq, Hkv=Hkv, dqk=dqk, dv=dv, bs=1, shared=True, ori_idx=None,
+                    ori_len=None, ori_mask="band", win_left=2, win_right=0, cmp_lens=clens, ratio=ratio,
+                    cfa=True, scale=0.5)
     else:
         raise ValueError(mode)
     par["do"] = rng.standard_normal((sum(meta["lens"]), meta["Hq"], meta["dv"]))
@@ -96,7 +107,9 @@ def _build(par, meta) -> Problem:
     kw = {}
     if "cmp_kv" in par:
         kw = dict(k_cmp=par["cmp_kv"], v_cmp=par["cmp_kv"][..., :dv], cmp_lens=meta["cmp_lens"],
-                  cmp_idx=meta["cmp_idx"], cmp_topk_len=meta["cmp_len"], cmp_ratio=meta["ratio"])
+                  cmp_ratio=meta["ratio"])
+        if "cmp_idx" in meta:
+            kw.update(cmp_idx=meta["cmp_idx"], cmp_topk_len=meta["cmp_len"])
     return Problem(q=par["q"], k_ori=k_ori, v_ori=v_ori, kv_shared=meta["shared"],
                    q_lens=meta["lens"], kv_lens=meta["lens"], Hq=meta["Hq"], Hkv=meta["Hkv"],
                    d_qk=meta["dqk"], d_v=dv, scale=meta["scale"], block_size=meta["bs"],
@@ -127,7 +140,7 @@ def _grads(par, meta) -> dict:
     return out
 
 
-MODES = ["block", "token", "swa_cmp"]
+MODES = ["block", "token", "swa_cmp", "cfa"]
 
 
 # ----------------------------------------------------------------------------
@@ -208,6 +221,9 @@ def _selection_counts(meta, tq, g, b, t, L, off):
             c = meta["cmp_idx"][tq, g, i]
             if c >= 0 and (c + 1) * meta["ratio"] - 1 <= t:
                 ccounts[c] += 1
+    elif meta.get("cfa"):
+        C = meta["cmp_lens"][b]
+        ccounts = np.array([1.0 if (c + 1) * meta["ratio"] - 1 <= t else 0.0 for c in range(C)])
     return counts, ccounts
 
 
@@ -623,3 +639,30 @@ def test_round_to_bf16_matches_torch_and_ties():
     # a float64 just above a bf16 tie rounds up, where float32 double rounding would not
     x = 1 + 2.0 ** -8 + 2.0 ** -40
     assert oracle.widen_bf16(oracle.round_to_bf16_bits(np.array([x])))[0] == 1 + 2.0 ** -7
+
+
+def test_cfa_equals_scfa_listing_every_compressed_row():
+    """CFA (every compressed row, no indices) is SCFA whose cmp index list names every
+    compressed row of the sequence in order: same rows, same order, same results."""
+    par, meta = _tiny_params("cfa", seed=81)
+    p_cfa = _build(par, meta)
+    Cmax = max(meta["cmp_lens"])
+    T = sum(meta["lens"])
+    cidx = np.full((T, meta["Hkv"], Cmax), -1, dtype=np.int64)
+    off = 0
+    for L, C in zip(meta["lens"], meta["cmp_lens"]):
+        cidx[off:off + L, :, :C] = np.arange(C)
+        off += L
+    meta2 = dict(meta, cmp_idx=cidx, cmp_len=np.full((T, meta["Hkv"]), Cmax))
+    meta2.pop("cfa")
+    p_scfa = _build(par, meta2)
+    O1, l1 = oracle.forward(p_cfa, rounded=False)
+    O2, l2 = oracle.forward(p_scfa, rounded=False)
+    np.testing.assert_array_equal(O1, O2)
+    np.testing.assert_array_equal(l1, l2)
+    r1 = oracle.backward(p_cfa, O1, l1, par["do"], rounded=False)
+    r2 = oracle.backward(p_scfa, O2, l2, par["do"], rounded=False)
+    for key in r1:
+        np.testing.assert_array_equal(r1[key], r2[key])
+    # and the compressed rows do take part: some token sees at least one
+    assert any(len(oracle.visible_rows(p_cfa, tq, 0)[1]) for tq in range(T))
