@@ -55,7 +55,8 @@
  *   ori: NONE; CAUSAL row r <= ta; BAND ta - ori_win_left <= r <= ta + ori_win_right.
  *   cmp: NONE; CAUSAL compressed row c visible iff (c + 1) * cmp_ratio - 1 <= ta.
  * Without ori indices the whole original KV enters the selection under the ori
- * mask (sliding window when BAND); cmp indices add compressed rows (SCFA).
+ * mask (sliding window when BAND); cmp indices add compressed rows (SCFA); a
+ * compressed KV without indices adds all its rows under the cmp mask (CFA).
  *
  * Empty rows.  A query row with no visible key and no sink gets lse = +inf and
  * O = 0 and contributes no gradient.  A call with no query tokens returns
@@ -177,7 +178,8 @@ typedef struct sa_args {
   int32_t kv_shared;       /* 1: K = V = kv, V is the first d_v columns of each kv row */
   int32_t block_size;      /* rows per ori index (1 = token-level); <= 64 or a multiple of 64 */
   int32_t topk;            /* ori index slots per (token, kv-head); 0 = no ori indices */
-  int32_t cmp_topk;        /* cmp index slots per (token, kv-head); 0 = no compressed KV */
+  int32_t cmp_topk;        /* cmp index slots per (token, kv-head); 0 = no cmp indices (then cmp_kv,
+                              when given with cmp_ratio > 1, contributes all its rows: CFA) */
   int32_t cmp_ratio;       /* >= 1; cmp_kv has len_kv / cmp_ratio rows per sequence */
   int32_t ori_mask_mode;   /* sa_mask */
   int32_t cmp_mask_mode;   /* SA_MASK_NONE or SA_MASK_CAUSAL */
@@ -189,12 +191,13 @@ typedef struct sa_args {
   const void* k;           /* bf16, required when !kv_shared */
   const void* v;           /* bf16, required when !kv_shared */
   const void* kv;          /* bf16, required when kv_shared */
-  const void* cmp_kv;      /* bf16, required when cmp_topk > 0 */
+  const void* cmp_kv;      /* bf16, required when cmp_topk > 0; without cmp indices and with
+                              cmp_ratio > 1 every compressed row takes part (CFA) */
   const int32_t* ori_idx;  /* required when topk > 0 */
   const int32_t* cmp_idx;  /* required when cmp_topk > 0 */
   const int32_t* cu_seqlens_q;   /* TND: B + 1 offsets, required */
   const int32_t* cu_seqlens_kv;  /* TND: B + 1 offsets, required */
-  const int32_t* cu_seqlens_cmp; /* TND with cmp_topk > 0: B + 1 offsets, required */
+  const int32_t* cu_seqlens_cmp; /* TND with a compressed KV: B + 1 offsets, required */
   const int32_t* ori_topk_len;   /* optional (NULL = all topk slots usable) */
   const int32_t* cmp_topk_len;   /* optional (NULL = all cmp_topk slots usable) */
   const int32_t* cmp_residual;   /* optional, [B]: len_kv mod cmp_ratio; accepted, not used */
@@ -209,7 +212,7 @@ typedef struct sa_fwd_out {
 
 /* Backward inputs and outputs (device).  o / lse are the forward's outputs.
  * dq is required.  dk and dv (separate K, V) or dkv (K = V) are required.
- * dcmp_kv is required when cmp_topk > 0, dsinks when sinks != NULL. */
+ * dcmp_kv is required with a compressed KV (cmp indices, or CFA), dsinks when sinks != NULL. */
 typedef struct sa_bwd_io {
   const void* o;           /* bf16 [.., Hq, d_v] */
   const void* d_o;         /* bf16 [.., Hq, d_v] */

@@ -71,7 +71,7 @@ def max_visible_rows(w) -> int:
         n += w.topk * max(w.block_size, 1) if w.block_size > 1 else w.topk
     else:
         n += (w.win_left + w.win_right + 1) if w.ori_mask == "band" else max(w.seq_lengths)
-    n += w.cmp_topk
+    n += w.cmp_topk if w.cmp_topk else (max(w.seq_lengths) // w.cmp_ratio if w.cmp_all else 0)
     return n
 
 

@@ -46,7 +46,13 @@ SMALL = {
     "token_h128_topk": (scaled("cfg3", "h128", S=300, Hq=128, topk=96, seed=36), {}),
     "swa_cmp_h64": (scaled("cfg4", "h64", seqlens=(100, 300, 37), Hq=64, cmp_topk=64,
                            cmp_len_range=(16, 64), seed=37), {}),
-    # 128 heads per KV head: the dim-split CTA pair (window + compressed rows + sinks)
+    # CFA: the window over the original KV plus every compressed row (no cmp indices), on the
+    # generic kernels (16 heads) and the tcgen05 token kernels (64 heads)
+    "cfa_h16": (scaled("cfg4", "cfa", seqlens=(100, 300, 37), Hq=16, cmp_topk=0, cmp_all=True, cmp_ratio=8,
+                       seed=39), {}),
+    "cfa_h64": (scaled("cfg4", "cfa64", seqlens=(200, 77), Hq=64, cmp_topk=0, cmp_all=True, cmp_ratio=8,
+                       seed=40), {}),
+    # 128 heads per KV head (window + compressed rows + sinks)
     "swa_cmp_h128": (scaled("cfg4", "h128", seqlens=(100, 300, 37), Hq=128, cmp_topk=64,
                             cmp_len_range=(16, 64), seed=38), {}),
     # G = 1 and 2: key-stationary tiles of 128 and 64 tokens with rows gathered one by one

@@ -26,16 +26,23 @@ struct Sizes {
   long long Tq, Tkv, Tcmp;
 };
 
+// Compressed rows take part when cmp indices are given (SCFA: Gather(cmpKv,
+// topkIndices)), or when a compressed KV comes without indices and a compression
+// ratio above 1 (CFA: concat(oriKv, cmpKv), every compressed row);
+// SparseFlashMlaGrad "Computation formula" Stage 1.
+bool cfa(const sa_args* a) { return a->cmp_topk == 0 && a->cmp_kv != nullptr && a->cmp_ratio > 1; }
+bool has_cmp(const sa_args* a) { return a->cmp_topk > 0 || cfa(a); }
+
 Sizes sizes_of(const sa_args* a) {
   Sizes s;
   if (a->layout_q == SA_LAYOUT_BSND) {
     s.Tq = (long long)a->batch * a->s_q;
     s.Tkv = (long long)a->batch * a->s_kv;
-    s.Tcmp = a->cmp_topk > 0 ? (long long)a->batch * (a->s_kv / (a->cmp_ratio > 0 ? a->cmp_ratio : 1)) : 0;
+    s.Tcmp = has_cmp(a) ? (long long)a->batch * (a->s_kv / (a->cmp_ratio > 0 ? a->cmp_ratio : 1)) : 0;
   } else {
     s.Tq = a->t_q;
     s.Tkv = a->t_kv;
-    s.Tcmp = a->cmp_topk > 0 ? a->t_cmp : 0;
+    s.Tcmp = has_cmp(a) ? a->t_cmp : 0;
   }
   return s;
 }
@@ -76,12 +83,12 @@ sa_status validate(const sa_args* a) {
     if (a->cmp_topk > 0 && (!a->cmp_kv || !a->cmp_idx)) return SA_ERR_NULLPTR;
     if (a->layout_q == SA_LAYOUT_TND) {
       if (!a->cu_seqlens_q || !a->cu_seqlens_kv) return SA_ERR_NULLPTR;
-      if (a->cmp_topk > 0 && !a->cu_seqlens_cmp) return SA_ERR_NULLPTR;
+      if (has_cmp(a) && !a->cu_seqlens_cmp) return SA_ERR_NULLPTR;
       if (a->batch < 1) return SA_ERR_PARAM;
     }
   }
   // combinations that are valid on the pages but not built here
-  if (a->cmp_topk > 0 && !a->kv_shared) return SA_ERR_UNSUPPORTED;
+  if (has_cmp(a) && !a->kv_shared) return SA_ERR_UNSUPPORTED;
   if (!sa::kernels_built(a->d_qk, a->d_v, a->kv_shared != 0)) return SA_ERR_UNSUPPORTED;
   return SA_OK;
 }
@@ -121,7 +128,7 @@ sa::Prob make_prob(const sa_args* a, int* status) {
     p.k = static_cast<const bf16*>(a->k);
     p.v = static_cast<const bf16*>(a->v);
   }
-  p.cmpk = a->cmp_topk > 0 ? static_cast<const bf16*>(a->cmp_kv) : nullptr;
+  p.cmpk = has_cmp(a) ? static_cast<const bf16*>(a->cmp_kv) : nullptr;
   p.ori_idx = a->topk > 0 ? a->ori_idx : nullptr;
   p.cmp_idx = a->cmp_topk > 0 ? a->cmp_idx : nullptr;
   p.cu_q = a->cu_seqlens_q;
@@ -149,13 +156,13 @@ bool use_kv_path(const sa_args* a) {
   if (a->flags & SA_FLAG_QUERY_STATIONARY_BWD) return false;
   const int G = a->n_heads_q / a->n_heads_kv;
   return a->layout_q == SA_LAYOUT_BSND && a->topk > 0 && a->block_size == 64 && a->s_q == a->s_kv &&
-         !a->kv_shared && a->cmp_topk == 0 && a->sinks == nullptr && G <= 128 &&
+         !a->kv_shared && !has_cmp(a) && a->sinks == nullptr && G <= 128 &&
          sa::kv_path_built(a->d_qk, a->d_v);
 }
 
 // Query-stationary block kernels (TMA-fed): 64-row blocks, separate K / V, no compressed KV.
 bool use_qb_path(const sa_args* a) {
-  return a->topk > 0 && a->topk <= sa::kQbMaxSlots && a->block_size == 64 && !a->kv_shared && a->cmp_topk == 0 &&
+  return a->topk > 0 && a->topk <= sa::kQbMaxSlots && a->block_size == 64 && !a->kv_shared && !has_cmp(a) &&
          sa::qb_path_built(a->d_qk, a->d_v);
 }
 
@@ -535,7 +542,7 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
   if (s.Tq == 0) return SA_OK;
   if (!io->o || !io->d_o || !io->lse || !io->dq) return SA_ERR_NULLPTR;
   if (args->kv_shared ? !io->dkv : (!io->dk || !io->dv)) return SA_ERR_NULLPTR;
-  if (args->cmp_topk > 0 && !io->dcmp_kv) return SA_ERR_NULLPTR;
+  if (has_cmp(args) && !io->dcmp_kv) return SA_ERR_NULLPTR;
   if (sinks && !io->dsinks) return SA_ERR_NULLPTR;
   BwdWs w = bwd_ws_layout(args);
   if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
@@ -556,7 +563,7 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
   out.dq = static_cast<bf16*>(io->dq);
   out.dk_acc = reinterpret_cast<float*>(base + w.dk);
   out.dv_acc = args->kv_shared ? nullptr : reinterpret_cast<float*>(base + w.dv);
-  out.dcmp_acc = args->cmp_topk > 0 ? reinterpret_cast<float*>(base + w.dcmp) : nullptr;
+  out.dcmp_acc = has_cmp(args) ? reinterpret_cast<float*>(base + w.dcmp) : nullptr;
   out.dsinks = sinks ? io->dsinks : nullptr;
   const long long nk = s.Tkv * args->n_heads_kv * args->d_qk;
   const long long nv = s.Tkv * args->n_heads_kv * args->d_v;
@@ -617,7 +624,7 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
       jobs[nj++] = sa::Cvt{out.dk_acc, static_cast<bf16*>(io->dk), nk};
       jobs[nj++] = sa::Cvt{out.dv_acc, static_cast<bf16*>(io->dv), nv};
     }
-    if (args->cmp_topk > 0) jobs[nj++] = sa::Cvt{out.dcmp_acc, static_cast<bf16*>(io->dcmp_kv), nc};
+    if (has_cmp(args)) jobs[nj++] = sa::Cvt{out.dcmp_acc, static_cast<bf16*>(io->dcmp_kv), nc};
     if (w.dq) jobs[nj++] = sa::Cvt{reinterpret_cast<float*>(base + w.dq), static_cast<bf16*>(io->dq),
                                    s.Tq * args->n_heads_q * args->d_qk};
     e = sa::launch_to_bf16_multi(jobs, nj, cs);

@@ -77,7 +77,7 @@ __device__ __forceinline__ Unit make_unit(const Prob& p, int tq, int g) {
     Lq = p.s_q;
     u.Lk = p.s_kv;
     u.kv0 = u.b * p.s_kv;
-    u.Lc = p.cmp_topk > 0 ? p.s_kv / p.ratio : 0;
+    u.Lc = p.cmpk ? p.s_kv / p.ratio : 0;
     u.cmp0 = u.b * u.Lc;
   } else {
     // offsets are clamped to the packed extents, so inconsistent cu_seqlens can
@@ -88,7 +88,7 @@ __device__ __forceinline__ Unit make_unit(const Prob& p, int tq, int g) {
     u.t = tq - q0;
     u.kv0 = min(max(__ldg(p.cu_kv + u.b), 0), p.Tkv);
     u.Lk = min(max(__ldg(p.cu_kv + u.b + 1), u.kv0), p.Tkv) - u.kv0;
-    if (p.cmp_topk > 0) {
+    if (p.cmpk) {
       u.cmp0 = min(max(__ldg(p.cu_cmp + u.b), 0), p.Tcmp);
       u.Lc = min(max(__ldg(p.cu_cmp + u.b + 1), u.cmp0), p.Tcmp) - u.cmp0;
     } else {
@@ -133,7 +133,8 @@ __device__ __forceinline__ Unit make_unit(const Prob& p, int tq, int g) {
     if (p.cmp_len) n = min(n, max(0, __ldg(p.cmp_len + ug)));
     u.n_cmp_slots = n;
   } else {
-    u.n_cmp_slots = 0;
+    // a compressed KV without indices (CFA): every compressed row, slot c = row c
+    u.n_cmp_slots = p.cmpk ? u.Lc : 0;
   }
   u.n_tiles = u.n_ori_tiles + (u.n_cmp_slots + kTileRows - 1) / kTileRows;
   return u;
@@ -215,7 +216,8 @@ __device__ __forceinline__ int slot_index(const Prob& p, const Unit& u, int tile
     return 0;
   }
   const int s = (tile - u.n_ori_tiles) * kTileRows + r;
-  return s < u.n_cmp_slots ? __ldg(p.cmp_idx + ug * p.cmp_topk + s) : -1;
+  if (s >= u.n_cmp_slots) return -1;
+  return p.cmp_idx ? __ldg(p.cmp_idx + ug * p.cmp_topk + s) : s;
 }
 
 // Resolve row r (0..63) of tile `tile` of unit u, whose slot holds index x (from

@@ -90,7 +90,7 @@ __device__ __forceinline__ int qb_slots(const QbArgs& a, const Unit& u, int* xs,
 }
 
 __device__ __forceinline__ Unit qb_unit(const QbArgs& a, int tq, int g) {
-  Prob p;
+  Prob p = {};  // only the sequence geometry is set: no indices, no compressed KV
   p.layout = a.layout;
   p.B = a.B;
   p.s_q = a.s_q;
@@ -100,8 +100,9 @@ __device__ __forceinline__ Unit qb_unit(const QbArgs& a, int tq, int g) {
   p.cu_q = a.cu_q;
   p.cu_kv = a.cu_kv;
   p.cu_cmp = nullptr;
-  p.topk = 0;  // only the sequence geometry is needed here
+  p.topk = 0;
   p.cmp_topk = 0;
+  p.cmpk = nullptr;
   p.ori_mask = kMaskNone;
   p.ratio = 1;
   p.Hkv = a.Hkv;

@@ -719,7 +719,7 @@ static bool tk_row_maps(const Prob& p, CUtensorMap* mkv, CUtensorMap* mcmp, int*
     return false;
   *has_cmp = 0;
   *mcmp = *mkv;
-  if (p.cmp_topk > 0 && p.cmpk && p.Tcmp > 0) {
+  if (p.cmpk && p.Tcmp > 0) {
     if (!make_tmap_bf16(mcmp, p.cmpk, (uint64_t)p.Tcmp, (uint64_t)p.Hkv * tk::DQK, (uint64_t)p.Hkv * tk::DQK * 2, 1))
       return false;
     *has_cmp = 1;
