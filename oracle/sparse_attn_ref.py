@@ -48,6 +48,9 @@ reason in the design notes of this repository):
     zero gradients;
   - with K = V, V is the first d_v columns of the shared KV row;
   - TND indices are positions local to their own sequence, like BSND;
+  - sequsedQ / sequsedOriKv / sequsedCmpKv shorten each sequence to the tokens
+    that take part: the effective lengths set the causal alignment and the
+    sequence end; a query row past sequsedQ selects nothing (an empty row);
   - the compressed rows are gathered through cmp indices when there are any
     (SCFA); a compressed KV without indices contributes all its rows (CFA);
   - each SoftmaxL1Norm output is normalised over its own slots (ori and cmp
@@ -134,7 +137,8 @@ class Problem:
                  d_qk, d_v, scale, block_size=1, ori_idx=None, ori_topk_len=None,
                  k_cmp=None, v_cmp=None, cmp_lens=None, cmp_idx=None,
                  cmp_topk_len=None, cmp_ratio=1, ori_mask="causal",
-                 cmp_mask="causal", win_left=0, win_right=0, sinks=None):
+                 cmp_mask="causal", win_left=0, win_right=0, sinks=None,
+                 q_used=None, kv_used=None, cmp_used=None):
         self.q = np.asarray(q)
         self.k_ori = np.asarray(k_ori)
         self.v_ori = np.asarray(v_ori)
@@ -163,6 +167,12 @@ class Problem:
         self.cmp_len = np.asarray(cmp_lens, dtype=np.int64)
         self.cmp_start = np.concatenate([[0], np.cumsum(self.cmp_len)])[:-1]
         self.T = int(self.q_len.sum())
+        # sequsedQ / sequsedOriKv / sequsedCmpKv: tokens of each sequence that take part
+        nb = len(self.q_len)
+        self.q_used = self.q_len.copy() if q_used is None else np.minimum(self.q_len, np.asarray(q_used))
+        self.kv_used = self.kv_len.copy() if kv_used is None else np.minimum(self.kv_len, np.asarray(kv_used))
+        self.cmp_used = self.cmp_len.copy() if cmp_used is None else np.minimum(self.cmp_len, np.asarray(cmp_used))
+        assert len(self.q_used) == len(self.kv_used) == len(self.cmp_used) == nb
         self._batch_of = np.repeat(np.arange(len(self.q_len)), self.q_len)
         assert self.q.shape == (self.T, Hq, d_qk)
 
@@ -212,6 +222,9 @@ class Problem:
                 kw["cmp_topk_len"] = inp["cmp_topk_len"].reshape(T, w.Hkv)
         if "sinks" in inp:
             kw["sinks"] = inp["sinks"].astype(np.float64)
+        for key, arg in (("seqused_q", "q_used"), ("seqused_kv", "kv_used"), ("seqused_cmp", "cmp_used")):
+            if key in inp:
+                kw[arg] = inp[key].astype(np.int64)
         return cls(q=q, k_ori=k_ori, v_ori=v_ori, kv_shared=w.kv_shared, q_lens=lens,
                    kv_lens=lens, Hq=w.Hq, Hkv=w.Hkv, d_qk=w.d_qk, d_v=w.d_v,
                    scale=w.scale, block_size=w.block_size, cmp_ratio=w.cmp_ratio,
@@ -231,8 +244,10 @@ def visible_rows(p: Problem, tq: int, g: int):
     """
     b = p.batch_of(tq)
     t = tq - int(p.q_start[b])
-    Lk = int(p.kv_len[b])
-    ta = t + (Lk - int(p.q_len[b]))           # query position on the key axis
+    Lk = int(p.kv_used[b])                    # the rows that take part (sequsedOriKv)
+    ta = t + (Lk - int(p.q_used[b]))          # query position on the key axis
+    if t >= int(p.q_used[b]):                 # past sequsedQ: the row selects nothing
+        return np.zeros(0, dtype=np.int64), np.zeros(0, dtype=np.int64)
 
     # original KV: gathered through the ori indices, else all of it (SWA / SCFA / CFA)
     if p.ori_idx is not None:
@@ -263,7 +278,7 @@ def visible_rows(p: Problem, tq: int, g: int):
             n = max(0, min(n, int(p.cmp_topk_len[tq, g])))
         c = p.cmp_idx[tq, g, :n]
         c = c[c >= 0]
-        if np.any(c >= int(p.cmp_len[b])):
+        if np.any(c >= int(p.cmp_used[b])):
             raise IndexError(f"cmp index out of range at token {tq}, kv-head {g}")
         if p.cmp_mask == "causal":
             c = c[(c + 1) * p.cmp_ratio - 1 <= ta]
@@ -272,7 +287,7 @@ def visible_rows(p: Problem, tq: int, g: int):
         cmp = c
     elif p.has_cmp:
         # CFA (Stage 1, the "else" case): every compressed row of the sequence
-        c = np.arange(int(p.cmp_len[b]), dtype=np.int64)
+        c = np.arange(int(p.cmp_used[b]), dtype=np.int64)
         if p.cmp_mask == "causal":
             c = c[(c + 1) * p.cmp_ratio - 1 <= ta]
         elif p.cmp_mask != "none":
@@ -449,8 +464,11 @@ def _slot_rows(p: Problem, tq: int, g: int, kind: str):
     visible_rows, slot by slot."""
     b = p.batch_of(tq)
     t = tq - int(p.q_start[b])
-    Lk = int(p.kv_len[b])
-    ta = t + (Lk - int(p.q_len[b]))
+    Lk = int(p.kv_used[b])
+    ta = t + (Lk - int(p.q_used[b]))
+    idx_all = p.ori_idx if kind == "ori" else p.cmp_idx
+    if t >= int(p.q_used[b]):                 # past sequsedQ: every slot is empty
+        return [np.zeros(0, dtype=np.int64) for _ in range(idx_all.shape[2])]
     out = []
     if kind == "ori":
         n_all = p.ori_idx.shape[2]
@@ -478,7 +496,7 @@ def _slot_rows(p: Problem, tq: int, g: int, kind: str):
             if s >= n or c < 0:
                 out.append(np.zeros(0, dtype=np.int64))
                 continue
-            if c >= int(p.cmp_len[b]):
+            if c >= int(p.cmp_used[b]):
                 raise IndexError(f"cmp index out of range at token {tq}, kv-head {g}")
             ok = p.cmp_mask != "causal" or (c + 1) * p.cmp_ratio - 1 <= ta
             out.append(np.array([c] if ok else [], dtype=np.int64))
