@@ -38,6 +38,8 @@ class Workload:
     cmp_ratio: int = 1
     cmp_topk: int = 0              # slots of cmp indices per (token, kv-head); 0 = none
     cmp_all: bool = False          # compressed KV without indices: every compressed row (CFA)
+    used: tuple = ()               # per sequence: tokens that take part (sequsedQ = sequsedOriKv;
+                                   # sequsedCmpKv = used // cmp_ratio); () = all
     cmp_len_range: tuple = (0, 0)  # inclusive range of the per-row cmp topk length
     ori_mask: str = "causal"       # "none" | "causal" | "band"
     cmp_mask: str = "causal"       # "none" | "causal"

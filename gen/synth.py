@@ -210,6 +210,13 @@ def make_inputs(w: Workload, *, allow_future: bool = False, cmp_any: bool = Fals
             cap[starts[b]:starts[b] + L] = n[:, None]
         out["cmp_topk_len"] = np.minimum(raw, cap).astype(np.int32).reshape(lead + (w.Hkv,))
 
+    if w.used:
+        assert len(w.used) == len(lens)
+        out["seqused_q"] = np.asarray(w.used, dtype=np.int32)
+        out["seqused_kv"] = np.asarray(w.used, dtype=np.int32)
+        if w.cmp_topk > 0 or w.cmp_all:
+            out["seqused_cmp"] = np.asarray([u // w.cmp_ratio for u in w.used], dtype=np.int32)
+
     if w.layout == "TND":
         out["cu_seqlens_q"] = starts.astype(np.int32)
         out["cu_seqlens_kv"] = starts.astype(np.int32)

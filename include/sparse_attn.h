@@ -58,6 +58,15 @@
  * mask (sliding window when BAND); cmp indices add compressed rows (SCFA); a
  * compressed KV without indices adds all its rows under the cmp mask (CFA).
  *
+ * Used lengths (SparseFlashMlaGrad "Parameter Description": sequsedQOptional,
+ * sequsedOriKvOptional, sequsedCmpKvOptional).  When given, sequence b takes part
+ * with its first seqused_q[b] query tokens, seqused_kv[b] KV rows and
+ * seqused_cmp[b] compressed rows (each clamped to the sequence's length): these
+ * effective lengths set the bottom-right alignment (ta = t + used_kv - used_q) and
+ * the sequence ends, an index past them selects nothing, and a query row past
+ * seqused_q is an empty row (below).  Problems with used lengths run on the
+ * generic and token-level kernels.
+ *
  * Empty rows.  A query row with no visible key and no sink gets lse = +inf and
  * O = 0 and contributes no gradient.  A call with no query tokens returns
  * SA_OK without launching anything.
@@ -101,7 +110,7 @@
 extern "C" {
 #endif
 
-#define SA_ABI_VERSION 2
+#define SA_ABI_VERSION 3
 
 typedef enum sa_status {
   SA_OK = 0,
@@ -202,6 +211,12 @@ typedef struct sa_args {
   const int32_t* cmp_topk_len;   /* optional (NULL = all cmp_topk slots usable) */
   const int32_t* cmp_residual;   /* optional, [B]: len_kv mod cmp_ratio; accepted, not used */
   const float* sinks;            /* optional, [Hq] fp32 sink logits */
+  const int32_t* seqused_q;      /* optional, [B]: query tokens of each sequence that take part
+                                    (sequsedQ); the rest select nothing */
+  const int32_t* seqused_kv;     /* optional, [B]: original KV tokens of each sequence that take
+                                    part (sequsedOriKv) */
+  const int32_t* seqused_cmp;    /* optional, [B]: compressed KV rows of each sequence that take
+                                    part (sequsedCmpKv) */
 } sa_args;
 
 /* Forward outputs (device): O bf16 [.., Hq, d_v]; lse fp32 [.., Hq]. */

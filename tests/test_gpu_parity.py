@@ -52,6 +52,12 @@ SMALL = {
                        seed=39), {}),
     "cfa_h64": (scaled("cfg4", "cfa64", seqlens=(200, 77), Hq=64, cmp_topk=0, cmp_all=True, cmp_ratio=8,
                        seed=40), {}),
+    # sequsedQ / sequsedOriKv / sequsedCmpKv: padded sequences of which only the first
+    # `used` tokens take part (generic kernels for blocks; tcgen05 token kernels at 64 heads)
+    "block_used": (scaled("cfg1", "used", B=2, S=256, Hq=8, Hkv=2, topk=3, used=(200, 97), seed=41), {}),
+    "token_used_h64": (scaled("cfg3", "used", S=400, Hq=64, topk=128, used=(301,), seed=42), {}),
+    "swa_cmp_used": (scaled("cfg4", "used", seqlens=(100, 300, 37), Hq=16, cmp_topk=64, cmp_len_range=(16, 64),
+                            used=(80, 213, 37), seed=43), {}),
     # 128 heads per KV head (window + compressed rows + sinks)
     "swa_cmp_h128": (scaled("cfg4", "h128", seqlens=(100, 300, 37), Hq=128, cmp_topk=64,
                             cmp_len_range=(16, 64), seed=38), {}),

@@ -75,6 +75,7 @@ class SaArgs(ctypes.Structure):
         ("ori_idx", _vp), ("cmp_idx", _vp),
         ("cu_seqlens_q", _vp), ("cu_seqlens_kv", _vp), ("cu_seqlens_cmp", _vp),
         ("ori_topk_len", _vp), ("cmp_topk_len", _vp), ("cmp_residual", _vp), ("sinks", _vp),
+        ("seqused_q", _vp), ("seqused_kv", _vp), ("seqused_cmp", _vp),
     ]
 
 

@@ -51,6 +51,9 @@ class SparseAttention:
     cu_seqlens_cmp: torch.Tensor | None = None
     cmp_residual: torch.Tensor | None = None
     sinks: torch.Tensor | None = None
+    seqused_q: torch.Tensor | None = None     # [B] int32: query tokens that take part
+    seqused_kv: torch.Tensor | None = None    # [B] int32: original KV tokens that take part
+    seqused_cmp: torch.Tensor | None = None   # [B] int32: compressed KV rows that take part
     ori_mask: str = "causal"
     cmp_mask: str = "causal"
     win_left: int = 0
@@ -98,6 +101,8 @@ class SparseAttention:
         a.ori_topk_len, a.cmp_topk_len = _ptr(self.ori_topk_len), _ptr(self.cmp_topk_len)
         a.cmp_residual = _ptr(self.cmp_residual)
         a.sinks = _ptr(self.sinks)
+        a.seqused_q, a.seqused_kv = _ptr(self.seqused_q), _ptr(self.seqused_kv)
+        a.seqused_cmp = _ptr(self.seqused_cmp)
         return a
 
     # ---- allocation helpers ------------------------------------------------
@@ -221,7 +226,8 @@ class SparseAttention:
         else:
             kw["k"], kw["v"] = t["k"], t["v"]
         for key in ("ori_idx", "ori_topk_len", "cmp_kv", "cmp_idx", "cmp_topk_len",
-                    "cu_seqlens_q", "cu_seqlens_kv", "cu_seqlens_cmp", "cmp_residual", "sinks"):
+                    "cu_seqlens_q", "cu_seqlens_kv", "cu_seqlens_cmp", "cmp_residual", "sinks",
+                    "seqused_q", "seqused_kv", "seqused_cmp"):
             if key in t:
                 kw[key] = t[key]
         if w.layout == "BSND":

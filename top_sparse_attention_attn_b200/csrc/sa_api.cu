@@ -32,6 +32,8 @@ struct Sizes {
 // SparseFlashMlaGrad "Computation formula" Stage 1.
 bool cfa(const sa_args* a) { return a->cmp_topk == 0 && a->cmp_kv != nullptr && a->cmp_ratio > 1; }
 bool has_cmp(const sa_args* a) { return a->cmp_topk > 0 || cfa(a); }
+// sequsedQ / sequsedOriKv / sequsedCmpKv given (the block kernels do not take them)
+bool has_used(const sa_args* a) { return a->seqused_q || a->seqused_kv || a->seqused_cmp; }
 
 Sizes sizes_of(const sa_args* a) {
   Sizes s;
@@ -137,6 +139,9 @@ sa::Prob make_prob(const sa_args* a, int* status) {
   p.ori_len = a->topk > 0 ? a->ori_topk_len : nullptr;
   p.cmp_len = a->cmp_topk > 0 ? a->cmp_topk_len : nullptr;
   p.sinks = a->sinks;
+  p.used_q = a->seqused_q;
+  p.used_kv = a->seqused_kv;
+  p.used_cmp = has_cmp(a) ? a->seqused_cmp : nullptr;
   p.status = status;
   return p;
 }
@@ -156,13 +161,13 @@ bool use_kv_path(const sa_args* a) {
   if (a->flags & SA_FLAG_QUERY_STATIONARY_BWD) return false;
   const int G = a->n_heads_q / a->n_heads_kv;
   return a->layout_q == SA_LAYOUT_BSND && a->topk > 0 && a->block_size == 64 && a->s_q == a->s_kv &&
-         !a->kv_shared && !has_cmp(a) && a->sinks == nullptr && G <= 128 &&
+         !a->kv_shared && !has_cmp(a) && !has_used(a) && a->sinks == nullptr && G <= 128 &&
          sa::kv_path_built(a->d_qk, a->d_v);
 }
 
 // Query-stationary block kernels (TMA-fed): 64-row blocks, separate K / V, no compressed KV.
 bool use_qb_path(const sa_args* a) {
-  return a->topk > 0 && a->topk <= sa::kQbMaxSlots && a->block_size == 64 && !a->kv_shared && !has_cmp(a) &&
+  return a->topk > 0 && a->topk <= sa::kQbMaxSlots && a->block_size == 64 && !a->kv_shared && !has_cmp(a) && !has_used(a) &&
          sa::qb_path_built(a->d_qk, a->d_v);
 }
 

@@ -33,6 +33,7 @@ struct Prob {
   int layout, B, s_q, s_kv;
   int Tq, Tkv, Tcmp;
   int Hq, Hkv, G, dqk, dv, shared, bs, topk, cmp_topk, ratio, ori_mask, cmp_mask;
+  const int *used_q, *used_kv, *used_cmp;  // sequsedQ / OriKv / CmpKv ([B]) or null
   long long wl, wr;
   float scale;        // scaleValue
   float scale_log2;   // scale * log2(e)
@@ -96,6 +97,11 @@ __device__ __forceinline__ Unit make_unit(const Prob& p, int tq, int g) {
       u.Lc = 0;
     }
   }
+  // the tokens that take part (sequsedQ / sequsedOriKv / sequsedCmpKv)
+  if (p.used_q) Lq = min(Lq, max(0, __ldg(p.used_q + u.b)));
+  if (p.used_kv) u.Lk = min(u.Lk, max(0, __ldg(p.used_kv + u.b)));
+  if (p.used_cmp) u.Lc = min(u.Lc, max(0, __ldg(p.used_cmp + u.b)));
+  const bool active = u.t < Lq;  // a row past sequsedQ selects nothing
   u.ta = u.t + u.Lk - Lq;
   const long long ug = (long long)tq * p.Hkv + g;
   u.tps = 1;
@@ -137,6 +143,12 @@ __device__ __forceinline__ Unit make_unit(const Prob& p, int tq, int g) {
     u.n_cmp_slots = p.cmpk ? u.Lc : 0;
   }
   u.n_tiles = u.n_ori_tiles + (u.n_cmp_slots + kTileRows - 1) / kTileRows;
+  if (!active) {
+    u.n_ori_slots = u.n_cmp_slots = 0;
+    u.n_ori_tiles = u.n_tiles = 0;
+    u.lo = 0;
+    u.hi = -1;
+  }
   return u;
 }
 
