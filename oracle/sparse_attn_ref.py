@@ -51,6 +51,8 @@ reason in the design notes of this repository):
   - sequsedQ / sequsedOriKv / sequsedCmpKv shorten each sequence to the tokens
     that take part: the effective lengths set the causal alignment and the
     sequence end; a query row past sequsedQ selects nothing (an empty row);
+  - a paged KV cache maps logical row r of sequence b to physical row
+    block_table[b, r // page_size] * page_size + r % page_size;
   - the compressed rows are gathered through cmp indices when there are any
     (SCFA); a compressed KV without indices contributes all its rows (CFA);
   - each SoftmaxL1Norm output is normalised over its own slots (ori and cmp
@@ -138,7 +140,7 @@ class Problem:
                  k_cmp=None, v_cmp=None, cmp_lens=None, cmp_idx=None,
                  cmp_topk_len=None, cmp_ratio=1, ori_mask="causal",
                  cmp_mask="causal", win_left=0, win_right=0, sinks=None,
-                 q_used=None, kv_used=None, cmp_used=None):
+                 q_used=None, kv_used=None, cmp_used=None, block_table=None, page_size=0):
         self.q = np.asarray(q)
         self.k_ori = np.asarray(k_ori)
         self.v_ori = np.asarray(v_ori)
@@ -173,6 +175,11 @@ class Problem:
         self.kv_used = self.kv_len.copy() if kv_used is None else np.minimum(self.kv_len, np.asarray(kv_used))
         self.cmp_used = self.cmp_len.copy() if cmp_used is None else np.minimum(self.cmp_len, np.asarray(cmp_used))
         assert len(self.q_used) == len(self.kv_used) == len(self.cmp_used) == nb
+        # paged KV cache (aclnnNsaSelectedAttentionInfer: "paged attention obtains the
+        # kvCache"): k_ori / v_ori are the cache, [pages * page_size, Hkv, d]; logical row r
+        # of sequence b lives in physical page block_table[b, r // page_size]
+        self.block_table = None if block_table is None else np.asarray(block_table, dtype=np.int64)
+        self.page_size = int(page_size)
         self._batch_of = np.repeat(np.arange(len(self.q_len)), self.q_len)
         assert self.q.shape == (self.T, Hq, d_qk)
 
@@ -296,11 +303,20 @@ def visible_rows(p: Problem, tq: int, g: int):
     return ori, cmp
 
 
+def kv_rows(p: Problem, b: int, rows) -> np.ndarray:
+    """Storage rows of sequence b's (sequence-local) original-KV rows: contiguous from
+    kv_start[b], or through the block table of a paged cache."""
+    rows = np.asarray(rows, dtype=np.int64)
+    if p.block_table is None:
+        return p.kv_start[b] + rows
+    return p.block_table[b, rows // p.page_size] * p.page_size + rows % p.page_size
+
+
 def _gather(p: Problem, tq: int, g: int):
     b = p.batch_of(tq)
     ori, cmp = visible_rows(p, tq, g)
-    K = as_f64(p.k_ori[p.kv_start[b] + ori, g])
-    V = as_f64(p.v_ori[p.kv_start[b] + ori, g])
+    K = as_f64(p.k_ori[kv_rows(p, b, ori), g])
+    V = as_f64(p.v_ori[kv_rows(p, b, ori), g])
     if len(cmp):
         K = np.concatenate([K, as_f64(p.k_cmp[p.cmp_start[b] + cmp, g])])
         V = np.concatenate([V, as_f64(p.v_cmp[p.cmp_start[b] + cmp, g])])
@@ -423,8 +439,8 @@ def backward(p: Problem, O, lse, dO, units=None, rounded: bool = True):
             dq[(tq, g)] = r["dQ"]
         b = p.batch_of(tq)
         no = len(r["ori"])
-        _scatter_add(dk[:, g], p.kv_start[b] + r["ori"], r["dK_rows"][:no])
-        _scatter_add(dv[:, g], p.kv_start[b] + r["ori"], r["dV_rows"][:no])
+        _scatter_add(dk[:, g], kv_rows(p, b, r["ori"]), r["dK_rows"][:no])
+        _scatter_add(dv[:, g], kv_rows(p, b, r["ori"]), r["dV_rows"][:no])
         if len(r["cmp"]):
             _scatter_add(dkc[:, g], p.cmp_start[b] + r["cmp"], r["dK_rows"][no:])
             _scatter_add(dvc[:, g], p.cmp_start[b] + r["cmp"], r["dV_rows"][no:])
@@ -534,7 +550,7 @@ def unit_softmax_l1norm(p: Problem, tq: int, g: int, lse, normalize: bool = True
             if len(rows) == 0:
                 continue
             if kind == "ori":
-                K = as_f64(p.k_ori[p.kv_start[b] + rows, g])
+                K = as_f64(p.k_ori[kv_rows(p, b, rows), g])
             else:
                 K = as_f64(p.k_cmp[p.cmp_start[b] + rows, g])
             P = np.exp(p.scale * (Q @ K.T) - lse[:, None])   # [G, rows of the slot]
