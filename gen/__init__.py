@@ -6,7 +6,7 @@ attention arithmetic.
 """
 
 from .configs import WORKLOADS, Workload, get_workload, scaled
-from .synth import make_inputs, bf16_bits_from_f32, f32_from_bf16_bits
+from .synth import make_inputs, make_paged_inputs, bf16_bits_from_f32, f32_from_bf16_bits
 
 __all__ = [
     "WORKLOADS",
@@ -14,6 +14,7 @@ __all__ = [
     "get_workload",
     "scaled",
     "make_inputs",
+    "make_paged_inputs",
     "bf16_bits_from_f32",
     "f32_from_bf16_bits",
 ]

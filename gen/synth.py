@@ -221,3 +221,44 @@ def make_inputs(w: Workload, *, allow_future: bool = False, cmp_any: bool = Fals
         out["cu_seqlens_q"] = starts.astype(np.int32)
         out["cu_seqlens_kv"] = starts.astype(np.int32)
     return out
+
+
+def make_paged_inputs(seed: int, *, B: int, s_q: int, kv_lens, page: int, Hq: int, Hkv: int, d_qk: int, d_v: int,
+                      kv_shared: bool, block_size: int, topk: int, sinks: bool = True, spare_pages: int = 3) -> dict:
+    """Decode-style inputs over a paged KV cache: s_q query tokens at the end of each
+    of B sequences (lengths kv_lens), the cache's pages in shuffled order behind a
+    per-sequence block table, and causal index sets (block_size-row blocks with the
+    diagonal block first, or tokens) drawn over each query's visible prefix.  Dense
+    tensors fp32 N(0, 1) -> bf16 (RNE) bit patterns; indices int32, -1 padded."""
+    rng = np.random.default_rng(seed)
+    kv_lens = np.asarray(kv_lens, dtype=np.int64)
+    max_pages = int(-(-int(kv_lens.max()) // page))
+    n_pages = B * max_pages + spare_pages
+    table = rng.permutation(n_pages)[:B * max_pages].reshape(B, max_pages).astype(np.int32)
+    rows = n_pages * page
+    out = {"q": bf16_bits_from_f32(rng.standard_normal((B * s_q, Hq, d_qk), dtype=np.float32))}
+    if kv_shared:
+        out["kv"] = bf16_bits_from_f32(rng.standard_normal((rows, Hkv, d_qk), dtype=np.float32))
+    else:
+        out["k"] = bf16_bits_from_f32(rng.standard_normal((rows, Hkv, d_qk), dtype=np.float32))
+        out["v"] = bf16_bits_from_f32(rng.standard_normal((rows, Hkv, d_v), dtype=np.float32))
+    idx = np.full((B * s_q, Hkv, topk), -1, dtype=np.int32)
+    for b in range(B):
+        for t in range(s_q):
+            ta = t + int(kv_lens[b]) - s_q                       # the query's position in its sequence
+            for g in range(Hkv):
+                if block_size > 1:
+                    diag = ta // block_size
+                    rest = rng.permutation(diag)[:topk - 1]
+                    sel = np.concatenate([[diag], rest])
+                else:
+                    sel = rng.permutation(ta + 1)[:topk]
+                idx[b * s_q + t, g, :len(sel)] = sel
+    out["ori_idx"] = idx
+    out["block_table"] = table
+    out["seqused_kv"] = kv_lens.astype(np.int32)
+    if sinks:
+        out["sinks"] = rng.standard_normal(Hq).astype(np.float32)
+    out["_meta"] = dict(B=B, s_q=s_q, s_kv=max_pages * page, t_kv=rows, page=page, Hq=Hq, Hkv=Hkv, d_qk=d_qk,
+                        d_v=d_v, kv_shared=kv_shared, block_size=block_size, topk=topk)
+    return out

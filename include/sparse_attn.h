@@ -58,6 +58,16 @@
  * mask (sliding window when BAND); cmp indices add compressed rows (SCFA); a
  * compressed KV without indices adds all its rows under the cmp mask (CFA).
  *
+ * Paged KV cache (aclnnNsaSelectedAttentionInfer: "paged attention obtains the
+ * kvCache", a few query tokens per sequence).  With block_table, k / v / kv are a
+ * cache of t_kv rows in pages of page_size rows; logical row r of sequence b is
+ * cache row block_table[b, r / page_size] * page_size + r % page_size.  s_kv is the
+ * logical capacity (at most max_pages * page_size) and seqused_kv gives each
+ * sequence's actual length; the queries sit at the end of their sequences (the
+ * bottom-right alignment).  BSND only, no compressed KV; the forward and
+ * sa_softmax_l1norm take it, the backward returns SA_ERR_UNSUPPORTED.  A page
+ * index outside the cache selects nothing and raises the index bit.
+ *
  * Used lengths (SparseFlashMlaGrad "Parameter Description": sequsedQOptional,
  * sequsedOriKvOptional, sequsedCmpKvOptional).  When given, sequence b takes part
  * with its first seqused_q[b] query tokens, seqused_kv[b] KV rows and
@@ -110,7 +120,7 @@
 extern "C" {
 #endif
 
-#define SA_ABI_VERSION 3
+#define SA_ABI_VERSION 4
 
 typedef enum sa_status {
   SA_OK = 0,
@@ -217,6 +227,9 @@ typedef struct sa_args {
                                     part (sequsedOriKv) */
   const int32_t* seqused_cmp;    /* optional, [B]: compressed KV rows of each sequence that take
                                     part (sequsedCmpKv) */
+  const int32_t* block_table;    /* optional, [B, max_pages]: paged KV cache (BSND only) */
+  int32_t page_size;             /* rows per cache page (with block_table) */
+  int32_t max_pages;             /* pages per sequence in block_table (with block_table) */
 } sa_args;
 
 /* Forward outputs (device): O bf16 [.., Hq, d_v]; lse fp32 [.., Hq]. */

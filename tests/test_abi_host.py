@@ -255,6 +255,24 @@ def test_dq_separate_is_ignored_past_the_block_kernels_slot_limit():
     assert _ws(a) == _ws(b)
 
 
+def test_paged_cache_validates_on_the_host():
+    """A paged KV cache: BSND only, page geometry covering s_kv, no compressed KV, and no
+    backward (SA_ERR_UNSUPPORTED); checked before any device work."""
+    ok = dict(block_table=FAKE, page_size=64, max_pages=2, t_kv=1024)
+    n = ctypes.c_size_t(0)
+    f = L.lib().sa_fwd_get_workspace_size
+    assert f(ctypes.byref(_args(**ok)), ctypes.byref(n)) == L.SA_OK
+    assert f(ctypes.byref(_args(**dict(ok, page_size=0))), ctypes.byref(n)) == L.SA_ERR_PARAM
+    assert f(ctypes.byref(_args(**dict(ok, max_pages=1))), ctypes.byref(n)) == L.SA_ERR_PARAM   # 64 < s_kv
+    assert f(ctypes.byref(_args(**dict(ok, t_kv=0))), ctypes.byref(n)) == L.SA_ERR_PARAM
+    tnd = dict(ok, layout_q=L.SA_LAYOUT_TND, layout_kv=L.SA_LAYOUT_TND, t_q=8, cu_seqlens_q=FAKE,
+               cu_seqlens_kv=FAKE)
+    assert f(ctypes.byref(_args(**tnd)), ctypes.byref(n)) == L.SA_ERR_UNSUPPORTED
+    assert L.lib().sa_bwd_get_workspace_size(ctypes.byref(_args(**ok)), ctypes.byref(n)) == L.SA_ERR_UNSUPPORTED
+    # the block kernels do not take a paged cache: the generic forward does
+    assert _plan(_args(**ok))[0] == L.SA_KERNEL_FWD_GENERIC
+
+
 def test_softmax_l1norm_validates_on_the_host():
     """sa_softmax_l1norm needs an output, its index list, and the forward's lse; all
     checked before any device work (no GPU here)."""

@@ -76,6 +76,7 @@ class SaArgs(ctypes.Structure):
         ("cu_seqlens_q", _vp), ("cu_seqlens_kv", _vp), ("cu_seqlens_cmp", _vp),
         ("ori_topk_len", _vp), ("cmp_topk_len", _vp), ("cmp_residual", _vp), ("sinks", _vp),
         ("seqused_q", _vp), ("seqused_kv", _vp), ("seqused_cmp", _vp),
+        ("block_table", _vp), ("page_size", ctypes.c_int32), ("max_pages", ctypes.c_int32),
     ]
 
 

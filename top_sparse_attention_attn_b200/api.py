@@ -54,6 +54,8 @@ class SparseAttention:
     seqused_q: torch.Tensor | None = None     # [B] int32: query tokens that take part
     seqused_kv: torch.Tensor | None = None    # [B] int32: original KV tokens that take part
     seqused_cmp: torch.Tensor | None = None   # [B] int32: compressed KV rows that take part
+    block_table: torch.Tensor | None = None   # [B, max_pages] int32: paged KV cache (k / v / kv are the cache)
+    page_size: int = 0
     ori_mask: str = "causal"
     cmp_mask: str = "causal"
     win_left: int = 0
@@ -103,6 +105,9 @@ class SparseAttention:
         a.sinks = _ptr(self.sinks)
         a.seqused_q, a.seqused_kv = _ptr(self.seqused_q), _ptr(self.seqused_kv)
         a.seqused_cmp = _ptr(self.seqused_cmp)
+        a.block_table = _ptr(self.block_table)
+        a.page_size = self.page_size
+        a.max_pages = 0 if self.block_table is None else int(self.block_table.shape[-1])
         return a
 
     # ---- allocation helpers ------------------------------------------------

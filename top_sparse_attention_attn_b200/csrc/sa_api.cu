@@ -34,12 +34,14 @@ bool cfa(const sa_args* a) { return a->cmp_topk == 0 && a->cmp_kv != nullptr && 
 bool has_cmp(const sa_args* a) { return a->cmp_topk > 0 || cfa(a); }
 // sequsedQ / sequsedOriKv / sequsedCmpKv given (the block kernels do not take them)
 bool has_used(const sa_args* a) { return a->seqused_q || a->seqused_kv || a->seqused_cmp; }
+// A paged KV cache (block_table): the forward only
+bool paged(const sa_args* a) { return a->block_table != nullptr; }
 
 Sizes sizes_of(const sa_args* a) {
   Sizes s;
   if (a->layout_q == SA_LAYOUT_BSND) {
     s.Tq = (long long)a->batch * a->s_q;
-    s.Tkv = (long long)a->batch * a->s_kv;
+    s.Tkv = paged(a) ? (long long)a->t_kv : (long long)a->batch * a->s_kv;  // a paged cache has t_kv rows
     s.Tcmp = has_cmp(a) ? (long long)a->batch * (a->s_kv / (a->cmp_ratio > 0 ? a->cmp_ratio : 1)) : 0;
   } else {
     s.Tq = a->t_q;
@@ -73,6 +75,12 @@ sa_status validate(const sa_args* a) {
   if (a->cmp_mask_mode != SA_MASK_NONE && a->cmp_mask_mode != SA_MASK_CAUSAL) return SA_ERR_PARAM;
   if (a->ori_mask_mode == SA_MASK_BAND && (a->ori_win_left < 0 || a->ori_win_right < 0)) return SA_ERR_PARAM;
   if (!isfinite(a->scale)) return SA_ERR_PARAM;
+  if (paged(a)) {
+    if (a->layout_q != SA_LAYOUT_BSND) return SA_ERR_UNSUPPORTED;
+    if (a->page_size < 1 || a->max_pages < 1 || a->t_kv < 1) return SA_ERR_PARAM;
+    if ((long long)a->max_pages * a->page_size < a->s_kv) return SA_ERR_PARAM;
+    if (has_cmp(a)) return SA_ERR_UNSUPPORTED;
+  }
   Sizes s = sizes_of(a);
   if (s.Tq >= (1ll << 30) || s.Tkv >= (1ll << 30) || s.Tcmp >= (1ll << 30)) return SA_ERR_PARAM;
   const int G = a->n_heads_q / a->n_heads_kv;
@@ -142,6 +150,9 @@ sa::Prob make_prob(const sa_args* a, int* status) {
   p.used_q = a->seqused_q;
   p.used_kv = a->seqused_kv;
   p.used_cmp = has_cmp(a) ? a->seqused_cmp : nullptr;
+  p.page_table = a->block_table;
+  p.page_size = a->page_size;
+  p.max_pages = a->max_pages;
   p.status = status;
   return p;
 }
@@ -161,13 +172,13 @@ bool use_kv_path(const sa_args* a) {
   if (a->flags & SA_FLAG_QUERY_STATIONARY_BWD) return false;
   const int G = a->n_heads_q / a->n_heads_kv;
   return a->layout_q == SA_LAYOUT_BSND && a->topk > 0 && a->block_size == 64 && a->s_q == a->s_kv &&
-         !a->kv_shared && !has_cmp(a) && !has_used(a) && a->sinks == nullptr && G <= 128 &&
+         !a->kv_shared && !has_cmp(a) && !has_used(a) && !paged(a) && a->sinks == nullptr && G <= 128 &&
          sa::kv_path_built(a->d_qk, a->d_v);
 }
 
 // Query-stationary block kernels (TMA-fed): 64-row blocks, separate K / V, no compressed KV.
 bool use_qb_path(const sa_args* a) {
-  return a->topk > 0 && a->topk <= sa::kQbMaxSlots && a->block_size == 64 && !a->kv_shared && !has_cmp(a) && !has_used(a) &&
+  return a->topk > 0 && a->topk <= sa::kQbMaxSlots && a->block_size == 64 && !a->kv_shared && !has_cmp(a) && !has_used(a) && !paged(a) &&
          sa::qb_path_built(a->d_qk, a->d_v);
 }
 
@@ -534,6 +545,7 @@ sa_status sa_bwd_get_workspace_size(const sa_args* args, size_t* ws_bytes) {
   if (!ws_bytes) return SA_ERR_NULLPTR;
   sa_status st = validate(args);
   if (st != SA_OK) return st;
+  if (paged(args)) return SA_ERR_UNSUPPORTED;  // a paged cache is an inference input: no backward
   *ws_bytes = bwd_ws_layout(args).total;
   return SA_OK;
 }
@@ -541,6 +553,7 @@ sa_status sa_bwd_get_workspace_size(const sa_args* args, size_t* ws_bytes) {
 sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_bytes, void* stream) {
   sa_status st = validate(args);
   if (st != SA_OK) return st;
+  if (paged(args)) return SA_ERR_UNSUPPORTED;
   if (!io) return SA_ERR_NULLPTR;
   Sizes s = sizes_of(args);
   const bool sinks = args->sinks != nullptr;

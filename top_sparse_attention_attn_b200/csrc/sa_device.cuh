@@ -34,6 +34,8 @@ struct Prob {
   int Tq, Tkv, Tcmp;
   int Hq, Hkv, G, dqk, dv, shared, bs, topk, cmp_topk, ratio, ori_mask, cmp_mask;
   const int *used_q, *used_kv, *used_cmp;  // sequsedQ / OriKv / CmpKv ([B]) or null
+  const int* page_table;                   // paged KV cache: [B, max_pages] or null
+  int page_size, max_pages;
   long long wl, wr;
   float scale;        // scaleValue
   float scale_log2;   // scale * log2(e)
@@ -232,6 +234,20 @@ __device__ __forceinline__ int slot_index(const Prob& p, const Unit& u, int tile
   return p.cmp_idx ? __ldg(p.cmp_idx + ug * p.cmp_topk + s) : s;
 }
 
+// Storage row code of sequence-local original-KV row `row` of unit u: contiguous
+// from kv0, or through the block table of a paged cache (-1, with the index bit,
+// for a page outside the cache).
+__device__ __forceinline__ int kv_code(const Prob& p, const Unit& u, long long row) {
+  if (!p.page_table) return u.kv0 + (int)row;
+  const int page = __ldg(p.page_table + (long long)u.b * p.max_pages + (int)(row / p.page_size));
+  const long long code = (long long)page * p.page_size + row % p.page_size;
+  if (page < 0 || code >= p.Tkv) {
+    if (p.status) atomicOr(p.status, kStatusIndexRange);
+    return -1;
+  }
+  return (int)code;
+}
+
 // Resolve row r (0..63) of tile `tile` of unit u, whose slot holds index x (from
 // slot_index), to a global row code, or -1.  An index past the end of its
 // sequence selects nothing and raises the status word's index bit.
@@ -249,7 +265,7 @@ __device__ __forceinline__ int resolve_row_x(const Prob& p, const Unit& u, int t
       }
       long long row = first + within;
       if (row >= u.Lk || !ori_mask_ok(p, u, (int)row)) return -1;
-      return u.kv0 + (int)row;
+      return kv_code(p, u, row);
     } else if (u.ori_mode == kOriToken) {
       if (x < 0) return -1;
       if (x >= u.Lk) {
@@ -257,11 +273,11 @@ __device__ __forceinline__ int resolve_row_x(const Prob& p, const Unit& u, int t
         return -1;
       }
       if (!ori_mask_ok(p, u, x)) return -1;
-      return u.kv0 + x;
+      return kv_code(p, u, x);
     } else {
       int row = u.lo + tile * kTileRows + r;
       if (row > u.hi) return -1;
-      return u.kv0 + row;
+      return kv_code(p, u, row);
     }
   }
   const int c = x;
