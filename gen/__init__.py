@@ -6,7 +6,7 @@ attention arithmetic.
 """
 
 from .configs import WORKLOADS, Workload, get_workload, scaled
-from .synth import make_inputs, make_paged_inputs, bf16_bits_from_f32, f32_from_bf16_bits
+from .synth import make_indexer_inputs, make_inputs, make_paged_inputs, bf16_bits_from_f32, f32_from_bf16_bits
 
 __all__ = [
     "WORKLOADS",
@@ -15,6 +15,7 @@ __all__ = [
     "scaled",
     "make_inputs",
     "make_paged_inputs",
+    "make_indexer_inputs",
     "bf16_bits_from_f32",
     "f32_from_bf16_bits",
 ]

@@ -262,3 +262,32 @@ def make_paged_inputs(seed: int, *, B: int, s_q: int, kv_lens, page: int, Hq: in
     out["_meta"] = dict(B=B, s_q=s_q, s_kv=max_pages * page, t_kv=rows, page=page, Hq=Hq, Hkv=Hkv, d_qk=d_qk,
                         d_v=d_v, kv_shared=kv_shared, block_size=block_size, topk=topk)
     return out
+
+
+def make_indexer_inputs(seed: int, *, lens, H: int, d: int, topk: int, layout: str = "TND") -> dict:
+    """Inputs of the indexer KL-loss backward: q [T, H, d] and k [T, d] (fp32 N(0, 1) ->
+    bf16 bits), w [T, H] fp32 N(0, 1) / sqrt(H), token indices drawn over each token's
+    visible prefix [0, t] (-1 padded, in random slot order), a per-token usable length,
+    and a target p: uniform random weights on the usable filled slots, normalised to 1."""
+    rng = np.random.default_rng(seed)
+    T = sum(lens)
+    q = bf16_bits_from_f32(rng.standard_normal((T, H, d), dtype=np.float32))
+    k = bf16_bits_from_f32(rng.standard_normal((T, d), dtype=np.float32))
+    w = (rng.standard_normal((T, H)) / np.sqrt(H)).astype(np.float32)
+    idx = np.full((T, topk), -1, dtype=np.int32)
+    off = 0
+    for L in lens:
+        for t in range(L):
+            sel = rng.permutation(t + 1)[:topk]
+            row = np.full(topk, -1, dtype=np.int32)
+            row[:len(sel)] = sel
+            idx[off + t] = rng.permutation(row)
+        off += L
+    tlen = rng.integers(topk // 2, topk + 1, T).astype(np.int32)
+    p = rng.random((T, topk)).astype(np.float32)
+    usable = (idx >= 0) & (np.arange(topk)[None, :] < tlen[:, None])
+    p = np.where(usable, p, 0.0).astype(np.float32)
+    s = p.sum(axis=1, keepdims=True)
+    p = np.where(s > 0, p / np.where(s > 0, s, 1), 0.0).astype(np.float32)
+    starts = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return dict(q=q, k=k, w=w, idx=idx, topk_len=tlen, p=p, cu_seqlens=starts, lens=tuple(lens), layout=layout)

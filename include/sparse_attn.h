@@ -320,6 +320,46 @@ size_t sa_bwd_no_alloc_max_workspace(void);
  * sa_fwd.  Asynchronous. */
 sa_status sa_softmax_l1norm(const sa_args* args, const float* lse, float* ori_out, float* cmp_out, void* stream);
 
+/* The lightning indexer's KL-loss backward (aclnnSparseLightningIndexerGradKLLoss,
+ * "Formula"): over token t's used slots j (index >= 0, before topk_len, inside the
+ * sequence, not in t's future),
+ *   I[t, j] = sum_h w[t, h] ReLU(q[t, h] . k[j]),  L = sum_t KL(p[t, :] || Softmax(I[t, :])),
+ *   dI = Softmax(I) - p,  dw[t, h] = sum_j ReLU(q[t, h] . k[j]) dI[t, j],
+ *   dS = w[t, h] (q[t, h] . k[j] > 0) dI[t, j],  dq[t] = dS k,  dk[j] += dS^T q[t].
+ * p's entries at unused slots are ignored; 0 log 0 = 0; no scale on q k^T. */
+typedef struct sa_indexer_args {
+  int32_t layout;          /* sa_layout of every tensor (BSND or TND) */
+  int32_t batch;           /* B */
+  int32_t s_q, s_kv;       /* BSND sequence lengths */
+  int32_t t_q, t_kv;       /* TND packed token counts */
+  int32_t n_heads;         /* indexer query heads H: 16, 32 or 64 */
+  int32_t d;               /* head dim: 64 or 128 */
+  int32_t topk;            /* index slots per token (>= 1) */
+  const void* q;           /* bf16 [.., H, d] */
+  const void* k;           /* bf16 [.., d] (one indexer key head) */
+  const float* w;          /* fp32 [.., H] per-token head weights */
+  const int32_t* idx;      /* [.., topk] token indices local to the sequence, -1 = empty */
+  const int32_t* topk_len; /* optional [..]: usable slots per token */
+  const float* p;          /* fp32 [.., topk] target distribution (e.g. sa_softmax_l1norm's ori_out) */
+  const int32_t* cu_seqlens_q;   /* TND: B + 1 offsets */
+  const int32_t* cu_seqlens_kv;  /* TND: B + 1 offsets */
+} sa_indexer_args;
+
+typedef struct sa_indexer_grads {
+  float* loss;             /* optional, fp32 [..]: each token's KL term */
+  void* dq;                /* bf16 [.., H, d] */
+  void* dk;                /* bf16 [.., d] */
+  float* dw;               /* fp32 [.., H] */
+} sa_indexer_grads;
+
+/* Workspace of sa_indexer_kl_grad: a status word and the fp32 dk accumulator. */
+sa_status sa_indexer_kl_grad_get_workspace_size(const sa_indexer_args* args, size_t* ws_bytes);
+/* Errors: SA_ERR_NULLPTR (a required pointer), SA_ERR_PARAM (sizes, alignment),
+ * SA_ERR_UNSUPPORTED (H or d not built), SA_ERR_WORKSPACE.  Asynchronous; an index
+ * past its sequence sets the status word's index bit (sa_read_status). */
+sa_status sa_indexer_kl_grad(const sa_indexer_args* args, const sa_indexer_grads* grads, void* ws,
+                             size_t ws_bytes, void* stream);
+
 /* rowsum(dO o O) alone -- the "FlashSoftmaxGrad(dO, O)" / "SoftmaxGrad(dO, O)"
  * term of aclnnSparseFlashAttentionGrad Phase 2 and SparseFlashMlaGrad Stage 2:
  * delta[token, h] = sum_c d_o[token, h, c] * o[token, h, c] in fp32.

@@ -255,6 +255,26 @@ def test_dq_separate_is_ignored_past_the_block_kernels_slot_limit():
     assert _ws(a) == _ws(b)
 
 
+def test_indexer_kl_grad_validates_on_the_host():
+    a = L.SaIndexerArgs()
+    a.layout, a.batch, a.s_q, a.s_kv = L.SA_LAYOUT_BSND, 2, 64, 64
+    a.n_heads, a.d, a.topk = 64, 128, 32
+    a.q = a.k = a.w = a.idx = a.p = FAKE
+    n = ctypes.c_size_t(0)
+    f = L.lib().sa_indexer_kl_grad_get_workspace_size
+    assert f(ctypes.byref(a), ctypes.byref(n)) == L.SA_OK
+    assert n.value >= 2 * 64 * 128 * 4                                # the fp32 dk accumulator
+    for field, val, want in (("n_heads", 48, L.SA_ERR_UNSUPPORTED), ("d", 96, L.SA_ERR_UNSUPPORTED),
+                             ("topk", 0, L.SA_ERR_PARAM), ("p", None, L.SA_ERR_NULLPTR), ("layout", 9, L.SA_ERR_PARAM)):
+        b = L.SaIndexerArgs.from_buffer_copy(a)
+        setattr(b, field, val)
+        assert f(ctypes.byref(b), ctypes.byref(n)) == want, field
+    g = L.SaIndexerGrads(loss=None, dq=FAKE, dk=FAKE, dw=None)
+    assert L.lib().sa_indexer_kl_grad(ctypes.byref(a), ctypes.byref(g), FAKE, 1 << 30, None) == L.SA_ERR_NULLPTR
+    g.dw = FAKE
+    assert L.lib().sa_indexer_kl_grad(ctypes.byref(a), ctypes.byref(g), FAKE, 16, None) == L.SA_ERR_WORKSPACE
+
+
 def test_paged_cache_validates_on_the_host():
     """A paged KV cache: BSND only, page geometry covering s_kv, no compressed KV, and no
     backward (SA_ERR_UNSUPPORTED); checked before any device work."""

@@ -7,6 +7,6 @@ a thin wrapper that marshals torch tensors into it.
 
 from . import _lib
 from ._lib import SaError
-from .api import SparseAttention
+from .api import SparseAttention, indexer_kl_grad
 
-__all__ = ["SparseAttention", "SaError", "_lib"]
+__all__ = ["SparseAttention", "SaError", "_lib", "indexer_kl_grad"]

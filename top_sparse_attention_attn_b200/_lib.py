@@ -80,6 +80,20 @@ class SaArgs(ctypes.Structure):
     ]
 
 
+class SaIndexerArgs(ctypes.Structure):
+    _fields_ = [
+        ("layout", ctypes.c_int32), ("batch", ctypes.c_int32), ("s_q", ctypes.c_int32), ("s_kv", ctypes.c_int32),
+        ("t_q", ctypes.c_int32), ("t_kv", ctypes.c_int32), ("n_heads", ctypes.c_int32), ("d", ctypes.c_int32),
+        ("topk", ctypes.c_int32),
+        ("q", _vp), ("k", _vp), ("w", _vp), ("idx", _vp), ("topk_len", _vp), ("p", _vp),
+        ("cu_seqlens_q", _vp), ("cu_seqlens_kv", _vp),
+    ]
+
+
+class SaIndexerGrads(ctypes.Structure):
+    _fields_ = [("loss", _vp), ("dq", _vp), ("dk", _vp), ("dw", _vp)]
+
+
 class SaFwdOut(ctypes.Structure):
     _fields_ = [("o", _vp), ("lse", _vp)]
 
@@ -103,7 +117,8 @@ EXPORTS = ["sa_fwd_get_workspace_size", "sa_fwd", "sa_bwd_get_workspace_size", "
            "sa_set_timing_events", "sa_kernel_launch_count", "sa_bwd_no_alloc",
            "sa_bwd_no_alloc_max_workspace", "sa_selftest_mma", "sa_selftest_wait_timeout",
            "sa_selftest_mma2", "sa_plan", "sa_read_status", "sa_bwd_no_alloc_read_status",
-           "sa_debug_block_index", "sa_selftest_gather4", "sa_softmax_l1norm"]
+           "sa_debug_block_index", "sa_selftest_gather4", "sa_softmax_l1norm",
+           "sa_indexer_kl_grad_get_workspace_size", "sa_indexer_kl_grad"]
 
 
 def lib() -> ctypes.CDLL:
@@ -121,6 +136,8 @@ def lib() -> ctypes.CDLL:
         L.sa_bwd.argtypes = [P(SaArgs), P(SaBwdIo), _vp, ctypes.c_size_t, _vp]
         L.sa_softmax_grad_preprocess.argtypes = [P(SaArgs), _vp, _vp, _vp, _vp]
         L.sa_softmax_l1norm.argtypes = [P(SaArgs), _vp, _vp, _vp, _vp]
+        L.sa_indexer_kl_grad_get_workspace_size.argtypes = [P(SaIndexerArgs), P(ctypes.c_size_t)]
+        L.sa_indexer_kl_grad.argtypes = [P(SaIndexerArgs), P(SaIndexerGrads), _vp, ctypes.c_size_t, _vp]
         L.sa_debug_resolve.argtypes = [P(SaArgs), _vp, _vp, ctypes.c_int32, _vp]
         L.sa_status_string.argtypes = [ctypes.c_int32]
         L.sa_status_string.restype = ctypes.c_char_p
@@ -213,6 +230,18 @@ def sa_selftest_wait_timeout(status: int, waited: int, stream: int = 0) -> None:
 def sa_softmax_grad_preprocess(args: SaArgs, o: int, d_o: int, delta: int, stream: int = 0) -> None:
     _check(lib().sa_softmax_grad_preprocess(ctypes.byref(args), o, d_o, delta, stream),
            "sa_softmax_grad_preprocess")
+
+
+def sa_indexer_kl_grad_get_workspace_size(args: SaIndexerArgs) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().sa_indexer_kl_grad_get_workspace_size(ctypes.byref(args), ctypes.byref(n)),
+           "sa_indexer_kl_grad_get_workspace_size")
+    return n.value
+
+
+def sa_indexer_kl_grad(args: SaIndexerArgs, grads: SaIndexerGrads, ws: int, ws_bytes: int, stream: int = 0) -> None:
+    _check(lib().sa_indexer_kl_grad(ctypes.byref(args), ctypes.byref(grads), ws, ws_bytes, stream),
+           "sa_indexer_kl_grad")
 
 
 def sa_softmax_l1norm(args: SaArgs, lse: int, ori_out, cmp_out, stream: int = 0) -> None:

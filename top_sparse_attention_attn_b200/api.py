@@ -246,3 +246,33 @@ class SparseAttention:
 
 def default_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)
+
+
+def indexer_kl_grad(q, k, w, idx, p, *, topk_len=None, cu_seqlens_q=None, cu_seqlens_kv=None, batch=None,
+                    stream=None):
+    """The lightning indexer's KL-loss backward (sa_indexer_kl_grad).
+
+    BSND: q [B, S, H, d], k [B, S_kv, d], w [B, S, H], idx / p [B, S, topk], topk_len
+    [B, S] (optional).  TND: the same without B (token-major) plus cu_seqlens_q / _kv.
+    Returns (loss per token fp32, dq bf16 like q, dk bf16 like k, dw fp32 like w)."""
+    tnd = cu_seqlens_q is not None
+    a = L.SaIndexerArgs()
+    a.layout = L.SA_LAYOUT_TND if tnd else L.SA_LAYOUT_BSND
+    if tnd:
+        a.batch = int(cu_seqlens_q.numel()) - 1 if batch is None else batch
+        a.t_q, a.t_kv = int(q.shape[0]), int(k.shape[0])
+    else:
+        a.batch, a.s_q, a.s_kv = int(q.shape[0]), int(q.shape[1]), int(k.shape[1])
+    a.n_heads, a.d, a.topk = int(q.shape[-2]), int(q.shape[-1]), int(idx.shape[-1])
+    a.q, a.k, a.w, a.idx, a.p = _ptr(q), _ptr(k), _ptr(w), _ptr(idx), _ptr(p)
+    a.topk_len = _ptr(topk_len)
+    a.cu_seqlens_q, a.cu_seqlens_kv = _ptr(cu_seqlens_q), _ptr(cu_seqlens_kv)
+    loss = torch.empty(q.shape[:-2], dtype=torch.float32, device=q.device)
+    dq, dk = torch.empty_like(q), torch.empty_like(k)
+    dw = torch.empty_like(w)
+    g = L.SaIndexerGrads(loss=_ptr(loss), dq=_ptr(dq), dk=_ptr(dk), dw=_ptr(dw))
+    n = L.sa_indexer_kl_grad_get_workspace_size(a)
+    ws = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
+    st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    L.sa_indexer_kl_grad(a, g, _ptr(ws), n, st)
+    return loss, dq, dk, dw

@@ -678,6 +678,82 @@ sa_status sa_softmax_l1norm(const sa_args* args, const float* lse, float* ori_ou
   return cuda_status(sa::launch_softmax_l1norm(p, lse, ori_out, cmp_out, static_cast<cudaStream_t>(stream)));
 }
 
+static sa_status ix_validate(const sa_indexer_args* a, long long* Tq, long long* Tkv) {
+  if (!a) return SA_ERR_NULLPTR;
+  if (a->layout != SA_LAYOUT_BSND && a->layout != SA_LAYOUT_TND) return SA_ERR_PARAM;
+  if (a->batch < 0 || a->topk < 1) return SA_ERR_PARAM;
+  if (a->layout == SA_LAYOUT_BSND) {
+    if (a->s_q < 0 || a->s_kv < 0) return SA_ERR_PARAM;
+    *Tq = (long long)a->batch * a->s_q;
+    *Tkv = (long long)a->batch * a->s_kv;
+  } else {
+    if (a->t_q < 0 || a->t_kv < 0) return SA_ERR_PARAM;
+    *Tq = a->t_q;
+    *Tkv = a->t_kv;
+  }
+  if (*Tq >= (1ll << 31) || *Tkv >= (1ll << 30)) return SA_ERR_PARAM;
+  if (!sa::ix_built(a->n_heads, a->d)) return SA_ERR_UNSUPPORTED;
+  if (*Tq > 0) {
+    if (!a->q || !a->k || !a->w || !a->idx || !a->p) return SA_ERR_NULLPTR;
+    if (a->layout == SA_LAYOUT_TND && (!a->cu_seqlens_q || !a->cu_seqlens_kv || a->batch < 1)) return SA_ERR_NULLPTR;
+    if (!aligned16(a->q) || !aligned16(a->k)) return SA_ERR_PARAM;
+  }
+  return SA_OK;
+}
+
+sa_status sa_indexer_kl_grad_get_workspace_size(const sa_indexer_args* args, size_t* ws_bytes) {
+  if (!ws_bytes) return SA_ERR_NULLPTR;
+  long long Tq = 0, Tkv = 0;
+  sa_status st = ix_validate(args, &Tq, &Tkv);
+  if (st != SA_OK) return st;
+  *ws_bytes = kAlign + align_up((size_t)Tkv * args->d * sizeof(float));
+  return SA_OK;
+}
+
+sa_status sa_indexer_kl_grad(const sa_indexer_args* args, const sa_indexer_grads* g, void* ws, size_t ws_bytes,
+                             void* stream) {
+  long long Tq = 0, Tkv = 0;
+  sa_status st = ix_validate(args, &Tq, &Tkv);
+  if (st != SA_OK) return st;
+  if (!g) return SA_ERR_NULLPTR;
+  if (Tq == 0) return SA_OK;
+  if (!g->dq || !g->dk || !g->dw) return SA_ERR_NULLPTR;
+  if (!aligned16(g->dq) || !aligned16(g->dk)) return SA_ERR_PARAM;
+  const size_t need = kAlign + align_up((size_t)Tkv * args->d * sizeof(float));
+  if (!ws || ws_bytes < need) return SA_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(ws);
+  if (cudaMemsetAsync(base, 0, need, cs) != cudaSuccess) return SA_ERR_CUDA;
+  sa::IxArgs a;
+  memset(&a, 0, sizeof(a));
+  a.layout = args->layout;
+  a.B = args->batch;
+  a.s_q = args->s_q;
+  a.s_kv = args->s_kv;
+  a.Tq = (int)Tq;
+  a.Tkv = (int)Tkv;
+  a.H = args->n_heads;
+  a.D = args->d;
+  a.topk = args->topk;
+  a.q = static_cast<const bf16*>(args->q);
+  a.k = static_cast<const bf16*>(args->k);
+  a.w = args->w;
+  a.idx = args->idx;
+  a.topk_len = args->topk_len;
+  a.p = args->p;
+  a.cu_q = args->cu_seqlens_q;
+  a.cu_kv = args->cu_seqlens_kv;
+  a.loss = g->loss;
+  a.dq = static_cast<bf16*>(g->dq);
+  a.dk_acc = reinterpret_cast<float*>(base + kAlign);
+  a.dw = g->dw;
+  a.status = reinterpret_cast<int*>(base);
+  cudaError_t e = sa::launch_indexer_kl(a, cs);
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+  if (Tkv > 0) e = sa::launch_to_bf16(a.dk_acc, static_cast<bf16*>(g->dk), Tkv * args->d, cs);
+  return cuda_status(e);
+}
+
 sa_status sa_debug_resolve(const sa_args* args, int32_t* rows, int32_t* counts, int32_t max_rows, void* stream) {
   sa_status st = validate(args);
   if (st != SA_OK) return st;

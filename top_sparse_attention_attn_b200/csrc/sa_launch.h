@@ -80,6 +80,24 @@ struct Cvt {
 };
 cudaError_t launch_to_bf16_multi(const Cvt* jobs, int njobs, cudaStream_t st);
 cudaError_t launch_check(const Prob& p, cudaStream_t st);
+// The lightning indexer's KL-loss backward (one CTA per token).
+struct IxArgs {
+  int layout, B, s_q, s_kv, Tq, Tkv, H, D, topk;
+  const bf16* q;        // [Tq, H, D]
+  const bf16* k;        // [Tkv, D]
+  const float* w;       // [Tq, H]
+  const int* idx;       // [Tq, topk]
+  const int* topk_len;  // [Tq] or null
+  const float* p;       // [Tq, topk]
+  const int *cu_q, *cu_kv;
+  float* loss;          // [Tq] or null
+  bf16* dq;             // [Tq, H, D]
+  float* dk_acc;        // [Tkv, D] fp32, zeroed by the caller
+  float* dw;            // [Tq, H]
+  int* status;
+};
+bool ix_built(int H, int D);
+cudaError_t launch_indexer_kl(const IxArgs& a, cudaStream_t st);
 // SoftmaxL1Norm outputs: ori_out [Tq, Hkv, topk] and / or cmp_out [Tq, Hkv,
 // cmp_topk] fp32 (either may be null), from the forward's lse.
 cudaError_t launch_softmax_l1norm(const Prob& p, const float* lse, float* ori_out, float* cmp_out, cudaStream_t st);
