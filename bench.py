@@ -577,7 +577,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     flags = 0
     for f in filter(None, args.flags.split(",")):
         flags |= {"dq_separate": L.SA_FLAG_DQ_SEPARATE, "query_stationary": L.SA_FLAG_QUERY_STATIONARY_BWD,
-                  "fwd_block_tc": L.SA_FLAG_FWD_BLOCK_TC}[f]
+                  "fwd_block_tc": L.SA_FLAG_FWD_BLOCK_TC, "token_fwd_unpaired": L.SA_FLAG_TOKEN_FWD_UNPAIRED}[f]
     sa, t, inputs, work = setup_problem(w, dev, flags, host_dense=False)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
@@ -771,7 +771,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager calls instead of CUDA-graph replays")
     ap.add_argument("--no-per-workload", action="store_true", help="skip the other workloads' figures")
-    ap.add_argument("--flags", default="", help="kernel variants for measurements: dq_separate | query_stationary | fwd_block_tc")
+    ap.add_argument("--flags", default="", help="kernel variants for measurements: dq_separate | query_stationary | fwd_block_tc | "
+                    "token_fwd_unpaired")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -164,6 +164,12 @@ typedef enum sa_dtype { SA_DTYPE_BF16 = 0, SA_DTYPE_FP16 = 1 } sa_dtype;
  * tcgen05 version instead (scores and output in TMEM, M = 128 key pairs against
  * the 16 heads of an item); it computes the same result and measured slower. */
 #define SA_FLAG_FWD_BLOCK_TC 8u
+/* Token-level tensor-core forward: with a multiple of 128 query heads per kv-head
+ * the two 64-head CTAs of a token run as a thread-block cluster and share the row
+ * gathers (each gathers every other 32-row sub-tile and copies it to the other
+ * over distributed shared memory).  This flag runs every 64-head CTA on its own
+ * instead; the result is bit-identical. */
+#define SA_FLAG_TOKEN_FWD_UNPAIRED 16u
 
 /* Kernels reported by sa_plan(). */
 typedef enum sa_kernel {

@@ -100,6 +100,39 @@ def test_block_level_forward_on_tcgen05(name):
     run_full_comparison(w, kw, flags=L.SA_FLAG_FWD_BLOCK_TC)
 
 
+TOKEN_H128 = {
+    **{k: SMALL[k] for k in ("token_h128_topk", "swa_cmp_h128")},
+    # a 2048-token sequence with top-2048: every sub-tile pattern of the paired gathers
+    "token_h128_s2048": (scaled("cfg3", "s2048", S=2048, Hq=128, seed=44), {}),
+}
+
+
+@pytest.mark.parametrize("name", list(TOKEN_H128))
+def test_token_forward_pair_equals_unpaired(name):
+    """128 heads per kv-head: the cluster-paired token forward (each CTA of a token
+    gathers every other sub-tile and copies it to the other) gives bit-identical O
+    and lse to the unpaired kernel (SA_FLAG_TOKEN_FWD_UNPAIRED), which the oracle
+    comparison then checks element by element."""
+    _need_gpu()
+    from top_sparse_attention_attn_b200 import _lib as L
+    from gpu_harness import device_problem
+    w, kw = TOKEN_H128[name]
+    inputs = make_inputs(w, **kw)
+    res = []
+    for flags in (0, L.SA_FLAG_TOKEN_FWD_UNPAIRED):
+        sa, _ = device_problem(w, inputs, flags)
+        assert sa.plan()[0] == L.SA_KERNEL_FWD_TOKEN_TC
+        ws = sa.fwd_workspace()
+        o, lse = sa.forward(ws=ws)
+        torch.cuda.synchronize()
+        assert sa.read_status(ws) == 0
+        res.append((o.view(torch.int16).cpu().numpy(), lse.cpu().numpy()))
+    np.testing.assert_array_equal(res[0][0], res[1][0])
+    np.testing.assert_array_equal(res[0][1], res[1][1])
+    if name != "token_h128_s2048":
+        run_full_comparison(w, kw, flags=L.SA_FLAG_TOKEN_FWD_UNPAIRED)
+
+
 @pytest.mark.parametrize("cfg", ["cfg2", "cfg1", "cfg5", "cfg4", "cfg3"])
 def test_full_size_sampled(cfg):
     _need_gpu()

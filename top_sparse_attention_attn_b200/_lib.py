@@ -33,6 +33,7 @@ SA_FLAG_CHECK = 1
 SA_FLAG_QUERY_STATIONARY_BWD = 2
 SA_FLAG_DQ_SEPARATE = 4
 SA_FLAG_FWD_BLOCK_TC = 8
+SA_FLAG_TOKEN_FWD_UNPAIRED = 16
 
 # sa_kernel (sa_plan)
 SA_KERNEL_FWD_BLOCK = 1

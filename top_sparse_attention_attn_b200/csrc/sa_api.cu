@@ -537,7 +537,8 @@ sa_status sa_fwd(const sa_args* args, const sa_fwd_out* out, void* ws, size_t ws
     return cuda_status(sa::launch_qb(q, args->k, args->v, false, cs));
   }
   if (choice == SA_KERNEL_FWD_TOKEN_TC)
-    return cuda_status(sa::launch_tk_fwd(p, static_cast<bf16*>(out->o), out->lse, cs));
+    return cuda_status(sa::launch_tk_fwd(p, static_cast<bf16*>(out->o), out->lse,
+                                         !(args->flags & SA_FLAG_TOKEN_FWD_UNPAIRED), cs));
   return cuda_status(sa::launch_fwd(p, static_cast<bf16*>(out->o), out->lse, cs));
 }
 

@@ -350,49 +350,59 @@ __global__ void __launch_bounds__(WITH_DQ ? 320 : 192, 1) kv_bwd_kernel(const __
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
       constexpr uint32_t idQ = idesc_bf16(128, WITH_DQ ? DQK : 64, false, true);
+      // operand descriptors at the buffers' starts (K-major "k", MN-major "n")
+      const uint64_t dKk = sdesc(sK, 16, 1024), dVk = sdesc(sV, 16, 1024), dKn = sdesc(sK, 8192, 1024);
+      const uint64_t dPSk = sdesc(sPS, 16, 1024), dPSn = sdesc(sPS, 16384, 1024);
       bool ok = mbar_wait(&bars.kv_full, 0, abort_flag, a.status);
       for (int i = 0; ok && i < ntiles; ++i) {
         const int st = i & 1;
         if (!mbar_wait(&bars.q_full[st], (i >> 1) & 1, abort_flag, a.status)) break;
         tc_fence_after();
         const uint32_t q = sQ + st * PL::kQStage, d = sDO + st * PL::kDOStage;
+        const uint64_t dQk = sdesc(q, 16, 1024), dDOk = sdesc(d, 16, 1024);
+        const uint64_t dQn = sdesc(q, 16384, 1024), dDOn = sdesc(d, 16384, 1024);
         // S = Q K^T, dP = dO V^T
+#pragma unroll
         for (int kk = 0; kk < DQK / 16; ++kk)
-          mma_bf16(tmem + PL::cS, sdesc(q + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                   sdesc(sK + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), idS, kk > 0);
+          mma_bf16(tmem + PL::cS, desc_add(dQk, (kk >> 2) * 16384 + (kk & 3) * 32),
+                   desc_add(dKk, (kk >> 2) * 8192 + (kk & 3) * 32), idS, kk > 0);
+#pragma unroll
         for (int kk = 0; kk < DV / 16; ++kk)
-          mma_bf16(tmem + PL::cDP, sdesc(d + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                   sdesc(sV + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), idS, kk > 0);
+          mma_bf16(tmem + PL::cDP, desc_add(dDOk, (kk >> 2) * 16384 + (kk & 3) * 32),
+                   desc_add(dVk, (kk >> 2) * 8192 + (kk & 3) * 32), idS, kk > 0);
         mma_commit(&bars.s_full);
         if (!mbar_wait(&bars.p_full, i & 1, abort_flag, a.status)) break;
         tc_fence_after();
         // dV^T += dO^T P
+#pragma unroll
         for (int t = 0; t < PL::NV; ++t) {
           const int M = min(128, DV - 128 * t);
           const uint32_t id = idesc_bf16(M, 64, true, true);
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_bf16(tmem + PL::cDV + 64 * t, sdesc(d + 2 * t * 16384 + kk * 2048, 16384, 1024),
-                     sdesc(sPS + kk * 2048, 16384, 1024), id, (i > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16(tmem + PL::cDV + 64 * t, desc_add(dDOn, 2 * t * 16384 + kk * 2048), desc_add(dPSn, kk * 2048), id,
+                     (i > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&bars.p_free);
         if (!mbar_wait(&bars.ds_full, i & 1, abort_flag, a.status)) break;
         tc_fence_after();
         // dK^T += Q^T dS
+#pragma unroll
         for (int t = 0; t < PL::NK; ++t) {
           const int M = min(128, DQK - 128 * t);
           const uint32_t id = idesc_bf16(M, 64, true, true);
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_bf16(tmem + ((uint32_t)PL::kDkLane << 16) + PL::cDK + 64 * t,
-                     sdesc(q + 2 * t * 16384 + kk * 2048, 16384, 1024),
-                     sdesc(sPS + kk * 2048, 16384, 1024), id, (i > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16(tmem + ((uint32_t)PL::kDkLane << 16) + PL::cDK + 64 * t, desc_add(dQn, 2 * t * 16384 + kk * 2048),
+                     desc_add(dPSn, kk * 2048), id, (i > 0 || kk > 0) ? 1u : 0u);
         }
         if (WITH_DQ) {
           if (i > 0 && !mbar_wait(&bars.dq_free, (i - 1) & 1, abort_flag, a.status)) break;
           tc_fence_after();
           // dQ = dS K_j  (K_j as an MN-major B: N = DQK columns in 64-wide slabs of 64 rows)
+#pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + PL::cDQ, sdesc(sPS + kk * 32, 16, 1024), sdesc(sK + kk * 2048, 8192, 1024), idQ,
-                     kk > 0);
+            mma_bf16(tmem + PL::cDQ, desc_add(dPSk, kk * 32), desc_add(dKn, kk * 2048), idQ, kk > 0);
         }
         mma_commit(&bars.q_empty[st]);
         mma_commit(&bars.tile_done);

@@ -50,6 +50,28 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, 
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// launch_pdl with thread-block clusters of `cluster_x` consecutive CTAs (grid a
+// multiple of cluster_x).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                               cudaStream_t st, unsigned cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // TMA tensor map over a [rows][cols] bf16 matrix (row stride in bytes), boxes
 // of box_rows x 64 columns, 128-byte swizzle, zero fill out of range.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
@@ -71,7 +93,7 @@ cudaError_t launch_to_bf16(const float* src, bf16* dst, long long n, cudaStream_
 bool tk_path_built(int dqk, int dv, int shared, int G);
 cudaError_t launch_tk_bwd(const Prob& p, const float* lse, const float* delta, const bf16* d_o, const BwdOut& out,
                           cudaStream_t st);
-cudaError_t launch_tk_fwd(const Prob& p, bf16* o, float* lse, cudaStream_t st);
+cudaError_t launch_tk_fwd(const Prob& p, bf16* o, float* lse, bool pair, cudaStream_t st);
 // Up to four fp32 -> bf16 conversions in one launch (each n a multiple of 8).
 struct Cvt {
   const float* src;

@@ -84,11 +84,25 @@ __device__ __forceinline__ uint32_t tk_kv_addr(uint32_t stage, int r, int c) {
 // copies have landed (TMA_SLABS < NSQ).  The next sub-tile's indices are loaded
 // while the current one is issued.  Stage reuse waits for kv_empty; on abort the
 // warp stops issuing.  Before returning it waits (bounded) for every copy to land.
-template <int NST, int TMA_SLABS>
+//
+// PAIR: the two CTAs of a cluster (two head slices of one token) select the same
+// rows.  Each gathers half of every sub-tile (rows 16 * rank .. + 15, 36 gathers)
+// into its own stage, completing half_full; the copier warp of tk_fwd_kernel then
+// copies that half into the same rows of the partner's stage.  kv_full needs both
+// halves: the copier's arrival once this CTA's half has landed, and the partner's
+// bytes (expected by the loader).  Before gathering into a stage again the loader
+// waits for copy_done (the partner has received this CTA's previous half, so the
+// copy has read it), then tells the partner through peer_ready that the stage may
+// take the partner's half (its previous use has been consumed).  Every
+// one of these barriers completes once per use of a stage (phase (i / NST) & 1).
+template <int NST, int TMA_SLABS, bool PAIR = false>
 __device__ void tk_load_rows(const Prob& p, const Unit& u, int g, int nsub, uint32_t sKV, int* codes,
                              const CUtensorMap* mapKV, const CUtensorMap* mapCmp, bool has_cmp, uint64_t* kv_full,
-                             uint64_t* kv_empty, uint64_t* codes_full, volatile int* abort_flag, int lane) {
+                             uint64_t* kv_empty, uint64_t* codes_full, volatile int* abort_flag, int lane,
+                             uint64_t* half_full = nullptr, uint64_t* peer_ready = nullptr,
+                             uint64_t* copy_done = nullptr, uint32_t crank = 0) {
   constexpr int CP_PIECES = (tk::NSQ - TMA_SLABS) * 8;  // 16-byte pieces of a row copied by cp.async
+  static_assert(!PAIR || CP_PIECES == 0, "a pair gathers every slab by TMA");
   int x_next = nsub > 0 ? slot_index(p, u, 0, lane) : -1;
   int issued = 0;
   for (int i = 0; i < nsub; ++i) {
@@ -96,7 +110,12 @@ __device__ void tk_load_rows(const Prob& p, const Unit& u, int g, int nsub, uint
     const int x = x_next;
     if (i + 1 < nsub) x_next = slot_index(p, u, (i + 1) >> 1, 32 * ((i + 1) & 1) + lane);  // prefetch
     bool ok = true;
-    if (lane == 0 && i >= NST) ok = mbar_wait(&kv_empty[st], ((i / NST) - 1) & 1, abort_flag, p.status);
+    if (lane == 0) {
+      if (i >= NST) ok = mbar_wait(&kv_empty[st], ((i / NST) - 1) & 1, abort_flag, p.status);
+      if (PAIR && ok && i >= NST) ok = mbar_wait_cluster(&copy_done[st], ((i / NST) - 1) & 1, abort_flag, p.status);
+      // the partner's half may land (once signalled, the stage is armed below and drained on exit)
+      if (PAIR && ok) mbar_arrive_remote(mapa_shared(smem_u32(&peer_ready[st]), crank ^ 1u));
+    }
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (!ok) break;
     const int code = resolve_row_x(p, u, tile, r, x);
@@ -107,20 +126,24 @@ __device__ void tk_load_rows(const Prob& p, const Unit& u, int g, int nsub, uint
     if (TMA_SLABS > 0) {
       const bool cmp_tile = tile >= u.n_ori_tiles && has_cmp;
       const int y = code >= 0 ? (code & ~kCmpFlag) : 0;  // invisible rows load row 0 (masked later)
-      if (lane == 0) mbar_arrive_tx(&kv_full[st], (uint32_t)(TMA_SLABS * tk::NK * 128));
+      uint64_t* gbar = PAIR ? &half_full[st] : &kv_full[st];
+      if (lane == 0) {
+        if (PAIR) mbar_arrive_tx(&kv_full[st], (uint32_t)(TMA_SLABS * 16 * 128));  // the partner's half
+        mbar_arrive_tx(gbar, (uint32_t)(TMA_SLABS * (PAIR ? 16 : tk::NK) * 128));
+      }
       __syncwarp();
       const int q4 = lane & 7;
       const int y0 = __shfl_sync(0xffffffffu, y, 4 * q4), y1 = __shfl_sync(0xffffffffu, y, 4 * q4 + 1);
       const int y2 = __shfl_sync(0xffffffffu, y, 4 * q4 + 2), y3 = __shfl_sync(0xffffffffu, y, 4 * q4 + 3);
-      if (lane < 8) {
+      if (lane < 8 && (!PAIR || (uint32_t)(lane >> 2) == crank)) {
         const CUtensorMap* map = cmp_tile ? mapCmp : mapKV;
         const uint32_t dst = stage + q4 * 4 * 128;
 #pragma unroll
         for (int s = 0; s < TMA_SLABS; ++s)
-          tma_gather4(dst + s * (tk::NK * 128), map, g * tk::DQK + 64 * s, y0, y1, y2, y3, &kv_full[st]);
+          tma_gather4(dst + s * (tk::NK * 128), map, g * tk::DQK + 64 * s, y0, y1, y2, y3, gbar);
       }
     }
-    if (CP_PIECES > 0) {
+    if constexpr (CP_PIECES > 0) {
       // lanes take consecutive 16-byte pieces of one row; invisible rows are zero-filled
       const int* cd = codes + (i & 3) * tk::NK;
 #pragma unroll 4
@@ -138,8 +161,11 @@ __device__ void tk_load_rows(const Prob& p, const Unit& u, int g, int nsub, uint
     issued = i + 1;
   }
   if (TMA_SLABS > 0 && lane == 0)
-    for (int i = issued > NST ? issued - NST : 0; i < issued; ++i) mbar_wait_drain(&kv_full[i % NST], (i / NST) & 1);
-  if (CP_PIECES > 0) cp_async_wait_none();
+    for (int i = issued > NST ? issued - NST : 0; i < issued; ++i) {
+      if (PAIR) mbar_wait_drain(&half_full[i % NST], (i / NST) & 1);
+      mbar_wait_drain(&kv_full[i % NST], (i / NST) & 1);
+    }
+  if constexpr (CP_PIECES > 0) cp_async_wait_none();
 }
 
 // ===========================================================================
@@ -251,43 +277,56 @@ __global__ void __launch_bounds__(320, 1) tk_bwd_kernel(const __grid_constant__ 
       constexpr uint32_t idKVR = idesc_bf16(64, 32, true, true);
       constexpr uint32_t idDQ = idesc_bf16(64, 256, false, true);
       constexpr uint32_t idDQR = idesc_bf16(64, 64, false, true);
+      // operand descriptors at the buffers' starts (K-major "k", MN-major "m" / "n")
+      const uint64_t dQk = sdesc(sQ, 16, 1024), dDOk = sdesc(sDO, 16, 1024);
+      const uint64_t dQm = sdesc(sQ, tk::H * 128, 1024), dDOm = sdesc(sDO, tk::H * 128, 1024);
+      const uint64_t dDSn = sdesc64(sDS, tk::H * 64, 512), dPn = sdesc64(sP, tk::H * 64, 512);
+      const uint64_t dDSk = sdesc64(sDS, 16, 512);
       bool ok = mbar_wait(&bars.q_full, 0, abort_flag, p.status);
       for (int i = 0; ok && i < nsub; ++i) {
         const int st = i % PL::NST;
         if (!mbar_wait(&bars.kv_full[st], (i / PL::NST) & 1, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t kv = sKV + st * tk::kKVStage;
+        const uint64_t dKVk = sdesc(kv, 16, 1024);
         // S = Q KV^T (lanes 0..15), dP = dO V^T (lanes 16..31)
+#pragma unroll
         for (int kk = 0; kk < tk::DQK / 16; ++kk)
-          mma_bf16(tmem + PL::cS, sdesc(sQ + (kk >> 2) * (tk::H * 128) + (kk & 3) * 32, 16, 1024),
-                   sdesc(kv + (kk >> 2) * (tk::NK * 128) + (kk & 3) * 32, 16, 1024), idS, kk > 0);
+          mma_bf16(tmem + PL::cS, desc_add(dQk, (kk >> 2) * (tk::H * 128) + (kk & 3) * 32),
+                   desc_add(dKVk, (kk >> 2) * (tk::NK * 128) + (kk & 3) * 32), idS, kk > 0);
+#pragma unroll
         for (int kk = 0; kk < tk::DV / 16; ++kk)
-          mma_bf16(tmem + (16u << 16) + PL::cS, sdesc(sDO + (kk >> 2) * (tk::H * 128) + (kk & 3) * 32, 16, 1024),
-                   sdesc(kv + (kk >> 2) * (tk::NK * 128) + (kk & 3) * 32, 16, 1024), idS, kk > 0);
+          mma_bf16(tmem + (16u << 16) + PL::cS, desc_add(dDOk, (kk >> 2) * (tk::H * 128) + (kk & 3) * 32),
+                   desc_add(dKVk, (kk >> 2) * (tk::NK * 128) + (kk & 3) * 32), idS, kk > 0);
         mma_commit(&bars.s_full);
         if (!mbar_wait(&bars.pds_full, i & 1, abort_flag, p.status)) break;
         if (i > 0 && !mbar_wait(&bars.dkv_free, (i - 1) & 1, abort_flag, p.status)) break;
         tc_fence_after();
         // dKV^T = Q^T dS + dO^T P over the 64 heads (fresh for every sub-tile)
+#pragma unroll
         for (int t = 0; t < 4; ++t) {
+#pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + PL::cKV + 32 * t, sdesc(sQ + 2 * t * (tk::H * 128) + kk * 2048, tk::H * 128, 1024),
-                     sdesc64(sDS + kk * 1024, tk::H * 64, 512), idKV, kk > 0);
+            mma_bf16(tmem + PL::cKV + 32 * t, desc_add(dQm, 2 * t * (tk::H * 128) + kk * 2048),
+                     desc_add(dDSn, kk * 1024), idKV, kk > 0);
+#pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + PL::cKV + 32 * t, sdesc(sDO + 2 * t * (tk::H * 128) + kk * 2048, tk::H * 128, 1024),
-                     sdesc64(sP + kk * 1024, tk::H * 64, 512), idKV, 1u);
+            mma_bf16(tmem + PL::cKV + 32 * t, desc_add(dDOm, 2 * t * (tk::H * 128) + kk * 2048),
+                     desc_add(dPn, kk * 1024), idKV, 1u);
         }
+#pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + PL::cKVR, sdesc(sQ + 8 * (tk::H * 128) + kk * 2048, tk::H * 128, 1024),
-                   sdesc64(sDS + kk * 1024, tk::H * 64, 512), idKVR, kk > 0);
+          mma_bf16(tmem + PL::cKVR, desc_add(dQm, 8 * (tk::H * 128) + kk * 2048), desc_add(dDSn, kk * 1024), idKVR,
+                   kk > 0);
         // dQ += dS KV (KV as an MN-major B: N = dims in 64-wide slabs of 32 rows)
+        const uint64_t dKVn = sdesc(kv, tk::NK * 128, 1024);
+#pragma unroll
         for (int kk = 0; kk < tk::NK / 16; ++kk) {
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          const uint64_t a = sdesc64(sDS + kk * 32, 16, 512);
-          mma_bf16(tmem + PL::cDQ, a, sdesc(kv + kk * 2048, tk::NK * 128, 1024), idDQ, acc);
-          mma_bf16(tmem + (16u << 16) + PL::cDQ, a, sdesc(kv + 4 * (tk::NK * 128) + kk * 2048, tk::NK * 128, 1024),
-                   idDQ, acc);
-          mma_bf16(tmem + PL::cDQR, a, sdesc(kv + 8 * (tk::NK * 128) + kk * 2048, tk::NK * 128, 1024), idDQR, acc);
+          const uint64_t a = desc_add(dDSk, kk * 32);
+          mma_bf16(tmem + PL::cDQ, a, desc_add(dKVn, kk * 2048), idDQ, acc);
+          mma_bf16(tmem + (16u << 16) + PL::cDQ, a, desc_add(dKVn, 4 * (tk::NK * 128) + kk * 2048), idDQ, acc);
+          mma_bf16(tmem + PL::cDQR, a, desc_add(dKVn, 8 * (tk::NK * 128) + kk * 2048), idDQR, acc);
         }
         // the stage is released by the reduction warps, which stage dKV^T in it once
         // every MMA of the sub-tile (dKV^T included) has completed
@@ -491,14 +530,22 @@ struct TkFwdBars {
   uint64_t q_full, kv_full[TkFwdPlan::NST], kv_empty[TkFwdPlan::NST], s_full[2], s_free[2], p_full[2],
       pv_done[2];
   uint64_t codes_full[4];
+  // cluster pair: this CTA's half of a stage has landed / the partner's stage may
+  // take this CTA's half / the partner has received this CTA's half
+  uint64_t half_full[TkFwdPlan::NST], peer_ready[TkFwdPlan::NST], copy_done[TkFwdPlan::NST];
   uint32_t tmem_base;
   int abort_flag;
 };
 
-__global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ CUtensorMap mapQ,
-                                                        const __grid_constant__ CUtensorMap mapKV,
-                                                        const __grid_constant__ CUtensorMap mapCmp, const int has_cmp,
-                                                        const Prob p, bf16* __restrict__ O, float* __restrict__ LSE) {
+// PAIR: launched in clusters of two CTAs, the two 64-head slices of one token
+// (G / 64 even), which share the row gathers (tk_load_rows); a seventh warp
+// copies the half of each stage this CTA gathered into the partner's stage.
+template <bool PAIR>
+__global__ void __launch_bounds__(PAIR ? 224 : 192, 1) tk_fwd_kernel(const __grid_constant__ CUtensorMap mapQ,
+                                                                     const __grid_constant__ CUtensorMap mapKV,
+                                                                     const __grid_constant__ CUtensorMap mapCmp,
+                                                                     const int has_cmp, const Prob p,
+                                                                     bf16* __restrict__ O, float* __restrict__ LSE) {
   using PL = TkFwdPlan;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ TkFwdBars bars;
@@ -506,8 +553,10 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
   if (smem_u32(smem) & 1023) {
     pdl_wait();
     if (threadIdx.x == 0 && p.status) atomicOr(p.status, kStatusSmemAlign);
+    if (PAIR) cluster_sync();  // the same outcome in both CTAs
     return;
   }
+  const uint32_t crank = PAIR ? cluster_ctarank() : 0u;
   const int nhs = p.G / tk::H;
   const int unit = blockIdx.x / nhs, hs = blockIdx.x - unit * nhs;
   const int tq = unit / p.Hkv, g = unit - tq * p.Hkv;
@@ -519,7 +568,7 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
     bars.abort_flag = 0;
     mbar_init(&bars.q_full, 1);
     for (int s = 0; s < PL::NST; ++s) {
-      mbar_init(&bars.kv_full[s], (PL::kTmaSlabs > 0 ? 1 : 0) + (PL::kTmaSlabs < tk::NSQ ? 32 : 0));
+      mbar_init(&bars.kv_full[s], PAIR ? 2 : (PL::kTmaSlabs > 0 ? 1 : 0) + (PL::kTmaSlabs < tk::NSQ ? 32 : 0));
       mbar_init(&bars.kv_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -529,6 +578,11 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
       mbar_init(&bars.pv_done[b], 1);
     }
     for (int s = 0; s < 4; ++s) mbar_init(&bars.codes_full[s], 1);
+    for (int s = 0; s < PL::NST; ++s) {
+      mbar_init(&bars.half_full[s], 1);
+      mbar_init(&bars.peer_ready[s], 1);
+      mbar_init(&bars.copy_done[s], 1);
+    }
     mbar_fence_init();
     tma_prefetch_desc(&mapQ);
     tma_prefetch_desc(&mapKV);
@@ -541,7 +595,10 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
   const int nsub = 2 * u.n_tiles;
   fence_async_smem();
   tc_fence_before();
-  __syncthreads();
+  if (PAIR)
+    cluster_sync();  // the partner's barriers are initialised before any remote arrive or copy
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
@@ -552,8 +609,9 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
       for (int s = 0; s < tk::NSQ; ++s)
         tma_load_2d(sQ + s * tk::H * 128, &mapQ, 64 * s, tq * p.Hq + head0, &bars.q_full);
     }
-    tk_load_rows<PL::NST, PL::kTmaSlabs>(p, u, g, nsub, sKV, codes, &mapKV, &mapCmp, has_cmp != 0, bars.kv_full,
-                                          bars.kv_empty, bars.codes_full, abort_flag, lane);
+    tk_load_rows<PL::NST, PL::kTmaSlabs, PAIR>(p, u, g, nsub, sKV, codes, &mapKV, &mapCmp, has_cmp != 0,
+                                                bars.kv_full, bars.kv_empty, bars.codes_full, abort_flag, lane,
+                                                bars.half_full, bars.peer_ready, bars.copy_done, crank);
     if (lane == 0) mbar_wait_drain(&bars.q_full, 0);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -561,17 +619,22 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(64, 32, false, false);
       constexpr uint32_t idPV = idesc_bf16(64, 256, false, true);
+      const uint64_t dQk = sdesc(sQ, 16, 1024);  // Q as the K-major A of S
       bool ok = mbar_wait(&bars.q_full, 0, abort_flag, p.status);
       for (int i = 0; ok && i <= nsub; ++i) {
         if (i < nsub) {
           const int st = i % PL::NST;
           if (!mbar_wait(&bars.kv_full[st], (i / PL::NST) & 1, abort_flag, p.status)) break;
+          if (PAIR)  // the partner's half has landed: the partner may gather into that stage again
+            mbar_arrive_remote(mapa_shared(smem_u32(&bars.copy_done[st]), crank ^ 1u));
           if (i >= 2 && !mbar_wait(&bars.s_free[i & 1], ((i - 2) >> 1) & 1, abort_flag, p.status)) break;
           tc_fence_after();
-          const uint32_t kv = sKV + st * tk::kKVStage;
+          const uint64_t dKVk = sdesc(sKV + st * tk::kKVStage, 16, 1024);
+          const uint32_t dS = tmem + PL::cS0 + 32 * (i & 1);
+#pragma unroll
           for (int kk = 0; kk < tk::DQK / 16; ++kk)
-            mma_bf16(tmem + PL::cS0 + 32 * (i & 1), sdesc(sQ + (kk >> 2) * (tk::H * 128) + (kk & 3) * 32, 16, 1024),
-                     sdesc(kv + (kk >> 2) * (tk::NK * 128) + (kk & 3) * 32, 16, 1024), idS, kk > 0);
+            mma_bf16(dS, desc_add(dQk, (kk >> 2) * (tk::H * 128) + (kk & 3) * 32),
+                     desc_add(dKVk, (kk >> 2) * (tk::NK * 128) + (kk & 3) * 32), idS, kk > 0);
           mma_commit(&bars.s_full[i & 1]);
         }
         if (i >= 1) {
@@ -579,16 +642,37 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
           if (!mbar_wait(&bars.p_full[j & 1], (j >> 1) & 1, abort_flag, p.status)) break;
           tc_fence_after();
           // O += P_j V_j (V = the first 512 dims of the KV rows, an MN-major B)
-          const uint32_t kv = sKV + stj * tk::kKVStage, pb = sP + (j & 1) * tk::kPBytes;
+          const uint64_t dVn = sdesc(sKV + stj * tk::kKVStage, tk::NK * 128, 1024);
+          const uint64_t dPk = sdesc64(sP + (j & 1) * tk::kPBytes, 16, 512);
+#pragma unroll
           for (int kk = 0; kk < tk::NK / 16; ++kk) {
             const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-            const uint64_t a = sdesc64(pb + kk * 32, 16, 512);
-            mma_bf16(tmem + PL::cO, a, sdesc(kv + kk * 2048, tk::NK * 128, 1024), idPV, acc);
-            mma_bf16(tmem + (16u << 16) + PL::cO, a, sdesc(kv + 4 * (tk::NK * 128) + kk * 2048, tk::NK * 128, 1024),
-                     idPV, acc);
+            const uint64_t a = desc_add(dPk, kk * 32);
+            mma_bf16(tmem + PL::cO, a, desc_add(dVn, kk * 2048), idPV, acc);
+            mma_bf16(tmem + (16u << 16) + PL::cO, a, desc_add(dVn, 4 * (tk::NK * 128) + kk * 2048), idPV, acc);
           }
           mma_commit(&bars.kv_empty[stj]);
           mma_commit(&bars.pv_done[j & 1]);
+        }
+      }
+    }
+  } else if (PAIR && warp == 6) {
+    // ------------------------------------------------------------ copier
+    // this CTA's half of each sub-tile, once landed, into the same rows of the
+    // partner's stage (16 rows x 128 bytes = 2 KB per slab) as soon as the
+    // partner's stage may take it
+    if (lane == 0) {
+      for (int i = 0; i < nsub; ++i) {
+        const int st = i % PL::NST, ph = (i / PL::NST) & 1;
+        if (!mbar_wait(&bars.half_full[st], ph, abort_flag, p.status)) break;
+        mbar_arrive(&bars.kv_full[st]);  // this CTA's half is in
+        if (!mbar_wait_cluster(&bars.peer_ready[st], ph, abort_flag, p.status)) break;
+        const uint32_t half = sKV + st * tk::kKVStage + crank * (16 * 128);
+        const uint32_t bar = mapa_shared(smem_u32(&bars.kv_full[st]), crank ^ 1u);
+#pragma unroll
+        for (int s = 0; s < tk::NSQ; ++s) {
+          const uint32_t src = half + s * (tk::NK * 128);
+          bulk_copy_to_peer(mapa_shared(src, crank ^ 1u), src, 16 * 128, bar);
         }
       }
     }
@@ -702,6 +786,8 @@ __global__ void __launch_bounds__(192, 1) tk_fwd_kernel(const __grid_constant__ 
     tmem_dealloc(tmem, PL::kAlloc);
     tmem_relinquish();
   }
+  // no CTA leaves while its partner may still copy into it or arrive on its barriers
+  if (PAIR) cluster_sync();
 }
 
 // ===========================================================================
@@ -748,7 +834,7 @@ cudaError_t launch_tk_bwd(const Prob& p, const float* lse, const float* delta, c
   return e;
 }
 
-cudaError_t launch_tk_fwd(const Prob& p, bf16* o, float* lse, cudaStream_t st) {
+cudaError_t launch_tk_fwd(const Prob& p, bf16* o, float* lse, bool pair, cudaStream_t st) {
   using PL = TkFwdPlan;
   if (!tk_path_built(p.dqk, p.dv, p.shared, p.G)) return cudaErrorInvalidValue;
   const long long grid = (long long)p.Tq * p.Hkv * (p.G / tk::H);
@@ -758,10 +844,19 @@ cudaError_t launch_tk_fwd(const Prob& p, bf16* o, float* lse, cudaStream_t st) {
   if (!make_tmap_bf16(&mq, p.q, (uint64_t)p.Tq * p.Hq, tk::DQK, (uint64_t)tk::DQK * 2, tk::H) ||
       !tk_row_maps(p, &mkv, &mcmp, &has_cmp))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(tk_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kSmem);
+  // the two 64-head slices of a token are consecutive CTAs: pair them when every token has an even count
+  pair = pair && (p.G / tk::H) % 2 == 0;
+  cudaError_t e = pair ? cudaFuncSetAttribute(tk_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              PL::kSmem)
+                       : cudaFuncSetAttribute(tk_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              PL::kSmem);
   if (e != cudaSuccess) return e;
   mark_begin(st, kTimeFwd);
-  e = launch_pdl(tk_fwd_kernel, (unsigned)grid, 192, PL::kSmem, st, mq, mkv, mcmp, has_cmp, p, o, lse);
+  if (pair)
+    e = launch_pdl_cluster(tk_fwd_kernel<true>, (unsigned)grid, 224, PL::kSmem, st, 2u, mq, mkv, mcmp, has_cmp, p,
+                           o, lse);
+  else
+    e = launch_pdl(tk_fwd_kernel<false>, (unsigned)grid, 192, PL::kSmem, st, mq, mkv, mcmp, has_cmp, p, o, lse);
   count_launch();
   mark_end(st, kTimeFwd);
   return e;
