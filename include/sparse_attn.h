@@ -27,8 +27,15 @@
  * returns without synchronising.  The library never allocates device memory:
  * the caller owns every buffer, including the workspace.
  *
- * Pointers.  Every tensor pointer is a DEVICE pointer (bf16 = 2-byte bfloat16,
- * row-major, innermost dimension contiguous, 16-byte aligned).  The sa_args /
+ * Pointers.  Every tensor pointer is a DEVICE pointer (row-major, innermost
+ * dimension contiguous, 16-byte aligned).  "bf16" below means the 2-byte element
+ * type sa_args.dtype names: bfloat16 (SA_DTYPE_BF16) or IEEE half
+ * (SA_DTYPE_FP16), the same for q, k, v, kv, cmp_kv, O, dO and the gradients
+ * (SparseFlashMlaGrad "Parameter Description": BFLOAT16 or FLOAT16, outputs of
+ * the inputs' type); lse, sinks, dSinks and the SoftmaxL1Norm outputs are fp32.
+ * The tensor-core kernels take bfloat16; fp16 problems run on the generic
+ * query-stationary kernels (fp16 MMA operands, fp32 accumulation), whatever the
+ * selection mode.  The sa_args /
  * sa_fwd_out / sa_bwd_io structs themselves are host memory read during the
  * call only.  `stream` is a cudaStream_t (NULL = the legacy default stream).
  *
@@ -126,7 +133,7 @@ typedef enum sa_status {
   SA_OK = 0,
   SA_ERR_NULLPTR = 1,      /* a required pointer is NULL */
   SA_ERR_PARAM = 2,        /* a size, mode or attribute is out of range */
-  SA_ERR_UNSUPPORTED = 3,  /* valid per the pages but not built (e.g. fp16, CFA) */
+  SA_ERR_UNSUPPORTED = 3,  /* valid per the pages but not built (e.g. mixed layouts) */
   SA_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than *_get_workspace_size */
   SA_ERR_INDEX = 5,        /* SA_FLAG_CHECK found an index past its sequence */
   SA_ERR_TIMEOUT = 6,      /* a bounded device wait gave up */
@@ -192,7 +199,7 @@ typedef enum sa_kernel {
 typedef struct sa_args {
   int32_t layout_q;        /* sa_layout of q, o, d_o, lse and the index tensors */
   int32_t layout_kv;       /* sa_layout of k, v, kv and cmp_kv (must equal layout_q) */
-  int32_t dtype;           /* sa_dtype; only SA_DTYPE_BF16 is built */
+  int32_t dtype;           /* sa_dtype: the 2-byte element type of every bf16 tensor */
   int32_t batch;           /* B >= 0 */
   int32_t s_q, s_kv;       /* BSND sequence lengths (ignored for TND) */
   int32_t t_q, t_kv, t_cmp;/* TND packed token counts (ignored for BSND) */

@@ -105,7 +105,7 @@ def _ws(a):
     (dict(), L.SA_OK),
     (dict(n_heads_q=15), L.SA_ERR_PARAM),
     (dict(n_heads_kv=0), L.SA_ERR_PARAM),
-    (dict(dtype=L.SA_DTYPE_FP16), L.SA_ERR_UNSUPPORTED),
+    (dict(dtype=L.SA_DTYPE_FP16), L.SA_OK),
     (dict(dtype=7), L.SA_ERR_PARAM),
     (dict(d_qk=96, d_v=96), L.SA_ERR_UNSUPPORTED),
     (dict(d_qk=100), L.SA_ERR_PARAM),
@@ -242,6 +242,11 @@ def test_plan_reports_the_kernel_each_problem_gets():
                block_size=1, topk=32)
     assert _plan(_args(**tok)) == (L.SA_KERNEL_FWD_TOKEN_TC, L.SA_KERNEL_BWD_TOKEN_TC)
     assert _plan(_args(**dict(tok, n_heads_q=16))) == (L.SA_KERNEL_FWD_GENERIC, L.SA_KERNEL_BWD_GENERIC)
+    # fp16 inputs run on the generic kernels (the tensor-core kernels take bf16)
+    f16 = L.SA_DTYPE_FP16
+    assert _plan(_args(dtype=f16)) == (L.SA_KERNEL_FWD_GENERIC, L.SA_KERNEL_BWD_GENERIC)
+    assert _plan(_args(**dict(tok, dtype=f16))) == (L.SA_KERNEL_FWD_GENERIC, L.SA_KERNEL_BWD_GENERIC)
+    assert _plan(_args(dtype=f16, flags=L.SA_FLAG_FWD_BLOCK_TC))[0] == L.SA_KERNEL_FWD_GENERIC
     with pytest.raises(L.SaError):
         _plan(_args(n_heads_q=15))
 

@@ -80,7 +80,7 @@ class SparseAttention:
         a = L.SaArgs()
         a.layout_q = L.LAYOUTS[self.layout]
         a.layout_kv = L.LAYOUTS[self.layout]
-        a.dtype = L.SA_DTYPE_BF16
+        a.dtype = L.SA_DTYPE_FP16 if self.q.dtype == torch.float16 else L.SA_DTYPE_BF16
         a.batch = self.batch
         a.s_q, a.s_kv = self.s_q, self.s_kv
         a.t_q, a.t_kv, a.t_cmp = self.t_q, self.t_kv, self.t_cmp
@@ -116,7 +116,7 @@ class SparseAttention:
 
     def alloc_fwd(self):
         dev = self.q.device
-        o = torch.empty(self._lead() + (self.Hq, self.d_v), dtype=torch.bfloat16, device=dev)
+        o = torch.empty(self._lead() + (self.Hq, self.d_v), dtype=self.q.dtype, device=dev)
         lse = torch.empty(self._lead() + (self.Hq,), dtype=torch.float32, device=dev)
         return o, lse
 

@@ -53,8 +53,7 @@ Sizes sizes_of(const sa_args* a) {
 
 sa_status validate(const sa_args* a) {
   if (!a) return SA_ERR_NULLPTR;
-  if (a->dtype == SA_DTYPE_FP16) return SA_ERR_UNSUPPORTED;
-  if (a->dtype != SA_DTYPE_BF16) return SA_ERR_PARAM;
+  if (a->dtype != SA_DTYPE_BF16 && a->dtype != SA_DTYPE_FP16) return SA_ERR_PARAM;
   if (a->layout_q != SA_LAYOUT_BSND && a->layout_q != SA_LAYOUT_TND) return SA_ERR_PARAM;
   if (a->layout_kv != SA_LAYOUT_BSND && a->layout_kv != SA_LAYOUT_TND) return SA_ERR_PARAM;
   if (a->layout_q != a->layout_kv) return SA_ERR_UNSUPPORTED;  // mixed layouts are not built
@@ -154,6 +153,7 @@ sa::Prob make_prob(const sa_args* a, int* status) {
   p.page_size = a->page_size;
   p.max_pages = a->max_pages;
   p.status = status;
+  p.f16 = a->dtype == SA_DTYPE_FP16 ? 1 : 0;
   return p;
 }
 
@@ -171,15 +171,15 @@ sa_status check_tensor_alignment(const sa_args* a) {
 bool use_kv_path(const sa_args* a) {
   if (a->flags & SA_FLAG_QUERY_STATIONARY_BWD) return false;
   const int G = a->n_heads_q / a->n_heads_kv;
-  return a->layout_q == SA_LAYOUT_BSND && a->topk > 0 && a->block_size == 64 && a->s_q == a->s_kv &&
-         !a->kv_shared && !has_cmp(a) && !has_used(a) && !paged(a) && a->sinks == nullptr && G <= 128 &&
-         sa::kv_path_built(a->d_qk, a->d_v);
+  return a->dtype == SA_DTYPE_BF16 && a->layout_q == SA_LAYOUT_BSND && a->topk > 0 && a->block_size == 64 &&
+         a->s_q == a->s_kv && !a->kv_shared && !has_cmp(a) && !has_used(a) && !paged(a) && a->sinks == nullptr &&
+         G <= 128 && sa::kv_path_built(a->d_qk, a->d_v);
 }
 
 // Query-stationary block kernels (TMA-fed): 64-row blocks, separate K / V, no compressed KV.
 bool use_qb_path(const sa_args* a) {
-  return a->topk > 0 && a->topk <= sa::kQbMaxSlots && a->block_size == 64 && !a->kv_shared && !has_cmp(a) && !has_used(a) && !paged(a) &&
-         sa::qb_path_built(a->d_qk, a->d_v);
+  return a->dtype == SA_DTYPE_BF16 && a->topk > 0 && a->topk <= sa::kQbMaxSlots && a->block_size == 64 &&
+         !a->kv_shared && !has_cmp(a) && !has_used(a) && !paged(a) && sa::qb_path_built(a->d_qk, a->d_v);
 }
 
 // SA_FLAG_DQ_SEPARATE applies only where the query-stationary block kernels do
@@ -351,7 +351,8 @@ sa_status run_check(const sa_args* a, int* status, cudaStream_t st) {
 // Kernel choices (sa_plan reports them; sa_fwd / sa_bwd dispatch on them).
 bool tk_path(const sa_args* a) {
   // the row gathers need at least one KV row to point at (an empty KV takes the generic path)
-  return sa::tk_path_built(a->d_qk, a->d_v, a->kv_shared, a->n_heads_q / a->n_heads_kv) && sizes_of(a).Tkv >= 1;
+  return a->dtype == SA_DTYPE_BF16 && sa::tk_path_built(a->d_qk, a->d_v, a->kv_shared, a->n_heads_q / a->n_heads_kv) &&
+         sizes_of(a).Tkv >= 1;
 }
 
 int32_t fwd_choice(const sa_args* a) {
@@ -598,7 +599,7 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
     // zero the accumulators and the status word (one memset), then Delta
     if (cudaMemsetAsync(base, 0, w.zero_end, cs) != cudaSuccess) return SA_ERR_CUDA;
     e = sa::launch_delta(static_cast<const bf16*>(io->o), static_cast<const bf16*>(io->d_o), delta,
-                         s.Tq * args->n_heads_q, args->d_v, cs);
+                         s.Tq * args->n_heads_q, args->d_v, cs, p.f16 != 0);
     if (e != cudaSuccess) return SA_ERR_CUDA;
   }
   if (sinks && cudaMemsetAsync(io->dsinks, 0, sizeof(float) * args->n_heads_q, cs) != cudaSuccess)
@@ -646,7 +647,7 @@ sa_status sa_bwd(const sa_args* args, const sa_bwd_io* io, void* ws, size_t ws_b
     if (has_cmp(args)) jobs[nj++] = sa::Cvt{out.dcmp_acc, static_cast<bf16*>(io->dcmp_kv), nc};
     if (w.dq) jobs[nj++] = sa::Cvt{reinterpret_cast<float*>(base + w.dq), static_cast<bf16*>(io->dq),
                                    s.Tq * args->n_heads_q * args->d_qk};
-    e = sa::launch_to_bf16_multi(jobs, nj, cs);
+    e = sa::launch_to_bf16_multi(jobs, nj, cs, p.f16 != 0);
   }
   return cuda_status(e);
 }
@@ -660,7 +661,8 @@ sa_status sa_softmax_grad_preprocess(const sa_args* args, const void* o, const v
   if (!o || !d_o || !delta) return SA_ERR_NULLPTR;
   if (!aligned16(o) || !aligned16(d_o)) return SA_ERR_PARAM;
   return cuda_status(sa::launch_delta(static_cast<const bf16*>(o), static_cast<const bf16*>(d_o), delta,
-                                      s.Tq * args->n_heads_q, args->d_v, static_cast<cudaStream_t>(stream)));
+                                      s.Tq * args->n_heads_q, args->d_v, static_cast<cudaStream_t>(stream),
+                                      args->dtype == SA_DTYPE_FP16));
 }
 
 sa_status sa_softmax_l1norm(const sa_args* args, const float* lse, float* ori_out, float* cmp_out, void* stream) {

@@ -12,6 +12,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -52,6 +53,7 @@ struct Prob {
   const int* cmp_len;
   const float* sinks;
   int* status;        // device status word (may be null)
+  int f16;            // the 2-byte tensors (q, k, v, cmp_kv, O, dO, dQ, dK, dV) hold fp16, else bf16
 };
 
 struct Unit {
@@ -357,6 +359,41 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// The element type of the 2-byte tensors for the mma.sync kernels: the tensors
+// move as raw 16-bit data (the pointers are typed bf16 for storage only), and
+// Elt<F16> supplies the arithmetic -- the m16n8k16 MMA on bf16 or fp16 operands
+// (fp32 accumulation either way), two fp32 values rounded to nearest even into
+// one 32-bit pair, and a pair widened to fp32.
+template <bool F16>
+struct Elt;
+template <>
+struct Elt<false> {
+  static __device__ __forceinline__ void mma(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    mma16816(c, a, b0, b1);
+  }
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi) { return pack_bf16(lo, hi); }
+  static __device__ __forceinline__ float2 widen(uint32_t x) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x));
+  }
+};
+template <>
+struct Elt<true> {
+  static __device__ __forceinline__ void mma(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+  static __device__ __forceinline__ float2 widen(uint32_t x) {
+    return __half22float2(*reinterpret_cast<const __half2*>(&x));
+  }
+};
+
 // A fragment (16 x 16) at rows r0.., k-chunk kc (k0 = 8*kc) of a row-major swizzled tile.
 template <int D>
 __device__ __forceinline__ void load_a(uint32_t (&a)[4], uint32_t base, int r0, int kc, int lane) {
@@ -401,8 +438,10 @@ __device__ __forceinline__ float warp_sum4(float v) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
-// Delta of one row: sum_d a[d] * b[d] over n bf16 (n a multiple of 8, 16-byte
-// aligned rows) in fp32, by one warp; every lane returns the sum.
+// Delta of one row: sum_d a[d] * b[d] over n 2-byte elements (bf16, or fp16 with
+// F16; n a multiple of 8, 16-byte aligned rows) in fp32, by one warp; every lane
+// returns the sum.
+template <bool F16 = false>
 __device__ __forceinline__ float warp_row_dot_bf16(const bf16* __restrict__ a, const bf16* __restrict__ b, int n,
                                                    int lane) {
   const uint4* a4 = reinterpret_cast<const uint4*>(a);
@@ -410,11 +449,10 @@ __device__ __forceinline__ float warp_row_dot_bf16(const bf16* __restrict__ a, c
   float acc = 0.f;
   for (int i = lane; i < n / 8; i += 32) {
     uint4 x = __ldg(a4 + i), y = __ldg(b4 + i);
-    const __nv_bfloat162* px = reinterpret_cast<const __nv_bfloat162*>(&x);
-    const __nv_bfloat162* py = reinterpret_cast<const __nv_bfloat162*>(&y);
+    const uint32_t px[4] = {x.x, x.y, x.z, x.w}, py[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      float2 fx = __bfloat1622float2(px[j]), fy = __bfloat1622float2(py[j]);
+      const float2 fx = Elt<F16>::widen(px[j]), fy = Elt<F16>::widen(py[j]);
       acc = fmaf(fx.x, fy.x, acc);
       acc = fmaf(fx.y, fy.y, acc);
     }

@@ -84,10 +84,11 @@ cudaError_t launch_fwd(const Prob& p, bf16* o, float* lse, cudaStream_t st);
 cudaError_t launch_bwd_dq(const Prob& p, const bf16* d_o, const float* lse, const float* delta,
                           const BwdOut& out, cudaStream_t st);
 cudaError_t launch_delta(const bf16* o, const bf16* d_o, float* delta, long long rows, int dv,
-                         cudaStream_t st);
+                         cudaStream_t st, bool f16 = false);
 cudaError_t launch_bwd(const Prob& p, const bf16* o, const bf16* d_o, const float* lse,
                        const float* delta, const BwdOut& out, cudaStream_t st);
-cudaError_t launch_to_bf16(const float* src, bf16* dst, long long n, cudaStream_t st);
+// fp32 -> the 2-byte output type (bf16, or fp16 with f16); n a multiple of 8.
+cudaError_t launch_to_bf16(const float* src, bf16* dst, long long n, cudaStream_t st, bool f16 = false);
 // Token-level backward over one shared KV head (d 576 / 512) on tcgen05: dQ to
 // bf16 directly, dKV (dCmpKv) into the fp32 accumulators, dSinks accumulated.
 bool tk_path_built(int dqk, int dv, int shared, int G);
@@ -100,7 +101,7 @@ struct Cvt {
   bf16* dst;
   long long n;
 };
-cudaError_t launch_to_bf16_multi(const Cvt* jobs, int njobs, cudaStream_t st);
+cudaError_t launch_to_bf16_multi(const Cvt* jobs, int njobs, cudaStream_t st, bool f16 = false);
 cudaError_t launch_check(const Prob& p, cudaStream_t st);
 // The lightning indexer's KL-loss backward (one CTA per token).
 struct IxArgs {

@@ -87,7 +87,7 @@ __device__ __forceinline__ void load_rows16(const bf16* base, int nh, uint32_t d
 // ---------------------------------------------------------------------------
 // forward
 // ---------------------------------------------------------------------------
-template <int DQK, int DV, bool SHARED>
+template <int DQK, int DV, bool SHARED, bool F16>
 __global__ void __launch_bounds__(128) fwd_kernel(const Prob p, bf16* __restrict__ O,
                                                   float* __restrict__ LSE) {
   using PL = Plan<DQK, DV, SHARED>;
@@ -153,8 +153,8 @@ __global__ void __launch_bounds__(128) fwd_kernel(const Prob p, bf16* __restrict
       uint32_t a[4], b[4];
       load_a<DQK>(a, sQ, 0, kc, lane);
       load_b_nk<DQK>(b, bK, warp * 16, kc, lane);
-      mma16816(s[0], a, b[0], b[1]);
-      mma16816(s[1], a, b[2], b[3]);
+      Elt<F16>::mma(s[0], a, b[0], b[1]);
+      Elt<F16>::mma(s[1], a, b[2], b[3]);
     }
     const int* rc = rowc + cur * 64 + warp * 16;
     float mx[2] = {-INFINITY, -INFINITY};
@@ -193,8 +193,8 @@ __global__ void __launch_bounds__(128) fwd_kernel(const Prob p, bf16* __restrict
       const int chunk = warp * 2 + nt;
       uint32_t a0 = swz<64>(sP, r0, chunk) + (lane & 3) * 4;
       uint32_t a1 = swz<64>(sP, r0 + 8, chunk) + (lane & 3) * 4;
-      asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(a0), "r"(pack_bf16(p0, p1)));
-      asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(a1), "r"(pack_bf16(p2, p3)));
+      asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(a0), "r"(Elt<F16>::pack(p0, p1)));
+      asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(a1), "r"(Elt<F16>::pack(p2, p3)));
     }
     ps[0] = warp_sum4(ps[0]);
     ps[1] = warp_sum4(ps[1]);
@@ -225,8 +225,8 @@ __global__ void __launch_bounds__(128) fwd_kernel(const Prob p, bf16* __restrict
       for (int j = 0; j < NT / 2; ++j) {
         uint32_t b[4];
         load_b_kn<DVS>(b, bV, kc * 8, warp * (NT) + 2 * j, lane);
-        mma16816(o[2 * j], a, b[0], b[1]);
-        mma16816(o[2 * j + 1], a, b[2], b[3]);
+        Elt<F16>::mma(o[2 * j], a, b[0], b[1]);
+        Elt<F16>::mma(o[2 * j + 1], a, b[2], b[3]);
       }
     }
   }
@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(128) fwd_kernel(const Prob p, bf16* __restrict
 #pragma unroll
     for (int i = 0; i < NT; ++i) {
       int col = i * 8 + 2 * (lane & 3);
-      *reinterpret_cast<uint32_t*>(orow + col) = pack_bf16(o[i][2 * r] * inv[r], o[i][2 * r + 1] * inv[r]);
+      *reinterpret_cast<uint32_t*>(orow + col) = Elt<F16>::pack(o[i][2 * r] * inv[r], o[i][2 * r + 1] * inv[r]);
     }
     if (warp == 0 && (lane & 3) == 0)
       LSE[(long long)tq * p.Hq + h0 + row] = l[r] > 0.f ? (m[r] + log2f(l[r])) * kLn2 : INFINITY;
@@ -272,7 +272,7 @@ __device__ __forceinline__ void issue_k_tile(const Prob& p, int g, const int* rc
   }
 }
 
-template <int DQK, int DV, bool SHARED>
+template <int DQK, int DV, bool SHARED, bool F16>
 __global__ void __launch_bounds__(128) l1_sum_kernel(const Prob p, const float* __restrict__ LSE,
                                                      float* __restrict__ ori_out, float* __restrict__ cmp_out) {
   using PL = Plan<DQK, DV, SHARED>;
@@ -322,8 +322,8 @@ __global__ void __launch_bounds__(128) l1_sum_kernel(const Prob p, const float* 
       uint32_t a[4], b[4];
       load_a<DQK>(a, sQ, 0, kc, lane);
       load_b_nk<DQK>(b, bK, warp * 16, kc, lane);
-      mma16816(s[0], a, b[0], b[1]);
-      mma16816(s[1], a, b[2], b[3]);
+      Elt<F16>::mma(s[0], a, b[0], b[1]);
+      Elt<F16>::mma(s[1], a, b[2], b[3]);
     }
     const int* rc = rowc + cur * 64 + warp * 16;
     // P summed over this thread's two heads, then over the 8 row groups of the warp
@@ -393,7 +393,7 @@ __device__ __forceinline__ void red_add2(float* addr, float a, float b) {
   atomicAdd(reinterpret_cast<float2*>(addr), make_float2(a, b));
 }
 
-template <int DQK, int DV, bool SHARED, bool SCATTER>
+template <int DQK, int DV, bool SHARED, bool SCATTER, bool F16>
 __global__ void __launch_bounds__(128) bwd_kernel(const Prob p, const bf16* __restrict__ dO,
                                                   const float* __restrict__ LSE,
                                                   const float* __restrict__ Delta, BwdOut out) {
@@ -466,16 +466,16 @@ __global__ void __launch_bounds__(128) bwd_kernel(const Prob p, const bf16* __re
       uint32_t a[4], b[4];
       load_a<DQK>(a, sQ, 0, kc, lane);
       load_b_nk<DQK>(b, bK, warp * 16, kc, lane);
-      mma16816(s[0], a, b[0], b[1]);
-      mma16816(s[1], a, b[2], b[3]);
+      Elt<F16>::mma(s[0], a, b[0], b[1]);
+      Elt<F16>::mma(s[1], a, b[2], b[3]);
     }
 #pragma unroll 4
     for (int kc = 0; kc < DV / 8; kc += 2) {
       uint32_t a[4], b[4];
       load_a<DV>(a, sDO, 0, kc, lane);
       load_b_nk<DVS>(b, bV, warp * 16, kc, lane);
-      mma16816(dp[0], a, b[0], b[1]);
-      mma16816(dp[1], a, b[2], b[3]);
+      Elt<F16>::mma(dp[0], a, b[0], b[1]);
+      Elt<F16>::mma(dp[1], a, b[2], b[3]);
     }
     // P = exp(S - lse), dS = P (dP - Delta)
 #pragma unroll
@@ -492,10 +492,10 @@ __global__ void __launch_bounds__(128) bwd_kernel(const Prob p, const bf16* __re
       }
       const int chunk = warp * 2 + nt;
       uint32_t a0 = (lane & 3) * 4;
-      asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(swz<64>(sP, r0, chunk) + a0), "r"(pack_bf16(pv[0], pv[1])));
-      asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(swz<64>(sP, r0 + 8, chunk) + a0), "r"(pack_bf16(pv[2], pv[3])));
-      asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(swz<64>(sDS, r0, chunk) + a0), "r"(pack_bf16(dsv[0], dsv[1])));
-      asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(swz<64>(sDS, r0 + 8, chunk) + a0), "r"(pack_bf16(dsv[2], dsv[3])));
+      asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(swz<64>(sP, r0, chunk) + a0), "r"(Elt<F16>::pack(pv[0], pv[1])));
+      asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(swz<64>(sP, r0 + 8, chunk) + a0), "r"(Elt<F16>::pack(pv[2], pv[3])));
+      asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(swz<64>(sDS, r0, chunk) + a0), "r"(Elt<F16>::pack(dsv[0], dsv[1])));
+      asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(swz<64>(sDS, r0 + 8, chunk) + a0), "r"(Elt<F16>::pack(dsv[2], dsv[3])));
     }
     __syncwarp();
     // scatter: dK rows (the warp's 16 tile rows) = scale dS^T Q  [+ P^T dO on the V columns]
@@ -521,8 +521,8 @@ __global__ void __launch_bounds__(128) bwd_kernel(const Prob p, const bf16* __re
         for (int j = 0; j < 4; ++j) {
           uint32_t b[4];
           load_b_kn<DQK>(b, sQ, 0, nc0 + 2 * j, lane);
-          mma16816(acc[2 * j], adsT, b[0], b[1]);
-          mma16816(acc[2 * j + 1], adsT, b[2], b[3]);
+          Elt<F16>::mma(acc[2 * j], adsT, b[0], b[1]);
+          Elt<F16>::mma(acc[2 * j + 1], adsT, b[2], b[3]);
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -536,8 +536,8 @@ __global__ void __launch_bounds__(128) bwd_kernel(const Prob p, const bf16* __re
           for (int j = 0; j < 4; ++j) {
             uint32_t b[4];
             load_b_kn<DV>(b, sDO, 0, nc0 + 2 * j, lane);
-            mma16816(acc[2 * j], apT, b[0], b[1]);
-            mma16816(acc[2 * j + 1], apT, b[2], b[3]);
+            Elt<F16>::mma(acc[2 * j], apT, b[0], b[1]);
+            Elt<F16>::mma(acc[2 * j + 1], apT, b[2], b[3]);
           }
         }
 #pragma unroll
@@ -559,8 +559,8 @@ __global__ void __launch_bounds__(128) bwd_kernel(const Prob p, const bf16* __re
           for (int j = 0; j < 4; ++j) {
             uint32_t b[4];
             load_b_kn<DV>(b, sDO, 0, nc0 + 2 * j, lane);
-            mma16816(acc[2 * j], apT, b[0], b[1]);
-            mma16816(acc[2 * j + 1], apT, b[2], b[3]);
+            Elt<F16>::mma(acc[2 * j], apT, b[0], b[1]);
+            Elt<F16>::mma(acc[2 * j + 1], apT, b[2], b[3]);
           }
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -581,8 +581,8 @@ __global__ void __launch_bounds__(128) bwd_kernel(const Prob p, const bf16* __re
       for (int j = 0; j < NQ / 2; ++j) {
         uint32_t b[4];
         load_b_kn<DQK>(b, bK, kc * 8, warp * NQ + 2 * j, lane);
-        mma16816(dq[2 * j], a, b[0], b[1]);
-        mma16816(dq[2 * j + 1], a, b[2], b[3]);
+        Elt<F16>::mma(dq[2 * j], a, b[0], b[1]);
+        Elt<F16>::mma(dq[2 * j + 1], a, b[2], b[3]);
       }
     }
   }
@@ -598,7 +598,7 @@ __global__ void __launch_bounds__(128) bwd_kernel(const Prob p, const bf16* __re
     for (int i = 0; i < NQ; ++i) {
       int col = i * 8 + 2 * (lane & 3);
       *reinterpret_cast<uint32_t*>(qrow + col) =
-          pack_bf16(dq[i][2 * r] * p.scale, dq[i][2 * r + 1] * p.scale);
+          Elt<F16>::pack(dq[i][2 * r] * p.scale, dq[i][2 * r + 1] * p.scale);
     }
   }
   // dSinks: -P_sink * sum_j P_j dP_j summed over this CTA's rows
@@ -624,6 +624,7 @@ __global__ void __launch_bounds__(128) bwd_kernel(const Prob p, const bf16* __re
 // ---------------------------------------------------------------------------
 // rowsum(dO o O), finalize, checks, inspection
 // ---------------------------------------------------------------------------
+template <bool F16>
 __global__ void __launch_bounds__(256) delta_kernel(const bf16* __restrict__ O, const bf16* __restrict__ dO,
                                                     float* __restrict__ delta, long long rows, int dv) {
   pdl_wait();
@@ -631,10 +632,12 @@ __global__ void __launch_bounds__(256) delta_kernel(const bf16* __restrict__ O, 
   long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   int lane = threadIdx.x & 31;
   if (row >= rows) return;
-  const float acc = warp_row_dot_bf16(O + row * dv, dO + row * dv, dv, lane);
+  const float acc = warp_row_dot_bf16<F16>(O + row * dv, dO + row * dv, dv, lane);
   if (lane == 0) delta[row] = acc;
 }
 
+// fp32 -> the output element type (bf16, or fp16 with F16), eight at a time.
+template <bool F16>
 __global__ void __launch_bounds__(256) to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__ dst,
                                                       long long n8) {
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
@@ -642,10 +645,10 @@ __global__ void __launch_bounds__(256) to_bf16_kernel(const float* __restrict__ 
     float4 a = __ldg(reinterpret_cast<const float4*>(src) + 2 * i);
     float4 b = __ldg(reinterpret_cast<const float4*>(src) + 2 * i + 1);
     uint4 r;
-    r.x = pack_bf16(a.x, a.y);
-    r.y = pack_bf16(a.z, a.w);
-    r.z = pack_bf16(b.x, b.y);
-    r.w = pack_bf16(b.z, b.w);
+    r.x = Elt<F16>::pack(a.x, a.y);
+    r.y = Elt<F16>::pack(a.z, a.w);
+    r.z = Elt<F16>::pack(b.x, b.y);
+    r.w = Elt<F16>::pack(b.z, b.w);
     reinterpret_cast<uint4*>(dst)[i] = r;
   }
 }
@@ -656,6 +659,7 @@ struct CvtJobs {
   int n;
 };
 
+template <bool F16>
 __global__ void __launch_bounds__(256) to_bf16_multi_kernel(const CvtJobs J) {
   pdl_wait();
   pdl_trigger();
@@ -668,10 +672,10 @@ __global__ void __launch_bounds__(256) to_bf16_multi_kernel(const CvtJobs J) {
     const float4* src = reinterpret_cast<const float4*>(J.job[k].src);
     float4 a = __ldg(src + 2 * li), b = __ldg(src + 2 * li + 1);
     uint4 r;
-    r.x = pack_bf16(a.x, a.y);
-    r.y = pack_bf16(a.z, a.w);
-    r.z = pack_bf16(b.x, b.y);
-    r.w = pack_bf16(b.z, b.w);
+    r.x = Elt<F16>::pack(a.x, a.y);
+    r.y = Elt<F16>::pack(a.z, a.w);
+    r.z = Elt<F16>::pack(b.x, b.y);
+    r.w = Elt<F16>::pack(b.z, b.w);
     reinterpret_cast<uint4*>(J.job[k].dst)[li] = r;
   }
 }
@@ -729,10 +733,10 @@ bool kernels_built(int dqk, int dv, bool shared) {
   return false;
 }
 
-template <int DQK, int DV, bool SHARED>
+template <int DQK, int DV, bool SHARED, bool F16>
 static cudaError_t fwd_t(const Prob& p, bf16* o, float* lse, cudaStream_t st) {
   using PL = Plan<DQK, DV, SHARED>;
-  auto k = fwd_kernel<DQK, DV, SHARED>;
+  auto k = fwd_kernel<DQK, DV, SHARED, F16>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kBytes);
   if (e != cudaSuccess) return e;
   long long grid = (long long)p.Tq * p.Hkv * ((p.G + 15) / 16);
@@ -743,11 +747,11 @@ static cudaError_t fwd_t(const Prob& p, bf16* o, float* lse, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int DQK, int DV, bool SHARED, bool SCATTER = true>
+template <int DQK, int DV, bool SHARED, bool SCATTER, bool F16>
 static cudaError_t bwd_t(const Prob& p, const bf16* d_o, const float* lse, const float* delta,
                          const BwdOut& out, cudaStream_t st) {
   using PL = Plan<DQK, DV, SHARED>;
-  auto k = bwd_kernel<DQK, DV, SHARED, SCATTER>;
+  auto k = bwd_kernel<DQK, DV, SHARED, SCATTER, F16>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kBytes);
   if (e != cudaSuccess) return e;
   long long grid = (long long)p.Tq * p.Hkv * ((p.G + 15) / 16);
@@ -759,10 +763,10 @@ static cudaError_t bwd_t(const Prob& p, const bf16* d_o, const float* lse, const
   return cudaGetLastError();
 }
 
-template <int DQK, int DV, bool SHARED>
+template <int DQK, int DV, bool SHARED, bool F16>
 static cudaError_t l1_t(const Prob& p, const float* lse, float* ori_out, float* cmp_out, cudaStream_t st) {
   using PL = Plan<DQK, DV, SHARED>;
-  auto k = l1_sum_kernel<DQK, DV, SHARED>;
+  auto k = l1_sum_kernel<DQK, DV, SHARED, F16>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kBytes);
   if (e != cudaSuccess) return e;
   const long long units = (long long)p.Tq * p.Hkv;
@@ -786,16 +790,18 @@ static cudaError_t l1_t(const Prob& p, const float* lse, float* ori_out, float* 
 }
 
 cudaError_t launch_softmax_l1norm(const Prob& p, const float* lse, float* ori_out, float* cmp_out, cudaStream_t st) {
-#define X(A, B, C) \
-  if (p.dqk == A && p.dv == B && (bool)p.shared == C) return l1_t<A, B, C>(p, lse, ori_out, cmp_out, st);
+#define X(A, B, C)                                                                                          \
+  if (p.dqk == A && p.dv == B && (bool)p.shared == C)                                                       \
+    return p.f16 ? l1_t<A, B, C, true>(p, lse, ori_out, cmp_out, st) : l1_t<A, B, C, false>(p, lse, ori_out, cmp_out, st);
   SA_FOR_EACH_SHAPE(X)
 #undef X
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_fwd(const Prob& p, bf16* o, float* lse, cudaStream_t st) {
-#define X(A, B, C) \
-  if (p.dqk == A && p.dv == B && (bool)p.shared == C) return fwd_t<A, B, C>(p, o, lse, st);
+#define X(A, B, C)                              \
+  if (p.dqk == A && p.dv == B && (bool)p.shared == C) \
+    return p.f16 ? fwd_t<A, B, C, true>(p, o, lse, st) : fwd_t<A, B, C, false>(p, o, lse, st);
   SA_FOR_EACH_SHAPE(X)
 #undef X
   return cudaErrorInvalidValue;
@@ -804,8 +810,10 @@ cudaError_t launch_fwd(const Prob& p, bf16* o, float* lse, cudaStream_t st) {
 cudaError_t launch_bwd(const Prob& p, const bf16* o, const bf16* d_o, const float* lse,
                        const float* delta, const BwdOut& out, cudaStream_t st) {
   (void)o;
-#define X(A, B, C) \
-  if (p.dqk == A && p.dv == B && (bool)p.shared == C) return bwd_t<A, B, C>(p, d_o, lse, delta, out, st);
+#define X(A, B, C)                                                         \
+  if (p.dqk == A && p.dv == B && (bool)p.shared == C)                          \
+    return p.f16 ? bwd_t<A, B, C, true, true>(p, d_o, lse, delta, out, st)     \
+                 : bwd_t<A, B, C, true, false>(p, d_o, lse, delta, out, st);
   SA_FOR_EACH_SHAPE(X)
 #undef X
   return cudaErrorInvalidValue;
@@ -814,31 +822,37 @@ cudaError_t launch_bwd(const Prob& p, const bf16* o, const bf16* d_o, const floa
 cudaError_t launch_bwd_dq(const Prob& p, const bf16* d_o, const float* lse, const float* delta,
                           const BwdOut& out, cudaStream_t st) {
   // dQ only (dK / dV come from the key-stationary kernel); dSinks needs no sinks here
-  if (p.dqk == 64 && p.dv == 64 && !p.shared) return bwd_t<64, 64, false, false>(p, d_o, lse, delta, out, st);
-  if (p.dqk == 128 && p.dv == 128 && !p.shared) return bwd_t<128, 128, false, false>(p, d_o, lse, delta, out, st);
-  if (p.dqk == 192 && p.dv == 128 && !p.shared) return bwd_t<192, 128, false, false>(p, d_o, lse, delta, out, st);
+  if (p.dqk == 64 && p.dv == 64 && !p.shared) return bwd_t<64, 64, false, false, false>(p, d_o, lse, delta, out, st);
+  if (p.dqk == 128 && p.dv == 128 && !p.shared)
+    return bwd_t<128, 128, false, false, false>(p, d_o, lse, delta, out, st);
+  if (p.dqk == 192 && p.dv == 128 && !p.shared)
+    return bwd_t<192, 128, false, false, false>(p, d_o, lse, delta, out, st);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_delta(const bf16* o, const bf16* d_o, float* delta, long long rows, int dv,
-                         cudaStream_t st) {
+                         cudaStream_t st, bool f16) {
   if (rows == 0) return cudaSuccess;
-  cudaError_t e = launch_pdl(delta_kernel, (unsigned)((rows + 7) / 8), 256, 0, st, o, d_o, delta, rows, dv);
+  cudaError_t e = f16 ? launch_pdl(delta_kernel<true>, (unsigned)((rows + 7) / 8), 256, 0, st, o, d_o, delta, rows, dv)
+                      : launch_pdl(delta_kernel<false>, (unsigned)((rows + 7) / 8), 256, 0, st, o, d_o, delta, rows, dv);
   count_launch();
   return e;
 }
 
-cudaError_t launch_to_bf16(const float* src, bf16* dst, long long n, cudaStream_t st) {
+cudaError_t launch_to_bf16(const float* src, bf16* dst, long long n, cudaStream_t st, bool f16) {
   if (n == 0) return cudaSuccess;
   long long n8 = n / 8;  // every caller's n is a multiple of 64
   long long blocks = (n8 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  to_bf16_kernel<<<(unsigned)blocks, 256, 0, st>>>(src, dst, n8);
+  if (f16)
+    to_bf16_kernel<true><<<(unsigned)blocks, 256, 0, st>>>(src, dst, n8);
+  else
+    to_bf16_kernel<false><<<(unsigned)blocks, 256, 0, st>>>(src, dst, n8);
   count_launch();
   return cudaGetLastError();
 }
 
-cudaError_t launch_to_bf16_multi(const Cvt* jobs, int njobs, cudaStream_t st) {
+cudaError_t launch_to_bf16_multi(const Cvt* jobs, int njobs, cudaStream_t st, bool f16) {
   CvtJobs J;
   J.n = 0;
   long long acc = 0;
@@ -852,7 +866,8 @@ cudaError_t launch_to_bf16_multi(const Cvt* jobs, int njobs, cudaStream_t st) {
   if (J.n == 0) return cudaSuccess;
   long long blocks = (acc + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  cudaError_t e = launch_pdl(to_bf16_multi_kernel, (unsigned)blocks, 256, 0, st, J);
+  cudaError_t e = f16 ? launch_pdl(to_bf16_multi_kernel<true>, (unsigned)blocks, 256, 0, st, J)
+                      : launch_pdl(to_bf16_multi_kernel<false>, (unsigned)blocks, 256, 0, st, J);
   count_launch();
   return e;
 }
