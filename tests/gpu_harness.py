@@ -107,9 +107,11 @@ def compare_grads(tag: str, got: dict, ref: dict, T: int, w):
     check_close(f"{tag}:dq", widen(got["dq"]).reshape(T, -1), widen(ref["dq"]).reshape(T, -1))
 
 
-def run_full_comparison(w, gen_kwargs=None, flags=0):
-    """Small workload: every output element compared with the oracle."""
-    inputs = make_inputs(w, **(gen_kwargs or {}))
+def run_full_comparison(w, gen_kwargs=None, flags=0, inputs=None):
+    """Small workload: every output element compared with the oracle (on ``inputs``
+    when given, else on the workload's generated inputs)."""
+    if inputs is None:
+        inputs = make_inputs(w, **(gen_kwargs or {}))
     p = oracle.Problem.from_inputs(w, inputs)
     T = w.T
     sa, t = device_problem(w, inputs, flags)

@@ -181,3 +181,37 @@ def test_calls_capture_in_a_cuda_graph(name):
             check_close(f"graph:{key}", got[key], ref_g[key])
         else:
             check_close(f"graph:{key}", widen(got[key]), widen(ref_g[key]))
+
+
+def _with_duplicates(inputs, key, every=3):
+    """A copy of the inputs in which, for every ``every``-th (token, kv-head) list, slot 1
+    repeats slot 0's index when slot 0 is in use (a selection that names a row or block
+    twice)."""
+    out = dict(inputs)
+    idx = np.array(inputs[key], copy=True)
+    flat = idx.reshape(-1, idx.shape[-1])
+    rows = np.arange(0, flat.shape[0], every)
+    take = rows[flat[rows, 0] >= 0]
+    flat[take, 1] = flat[take, 0]
+    out[key] = idx
+    return out, len(take)
+
+
+DUP_CASES = {
+    "token_h64_dup": ("token_h64_topk", "ori_idx"),      # tcgen05 token kernels
+    "block_cfg2_dup": ("cfg2_small", "ori_idx"),         # TMA-fed block forward, key-stationary backward
+    "block_bs16_dup": ("block_bs16_d64", "ori_idx"),     # generic kernels
+    "swa_cmp_dup": ("swa_cmp_h64", "cmp_idx"),           # token kernels, repeated compressed rows
+}
+
+
+@pytest.mark.parametrize("name", list(DUP_CASES))
+def test_duplicate_indices_count_twice(name):
+    """A row or block named twice in one selection list contributes twice, as the oracle's
+    slot-by-slot gather counts it (duplicate indices are taken with multiplicity)."""
+    _need_gpu()
+    base, key = DUP_CASES[name]
+    w, kw = SMALL[base]
+    inputs, n = _with_duplicates(make_inputs(w, **kw), key)
+    assert n > 0
+    run_full_comparison(w, inputs=inputs)
