@@ -23,6 +23,9 @@
 // running maximum moves only when a sub-tile's maximum exceeds it by more than 8
 // (a factor of 256 in the exponentials): O and the running sum are then rescaled
 // once, after the previous P V has landed.  Sinks start the running state.
+// With 128 query heads per kv-head the two 64-head CTAs of a token run as a
+// two-CTA cluster: each gathers half of every sub-tile and copies it into the
+// other's stage over distributed shared memory (tk_load_rows, PAIR).
 //
 // Backward (SparseFlashMlaGrad Stages 2-3: P recomputed from lse, dP = dO V^T,
 // dS = P o (dP - Delta), dQ = dS K scale, dKV = dS^T Q scale + P^T dO), per
