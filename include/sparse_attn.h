@@ -175,7 +175,9 @@ typedef enum sa_dtype { SA_DTYPE_BF16 = 0, SA_DTYPE_FP16 = 1 } sa_dtype;
  * the two 64-head CTAs of a token run as a thread-block cluster and share the row
  * gathers (each gathers every other 32-row sub-tile and copies it to the other
  * over distributed shared memory).  This flag runs every 64-head CTA on its own
- * instead; the result is bit-identical. */
+ * instead; the result is bit-identical.  It also serves where a two-CTA cluster of
+ * this kernel's shared memory cannot be scheduled (the launch then fails and
+ * sa_fwd returns SA_ERR_CUDA): the unpaired kernel needs no clusters. */
 #define SA_FLAG_TOKEN_FWD_UNPAIRED 16u
 
 /* Kernels reported by sa_plan(). */
