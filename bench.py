@@ -388,10 +388,10 @@ def compulsory_bytes(w, work) -> dict:
 
 def fractions(work, comp, peaks, fwd_ms, bwd_ms) -> dict:
     """Roofline fractions (burst tensor peak, measured HBM bandwidth):
-    the benchmark spec -- the slower of FLOPs at the tensor peak and gathered + compulsory
-                  bytes at HBM bandwidth, over the measured time;
-    tensor     -- the slower of FLOPs at the tensor peak and compulsory bytes only
-                  (the stricter figure: gathers that hit L2 or are avoided do not count).
+    gather_model -- the slower of FLOPs at the tensor peak and gathered + compulsory
+                    bytes at HBM bandwidth, over the measured time;
+    tensor       -- the slower of FLOPs at the tensor peak and compulsory bytes only
+                    (the stricter figure: gathers that hit L2 or are avoided do not count).
     A fraction above 1 means that model does not bind (the kernel beat it)."""
     P, BW = peaks["bf16_tflops"] * 1e12, peaks["hbm_gbs"] * 1e9
     out = {}
@@ -399,9 +399,9 @@ def fractions(work, comp, peaks, fwd_ms, bwd_ms) -> dict:
                                     ("bwd", bwd_ms, work["bwd_flops"], work["bwd_main_bytes"])):
         ns = max(flops / P, gbytes / BW) * 1e3 / ms
         tc = max(flops / P, comp[side] / BW) * 1e3 / ms
-        out[f"{side}_north_star_frac"] = ns
+        out[f"{side}_gather_model_frac"] = ns
         out[f"{side}_tensor_frac"] = tc
-        out[f"{side}_north_star_binding"] = ns <= 1.0
+        out[f"{side}_gather_model_binding"] = ns <= 1.0
     return out
 
 
@@ -553,7 +553,7 @@ def dominant_kernel_roofline(w, work, comp, peaks, peak_src, plan, m) -> dict:
             "peak_source": ("measured MEASURED_PEAKS.json (bf16 burst; HBM copy)" if peak_src == "measured"
                             else "fallback"),
             "t_roof_ms": max(t_f, t_b) * 1e3,
-            "north_star_frac": ns, "north_star_binding": ns <= 1.0,
+            "gather_model_frac": ns, "gather_model_binding": ns <= 1.0,
             "dram_over_compulsory": None if traffic is None else traffic / cbytes}
 
 
@@ -661,7 +661,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
                     "bwd_tflops": work2["bwd_flops"] / (m2["bwd_ms"] * 1e-3) / 1e12,
                     "fwd_kernel": KERNEL_NAMES[plan2[0]], "bwd_kernel": KERNEL_NAMES[plan2[1]],
                     **fr,
-                    "bwd_north_star_frac_in_step": fr_step["bwd_north_star_frac"],
+                    "bwd_gather_model_frac_in_step": fr_step["bwd_gather_model_frac"],
                     "bwd_tensor_frac_in_step": fr_step["bwd_tensor_frac"],
                     "roofline": roof2, "clocks": clk2.summary(),
                     "config": config_of(w2, work2, world, "")}
@@ -707,7 +707,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         # the backward as part of a one-graph step (forward then backward), minus the
         # forward alone: the fixed cost of starting a graph of its own drops out
         "step_graph_ms": m["step_graph_ms"], "bwd_in_step_ms": m["bwd_in_step_ms"],
-        "bwd_north_star_frac_in_step": fr_step["bwd_north_star_frac"],
+        "bwd_gather_model_frac_in_step": fr_step["bwd_gather_model_frac"],
         "bwd_tensor_frac_in_step": fr_step["bwd_tensor_frac"],
         "roofline": roof, "clocks": clk.summary(), "gpu_launches": m["launches"],
         # fp32 dQ / dK / dV reductions (L2 read-modify-writes, not DRAM bytes) of the

@@ -85,8 +85,8 @@ def test_roofline_fractions():
     assert comp["fwd"] < work["fwd_bytes"] and comp["bwd"] < work["bwd_main_bytes"] + comp["bwd"]
     peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}
     fr = bench.fractions(work, comp, peaks, fwd_ms=0.05, bwd_ms=0.05)
-    assert fr["fwd_tensor_frac"] <= fr["fwd_north_star_frac"]
-    assert fr["bwd_tensor_frac"] <= fr["bwd_north_star_frac"]
+    assert fr["fwd_tensor_frac"] <= fr["fwd_gather_model_frac"]
+    assert fr["bwd_tensor_frac"] <= fr["bwd_gather_model_frac"]
     # a time at exactly the spec roofline is a fraction of one
     t_ns = max(work["bwd_flops"] / 1e15, work["bwd_main_bytes"] / 5e12) * 1e3
-    assert abs(bench.fractions(work, comp, peaks, 1.0, t_ns)["bwd_north_star_frac"] - 1.0) < 1e-9
+    assert abs(bench.fractions(work, comp, peaks, 1.0, t_ns)["bwd_gather_model_frac"] - 1.0) < 1e-9
