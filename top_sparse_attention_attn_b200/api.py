@@ -20,6 +20,17 @@ def _ptr(t) -> int | None:
     return None if t is None else int(t.data_ptr())
 
 
+_ELEMENT_TYPES = {torch.bfloat16: L.SA_DTYPE_BF16, torch.float16: L.SA_DTYPE_FP16}
+
+
+def _same_element_type(ref: torch.Tensor, **tensors) -> None:
+    """The C ABI takes raw pointers: every 2-byte tensor of a call must hold the
+    element type sa_args.dtype names (that of q)."""
+    for name, t in tensors.items():
+        if t is not None and t.dtype != ref.dtype:
+            raise TypeError(f"{name} is {t.dtype}, q is {ref.dtype}: one element type per call")
+
+
 @dataclass
 class SparseAttention:
     layout: str                  # "BSND" | "TND"
@@ -80,7 +91,10 @@ class SparseAttention:
         a = L.SaArgs()
         a.layout_q = L.LAYOUTS[self.layout]
         a.layout_kv = L.LAYOUTS[self.layout]
-        a.dtype = L.SA_DTYPE_FP16 if self.q.dtype == torch.float16 else L.SA_DTYPE_BF16
+        if self.q.dtype not in _ELEMENT_TYPES:
+            raise TypeError(f"q is {self.q.dtype}: bfloat16 or float16 expected")
+        _same_element_type(self.q, k=self.k, v=self.v, kv=self.kv, cmp_kv=self.cmp_kv)
+        a.dtype = _ELEMENT_TYPES[self.q.dtype]
         a.batch = self.batch
         a.s_q, a.s_kv = self.s_q, self.s_kv
         a.t_q, a.t_kv, a.t_cmp = self.t_q, self.t_kv, self.t_cmp
@@ -147,6 +161,7 @@ class SparseAttention:
             o, lse = self.alloc_fwd()
         if ws is None:
             ws = self.fwd_workspace()
+        _same_element_type(self.q, o=o)
         out = L.SaFwdOut(o=_ptr(o), lse=_ptr(lse))
         st = torch.cuda.current_stream().cuda_stream if stream is None else stream
         L.sa_fwd(self.args(), out, _ptr(ws), ws.numel(), st)
@@ -157,6 +172,8 @@ class SparseAttention:
             grads = self.alloc_bwd()
         if ws is None:
             ws = self.bwd_workspace()
+        _same_element_type(self.q, o=o, d_o=d_o, dq=grads["dq"], dk=grads.get("dk"), dv=grads.get("dv"),
+                           dkv=grads.get("dkv"), dcmp=grads.get("dcmp"))
         io = L.SaBwdIo(o=_ptr(o), d_o=_ptr(d_o), lse=_ptr(lse), dq=_ptr(grads["dq"]),
                        dk=_ptr(grads.get("dk")), dv=_ptr(grads.get("dv")),
                        dkv=_ptr(grads.get("dkv")), dcmp_kv=_ptr(grads.get("dcmp")),
@@ -166,6 +183,7 @@ class SparseAttention:
         return grads
 
     def delta(self, o, d_o, stream=None) -> torch.Tensor:
+        _same_element_type(self.q, o=o, d_o=d_o)
         out = torch.empty(self._lead() + (self.Hq,), dtype=torch.float32, device=self.q.device)
         st = torch.cuda.current_stream().cuda_stream if stream is None else stream
         L.sa_softmax_grad_preprocess(self.args(), _ptr(o), _ptr(d_o), _ptr(out), st)
